@@ -1,0 +1,357 @@
+"""Oracle: group-wise INT4 (asymmetric, RTN) and NF4 (double-quantized) weight
+quantization, packing, dequantization and the fp64 matmul reference.
+
+TEST INFRASTRUCTURE ONLY -- see the package docstring for who may import it.
+
+Page titles cited below (the five source pages):
+
+* [Survey]     "大模型量化选型：五种主流方案对比与实战"
+* [Primer]     the aicoding.csdn.net primer whose first heading is
+               "一、量化究竟做了什么"
+* [Handbook]   "这不是理论课，是能立刻上手的LLM量化实操手册"
+* [Guide]      "开源模型量化实战指南：GGUF、GPTQ、AWQ选型与本地部署"
+* [Comparison] "【推理与部署篇05】模型量化部署深度对比：GPTQ、AWQ、GGUF与FP8实战指南"
+
+Readings taken where the pages leave a step open (each is listed, with its
+reason, in the design notes):
+
+R1  the group range includes 0 (``mn = min(min w, 0)``, ``mx = max(max w, 0)``)
+    so that the zero point always fits in 4 bits;
+R2  the scale is stored in fp16 and every later step uses the fp16 value; a
+    zero scale becomes 1.0;
+R3  "round" is round-half-to-even (``numpy.rint``);
+R4  nibble order: even k in the low nibble of byte k // 2;
+R5  the dequantized weight is the bf16 (round-to-nearest-even) of the exact
+    fp32 product ``(q - zp) * scale``;
+R6  NF4 levels are the normal-quantile construction with an exact zero
+    (8 positive, 7 negative quantiles, normalised to [-1, 1]);
+R7  an NF4 value on a midpoint takes the lower code;
+R8  double quantization: per run of 256 consecutive blocks,
+    ``s2 = max(absmax) / 255``, ``c = rint(absmax / s2)`` in [0, 255],
+    ``absmax' = c * s2`` in fp32; codes are chosen with the unquantized absmax;
+R9  NF4 dequant is ``bf16(fp32(T[q] * absmax'))``.
+
+All floating-point steps are numpy float32 operations (IEEE, round to nearest
+even) unless stated as fp64; the matmul accumulates in fp64.
+"""
+from __future__ import annotations
+
+import math
+import statistics
+from fractions import Fraction
+
+import numpy as np
+
+__all__ = [
+    "bf16_round_bits", "bf16_bits_to_f64", "bf16_bits_to_f32",
+    "group_index", "rtn_params", "quantize_rtn", "pack_nibbles", "unpack_nibbles",
+    "dequant_rtn_f32", "dequant_rtn", "nf4_table", "nf4_midpoints", "nf4_absmax",
+    "nf4_codes", "nf4_double_quant", "nf4_quantize", "nf4_dequant", "matmul_ref",
+    "matmul_exact_small", "ulp_bf16", "tolerance", "check_matmul",
+    "weight_bytes", "code_bytes", "nf4_weight_bytes",
+]
+
+F32 = np.float32
+
+
+# ---------------------------------------------------------------------------
+# bf16 rounding (R5): keep the top 16 bits of the fp32 pattern, rounding the
+# discarded low 16 bits to nearest, ties to the even result.
+# ---------------------------------------------------------------------------
+
+def bf16_round_bits(f: np.ndarray) -> np.ndarray:
+    """fp32 values -> bf16 bit patterns (uint16), round to nearest even.
+
+    Finite inputs only (no NaN handling is needed: the path never produces
+    NaN from finite inputs)."""
+    u = np.ascontiguousarray(f, dtype=F32).view(np.uint32).astype(np.uint64)
+    keep_lsb = (u >> np.uint64(16)) & np.uint64(1)
+    rounded = (u + np.uint64(0x7FFF) + keep_lsb) >> np.uint64(16)
+    return rounded.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(F32)
+
+
+def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    return bf16_bits_to_f32(b).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# INT4 asymmetric round-to-nearest, group-wise along K.
+# [Comparison] §2.3 gives the asymmetric min-max formulas for 8 bits
+# (scale = (max - min)/255, zero_point = round(-min/scale), range [0, 255]);
+# with 4 bits the denominator is 2^4 - 1 = 15 and the range is [0, 15].
+# [Comparison] §2.2 and [Primer] §二 give per-group granularity (one scale per
+# group of G weights, G = 128/64/32); [Primer] §四 names plain rounding (RTN).
+# ---------------------------------------------------------------------------
+
+def group_index(K: int, G: int, g_idx: np.ndarray | None) -> np.ndarray:
+    """Group id of every input channel k.  Without act-order the groups are the
+    contiguous runs [gG, (g+1)G); with act-order ([Survey] §3.2 desc_act,
+    [Guide] §3.2: inference must reorder) channel k belongs to g_idx[k]."""
+    if K % G:
+        raise ValueError("K must be a multiple of G")
+    if g_idx is None:
+        return np.arange(K, dtype=np.int64) // G
+    g = np.asarray(g_idx).astype(np.int64)
+    if g.shape != (K,):
+        raise ValueError("g_idx must have shape [K]")
+    if g.size and (g.min() < 0 or g.max() >= K // G):
+        raise ValueError("g_idx values must lie in [0, K/G)")
+    return g
+
+
+def _group_minmax(W: np.ndarray, G: int, gk: np.ndarray, contiguous: bool):
+    N, K = W.shape
+    ng = K // G
+    if contiguous:
+        Wg = W.reshape(N, ng, G)
+        return Wg.min(axis=2), Wg.max(axis=2)
+    mn = np.zeros((N, ng), F32)
+    mx = np.zeros((N, ng), F32)
+    for g in range(ng):
+        cols = np.nonzero(gk == g)[0]
+        if cols.size:
+            sub = W[:, cols]
+            mn[:, g] = sub.min(axis=1)
+            mx[:, g] = sub.max(axis=1)
+    return mn, mx
+
+
+def rtn_params(W: np.ndarray, G: int, g_idx: np.ndarray | None = None):
+    """Per (row, group) fp16 scale and zero point (R1, R2, R3).
+
+    Returns (scale_fp16 [N, K/G], zero_uint8 [N, K/G])."""
+    W = np.ascontiguousarray(W, dtype=F32)
+    N, K = W.shape
+    gk = group_index(K, G, g_idx)
+    mn, mx = _group_minmax(W, G, gk, g_idx is None)
+    mn = np.minimum(mn, F32(0))                      # R1
+    mx = np.maximum(mx, F32(0))
+    s32 = (mx - mn) / F32(15.0)                      # scale = (max - min) / (2^4 - 1)
+    s16 = s32.astype(np.float16)                     # R2: stored fp16 (round to nearest even)
+    s16[s16 == 0] = np.float16(1.0)
+    sf = s16.astype(F32)
+    zp = np.clip(np.rint(-mn / sf), 0, 15)           # zero_point = round(-min / scale)
+    return s16, zp.astype(np.uint8)
+
+
+def quantize_rtn(W: np.ndarray, G: int, g_idx: np.ndarray | None = None):
+    """Codes q = clamp(round(w / scale) + zp, 0, 15) (one uint8 per weight).
+
+    Returns (codes uint8 [N, K], scale fp16 [N, K/G], zero uint8 [N, K/G])."""
+    W = np.ascontiguousarray(W, dtype=F32)
+    N, K = W.shape
+    gk = group_index(K, G, g_idx)
+    s16, zp = rtn_params(W, G, g_idx)
+    sk = s16.astype(F32)[:, gk]
+    zk = zp.astype(F32)[:, gk]
+    q = np.clip(np.rint(W / sk) + zk, 0, 15)
+    return q.astype(np.uint8), s16, zp
+
+
+def pack_nibbles(codes: np.ndarray) -> np.ndarray:
+    """Two 4-bit codes per byte, even k in the low nibble (R4); [Guide] §1.1:
+    an INT4 value takes half a byte."""
+    c = np.asarray(codes, dtype=np.uint8)
+    if c.shape[-1] % 2:
+        raise ValueError("K must be even")
+    return (c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)
+
+
+def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def dequant_rtn_f32(Wq: np.ndarray, scales: np.ndarray, zeros: np.ndarray, G: int,
+                    g_idx: np.ndarray | None = None) -> np.ndarray:
+    """Exact fp32 value (q - zp) * scale before the bf16 rounding.  The product
+    of a |q - zp| <= 15 integer and an 11-bit fp16 significand is exact in fp32."""
+    q = unpack_nibbles(Wq).astype(F32)
+    K = q.shape[1]
+    gk = group_index(K, G, g_idx)
+    sk = np.asarray(scales, dtype=np.float16).astype(F32)[:, gk]
+    zk = np.asarray(zeros, dtype=np.uint8).astype(F32)[:, gk]
+    return (q - zk) * sk
+
+
+def dequant_rtn(Wq, scales, zeros, G, g_idx=None) -> np.ndarray:
+    """Dequantized weight as bf16 bits [N, K] (R5); the pages dequantize to the
+    bf16 compute dtype before the matmul ([Survey] §6.2, [Primer] §七)."""
+    return bf16_round_bits(dequant_rtn_f32(Wq, scales, zeros, G, g_idx))
+
+
+# ---------------------------------------------------------------------------
+# NF4.  [Survey] §6.1: 16 levels placed at quantiles of the normal
+# distribution, denser near zero; [Comparison] §6.2: non-uniform, follows the
+# normal CDF; [Survey] §6.3: block-wise, one scale per 64 weights by default;
+# [Survey] §6.2 and [Comparison] §6.1: double quantization of the scales.
+# ---------------------------------------------------------------------------
+
+def nf4_table() -> np.ndarray:
+    """16 NF4 levels (R6), evaluated in fp64, rounded once to fp32.
+
+    Quantile points: delta = 1 - (1/30 + 1/32)/2.  Eight positive levels at
+    the first 8 of 9 equally spaced probabilities from delta down to 1/2,
+    seven negative levels (mirrored) at the first 7 of 8 such probabilities,
+    plus an exact zero; divided by the largest level so the table spans
+    [-1, 1]."""
+    nd = statistics.NormalDist()
+    delta = 1.0 - 0.5 * (1.0 / 30.0 + 1.0 / 32.0)
+    pos = [nd.inv_cdf(delta + (0.5 - delta) * i / 8.0) for i in range(8)]
+    neg = [-nd.inv_cdf(delta + (0.5 - delta) * i / 7.0) for i in range(7)]
+    levels = sorted(neg + [0.0] + pos)
+    top = nd.inv_cdf(delta)
+    return np.array([v / top for v in levels], dtype=np.float64).astype(F32)
+
+
+def nf4_midpoints() -> np.ndarray:
+    """Decision thresholds t_i = fp32((T[i] + T[i+1]) / 2), i = 0..14."""
+    T = nf4_table().astype(np.float64)
+    return ((T[:-1] + T[1:]) / 2.0).astype(F32)
+
+
+def _blocks(W: np.ndarray, blocksize: int) -> np.ndarray:
+    flat = np.ascontiguousarray(W, dtype=F32).reshape(-1)
+    if flat.size % blocksize:
+        raise ValueError("N*K must be a multiple of the block size")
+    return flat.reshape(-1, blocksize)
+
+
+def nf4_absmax(W: np.ndarray, blocksize: int = 64) -> np.ndarray:
+    """fp32 absmax of each block of `blocksize` consecutive row-major weights."""
+    return np.abs(_blocks(W, blocksize)).max(axis=1)
+
+
+def nf4_codes(W: np.ndarray, blocksize: int = 64) -> np.ndarray:
+    """Code of each weight: v = w / absmax (fp32 divide; 0 if absmax is 0),
+    q = number of thresholds t_i with v > t_i (R7).  Returns uint8 [N, K]."""
+    B = _blocks(W, blocksize)
+    a = np.abs(B).max(axis=1)
+    safe = np.where(a > 0, a, F32(1.0)).astype(F32)
+    v = np.where(a[:, None] > 0, B / safe[:, None], F32(0.0)).astype(F32)
+    q = np.searchsorted(nf4_midpoints(), v, side="left")   # count of t_i < v
+    return q.astype(np.uint8).reshape(np.shape(W))
+
+
+def nf4_double_quant(absmax: np.ndarray, dq_group: int = 256):
+    """R8: returns (c uint8 [nblocks], s2 fp32 [ceil(nblocks/dq_group)])."""
+    a = np.asarray(absmax, dtype=F32)
+    nb = a.size
+    nruns = (nb + dq_group - 1) // dq_group
+    c = np.empty(nb, np.uint8)
+    s2 = np.empty(nruns, F32)
+    for r in range(nruns):
+        run = a[r * dq_group:(r + 1) * dq_group]
+        s = run.max() / F32(255.0)
+        if s == 0:
+            s = F32(1.0)
+        s2[r] = s
+        c[r * dq_group:(r + 1) * dq_group] = np.clip(np.rint(run / s), 0, 255).astype(np.uint8)
+    return c, s2
+
+
+def nf4_quantize(W: np.ndarray, blocksize: int = 64, dq_group: int = 256):
+    """Returns (packed codes uint8 [N, K/2], absmax codes uint8 [N*K/blocksize],
+    s2 fp32 [ceil(N*K/blocksize/dq_group)])."""
+    q = nf4_codes(W, blocksize)
+    c, s2 = nf4_double_quant(nf4_absmax(W, blocksize), dq_group)
+    return pack_nibbles(q), c, s2
+
+
+def nf4_dequant(Wq: np.ndarray, absmax_q: np.ndarray, s2: np.ndarray,
+                blocksize: int = 64, dq_group: int = 256) -> np.ndarray:
+    """R9: bf16 bits [N, K] of fp32(T[q] * absmax'), absmax' = fp32(c * s2)."""
+    q = unpack_nibbles(Wq)
+    shape = q.shape
+    qb = q.reshape(-1, blocksize)
+    nb = qb.shape[0]
+    c = np.asarray(absmax_q, dtype=np.uint8)[:nb].astype(F32)
+    s = np.asarray(s2, dtype=F32)[np.arange(nb) // dq_group]
+    a_dq = c * s                                              # fp32 product
+    vals = nf4_table()[qb] * a_dq[:, None]                    # fp32 product
+    return bf16_round_bits(vals.reshape(shape))
+
+
+# ---------------------------------------------------------------------------
+# Matmul reference: y[m, n] = sum_k x[m, k] * w_hat[n, k] in fp64, and the
+# tolerance |y - y_ref| <= 1e-3 * sum_k |x w_hat| + ulp_bf16(y_ref).
+# ---------------------------------------------------------------------------
+
+def matmul_ref(x_bits: np.ndarray, what_bits: np.ndarray):
+    """(y_ref, abs_ref) in fp64 for bf16 X [M, K] and bf16 W_hat [N, K]."""
+    x = bf16_bits_to_f64(x_bits)
+    w = bf16_bits_to_f64(what_bits)
+    return x @ w.T, np.abs(x) @ np.abs(w).T
+
+
+def matmul_exact_small(x_bits: np.ndarray, what_bits: np.ndarray) -> list:
+    """Exact rational products and sums by pure-Python loops (tiny inputs)."""
+    x = bf16_bits_to_f32(x_bits)
+    w = bf16_bits_to_f32(what_bits)
+    M, K = x.shape
+    N = w.shape[0]
+    out = []
+    for m in range(M):
+        row = []
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                acc += Fraction(float(x[m, k])) * Fraction(float(w[n, k]))
+            row.append(acc)
+        out.append(row)
+    return out
+
+
+def ulp_bf16(y: np.ndarray) -> np.ndarray:
+    """Spacing of the bf16 grid at |y| (8 significant bits); at 0 and in the
+    subnormal range it is the smallest subnormal, 2^-133."""
+    a = np.abs(np.asarray(y, dtype=np.float64))
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.where(a > 0, e, -200.0)
+    return np.where(e < -126, 2.0 ** -133, np.exp2(e - 7))
+
+
+def tolerance(y_ref: np.ndarray, abs_ref: np.ndarray) -> np.ndarray:
+    return 1e-3 * np.asarray(abs_ref, np.float64) + ulp_bf16(y_ref)
+
+
+def check_matmul(y_bits: np.ndarray, y_ref: np.ndarray, abs_ref: np.ndarray):
+    """Returns (ok, worst error / tolerance ratio)."""
+    y = bf16_bits_to_f64(y_bits)
+    err = np.abs(y - y_ref)
+    tol = tolerance(y_ref, abs_ref)
+    ratio = float((err / tol).max()) if err.size else 0.0
+    return bool(np.all(err <= tol)), ratio
+
+
+# ---------------------------------------------------------------------------
+# Storage sizes.  [Primer] opening: a 7B model is ~14 GB in FP16 and ~3.5 GB in
+# 4 bits; [Survey] §6.2 and [Comparison] §1: 70B goes from 140 GB to ~35 GB;
+# [Handbook] §4.1: codes (params x bits / 8), plus one fp16 scale and one zero
+# per group of 128.
+# ---------------------------------------------------------------------------
+
+def code_bytes(n_params: int, bits: int = 4) -> int:
+    return n_params * bits // 8
+
+
+def weight_bytes(N: int, K: int, G: int, zero_bytes: float = 0.5,
+                 scale_bytes: float = 2.0) -> float:
+    """Bytes of one INT4 layer: codes + per-group scale + per-group zero.
+    This library stores zeros as 4-bit values (0.5 B); the handbook's worked
+    example counts them at 2 B like the scales."""
+    groups = N * (K // G)
+    return code_bytes(N * K) + groups * scale_bytes + groups * zero_bytes
+
+
+def nf4_weight_bytes(N: int, K: int, blocksize: int = 64, dq_group: int = 256) -> float:
+    nb = N * K // blocksize
+    return code_bytes(N * K) + nb + 4 * math.ceil(nb / dq_group)

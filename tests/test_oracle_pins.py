@@ -1,0 +1,438 @@
+"""Pins for the CPU oracle: what the pages and the mathematics fix, checked
+against the oracle without re-typing its formulas.
+
+Each pin is chosen so that a plausible slip in the oracle (a dropped term, a
+wrong sign or index, truncation instead of round-half-even, swapped nibbles, a
+transposed operand) fails at least one of them; ``test_planted_mistakes``
+checks exactly that by planting such slips in copies of oracle functions.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from weight_only_bit_gemm_b200 import synthetic as S
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _parse_worked(path):
+    cases, cur = [], None
+    for line in open(path, encoding="utf-8"):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        key, *vals = line.split()
+        if key == "name":
+            cur = {"name": vals[0]}
+            cases.append(cur)
+        else:
+            cur[key] = vals
+    return cases
+
+
+WORKED = _parse_worked(os.path.join(GOLDEN, "int4_rtn_worked.txt"))
+
+
+# ---------------------------------------------------------------- worked examples
+
+@pytest.mark.parametrize("case", WORKED, ids=lambda c: c["name"])
+def test_int4_worked_examples(case):
+    G = int(case["G"][0])
+    w = np.array([float(v) for v in case["w"]], np.float32)[None, :]
+    codes, s16, zp = O.quantize_rtn(w, G)
+    assert s16.view(np.uint16)[0, 0] == int(case["scale_f16_bits"][0], 16)
+    assert zp[0, 0] == int(case["zero"][0])
+    assert codes[0].tolist() == [int(v) for v in case["codes"]]
+    packed = O.pack_nibbles(codes)
+    assert packed[0].tolist() == [int(v, 16) for v in case["packed_hex"]]
+    if "what_f32" in case:
+        f = O.dequant_rtn_f32(packed, s16, zp, G)
+        assert f[0].tolist() == [float(v) for v in case["what_f32"]]
+    what = O.bf16_bits_to_f32(O.dequant_rtn(packed, s16, zp, G))
+    assert what[0].tolist() == [float(v) for v in case["what"]]
+
+
+def test_sizes_closed_forms():
+    # primer: 7B fp16 ~14 GB, 4-bit ~3.5 GB; survey / comparison: 70B 140 -> 35 GB
+    assert 7_000_000_000 * 2 == 14_000_000_000
+    assert O.code_bytes(7_000_000_000) == 3_500_000_000
+    assert O.code_bytes(70_000_000_000) == 35_000_000_000
+    # handbook §4.1: 1.5e9 params, group 128.  Codes (1.5e9*4)/8 B divided by
+    # 1024^2 is 715.3 (MiB), printed "0.71GB"; scales 1.5e9/128*2 B = 23.4 MB,
+    # printed "0.023GB".  The byte counts are exact; the printed figures carry
+    # a unit slip, so they are matched to their printed digits only.
+    p = 1_500_000_000
+    assert O.code_bytes(p) == 750_000_000
+    assert abs(O.code_bytes(p) / 1024 ** 2 / 1000 - 0.71) < 0.01
+    scale_total = O.weight_bytes(1, p, 128, zero_bytes=0) - O.code_bytes(p)
+    assert scale_total == 23_437_500
+    assert abs(scale_total / 1e9 - 0.023) < 0.001
+    # the handbook counts a 2-byte zero point per group; this library stores 4 bits
+    pages = O.weight_bytes(1, p, 128, zero_bytes=2.0)
+    ours = O.weight_bytes(1, p, 128)
+    assert pages - ours == (p // 128) * 1.5
+    # a Llama-7B-shaped layer: K=4096, N=12288 at G=128
+    assert O.weight_bytes(12288, 4096, 128) == 12288 * 2048 + 12288 * 32 * 2.5
+
+
+# ---------------------------------------------------------------- library agreement
+
+def test_bf16_rounding_matches_torch_cast():
+    rng = np.random.default_rng(11)
+    vals = np.concatenate([
+        rng.standard_normal(200_000).astype(np.float32) * np.float32(3.0),
+        (rng.standard_normal(20_000) * 1e-30).astype(np.float32),
+        (rng.standard_normal(20_000) * 1e30).astype(np.float32),
+        np.array([0.0, -0.0, 1.0, 1.00390625, 1.01171875, 3.0e38, -3.0e38], np.float32),
+    ])
+    # exact ties: low 16 bits 0x8000 with even and odd kept LSB
+    u = rng.integers(0, 2 ** 31 - 2 ** 24, 50_000, dtype=np.uint64).astype(np.uint32)
+    ties = ((u & np.uint32(0xFFFF0000)) | np.uint32(0x8000)).view(np.float32)
+    vals = np.concatenate([vals, ties[np.isfinite(ties)]])
+    ours = O.bf16_round_bits(vals)
+    ref = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_fp16_scale_rounding_matches_torch_cast():
+    rng = np.random.default_rng(12)
+    s = np.abs(rng.standard_normal(100_000)).astype(np.float32) * np.float32(0.01)
+    s = np.concatenate([s, np.float32(2.0) ** np.arange(-30, 16, dtype=np.float32)])
+    ref = torch.from_numpy(s).to(torch.float16).numpy()
+    assert np.array_equal(s.astype(np.float16).view(np.uint16), ref.view(np.uint16))
+
+
+# ---------------------------------------------------------------- INT4 invariants
+
+def _rand_w(N, K, seed, sigma=0.02):
+    return S.draw_w(N, K, sigma, seed=seed, tag=99)
+
+
+@pytest.mark.parametrize("G", [32, 64, 128])
+def test_int4_codes_and_error_bound(G):
+    W = _rand_w(64, 1024, G)
+    W[3, :G] = 0.0                     # all-zero group
+    W[4, G:2 * G] = 0.0173             # constant positive group
+    W[5, :G] = -0.0311                 # constant negative group
+    q, s16, zp = O.quantize_rtn(W, G)
+    assert q.min() >= 0 and q.max() <= 15
+    assert zp.min() >= 0 and zp.max() <= 15
+    sf = s16.astype(np.float32)
+    gk = np.arange(W.shape[1]) // G
+    what = O.dequant_rtn_f32(O.pack_nibbles(q), s16, zp, G)
+    err = np.abs(W.astype(np.float64) - what)
+    bound = sf[:, gk].astype(np.float64)
+    unclamped = (q > 0) & (q < 15)
+    assert np.all(err[unclamped] <= bound[unclamped] / 2)
+    # clamped codes: fp16 rounding of the scale can push the end of the range
+    # by at most 15 * 2^-11 * scale
+    clamped = ~unclamped
+    assert np.all(err[clamped] <= bound[clamped] * (0.5 + 15 * 2.0 ** -11))
+    # group min -> code near 0, group max -> code near 15 (for mixed-sign groups)
+    Wg = W.reshape(64, -1, G)
+    qg = q.reshape(64, -1, G)
+    mixed = (Wg.min(-1) < 0) & (Wg.max(-1) > 0)
+    qmin = np.take_along_axis(qg, Wg.argmin(-1)[..., None], -1)[..., 0]
+    qmax = np.take_along_axis(qg, Wg.argmax(-1)[..., None], -1)[..., 0]
+    assert np.all(qmin[mixed] <= 1) and np.all(qmax[mixed] >= 14)
+    # constant and zero groups dequantize without error beyond bf16 rounding
+    w_bf = O.bf16_bits_to_f32(O.dequant_rtn(O.pack_nibbles(q), s16, zp, G))
+    assert np.all(w_bf[3, :G] == 0)
+    assert np.allclose(w_bf[4, G:2 * G], 0.0173, rtol=2 ** -8)
+    assert np.allclose(w_bf[5, :G], -0.0311, rtol=2 ** -8)
+
+
+def test_int4_brute_force_nearest_level():
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((40, 16)) * 0.05).astype(np.float32)
+    W[0, :4] = np.array([-0.1, 0.05, 0.0, 0.2], np.float32)
+    G = 4
+    q, s16, zp = O.quantize_rtn(W, G)
+    sf = s16.astype(np.float64)
+    for n in range(W.shape[0]):
+        for k in range(W.shape[1]):
+            g = k // G
+            # the code picked by round(w/s)+zp is a nearest of the 16 levels,
+            # measured in units of the scale (no clamping happens here)
+            t = float(np.float32(W[n, k]) / np.float32(sf[n, g]))
+            dist = [abs(t - (lv - int(zp[n, g]))) for lv in range(16)]
+            best = min(dist)
+            assert abs(dist[int(q[n, k])] - best) < 1e-12
+
+
+def test_int4_requantize_round_trip():
+    W = _rand_w(32, 512, 3)
+    q, s16, zp = O.quantize_rtn(W, 128)
+    f = O.dequant_rtn_f32(O.pack_nibbles(q), s16, zp, 128)
+    sk = s16.astype(np.float32)[:, np.arange(512) // 128]
+    zk = zp.astype(np.float32)[:, np.arange(512) // 128]
+    q2 = np.clip(np.rint(f.astype(np.float32) / sk) + zk, 0, 15)
+    assert np.array_equal(q2.astype(np.uint8), q)
+
+
+def test_pack_unpack_bijective():
+    rng = np.random.default_rng(2)
+    q = rng.integers(0, 16, (7, 64), dtype=np.uint8)
+    p = O.pack_nibbles(q)
+    assert p.shape == (7, 32)
+    assert np.array_equal(O.unpack_nibbles(p), q)
+    assert np.array_equal(p & 0xF, q[:, 0::2])
+
+
+# ---------------------------------------------------------------- act-order
+
+def test_act_order_identity_equals_contiguous():
+    W = _rand_w(16, 512, 4)
+    g_id = (np.arange(512) // 64).astype(np.int32)
+    a = O.quantize_rtn(W, 64)
+    b = O.quantize_rtn(W, 64, g_id)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+    assert np.array_equal(O.dequant_rtn(O.pack_nibbles(a[0]), a[1], a[2], 64),
+                          O.dequant_rtn(O.pack_nibbles(b[0]), b[1], b[2], 64, g_id))
+
+
+def test_act_order_equals_permuted_contiguous():
+    # quantizing with g_idx[perm[j]] = j // G is the same as quantizing the
+    # column-permuted matrix W[:, perm] with contiguous groups
+    K, G = 256, 32
+    W = _rand_w(12, K, 6)
+    perm = S.draw_perm(K, seed=1, tag=5, N=12)
+    g_idx = S.act_order_g_idx(perm, G)
+    q, s, z = O.quantize_rtn(W, G, g_idx)
+    qp, sp, zpp = O.quantize_rtn(W[:, perm], G)
+    assert np.array_equal(q[:, perm], qp)
+    assert np.array_equal(s, sp) and np.array_equal(z, zpp)
+    d = O.dequant_rtn(O.pack_nibbles(q), s, z, G, g_idx)
+    dp = O.dequant_rtn(O.pack_nibbles(qp), sp, zpp, G)
+    assert np.array_equal(d[:, perm], dp)
+
+
+def test_g_idx_validation():
+    W = _rand_w(2, 64, 1)
+    with pytest.raises(ValueError):
+        O.quantize_rtn(W, 32, np.full(64, 2, np.int32))
+    with pytest.raises(ValueError):
+        O.quantize_rtn(W, 32, np.full(64, -1, np.int32))
+
+
+# ---------------------------------------------------------------- NF4
+
+def test_nf4_table_invariants():
+    T = O.nf4_table().astype(np.float64)
+    assert T.shape == (16,)
+    assert np.all(np.diff(T) > 0)                      # 16 distinct increasing levels
+    assert T[0] == -1.0 and T[15] == 1.0               # normalised to [-1, 1]
+    assert T[7] == 0.0 and np.count_nonzero(T == 0) == 1
+    assert np.count_nonzero(T < 0) == 7 and np.count_nonzero(T > 0) == 8
+    gaps = np.diff(T)
+    # denser near zero: gaps grow monotonically away from zero on each side
+    assert np.all(np.diff(gaps[7:]) > 0) and np.all(np.diff(gaps[:7]) < 0)
+    # quantile spacing: the positive levels sit at equally spaced probabilities
+    # of the standard normal (a property, checked through the normal CDF)
+    top = math.sqrt(2) * _erfinv_pos(2 * (1 - 0.5 * (1 / 30 + 1 / 32)) - 1)
+    p = [0.5 * (1 + math.erf(t * top / math.sqrt(2))) for t in T[8:]]
+    d = np.diff(p)
+    assert np.allclose(d, d[0], rtol=1e-5)
+
+
+def _erfinv_pos(y):
+    # bisection on math.erf (independent of statistics.NormalDist.inv_cdf)
+    lo, hi = 0.0, 6.0
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        if math.erf(mid) < y:
+            lo = mid
+        else:
+            hi = mid
+    return 0.5 * (lo + hi)
+
+
+def test_nf4_codes_brute_force_nearest():
+    rng = np.random.default_rng(8)
+    W = (rng.standard_normal((6, 128)) * 0.02).astype(np.float32)
+    W[1, :64] = 0.0                                    # all-zero block
+    q = O.nf4_codes(W)
+    T = O.nf4_table().astype(np.float64)
+    a = O.nf4_absmax(W)
+    for b in range(a.size):
+        n, j = divmod(b * 64, 128)
+        for i in range(64):
+            w = W[n, j + i]
+            v = float(np.float32(w) / np.float32(a[b])) if a[b] > 0 else 0.0
+            dist = np.abs(v - T)
+            qq = int(q[n, j + i])
+            assert dist[qq] <= dist.min() + 1e-7
+    assert np.all(q[1, :64] == 7)
+    # the block maximum magnitude maps to an end level
+    for b in range(a.size):
+        n, j = divmod(b * 64, 128)
+        blk = W[n, j:j + 64]
+        if a[b] > 0:
+            i = int(np.argmax(np.abs(blk)))
+            assert int(q[n, j + i]) in (0, 15)
+
+
+def test_nf4_double_quant_bound_and_zero_block():
+    W = S.draw_w(40, 1024, 0.02, seed=3, tag=3)
+    W[0, :64] = 0.0
+    Wq, c, s2 = O.nf4_quantize(W)
+    a = O.nf4_absmax(W).astype(np.float64)
+    nb = a.size
+    assert c.shape == (nb,) and s2.shape == ((nb + 255) // 256,)
+    s = s2.astype(np.float64)[np.arange(nb) // 256]
+    a_dq = c.astype(np.float64) * s
+    assert np.all(np.abs(a - a_dq) <= s / 2 * (1 + 1e-6))
+    # the largest absmax of each run is reproduced by code 255 (up to fp32)
+    for r in range(s2.size):
+        run = slice(r * 256, (r + 1) * 256)
+        assert c[run].max() == 255
+    what = O.bf16_bits_to_f32(O.nf4_dequant(Wq, c, s2))
+    assert np.all(what[0, :64] == 0.0)
+    # dequantized values are T[q] * absmax' up to one bf16 rounding
+    q = O.unpack_nibbles(Wq).reshape(-1, 64)
+    ref = O.nf4_table()[q].astype(np.float64) * a_dq[:, None]
+    assert np.allclose(what.reshape(-1, 64), ref, rtol=2 ** -8, atol=0)
+
+
+# ---------------------------------------------------------------- matmul
+
+def test_matmul_exact_small_brute_force():
+    wl = S.TINY
+    K, N = 64, 24
+    W = S.draw_w(N, K, 0.02, seed=0, tag=wl["tag"])
+    q, s, z = O.quantize_rtn(W, 32)
+    what = O.dequant_rtn(O.pack_nibbles(q), s, z, 32)
+    x = S.draw_x(3, K, seed=0, tag=1, N=N)
+    y, ab = O.matmul_ref(x, what)
+    exact = O.matmul_exact_small(x, what)
+    for m in range(3):
+        for n in range(N):
+            # fp64 accumulation of exact bf16 x bf16 products: relative error
+            # is far below the 1e-3 tolerance of the GPU check
+            assert abs(Fraction(float(y[m, n])) - exact[m][n]) <= Fraction(1, 10 ** 12) * \
+                Fraction(float(ab[m, n]) + 1e-30)
+
+
+def test_matmul_unit_vector_picks_column():
+    K, N = 256, 16
+    W = _rand_w(N, K, 9)
+    q, s, z = O.quantize_rtn(W, 128)
+    what = O.dequant_rtn(O.pack_nibbles(q), s, z, 128)
+    for k in (0, 1, 77, 255):
+        e = np.zeros((1, K), np.float32)
+        e[0, k] = 1.0
+        y, ab = O.matmul_ref(S.to_bf16_bits(e), what)
+        assert np.array_equal(y[0], O.bf16_bits_to_f64(what[:, k]))
+
+
+def test_matmul_constant_group_closed_form():
+    # W constant c on a group: every code dequantizes to the same bf16 value v,
+    # so y = v * sum(x) over the group
+    K, G = 128, 128
+    W = np.full((1, K), 0.0123, np.float32)
+    q, s, z = O.quantize_rtn(W, G)
+    what = O.dequant_rtn(O.pack_nibbles(q), s, z, G)
+    v = O.bf16_bits_to_f64(what[0, 0])
+    assert np.all(O.bf16_bits_to_f64(what) == v)
+    x = S.draw_x(2, K, seed=4, tag=1)
+    y, _ = O.matmul_ref(x, what)
+    assert np.allclose(y[:, 0], v * O.bf16_bits_to_f64(x).sum(1), rtol=1e-14)
+
+
+def test_matmul_ref_matches_float64_numpy_layer():
+    wl = S.LLAMA7B_DECODE
+    K, N = 1024, 512
+    W = S.draw_w(N, K, 0.02, seed=0, tag=wl["tag"])
+    q, s, z = O.quantize_rtn(W, 128)
+    what = O.dequant_rtn(O.pack_nibbles(q), s, z, 128)
+    x = S.draw_x(4, K, seed=0, tag=2, N=N, outlier_frac=0.001, outlier_scale=50.0)
+    y, ab = O.matmul_ref(x, what)
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).double()
+    wf = torch.from_numpy(what.view(np.int16)).view(torch.bfloat16).double()
+    yt = (xf @ wf.T).numpy()
+    assert np.allclose(y, yt, rtol=1e-12, atol=1e-12)
+    assert np.all(ab >= np.abs(y))
+
+
+def test_tolerance_ulp():
+    assert O.ulp_bf16(np.array([1.0]))[0] == 2.0 ** -7
+    assert O.ulp_bf16(np.array([1.5]))[0] == 2.0 ** -7
+    assert O.ulp_bf16(np.array([-2.0]))[0] == 2.0 ** -6
+    assert O.ulp_bf16(np.array([0.0]))[0] == 2.0 ** -133
+    ok, r = O.check_matmul(S.to_bf16_bits(np.array([[1.0]], np.float32)),
+                           np.array([[1.0 + 2 ** -8]]), np.array([[0.0]]))
+    assert ok and r <= 0.5
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def _pins_fail(monkeypatch, name, fn):
+    """Replace one oracle function by a mutated copy and report whether any
+    of the core pins catches it."""
+    import oracle.w4_oracle as M
+    monkeypatch.setattr(M, name, fn)
+    monkeypatch.setattr(O, name, fn)
+    checks = [
+        lambda: [test_int4_worked_examples(c) for c in WORKED],
+        lambda: test_int4_codes_and_error_bound(32),
+        lambda: test_nf4_codes_brute_force_nearest(),
+        lambda: test_nf4_double_quant_bound_and_zero_block(),
+    ]
+    for chk in checks:
+        try:
+            chk()
+        except AssertionError:
+            return True
+    return False
+
+
+def test_planted_mistakes(monkeypatch):
+    import oracle.w4_oracle as M
+    orig_pack = M.pack_nibbles
+
+    def swapped_nibbles(codes):
+        p = orig_pack(codes)
+        return ((p >> 4) | (p << 4)).astype(np.uint8)
+    assert _pins_fail(monkeypatch, "pack_nibbles", swapped_nibbles)
+    monkeypatch.undo()
+
+    orig_round = M.bf16_round_bits
+
+    def truncating(f):
+        return (np.ascontiguousarray(f, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert _pins_fail(monkeypatch, "bf16_round_bits", truncating)
+    monkeypatch.undo()
+    assert M.bf16_round_bits is orig_round
+
+    def half_up_quant(W, G, g_idx=None):
+        W = np.ascontiguousarray(W, np.float32)
+        gk = M.group_index(W.shape[1], G, g_idx)
+        s16, zp = M.rtn_params(W, G, g_idx)
+        sk = s16.astype(np.float32)[:, gk]
+        q = np.clip(np.floor(W / sk + np.float32(0.5)) + zp.astype(np.float32)[:, gk], 0, 15)
+        return q.astype(np.uint8), s16, zp
+    assert _pins_fail(monkeypatch, "quantize_rtn", half_up_quant)
+    monkeypatch.undo()
+
+    def zero_sign_flipped(W, G, g_idx=None):
+        s16, zp = rtn_orig(W, G, g_idx)
+        return s16, np.clip(15 - zp.astype(np.int32), 0, 15).astype(np.uint8)
+    rtn_orig = M.rtn_params
+    assert _pins_fail(monkeypatch, "rtn_params", zero_sign_flipped)
+    monkeypatch.undo()
+
+    orig_dq = M.nf4_double_quant
+
+    def dq_truncating(absmax, dq_group=256):
+        c, s2 = orig_dq(absmax, dq_group)
+        a = np.asarray(absmax, np.float32)
+        s = s2[np.arange(a.size) // dq_group]
+        return np.floor(a / s).astype(np.uint8), s2
+    assert _pins_fail(monkeypatch, "nf4_double_quant", dq_truncating)
+    monkeypatch.undo()
