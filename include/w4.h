@@ -1,0 +1,205 @@
+/*
+ * w4.h -- C ABI of the group-wise 4-bit weight-only linear layer for NVIDIA
+ * B200 (sm_100a):  Y[M,N] = X[M,K] . dequant(Wq)^T
+ *
+ * Source pages (cited by title and section):
+ *   [Survey]     "大模型量化选型：五种主流方案对比与实战"
+ *   [Primer]     aicoding.csdn.net primer, "一、量化究竟做了什么" onwards
+ *   [Handbook]   "这不是理论课，是能立刻上手的LLM量化实操手册"
+ *   [Guide]      "开源模型量化实战指南：GGUF、GPTQ、AWQ选型与本地部署"
+ *   [Comparison] "【推理与部署篇05】模型量化部署深度对比：GPTQ、AWQ、GGUF与FP8实战指南"
+ *
+ * Conventions for every entry point
+ *   - All array pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains them.  Arrays are dense, row-major,
+ *     16-byte aligned unless stated otherwise.
+ *   - fp16 and bf16 values are passed as their uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues work and returns; results are ready when the stream
+ *     has reached that point.
+ *   - Return value: W4_OK, or an error found on the host BEFORE anything is
+ *     launched (bad sizes, null or misaligned pointers, unsupported shapes),
+ *     or W4_ERR_CUDA if a launch failed.  Errors that only the device can see
+ *     (g_idx out of range, a pipeline wait that timed out) set a per-device
+ *     error word that w4_device_status() reads.
+ *   - No CPU fallback: every computation runs in this library's kernels.
+ *
+ * Layouts
+ *   W       fp32 [N, K]        row n = output channel, K contiguous
+ *   Wq      uint8 [N, K/2]     two 4-bit codes per byte, even k in the low
+ *                              nibble ([Guide] §1.1: INT4 is half a byte)
+ *   scales  fp16 [N, K/G]      one scale per (row, group)
+ *   zeros   uint8 [N, K/G]     one zero point per (row, group), value 0..15
+ *   g_idx   int32 [K]          act-order group of each input channel, or NULL
+ *   X       bf16 [M, K]        activations
+ *   Y       bf16 [M, N]        output
+ *   Wp      uint8 opaque       pre-shuffled weights (w4_prepack / nf4_prepack)
+ */
+#ifndef W4_H_
+#define W4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int w4_status;
+typedef void* w4_stream; /* a cudaStream_t */
+
+enum {
+  W4_OK = 0,
+  W4_ERR_INVALID_ARG = 1, /* null/misaligned pointer, size out of range      */
+  W4_ERR_UNSUPPORTED = 2, /* valid but not supported by this build           */
+  W4_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed            */
+  W4_ERR_TIMEOUT = 4,     /* a device pipeline wait gave up (device status)  */
+  W4_ERR_DEVICE_INPUT = 5 /* the device found bad input data (device status) */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* w4_status_string(w4_status s);
+
+/* ABI version (major * 100 + minor). */
+int w4_version(void);
+
+/* Waits for `stream`, then returns and clears the error word that kernels of
+ * this library set on the current device: W4_OK, W4_ERR_TIMEOUT or
+ * W4_ERR_DEVICE_INPUT (or W4_ERR_CUDA if the synchronisation itself failed). */
+w4_status w4_device_status(w4_stream stream);
+
+/* ------------------------------------------------------------------------
+ * INT4 asymmetric round-to-nearest quantization, group-wise along K.
+ * [Comparison] §2.3: scale = (max - min) / (2^b - 1), zero_point =
+ * round(-min / scale), codes in [0, 2^b - 1] (printed for b = 8; here b = 4);
+ * [Comparison] §2.2 / [Primer] §二: one scale per group of G weights;
+ * [Primer] §四: plain rounding (RTN).  Per (row n, group g):
+ *   mn = min(min_k w, 0), mx = max(max_k w, 0)                     (fp32)
+ *   scale = fp16((mx - mn) / 15), or 1.0 if that is 0
+ *   zp = clamp(rint(-mn / scale), 0, 15)
+ *   q_k = clamp(rint(w_k / scale) + zp, 0, 15)     (rint: half to even)
+ * Group g is {k : k / G == g}, or {k : g_idx[k] == g} when g_idx is given
+ * (GPTQ act-order, [Survey] §3.2 desc_act).
+ *   W        in   fp32 [N, K]
+ *   N, K, G  N >= 1; G in {32, 64, 128}; K >= G, K % G == 0, K % 2 == 0
+ *   g_idx    in   int32 [K], values in [0, K/G), or NULL.  Out-of-range
+ *                 values are skipped and reported as W4_ERR_DEVICE_INPUT.
+ *   Wq       out  uint8 [N, K/2]
+ *   scales   out  fp16 bits [N, K/G]
+ *   zeros    out  uint8 [N, K/G]
+ * Bit-exact with the CPU definition above.  |w| must be finite and below
+ * 491520 (so that the fp16 scale is finite). */
+w4_status w4_quantize_rtn(const float* W, int N, int K, int G, const int32_t* g_idx,
+                          uint8_t* Wq, uint16_t* scales, uint8_t* zeros,
+                          w4_stream stream);
+
+/* Dequantization to the bf16 compute dtype ([Survey] §6.2, [Primer] §七):
+ *   w_hat[n,k] = bf16_rne( float(q - zp) * float(scale) )
+ * (the fp32 product is exact, so there is exactly one rounding).
+ *   Wq, scales, zeros, g_idx   in, as produced by w4_quantize_rtn
+ *   W_out                      out  bf16 bits [N, K]                        */
+w4_status w4_dequant(const uint8_t* Wq, const uint16_t* scales, const uint8_t* zeros,
+                     const int32_t* g_idx, int N, int K, int G, uint16_t* W_out,
+                     w4_stream stream);
+
+/* Bytes of the canonical INT4 storage of one [N, K] layer: codes N*K/2,
+ * fp16 scales 2 B and 4-bit zero points 0.5 B per group ([Handbook] §4.1
+ * counts codes as params*bits/8 plus per-group constants). */
+double w4_weight_bytes(int N, int K, int G);
+
+/* ------------------------------------------------------------------------
+ * Pre-shuffled device layout (no counterpart on the pages: it is the
+ * B200-specific part).  Wp holds, for each tile of 128 output rows and each
+ * stage of 128 input channels, one contiguous block that a single bulk copy
+ * brings into shared memory:
+ *   codes   8192 B: [chunk c < 4][row r < 128][16 B], chunk c covering the 32
+ *           channels 32c..32c+31 of the stage; in each 32-bit word of 8
+ *           channels k0..k0+7, bits 4j..4j+3 hold code k0+2j and bits
+ *           16+4j..19+4j hold code k0+2j+1 (j < 4)
+ *   scales  128 * (128/G) fp16, [row][group within the stage]
+ *   zeros   128 * (128/G) 4-bit values, [row][group], even index in the low
+ *           nibble
+ * Rows >= N and channels >= K are padding (code 0, scale 0, zero 0).  With
+ * act_order, the channels are taken in the order that makes each group
+ * contiguous (a stable sort of k by g_idx[k]) and that permutation, int32
+ * [K], follows the tiles.  Act-order needs exactly G channels per group
+ * (the GPTQ layout); otherwise the device reports W4_ERR_DEVICE_INPUT.   */
+size_t w4_prepacked_bytes(int N, int K, int G, int act_order);
+
+/* Canonical (Wq, scales, zeros, g_idx) -> Wp.  Wp must hold
+ * w4_prepacked_bytes(N, K, G, g_idx != NULL) bytes. */
+w4_status w4_prepack(const uint8_t* Wq, const uint16_t* scales, const uint8_t* zeros,
+                     const int32_t* g_idx, int N, int K, int G, uint8_t* Wp,
+                     w4_stream stream);
+
+/* Inverse of w4_prepack for the permuted-channel view: writes the codes,
+ * scales and zeros in the prepacked channel order (identical to the
+ * canonical arrays when act_order == 0) and, if perm != NULL and act_order,
+ * the channel permutation int32 [K]. */
+w4_status w4_unprepack(const uint8_t* Wp, int N, int K, int G, int act_order,
+                       uint8_t* Wq, uint16_t* scales, uint8_t* zeros, int32_t* perm,
+                       w4_stream stream);
+
+/* ------------------------------------------------------------------------
+ * W4A16 linear: Y = X . w_hat^T with w_hat as in w4_dequant, bf16 products,
+ * fp32 accumulation, bf16 (round to nearest even) output.  One kernel path:
+ * tcgen05 tensor-core MMAs with the dequantized weight tile in tensor memory
+ * (the swapped product Y^T = W_hat . X^T), M split into tiles of 16..256
+ * tokens; the decode shapes (M <= 16) stream the packed weights once
+ * ([Survey] §4.3: AWQ "GEMV" for single requests, "GEMM" for batches).
+ *   X          in   bf16 [M, K], 16-byte aligned, K % 64 == 0
+ *   Wp         in   from w4_prepack (act_order must match)
+ *   M, N, K, G M >= 1, N >= 1
+ *   Y          out  bf16 [M, N]
+ *   workspace  device scratch of at least w4_workspace_bytes(M,N,K,G,act_order)
+ *              bytes, 256-byte aligned, ZEROED ONCE before its first use; the
+ *              library leaves it zeroed after every call (split-K counters).
+ *              Calls that share a workspace must be ordered on one stream.  */
+size_t w4_workspace_bytes(int M, int N, int K, int G, int act_order);
+w4_status w4a16_gemm(const uint16_t* X, const uint8_t* Wp, int M, int N, int K, int G,
+                     int act_order, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                     w4_stream stream);
+
+/* ------------------------------------------------------------------------
+ * NF4 ([Survey] §6.1: 16 levels at normal-distribution quantiles, denser near
+ * zero; [Comparison] §6.2; [Survey] §6.3: block-wise absmax, one scale per 64
+ * weights; [Survey] §6.2 / [Comparison] §6.1: double quantization of the
+ * scales).  Blocks are 64 consecutive weights of a row (K % 64 == 0).
+ *   a = max |w| over the block (fp32); v = w / a (0 if a == 0);
+ *   q = #{ i < 15 : v > t_i }, t_i = (T[i] + T[i+1]) / 2  (lower code on ties)
+ *   per run of dq_group consecutive blocks: s2 = max(a) / 255 (1 if 0),
+ *   c = clamp(rint(a / s2), 0, 255), a' = fp32(c * s2)
+ *   w_hat = bf16_rne(fp32(T[q] * a'))
+ *   W          in   fp32 [N, K]
+ *   blocksize  64 (only value supported); dq_group in [1, 1024]
+ *   Wq         out  uint8 [N, K/2]
+ *   absmax_q   out  uint8 [N*K/64]
+ *   s2         out  fp32 [ceil(N*K/64/dq_group)]                           */
+w4_status nf4_quantize(const float* W, int N, int K, int blocksize, int dq_group,
+                       uint8_t* Wq, uint8_t* absmax_q, float* s2, w4_stream stream);
+w4_status nf4_dequant(const uint8_t* Wq, const uint8_t* absmax_q, const float* s2, int N,
+                      int K, int blocksize, int dq_group, uint16_t* W_out,
+                      w4_stream stream);
+
+/* The 16 NF4 levels this library uses (host memory, fp32). */
+void nf4_levels(float out[16]);
+
+/* NF4 pre-shuffled layout: as for INT4 (same codes block per 128 rows x 128
+ * channels) followed by the absmax codes [row][2] (two 64-blocks per stage).
+ * s2 stays in its canonical array. */
+size_t nf4_prepacked_bytes(int N, int K);
+w4_status nf4_prepack(const uint8_t* Wq, const uint8_t* absmax_q, int N, int K,
+                      uint8_t* Wp, w4_stream stream);
+
+/* Y = X . w_hat^T for NF4 weights (same kernel family as w4a16_gemm).
+ *   X bf16 [M,K]; Wp from nf4_prepack; s2 as from nf4_quantize; Y bf16 [M,N]. */
+size_t nf4_workspace_bytes(int M, int N, int K);
+w4_status nf4_gemm(const uint16_t* X, const uint8_t* Wp, const float* s2, int M, int N,
+                   int K, int dq_group, uint16_t* Y, void* workspace,
+                   size_t workspace_bytes, w4_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4_H_ */

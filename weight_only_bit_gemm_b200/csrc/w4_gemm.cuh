@@ -1,0 +1,124 @@
+// w4_gemm.cuh -- fused unpack -> dequant -> tcgen05 MMA for the W4A16 / NF4
+// linear layer, Y = X . W_hat^T, computed as the swapped product
+// Y^T = W_hat . X^T so that the dequantized weight tile is the MMA's A
+// operand and lives in tensor memory:
+//
+//   warp 0      producer: one bulk copy of the prepacked weight stage and two
+//               TMA tiles of X per stage into a shared-memory ring
+//   warp 1      tensor-memory allocation and the single MMA-issuing thread
+//   warps 2..9  dequantize: each thread owns one weight row (TMEM lane) and
+//               one 64-channel half of a stage, turns 32 packed bytes into 64
+//               bf16 values and writes them to TMEM with tcgen05.st; at the
+//               end they read the fp32 accumulator back and store Y (or a
+//               split-K partial)
+//
+// "这不是理论课...LLM量化实操手册" §4.2 measures a separate 4-bit decode +
+// dequant kernel next to the cuBLASLt matmul; here the two are one kernel and
+// the dequantized tile never leaves the SM.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "w4_prepack.cuh"
+#include "w4_ptx.cuh"
+#include "w4_quant.cuh"
+
+namespace w4 {
+
+enum WeightFormat : int { kFmtInt4 = 0, kFmtNf4 = 1 };
+
+template <int MT_, int STAGES_, int FMT_, int G_>
+struct GemmCfg {
+  static constexpr int MT = MT_;          // tokens per tile (MMA N)
+  static constexpr int STAGES = STAGES_;  // shared-memory ring depth
+  static constexpr int FMT = FMT_;
+  static constexpr int G = G_;            // INT4 group size (ignored for NF4)
+  static constexpr int kXBoxBytes = MT * 128;         // [MT][64] bf16, 128-byte rows
+  static constexpr int kXStageBytes = 2 * kXBoxBytes;  // 128 channels
+  static constexpr int kWStageBytes = FMT == kFmtInt4 ? int4_stage_bytes(G) : nf4_stage_bytes();
+  static constexpr int kWSlot = (kWStageBytes + 127) / 128 * 128;
+  static constexpr int kASlots = 3;                   // TMEM A ring (64 columns each)
+  static constexpr int kDCol = 0;
+  static constexpr int kACol = MT;                    // A slots after the accumulator
+  static constexpr int kColsNeeded = MT + kASlots * 64;
+  static constexpr int kTmemCols = kColsNeeded <= 32 ? 32
+                                   : kColsNeeded <= 64 ? 64
+                                   : kColsNeeded <= 128 ? 128
+                                   : kColsNeeded <= 256 ? 256 : 512;
+  static constexpr int kDqWarps = 8;
+  static constexpr int kThreads = 64 + kDqWarps * 32;
+  static constexpr int kNumBars = 2 * STAGES + 2 * kASlots + 3;
+  static constexpr int kSmemBytes =
+      1024 /* alignment slack */ + STAGES * (kXStageBytes + kWSlot) + kNumBars * 8 + 16 + 64;
+  static constexpr int kMinBlocks = kTmemCols <= 256 && kSmemBytes <= 113 * 1024 ? 2 : 1;
+  static_assert(MT % 16 == 0 && MT >= 16 && MT <= 256, "MMA N for M=128 is 16..256 step 16");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static_assert(kColsNeeded <= 512, "tensor memory");
+};
+
+__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) {
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ __nv_bfloat162 bits_bf2(uint32_t v) {
+  return *reinterpret_cast<__nv_bfloat162*>(&v);
+}
+
+// Exact INT4 dequant of one 32-bit word (8 codes) into 4 bf16 pairs:
+//   w_hat = bf16_rne((q - z) * s)
+// with s (fp16) split as s_hi + s_lo, both exact in bf16 (s_lo has <= 4
+// significant bits).  q is made as the bf16 value 128 + q by OR-ing the code
+// into the mantissa of 128.0; d = (128+q) - (128+z) is exact; d*s_lo is exact
+// (<= 8 bits); and one fused multiply-add d*s_hi + d*s_lo rounds the exact
+// product d*s once to bf16.
+struct Int4Dq {
+  __nv_bfloat162 zm, shi, slo;
+};
+
+__device__ __forceinline__ Int4Dq int4_dq_params(uint16_t s16, uint32_t z) {
+  const float sf = __half2float(__ushort_as_half(s16));
+  const __nv_bfloat16 hi = __float2bfloat16_rn(sf);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(sf - __bfloat162float(hi));
+  const __nv_bfloat16 zm = __float2bfloat16_rn(128.0f + static_cast<float>(z));
+  Int4Dq p;
+  p.zm = __halves2bfloat162(zm, zm);
+  p.shi = __halves2bfloat162(hi, hi);
+  p.slo = __halves2bfloat162(lo, lo);
+  return p;
+}
+
+__device__ __forceinline__ void int4_dq_word(uint32_t w, const Int4Dq& p, uint32_t* out) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t t = ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
+    const __nv_bfloat162 d = __hsub2(bits_bf2(t), p.zm);
+    const __nv_bfloat162 l = __hmul2(d, p.slo);
+    out[j] = bf2_bits(__hfma2(d, p.shi, l));
+  }
+}
+
+// NF4 dequant of one word: w_hat = bf16_rne(fp32(T[q] * a')), T in shared memory.
+__device__ __forceinline__ void nf4_dq_word(uint32_t w, float a, const float* __restrict__ T,
+                                            uint32_t* out) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float f0 = __fmul_rn(T[(w >> (4 * j)) & 0xFu], a);
+    const float f1 = __fmul_rn(T[(w >> (16 + 4 * j)) & 0xFu], a);
+    out[j] = bf2_bits(__floats2bfloat162_rn(f0, f1));
+  }
+}
+
+struct GemmArgs {
+  const uint8_t* Wp;      // prepacked weights (tiles x stages blocks)
+  const float* s2;        // NF4 second-level scales (NF4 only)
+  uint16_t* Y;            // bf16 [M, N]
+  float* partial;         // split-K partials [tile][split][MT][128]
+  unsigned int* counter;  // split-K arrival counters [tile]
+  int M, N, K;
+  int KS;                 // stages per tile row = ceil(K / 128)
+  int tiles_n;
+  int splits;
+  int dq_group;           // NF4 double-quant run length
+};
+
+}  // namespace w4

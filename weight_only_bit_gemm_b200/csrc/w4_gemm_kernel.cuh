@@ -1,0 +1,262 @@
+// w4_gemm_kernel.cuh -- the warp-specialised tcgen05 kernel (see w4_gemm.cuh).
+#pragma once
+
+#include "w4_gemm.cuh"
+
+namespace w4 {
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
+    w4_tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* xs = smem;                                   // STAGES x kXStageBytes
+  uint8_t* wsl = xs + C::STAGES * C::kXStageBytes;      // STAGES x kWSlot
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wsl + C::STAGES * C::kWSlot);
+  uint64_t* full = bars;                                // X + W landed       (tx)
+  uint64_t* empty = full + C::STAGES;                   // MMAs done reading  (commit)
+  uint64_t* afull = empty + C::STAGES;                  // A slot written     (8 warps)
+  uint64_t* aempty = afull + C::kASlots;                // A slot consumed    (commit)
+  uint64_t* accf = aempty + C::kASlots;                 // accumulator ready  (commit)
+  uint64_t* epi1 = accf + 1;                            // partials stored    (8 warps)
+  uint64_t* epi2 = epi1 + 1;                            // last-arrival known (1)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi2 + 1);
+  int* last_flag = reinterpret_cast<int*>(tmem_holder + 1);
+  float* Ts = reinterpret_cast<float*>(tmem_holder + 4);  // NF4 levels [16]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nt = blockIdx.x / args.splits;
+  const int split = blockIdx.x % args.splits;
+  const int mtile = blockIdx.y;
+  const int s0 = static_cast<int>(static_cast<long long>(split) * args.KS / args.splits);
+  const int s1 = static_cast<int>(static_cast<long long>(split + 1) * args.KS / args.splits);
+  const int nst = s1 - s0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < C::kASlots; ++i) {
+      mbar_init(&afull[i], C::kDqWarps);
+      mbar_init(&aempty[i], 1);
+    }
+    mbar_init(accf, 1);
+    mbar_init(epi1, C::kDqWarps);
+    mbar_init(epi2, 1);
+    fence_barrier_init();
+  }
+  if (C::FMT == kFmtNf4 && threadIdx.x < 16) Ts[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&xmap);
+      const uint64_t pol_w = policy_evict_first();  // weights are read once per M tile
+      const uint64_t pol_x = policy_evict_last();   // X is shared by every CTA
+      const uint8_t* wsrc =
+          args.Wp + (static_cast<size_t>(nt) * args.KS + s0) * C::kWStageBytes;
+      int issued = 0;
+      for (int it = 0; it < nst; ++it) {
+        const int s = it % C::STAGES;
+        if (it >= C::STAGES && !mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1)) break;
+        mbar_arrive_expect_tx(&full[s], C::kXStageBytes + C::kWStageBytes);
+        const int k0 = (s0 + it) * kStageK;
+        uint8_t* xdst = xs + s * C::kXStageBytes;
+        tma_load_2d(xdst, &xmap, k0, mtile * C::MT, &full[s], pol_x);
+        tma_load_2d(xdst + C::kXBoxBytes, &xmap, k0 + 64, mtile * C::MT, &full[s], pol_x);
+        bulk_g2s(wsl + s * C::kWSlot, wsrc + static_cast<size_t>(it) * C::kWStageBytes,
+                 C::kWStageBytes, &full[s], pol_w);
+        ++issued;
+      }
+      // never leave with copies in flight: wait for the last issued stages
+      for (int it = issued - 1; it >= 0 && it >= issued - C::STAGES; --it)
+        mbar_wait(&full[it % C::STAGES], (it / C::STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, C::MT);
+      const uint32_t d_tmem = tmem + C::kDCol;
+      for (int it = 0; it < nst; ++it) {
+        const int s = it % C::STAGES;
+        const int a = it % C::kASlots;
+        if (!mbar_wait(&full[s], (it / C::STAGES) & 1)) break;
+        if (!mbar_wait(&afull[a], (it / C::kASlots) & 1)) break;
+        tc_fence_after();
+        const uint32_t xaddr = smem_u32(xs + s * C::kXStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bdesc =
+              smem_desc_sw128(xaddr + (kk >> 2) * C::kXBoxBytes + (kk & 3) * 32);
+          const uint32_t a_tmem = tmem + C::kACol + a * 64 + kk * 8;
+          mma_bf16_ts(d_tmem, a_tmem, bdesc, idesc, (it | kk) != 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+        mma_commit(&aempty[a]);
+      }
+      mma_commit(accf);  // also on an early exit, so that TMEM is quiet before dealloc
+    }
+  } else {
+    // ------------------------------------------------------------ dequant
+    const int dw = warp - 2;        // 0..7
+    const int quad = warp & 3;      // TMEM lane quadrant this warp may access
+    const int h = dw >> 2;          // 64-channel half of each stage
+    const int row = quad * 32 + lane;
+    const int n = nt * kTileRows + row;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < nst && ok; ++it) {
+      const int s = it % C::STAGES;
+      const int a = it % C::kASlots;
+      // warp-uniform waits: the tcgen05 loads/stores below are .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (it / C::STAGES) & 1))) {
+        ok = false;
+        break;
+      }
+      const uint8_t* wb = wsl + s * C::kWSlot;
+      const uint4 c0 = *reinterpret_cast<const uint4*>(wb + (2 * h) * 2048 + row * 16);
+      const uint4 c1 = *reinterpret_cast<const uint4*>(wb + (2 * h + 1) * 2048 + row * 16);
+      uint32_t out[32];
+      if constexpr (C::FMT == kFmtInt4) {
+        constexpr int gps = kStageK / C::G;
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(wb + kCodeBytes);
+        const uint8_t* zb = wb + kCodeBytes + kTileRows * gps * 2;
+        // groups of chunks 2h and 2h+1
+        const int gl0 = (2 * h * 32) / C::G;
+        const int gl1 = ((2 * h + 1) * 32) / C::G;
+        const int i0 = row * gps + gl0, i1 = row * gps + gl1;
+        const Int4Dq p0 = int4_dq_params(sc[i0], (zb[i0 >> 1] >> ((i0 & 1) * 4)) & 0xFu);
+        const Int4Dq p1 = (gl1 == gl0) ? p0
+                          : int4_dq_params(sc[i1], (zb[i1 >> 1] >> ((i1 & 1) * 4)) & 0xFu);
+        int4_dq_word(c0.x, p0, out + 0);
+        int4_dq_word(c0.y, p0, out + 4);
+        int4_dq_word(c0.z, p0, out + 8);
+        int4_dq_word(c0.w, p0, out + 12);
+        int4_dq_word(c1.x, p1, out + 16);
+        int4_dq_word(c1.y, p1, out + 20);
+        int4_dq_word(c1.z, p1, out + 24);
+        int4_dq_word(c1.w, p1, out + 28);
+      } else {
+        const int blk_in_row = (s0 + it) * 2 + h;
+        float aq = 0.0f;
+        if (n < args.N && blk_in_row * 64 < args.K) {
+          const uint32_t c = wb[kCodeBytes + row * 2 + h];
+          const long long b = static_cast<long long>(n) * (args.K / 64) + blk_in_row;
+          aq = __fmul_rn(static_cast<float>(c), __ldg(args.s2 + b / args.dq_group));
+        }
+        nf4_dq_word(c0.x, aq, Ts, out + 0);
+        nf4_dq_word(c0.y, aq, Ts, out + 4);
+        nf4_dq_word(c0.z, aq, Ts, out + 8);
+        nf4_dq_word(c0.w, aq, Ts, out + 12);
+        nf4_dq_word(c1.x, aq, Ts, out + 16);
+        nf4_dq_word(c1.y, aq, Ts, out + 20);
+        nf4_dq_word(c1.z, aq, Ts, out + 24);
+        nf4_dq_word(c1.w, aq, Ts, out + 28);
+      }
+      if (it >= C::kASlots &&
+          !__all_sync(0xffffffffu, mbar_wait(&aempty[a], ((it / C::kASlots) - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tmem_st32(tmem + lane_base + C::kACol + a * 64 + h * 32, out);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[a]);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok && __all_sync(0xffffffffu, mbar_wait(accf, 0))) {
+      tc_fence_after();
+      constexpr int kHalfCols = C::MT / 2;
+      const int m_base = mtile * C::MT + h * kHalfCols;
+      const int tile_id = mtile * args.tiles_n + nt;
+      float* part = args.partial +
+                    ((static_cast<size_t>(tile_id) * args.splits + split) * C::MT + h * kHalfCols) *
+                        kTileRows;
+#pragma unroll 1
+      for (int cb = 0; cb < kHalfCols; cb += 8) {
+        uint32_t v[8];
+        tmem_ld8(tmem + lane_base + C::kDCol + h * kHalfCols + cb, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int m = m_base + cb + j;
+          const float acc = __uint_as_float(v[j]);
+          if (args.splits == 1) {
+            if (m < args.M && n < args.N)
+              args.Y[static_cast<size_t>(m) * args.N + n] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+          } else {
+            part[(cb + j) * kTileRows + row] = acc;
+          }
+        }
+      }
+      tc_fence_before();
+      if (args.splits > 1) {
+        // the last CTA of this tile to arrive sums the partials in split order
+        // (mbarriers with bounded waits, not bar.sync, so that a warp that gave
+        // up earlier cannot leave the others blocked)
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi1);
+        bool have_flag = true;
+        if (threadIdx.x == 64) {
+          if (mbar_wait(epi1, 0)) {
+            const unsigned prev = atomicAdd(args.counter + tile_id, 1u);
+            *last_flag = (prev == static_cast<unsigned>(args.splits - 1)) ? 1 : 0;
+          } else {
+            *last_flag = 0;
+          }
+          mbar_arrive(epi2);
+        }
+        have_flag = __all_sync(0xffffffffu, mbar_wait(epi2, 0));
+        if (have_flag && *last_flag) {
+          __threadfence();
+          const float* base =
+              args.partial + static_cast<size_t>(tile_id) * args.splits * C::MT * kTileRows;
+#pragma unroll 1
+          for (int c = 0; c < kHalfCols; ++c) {
+            const int ml = h * kHalfCols + c;
+            const int m = mtile * C::MT + ml;
+            float acc = 0.0f;
+            for (int sp = 0; sp < args.splits; ++sp)
+              acc += __ldcg(base + (static_cast<size_t>(sp) * C::MT + ml) * kTileRows + row);
+            if (m < args.M && n < args.N)
+              args.Y[static_cast<size_t>(m) * args.N + n] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+          }
+          if (threadIdx.x == 64) args.counter[tile_id] = 0u;  // leave the workspace zeroed
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    mbar_wait(accf, 0);  // every issued MMA has completed
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// act-order: X'[m, j] = X[m, perm[j]]
+__global__ void gather_x_kernel(const uint16_t* __restrict__ X, const int32_t* __restrict__ perm,
+                                int M, int K, uint16_t* __restrict__ Xp) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  const int m = blockIdx.y;
+  if (j < K && m < M) Xp[static_cast<size_t>(m) * K + j] = X[static_cast<size_t>(m) * K + perm[j]];
+}
+
+}  // namespace w4

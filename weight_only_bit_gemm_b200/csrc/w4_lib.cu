@@ -1,0 +1,200 @@
+// w4_lib.cu -- the C ABI (include/w4.h): host-side argument checks and kernel
+// launches.  One translation unit so that the per-device error word is a
+// single object.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/w4.h"
+#include "w4_gemm_kernel.cuh"
+#include "w4_prepack.cuh"
+#include "w4_quant.cuh"
+#include "w4_ptx.cuh"
+
+using namespace w4;
+
+namespace {
+
+inline cudaStream_t as_stream(w4_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+inline bool valid_group(int G) { return G == 32 || G == 64 || G == 128; }
+inline w4_status launch_status(cudaError_t e) { return e == cudaSuccess ? W4_OK : W4_ERR_CUDA; }
+inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+bool int4_shape_ok(int N, int K, int G) {
+  return N >= 1 && K >= 1 && valid_group(G) && K >= G && K % G == 0 && K % 2 == 0 &&
+         static_cast<long long>(N) * K <= (1LL << 40);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* w4_status_string(w4_status s) {
+  switch (s) {
+    case W4_OK: return "ok";
+    case W4_ERR_INVALID_ARG: return "invalid argument";
+    case W4_ERR_UNSUPPORTED: return "unsupported";
+    case W4_ERR_CUDA: return "CUDA error";
+    case W4_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case W4_ERR_DEVICE_INPUT: return "device found invalid input data";
+    default: return "unknown status";
+  }
+}
+
+int w4_version(void) { return 100; }
+
+w4_status w4_device_status(w4_stream stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return W4_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(v)) != cudaSuccess) return W4_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return W4_ERR_CUDA;
+  }
+  if (v & W4_DEV_ERR_TIMEOUT) return W4_ERR_TIMEOUT;
+  if (v & W4_DEV_ERR_INPUT) return W4_ERR_DEVICE_INPUT;
+  return W4_OK;
+}
+
+double w4_weight_bytes(int N, int K, int G) {
+  if (!int4_shape_ok(N, K, G)) return 0.0;
+  const double groups = static_cast<double>(N) * (K / G);
+  return static_cast<double>(N) * K / 2.0 + groups * 2.0 + groups * 0.5;
+}
+
+// ---------------------------------------------------------------- INT4 RTN
+w4_status w4_quantize_rtn(const float* W, int N, int K, int G, const int32_t* g_idx,
+                          uint8_t* Wq, uint16_t* scales, uint8_t* zeros, w4_stream stream) {
+  if (!W || !Wq || !scales || !zeros) return W4_ERR_INVALID_ARG;
+  if (!int4_shape_ok(N, K, G)) return W4_ERR_INVALID_ARG;
+  if (!aligned(W, 4) || !aligned(scales, 2) || (g_idx && !aligned(g_idx, 4)))
+    return W4_ERR_INVALID_ARG;
+  const int ng = K / G;
+  const size_t smem = static_cast<size_t>(ng) * 16;
+  if (smem > 200 * 1024) return W4_ERR_UNSUPPORTED;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaFuncSetAttribute(rtn_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         200 * 1024);
+  });
+  rtn_quantize_kernel<<<N, 256, smem, as_stream(stream)>>>(W, N, K, G, g_idx, Wq, scales, zeros);
+  return launch_status(cudaGetLastError());
+}
+
+w4_status w4_dequant(const uint8_t* Wq, const uint16_t* scales, const uint8_t* zeros,
+                     const int32_t* g_idx, int N, int K, int G, uint16_t* W_out,
+                     w4_stream stream) {
+  if (!Wq || !scales || !zeros || !W_out) return W4_ERR_INVALID_ARG;
+  if (!int4_shape_ok(N, K, G) || K % 8 != 0) return W4_ERR_INVALID_ARG;
+  if (!aligned(Wq, 4) || !aligned(W_out, 16) || !aligned(scales, 2) ||
+      (g_idx && !aligned(g_idx, 4)))
+    return W4_ERR_INVALID_ARG;
+  const long long total = static_cast<long long>(N) * (K / 8);
+  rtn_dequant_kernel<<<ceil_div(total, 256), 256, 0, as_stream(stream)>>>(Wq, scales, zeros,
+                                                                           g_idx, N, K, G, W_out);
+  return launch_status(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- prepack
+size_t w4_prepacked_bytes(int N, int K, int G, int act_order) {
+  if (!int4_shape_ok(N, K, G)) return 0;
+  const size_t tiles = ceil_div(N, kTileRows), ks = ceil_div(K, kStageK);
+  return tiles * ks * int4_stage_bytes(G) + (act_order ? static_cast<size_t>(K) * 4 : 0);
+}
+
+static int32_t* perm_region(uint8_t* Wp, int N, int K, int G) {
+  const size_t tiles = ceil_div(N, kTileRows), ks = ceil_div(K, kStageK);
+  return reinterpret_cast<int32_t*>(Wp + tiles * ks * int4_stage_bytes(G));
+}
+
+w4_status w4_prepack(const uint8_t* Wq, const uint16_t* scales, const uint8_t* zeros,
+                     const int32_t* g_idx, int N, int K, int G, uint8_t* Wp, w4_stream stream) {
+  if (!Wq || !scales || !zeros || !Wp) return W4_ERR_INVALID_ARG;
+  if (!int4_shape_ok(N, K, G)) return W4_ERR_INVALID_ARG;
+  if (!aligned(Wp, 16) || !aligned(scales, 2) || (g_idx && !aligned(g_idx, 4)))
+    return W4_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  int32_t* perm = nullptr;
+  if (g_idx) {
+    perm = perm_region(Wp, N, K, G);
+    act_order_perm_kernel<<<1, 1024, 0, st>>>(g_idx, K, G, perm);
+    if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+  }
+  dim3 grid(ceil_div(K, kStageK), ceil_div(N, kTileRows));
+  int4_prepack_kernel<<<grid, kTileRows, 0, st>>>(Wq, scales, zeros, perm, N, K, G, Wp);
+  return launch_status(cudaGetLastError());
+}
+
+w4_status w4_unprepack(const uint8_t* Wp, int N, int K, int G, int act_order, uint8_t* Wq,
+                       uint16_t* scales, uint8_t* zeros, int32_t* perm, w4_stream stream) {
+  if (!Wp || !Wq || !scales || !zeros) return W4_ERR_INVALID_ARG;
+  if (!int4_shape_ok(N, K, G) || !aligned(Wp, 16)) return W4_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  dim3 grid(ceil_div(K, kStageK), ceil_div(N, kTileRows));
+  int4_unprepack_kernel<<<grid, kTileRows, 0, st>>>(Wp, N, K, G, Wq, scales, zeros);
+  if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+  if (act_order && perm) {
+    const int32_t* src = perm_region(const_cast<uint8_t*>(Wp), N, K, G);
+    if (cudaMemcpyAsync(perm, src, static_cast<size_t>(K) * 4, cudaMemcpyDeviceToDevice, st) !=
+        cudaSuccess)
+      return W4_ERR_CUDA;
+  }
+  return W4_OK;
+}
+
+// ---------------------------------------------------------------- NF4
+void nf4_levels(float out[16]) {
+  if (out) std::memcpy(out, kNf4LevelBitsHost, sizeof(kNf4LevelBitsHost));
+}
+
+static bool nf4_shape_ok(int N, int K, int blocksize, int dq_group) {
+  return N >= 1 && K >= 64 && K % 64 == 0 && blocksize == 64 && dq_group >= 1 &&
+         dq_group <= 1024 && static_cast<long long>(N) * K <= (1LL << 40);
+}
+
+w4_status nf4_quantize(const float* W, int N, int K, int blocksize, int dq_group, uint8_t* Wq,
+                       uint8_t* absmax_q, float* s2, w4_stream stream) {
+  if (!W || !Wq || !absmax_q || !s2) return W4_ERR_INVALID_ARG;
+  if (!nf4_shape_ok(N, K, blocksize, dq_group)) return W4_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(s2, 4)) return W4_ERR_INVALID_ARG;
+  const long long nb = static_cast<long long>(N) * K / 64;
+  const int runs = ceil_div(nb, dq_group);
+  nf4_quantize_kernel<<<runs, dq_group, dq_group * sizeof(float), as_stream(stream)>>>(
+      W, nb, dq_group, Wq, absmax_q, s2);
+  return launch_status(cudaGetLastError());
+}
+
+w4_status nf4_dequant(const uint8_t* Wq, const uint8_t* absmax_q, const float* s2, int N, int K,
+                      int blocksize, int dq_group, uint16_t* W_out, w4_stream stream) {
+  if (!Wq || !absmax_q || !s2 || !W_out) return W4_ERR_INVALID_ARG;
+  if (!nf4_shape_ok(N, K, blocksize, dq_group)) return W4_ERR_INVALID_ARG;
+  if (!aligned(Wq, 4) || !aligned(W_out, 16) || !aligned(s2, 4)) return W4_ERR_INVALID_ARG;
+  const long long total8 = static_cast<long long>(N) * K / 8;
+  nf4_dequant_kernel<<<ceil_div(total8, 256), 256, 0, as_stream(stream)>>>(
+      Wq, absmax_q, s2, total8, dq_group, W_out);
+  return launch_status(cudaGetLastError());
+}
+
+size_t nf4_prepacked_bytes(int N, int K) {
+  if (!nf4_shape_ok(N, K, 64, 256)) return 0;
+  return static_cast<size_t>(ceil_div(N, kTileRows)) * ceil_div(K, kStageK) * nf4_stage_bytes();
+}
+
+w4_status nf4_prepack(const uint8_t* Wq, const uint8_t* absmax_q, int N, int K, uint8_t* Wp,
+                      w4_stream stream) {
+  if (!Wq || !absmax_q || !Wp) return W4_ERR_INVALID_ARG;
+  if (!nf4_shape_ok(N, K, 64, 256) || !aligned(Wp, 16)) return W4_ERR_INVALID_ARG;
+  dim3 grid(ceil_div(K, kStageK), ceil_div(N, kTileRows));
+  nf4_prepack_kernel<<<grid, kTileRows, 0, as_stream(stream)>>>(Wq, absmax_q, N, K, Wp);
+  return launch_status(cudaGetLastError());
+}
+
+}  // extern "C"
+
+#include "w4_gemm_host.inc"

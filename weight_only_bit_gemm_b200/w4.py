@@ -1,0 +1,242 @@
+"""ctypes binding of ``libw4b200.so`` (C ABI in ``include/w4.h``).
+
+Argument marshalling only: every computation runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (torch provides device memory and the
+current stream); there is no CPU path, and importing this module fails loudly
+when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libw4b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "w4.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m weight_only_bit_gemm_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+_SIGS = {
+    "w4_status_string": (ctypes.c_char_p, [_i]),
+    "w4_version": (_i, []),
+    "w4_device_status": (_i, [_p]),
+    "w4_weight_bytes": (ctypes.c_double, [_i, _i, _i]),
+    "w4_quantize_rtn": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p]),
+    "w4_dequant": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
+    "w4_prepacked_bytes": (_sz, [_i, _i, _i, _i]),
+    "w4_prepack": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
+    "w4_unprepack": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p, _p]),
+    "w4_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "w4a16_gemm": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "nf4_quantize": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p]),
+    "nf4_dequant": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p]),
+    "nf4_levels": (None, [_p]),
+    "nf4_prepacked_bytes": (_sz, [_i, _i]),
+    "nf4_prepack": (_i, [_p, _p, _i, _i, _p, _p]),
+    "nf4_workspace_bytes": (_sz, [_i, _i, _i]),
+    "nf4_gemm": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA, W4_ERR_TIMEOUT, \
+    W4_ERR_DEVICE_INPUT = range(6)
+
+
+class W4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib.w4_status_string(status).decode()} ({status})")
+
+
+def header_functions() -> list:
+    """Names of the functions declared in include/w4.h."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(\w+)\s*\(", text)) - {"defined", "if"})
+
+
+def _check(status: int, what: str) -> None:
+    if status != W4_OK:
+        raise W4Error(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _cuda(t, dtype, name):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    return t
+
+
+def device_status() -> int:
+    """Synchronise the current stream and return/clear the device error word."""
+    return lib.w4_device_status(_stream())
+
+
+# ----------------------------------------------------------------- INT4 RTN
+
+def quantize_rtn(W, G, g_idx=None):
+    """fp32 W [N, K] -> (Wq uint8 [N, K/2], scales fp16 [N, K/G], zeros uint8 [N, K/G])."""
+    _cuda(W, torch.float32, "W")
+    N, K = W.shape
+    dev = W.device
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    sc = torch.empty((N, K // G), dtype=torch.float16, device=dev)
+    zr = torch.empty((N, K // G), dtype=torch.uint8, device=dev)
+    if g_idx is not None:
+        _cuda(g_idx, torch.int32, "g_idx")
+    _check(lib.w4_quantize_rtn(_ptr(W), N, K, G, _ptr(g_idx), _ptr(Wq), _ptr(sc), _ptr(zr),
+                               _stream()), "w4_quantize_rtn")
+    return Wq, sc, zr
+
+
+def dequant(Wq, scales, zeros, G, g_idx=None):
+    N, K = Wq.shape[0], Wq.shape[1] * 2
+    out = torch.empty((N, K), dtype=torch.bfloat16, device=Wq.device)
+    _check(lib.w4_dequant(_ptr(Wq), _ptr(scales), _ptr(zeros), _ptr(g_idx), N, K, G, _ptr(out),
+                          _stream()), "w4_dequant")
+    return out
+
+
+def prepacked_bytes(N, K, G, act_order=False) -> int:
+    return lib.w4_prepacked_bytes(N, K, G, int(bool(act_order)))
+
+
+def prepack(Wq, scales, zeros, G, g_idx=None):
+    N, K = Wq.shape[0], Wq.shape[1] * 2
+    nbytes = prepacked_bytes(N, K, G, g_idx is not None)
+    if nbytes == 0:
+        raise W4Error(W4_ERR_INVALID_ARG, "w4_prepacked_bytes")
+    Wp = torch.empty(nbytes, dtype=torch.uint8, device=Wq.device)
+    _check(lib.w4_prepack(_ptr(Wq), _ptr(scales), _ptr(zeros), _ptr(g_idx), N, K, G, _ptr(Wp),
+                          _stream()), "w4_prepack")
+    return Wp
+
+
+def unprepack(Wp, N, K, G, act_order=False):
+    dev = Wp.device
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    sc = torch.empty((N, K // G), dtype=torch.float16, device=dev)
+    zr = torch.empty((N, K // G), dtype=torch.uint8, device=dev)
+    perm = torch.empty(K, dtype=torch.int32, device=dev) if act_order else None
+    _check(lib.w4_unprepack(_ptr(Wp), N, K, G, int(bool(act_order)), _ptr(Wq), _ptr(sc),
+                            _ptr(zr), _ptr(perm), _stream()), "w4_unprepack")
+    return Wq, sc, zr, perm
+
+
+class Workspace:
+    """Per-device scratch buffer, zero-filled once when (re)allocated; the
+    library leaves it zeroed after each call."""
+
+    def __init__(self):
+        self._buf = {}
+
+    def get(self, nbytes: int, device) -> torch.Tensor:
+        dev = torch.device(device)
+        key = dev.index if dev.index is not None else torch.cuda.current_device()
+        buf = self._buf.get(key)
+        if buf is None or buf.numel() < nbytes:
+            size = max(nbytes, 1 << 20)
+            buf = torch.zeros(size + 256, dtype=torch.uint8, device=dev)
+            self._buf[key] = buf
+        return buf
+
+
+_WS = Workspace()
+
+
+def _ws_view(buf):
+    off = (-buf.data_ptr()) % 256
+    return buf[off:]
+
+
+def workspace_bytes(M, N, K, G, act_order=False) -> int:
+    return lib.w4_workspace_bytes(M, N, K, G, int(bool(act_order)))
+
+
+def w4a16_gemm(X, Wp, N, K, G, act_order=False, out=None, workspace=None):
+    """Y[M, N] = X . dequant(W)^T for bf16 X [M, K] and prepacked Wp."""
+    _cuda(X, torch.bfloat16, "X")
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    need = workspace_bytes(M, N, K, G, act_order)
+    ws = _ws_view(workspace if workspace is not None else _WS.get(need, X.device))
+    _check(lib.w4a16_gemm(_ptr(X), _ptr(Wp), M, N, K, G, int(bool(act_order)), _ptr(out),
+                          _ptr(ws), ws.numel(), _stream()), "w4a16_gemm")
+    return out
+
+
+# ----------------------------------------------------------------- NF4
+
+def nf4_levels():
+    buf = (ctypes.c_float * 16)()
+    lib.nf4_levels(ctypes.cast(buf, ctypes.c_void_p))
+    return list(buf)
+
+
+def nf4_quantize(W, blocksize=64, dq_group=256):
+    _cuda(W, torch.float32, "W")
+    N, K = W.shape
+    dev = W.device
+    nb = N * K // blocksize
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    aq = torch.empty(nb, dtype=torch.uint8, device=dev)
+    s2 = torch.empty((nb + dq_group - 1) // dq_group, dtype=torch.float32, device=dev)
+    _check(lib.nf4_quantize(_ptr(W), N, K, blocksize, dq_group, _ptr(Wq), _ptr(aq), _ptr(s2),
+                            _stream()), "nf4_quantize")
+    return Wq, aq, s2
+
+
+def nf4_dequant(Wq, absmax_q, s2, dq_group=256, blocksize=64):
+    N, K = Wq.shape[0], Wq.shape[1] * 2
+    out = torch.empty((N, K), dtype=torch.bfloat16, device=Wq.device)
+    _check(lib.nf4_dequant(_ptr(Wq), _ptr(absmax_q), _ptr(s2), N, K, blocksize, dq_group,
+                           _ptr(out), _stream()), "nf4_dequant")
+    return out
+
+
+def nf4_prepack(Wq, absmax_q):
+    N, K = Wq.shape[0], Wq.shape[1] * 2
+    nbytes = lib.nf4_prepacked_bytes(N, K)
+    if nbytes == 0:
+        raise W4Error(W4_ERR_INVALID_ARG, "nf4_prepacked_bytes")
+    Wp = torch.empty(nbytes, dtype=torch.uint8, device=Wq.device)
+    _check(lib.nf4_prepack(_ptr(Wq), _ptr(absmax_q), N, K, _ptr(Wp), _stream()), "nf4_prepack")
+    return Wp
+
+
+def nf4_workspace_bytes(M, N, K) -> int:
+    return lib.nf4_workspace_bytes(M, N, K)
+
+
+def nf4_gemm(X, Wp, s2, N, K, dq_group=256, out=None, workspace=None):
+    _cuda(X, torch.bfloat16, "X")
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    need = nf4_workspace_bytes(M, N, K)
+    ws = _ws_view(workspace if workspace is not None else _WS.get(need, X.device))
+    _check(lib.nf4_gemm(_ptr(X), _ptr(Wp), _ptr(s2), M, N, K, dq_group, _ptr(out), _ptr(ws),
+                        ws.numel(), _stream()), "nf4_gemm")
+    return out
