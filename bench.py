@@ -331,3 +331,275 @@ def measure_e2e(step, args, pg):
     d2h = sum(t.numel() * 2 for t in hy)
     del g
     return ms, n, h2d, d2h
+
+
+# --------------------------------------------------------------------- other rows
+
+def _replicas_for(nbytes_each: int, l2: int) -> int:
+    return max(2, -(-4 * l2 // max(1, nbytes_each)))
+
+
+def measure_rows(w4, peaks):
+    """The other steps of the path, each timed alone (device time, CUDA events)."""
+    rows = {}
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    hbm = peaks["hbm_gbs"]
+
+    # a1+a2: INT4 RTN quantize + pack, and a6: standalone dequant, a4: prepack
+    K, N, G = 4096, 22016, 128
+    W = torch.from_numpy(S.layer_w(WL, K, N)).cuda()
+    Wq, sc, zr = w4.quantize_rtn(W, G)
+    t = time_calls([lambda: w4.quantize_rtn(W, G)], reps=5)[0]
+    qb = N * K * 4 + N * K / 2 + N * (K // G) * 3
+    rows["quantize_rtn"] = {"shape": [N, K], "G": G, "ms": t, "GB/s": qb / t / 1e6,
+                            "frac_of_hbm": qb / t / 1e6 / hbm}
+    t = time_calls([lambda: w4.dequant(Wq, sc, zr, G)], reps=5)[0]
+    db = N * K / 2 + N * (K // G) * 3 + N * K * 2
+    rows["dequant"] = {"shape": [N, K], "G": G, "ms": t, "GB/s": db / t / 1e6,
+                       "frac_of_hbm": db / t / 1e6 / hbm}
+    t = time_calls([lambda: w4.prepack(Wq, sc, zr, G)], reps=5)[0]
+    pb = 2 * (N * K / 2 + N * (K // G) * 2.5)
+    rows["prepack"] = {"shape": [N, K], "G": G, "ms": t, "GB/s": pb / t / 1e6}
+    del W, Wq, sc, zr
+
+    # a5: NF4 quantize; a7: NF4 decode / small batch
+    nf = S.NF4_DECODE
+    calls, nbytes = [], []
+    for (K, N) in nf["shapes"]:
+        W = torch.from_numpy(S.layer_w(nf, K, N)).cuda()
+        q4, c4, s24 = w4.nf4_quantize(W)
+        if (K, N) == nf["shapes"][0]:
+            t = time_calls([lambda: w4.nf4_quantize(W)], reps=5)[0]
+            b = N * K * 4 + N * K / 2 + N * K / 64
+            rows["nf4_quantize"] = {"shape": [N, K], "ms": t, "GB/s": b / t / 1e6}
+        wp = w4.nf4_prepack(q4, c4)
+        reps = [wp] + [wp.clone() for _ in range(_replicas_for(wp.numel(), l2) - 1)]
+        for M in nf["Ms"]:
+            X = bf16_dev(S.layer_x(nf, M, K, N))
+            for r in reps:
+                calls.append(lambda X=X, r=r, s=s24, N=N, K=K: w4.nf4_gemm(X, r, s, N, K))
+                nbytes.append(nf4_bytes(M, N, K))
+        del W
+    ts = time_calls(calls, reps=5)
+    rows["nf4_gemm_decode"] = {"configs": "(K,N) in {(4096,14336),(14336,4096)} x M in {1,8,32}",
+                               "TB/s": sum(nbytes) / sum(ts) / 1e9,
+                               "frac_of_hbm": sum(nbytes) / sum(ts) / 1e6 / hbm}
+
+    # a3: act-order (g_idx) decode and M=256, group 32
+    ao = S.ACT_ORDER_13B
+    dec_calls, dec_bytes, big_calls, big_flops = [], [], [], []
+    for (K, N) in ao["shapes"]:
+        G = ao["G"]
+        W = torch.from_numpy(S.layer_w(ao, K, N)).cuda()
+        g_idx = torch.from_numpy(S.act_order_g_idx(S.draw_perm(K, tag=ao["tag"], N=N), G)).cuda()
+        Wq, sc, zr = w4.quantize_rtn(W, G, g_idx)
+        wp = w4.prepack(Wq, sc, zr, G, g_idx)
+        reps = [wp] + [wp.clone() for _ in range(_replicas_for(wp.numel(), l2) - 1)]
+        for M in ao["Ms"]:
+            X = bf16_dev(S.layer_x(ao, M, K, N))
+            for r in reps:
+                f = (lambda X=X, r=r, N=N, K=K, G=G: w4.w4a16_gemm(X, r, N, K, G, True))
+                if M <= 16:
+                    dec_calls.append(f)
+                    dec_bytes.append(int4_bytes(M, N, K, G) + 4 * K)
+                else:
+                    big_calls.append(f)
+                    big_flops.append(2.0 * M * N * K)
+        del W, Wq, sc, zr
+    ts = time_calls(dec_calls, reps=5)
+    rows["act_order_decode"] = {"configs": "(K,N) in {(5120,13824),(13824,5120)} x M in {1,16}, G=32",
+                                "TB/s": sum(dec_bytes) / sum(ts) / 1e9,
+                                "frac_of_hbm": sum(dec_bytes) / sum(ts) / 1e6 / hbm}
+    ts = time_calls(big_calls, reps=5)
+    rows["act_order_m256"] = {"configs": "M=256, G=32", "TFLOP/s": sum(big_flops) / sum(ts) / 1e9}
+
+    # a8: prefill tensor-core GEMM (70B MLP shapes)
+    pf = S.PREFILL_70B
+    out = {}
+    for (K, N) in pf["shapes"]:
+        G = pf["G"]
+        W = torch.from_numpy(S.layer_w(pf, K, N)).cuda()
+        Wq, sc, zr = w4.quantize_rtn(W, G)
+        wp = w4.prepack(Wq, sc, zr, G)
+        Wd = w4.dequant(Wq, sc, zr, G)
+        del W, Wq, sc, zr
+        for M in pf["Ms"]:
+            X = bf16_dev(S.layer_x(pf, M, K, N))
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            t = time_calls([lambda: w4.w4a16_gemm(X, wp, N, K, G, out=Y)], reps=3)[0]
+            tc = time_calls([lambda: torch.matmul(X, Wd.t())], reps=3)[0]
+            fl = 2.0 * M * N * K
+            out[f"K{K}_N{N}_M{M}"] = {"ms": t, "flops": fl, "TFLOP/s": fl / t / 1e9,
+                                      "frac_of_bf16_peak": fl / t / 1e9 / peaks["bf16_tflops"],
+                                      "cublas_bf16_dense_TFLOP/s": fl / tc / 1e9}
+            del X, Y
+        del Wd, wp
+        torch.cuda.empty_cache()
+    tot_fl = sum(v["flops"] for v in out.values())
+    tot_ms = sum(v["ms"] for v in out.values())
+    rows["prefill_gemm"] = {"per_shape": out, "TFLOP/s": tot_fl / tot_ms / 1e9,
+                            "frac_of_bf16_peak": tot_fl / tot_ms / 1e9 / peaks["bf16_tflops"]}
+    return rows
+
+
+# --------------------------------------------------------------------- CPU oracle
+
+def _oracle_layer(K, N, rows):
+    """Oracle-side data for the first `rows` output rows of a decode layer
+    (rows are independent, so a row subset is a faithful sample)."""
+    import oracle as O
+    W = S.layer_w(WL, K, N)[:rows]
+    q, s, z = O.quantize_rtn(W, WL["G"])             # offline step, not timed
+    return O.pack_nibbles(q), s, z, S.layer_x(WL, 1, K, N)
+
+
+def _oracle_call(Wq, s, z, xb):
+    import oracle as O
+    O.matmul_ref(xb, O.dequant_rtn(Wq, s, z, WL["G"]))
+
+
+def oracle_sample(rows=4096):
+    """Time the CPU oracle (dequant + fp64 matmul) on the decode workload: the
+    first `rows` output rows of each of the 4 layer shapes at M = 1, BLAS
+    limited to one thread.  Returns (bytes, seconds, description)."""
+    from threadpoolctl import threadpool_limits
+    tot_b, tot_s = 0.0, 0.0
+    with threadpool_limits(limits=1):
+        for (K, N) in WL["shapes"]:
+            r = min(rows, N)
+            Wq, s, z, xb = _oracle_layer(K, N, r)
+            t0 = time.perf_counter()
+            _oracle_call(Wq, s, z, xb)
+            tot_s += time.perf_counter() - t0
+            tot_b += int4_bytes(1, r, K, WL["G"])
+    return tot_b, tot_s, (f"first {rows} output rows of each of the 4 layer shapes at M=1: "
+                          "numpy dequant + fp64 matmul, 1 thread")
+
+
+def run_reference(args, world, rank):
+    """`--impl reference`: the CPU oracle as the reference arm, same metric and
+    config.  Each step is one oracle decode call at M = 1 on a row subset of a
+    layer (rotating over the 4 shapes), the subset sized so that the whole run
+    takes about two minutes."""
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_limits
+    n_total = args.warmup + args.steps
+    budget = max(0.002, 90.0 / n_total)             # seconds per step
+    with threadpool_limits(limits=1):
+        # calibrate seconds per row on a 1024-row slice of the deepest layer
+        Wq, s, z, xb = _oracle_layer(11008, 4096, 1024)
+        _oracle_call(Wq, s, z, xb)
+        t0 = time.perf_counter()
+        _oracle_call(Wq, s, z, xb)
+        per_row = 1.5 * (time.perf_counter() - t0) / 1024
+        rows = int(max(8, min(4096, budget / max(per_row, 1e-9))))
+        prepared = [(K, N, *_oracle_layer(K, N, min(rows, N))) for (K, N) in WL["shapes"]]
+        tot_b, tot_s = 0.0, 0.0
+        for i in range(n_total):
+            K, N, Wq, s, z, xb = prepared[i % len(prepared)]
+            t0 = time.perf_counter()
+            _oracle_call(Wq, s, z, xb)
+            dt = time.perf_counter() - t0
+            if i >= args.warmup:
+                tot_s += dt
+                tot_b += int4_bytes(1, Wq.shape[0], K, WL["G"])
+    v = tot_b / tot_s / 1e12
+    sample = (f"one M=1 decode call per step on the first {rows} output rows of a layer, "
+              "4 layer shapes rotating; numpy dequant + fp64 matmul, 1 thread")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_s * 1e3 / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": v, "unit": "TB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-rows", action="store_true", help="skip the other-row measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+
+    world, rank, local, pg = dist_setup()
+    from weight_only_bit_gemm_b200 import build
+    build.build()
+    from weight_only_bit_gemm_b200 import w4
+
+    peaks = load_peaks()
+    step = DecodeStep(w4)
+    ms, per_call, clocks = measure_decode(step, args, pg, local)
+    ms = max_over_ranks(pg, ms)
+    total_bytes = sum_over_ranks(pg, step.step_bytes * args.steps)
+    value = total_bytes / (ms * 1e-3) / 1e12
+    e2e_ms, e2e_n, h2d, d2h = measure_e2e(step, args, pg)
+    e2e_value = sum_over_ranks(pg, step.step_bytes * e2e_n) / (e2e_ms * 1e-3) / 1e12
+    if w4.device_status() != w4.W4_OK:
+        raise RuntimeError("device error during the benchmark")
+
+    kern_ms = sum(per_call)
+    achieved = step.step_bytes / (kern_ms * 1e-3) / 1e9
+    per_shape = {}
+    for c, t in zip(step.calls, per_call):
+        per_shape[f"K{c['K']}_N{c['N']}_M{c['M']}"] = {
+            "us": round(t * 1e3, 3), "TB/s": round(c["bytes"] / (t * 1e-3) / 1e12, 3)}
+
+    rows = None
+    cpu = None
+    if rank == 0 and world == 1:
+        if not args.no_rows:
+            rows = measure_rows(w4, peaks)
+        if not args.no_cpu:
+            b, sec, desc = oracle_sample()
+            cpu = {"value": b / sec / 1e12, "unit": "TB/s", "cores": 1, "kind": "oracle",
+                   "sample": desc, "seconds": sec}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "calls_per_step": len(step.calls),
+                       "bytes_per_step": step.step_bytes,
+                       "l2": f"inputs larger than L2: {step.replicas} weight replicas per layer, "
+                             f"{step.replica_bytes / 1e6:.0f} MB total, each call reads its own",
+                       "parallelism": f"replicas x{world} (independent problems per GPU)",
+                       "timing": "CUDA graph of one step, CUDA events on the launching stream"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": None, "peak_source": peaks["source"],
+                         "kernel": "w4_tc_gemm_kernel (per-call device time)",
+                         "per_call": per_shape},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * len(step.calls),
+            "clocks": clocks,
+        }
+        if rows is not None:
+            line["rows"] = rows
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
