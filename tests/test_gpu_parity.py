@@ -237,3 +237,21 @@ def test_nf4_gemm_tolerance(w4, M, N, K):
     y = w4.nf4_gemm(x_dev(xb), Wp, dev(s2_r), N, K)
     status_ok(w4)
     _check(y, xb, what)
+
+
+def test_workspace_shared_across_shapes(w4):
+    # split-K calls of different tile counts share one workspace: the counters
+    # of one call must never be overwritten by another call's partial sums
+    ws = torch.zeros(64 << 20, dtype=torch.uint8, device="cuda")
+    layers = [(4, 256, 8192, 128), (1, 4096, 4096, 128), (16, 1024, 2048, 64),
+              (3, 2048, 6144, 128)]
+    built = [(M, N, K, G, *_int4_layer(w4, N, K, G, False, seed=20 + i))
+             for i, (M, N, K, G) in enumerate(layers)]
+    for _ in range(2):
+        for M, N, K, G, what, Wp in built:
+            xb = S.draw_x(M, K, seed=M, tag=2, N=N)
+            y = w4.w4a16_gemm(x_dev(xb), Wp, N, K, G, workspace=ws)
+            status_ok(w4)
+            _check(y, xb, what)
+    # the counter region is left zeroed
+    assert int(ws[: 65536 * 4].count_nonzero()) == 0

@@ -47,6 +47,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     mbar_init(epi1, C::kDqWarps);
     mbar_init(epi2, 1);
     fence_barrier_init();
+    grid_dep_launch();  // the next kernel on the stream may start its prologue
   }
   if (C::FMT == kFmtNf4 && threadIdx.x < 16) Ts[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
   if (warp == 1) {
@@ -66,18 +67,33 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
       const uint64_t pol_x = policy_evict_last();   // X is shared by every CTA
       const uint8_t* wsrc =
           args.Wp + (static_cast<size_t>(nt) * args.KS + s0) * C::kWStageBytes;
+      // The weights do not depend on the previous kernel: start streaming the
+      // first ring's worth before waiting for it, then add the X tiles.
+      const int first = nst < C::STAGES ? nst : C::STAGES;
+      for (int it = 0; it < first; ++it) {
+        mbar_arrive_expect_tx(&full[it], C::kXStageBytes + C::kWStageBytes);
+        bulk_g2s(wsl + it * C::kWSlot, wsrc + static_cast<size_t>(it) * C::kWStageBytes,
+                 C::kWStageBytes, &full[it], pol_w);
+      }
+      grid_dep_wait();
       int issued = 0;
       for (int it = 0; it < nst; ++it) {
         const int s = it % C::STAGES;
-        if (it >= C::STAGES && !mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1)) break;
-        mbar_arrive_expect_tx(&full[s], C::kXStageBytes + C::kWStageBytes);
+        if (it >= C::STAGES) {
+          if (!mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1)) break;
+          mbar_arrive_expect_tx(&full[s], C::kXStageBytes + C::kWStageBytes);
+          bulk_g2s(wsl + s * C::kWSlot, wsrc + static_cast<size_t>(it) * C::kWStageBytes,
+                   C::kWStageBytes, &full[s], pol_w);
+        }
         const int k0 = (s0 + it) * kStageK;
         uint8_t* xdst = xs + s * C::kXStageBytes;
         tma_load_2d(xdst, &xmap, k0, mtile * C::MT, &full[s], pol_x);
         tma_load_2d(xdst + C::kXBoxBytes, &xmap, k0 + 64, mtile * C::MT, &full[s], pol_x);
-        bulk_g2s(wsl + s * C::kWSlot, wsrc + static_cast<size_t>(it) * C::kWStageBytes,
-                 C::kWStageBytes, &full[s], pol_w);
         ++issued;
+      }
+      if (issued < first) {
+        // stopped early: the weight copies of the first ring are still counted
+        for (int it = issued; it < first; ++it) mbar_wait(&full[it], 0);
       }
       // never leave with copies in flight: wait for the last issued stages
       for (int it = issued - 1; it >= 0 && it >= issued - C::STAGES; --it)
@@ -179,6 +195,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     // ------------------------------------------------------------ epilogue
     if (ok && __all_sync(0xffffffffu, mbar_wait(accf, 0))) {
       tc_fence_after();
+      grid_dep_wait();  // Y and the workspace may still be in use by the previous kernel
       constexpr int kHalfCols = C::MT / 2;
       const int m_base = mtile * C::MT + h * kHalfCols;
       const int tile_id = mtile * args.tiles_n + nt;
