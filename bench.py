@@ -518,6 +518,29 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_single(w4, args):
+    fmt, K, N, M = args.single[0], *map(int, args.single[1:])
+    if fmt == "nf4":
+        W = torch.from_numpy(S.layer_w(S.NF4_DECODE, K, N)).cuda()
+        q, c, s2 = w4.nf4_quantize(W)
+        wp = w4.nf4_prepack(q, c)
+        X = bf16_dev(S.layer_x(S.NF4_DECODE, M, K, N))
+        f = (lambda: w4.nf4_gemm(X, wp, s2, N, K))
+        nbytes, flops = nf4_bytes(M, N, K), 2.0 * M * N * K
+    else:
+        G = WL["G"]
+        W = torch.from_numpy(S.layer_w(WL, K, N)).cuda()
+        Wq, sc, zr = w4.quantize_rtn(W, G)
+        wp = w4.prepack(Wq, sc, zr, G)
+        X = bf16_dev(S.layer_x(WL, M, K, N))
+        f = (lambda: w4.w4a16_gemm(X, wp, N, K, G))
+        nbytes, flops = int4_bytes(M, N, K, G), 2.0 * M * N * K
+    del W
+    t = time_calls([f], reps=max(1, args.steps), warm=args.warmup)[0]
+    print(json.dumps({"single": [fmt, K, N, M], "us": t * 1e3, "TB/s": nbytes / t / 1e9,
+                      "TFLOP/s": flops / t / 1e9}), flush=True)
+
+
 # --------------------------------------------------------------------- main
 
 def main():
@@ -528,6 +551,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-rows", action="store_true", help="skip the other-row measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--single", nargs=4, metavar=("FMT", "K", "N", "M"),
+                    help="profiling aid: run one layer call (FMT int4|nf4) warmup+steps times "
+                         "eagerly and print its mean device time")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -542,6 +568,10 @@ def main():
     from weight_only_bit_gemm_b200 import build
     build.build()
     from weight_only_bit_gemm_b200 import w4
+
+    if args.single:
+        run_single(w4, args)
+        return
 
     peaks = load_peaks()
     step = DecodeStep(w4)

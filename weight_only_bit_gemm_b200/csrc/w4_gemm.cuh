@@ -39,9 +39,13 @@ struct GemmCfg {
   static constexpr int kWStageBytes = FMT == kFmtInt4 ? int4_stage_bytes(G) : nf4_stage_bytes();
   static constexpr int kWSlot = (kWStageBytes + 127) / 128 * 128;
   static constexpr int kASlots = 3;                   // TMEM A ring (64 columns each)
+  // Independent accumulators: consecutive MMAs of a stage write different
+  // ones, so that narrow (decode) tiles are not serialised on the
+  // accumulator dependency; the epilogue sums them in a fixed order.
+  static constexpr int kAcc = MT <= 16 ? 4 : MT <= 32 ? 2 : 1;
   static constexpr int kDCol = 0;
-  static constexpr int kACol = MT;                    // A slots after the accumulator
-  static constexpr int kColsNeeded = MT + kASlots * 64;
+  static constexpr int kACol = kAcc * MT;             // A slots after the accumulators
+  static constexpr int kColsNeeded = kAcc * MT + kASlots * 64;
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32
                                    : kColsNeeded <= 64 ? 64
                                    : kColsNeeded <= 128 ? 128

@@ -116,7 +116,9 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
           const uint64_t bdesc =
               smem_desc_sw128(xaddr + (kk >> 2) * C::kXBoxBytes + (kk & 3) * 32);
           const uint32_t a_tmem = tmem + C::kACol + a * 64 + kk * 8;
-          mma_bf16_ts(d_tmem, a_tmem, bdesc, idesc, (it | kk) != 0 ? 1u : 0u);
+          const int acc = kk % C::kAcc;
+          mma_bf16_ts(d_tmem + acc * C::MT, a_tmem, bdesc, idesc,
+                      (it > 0 || kk >= C::kAcc) ? 1u : 0u);
         }
         mma_commit(&empty[s]);
         mma_commit(&aempty[a]);
@@ -204,13 +206,20 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
                         kTileRows;
 #pragma unroll 1
       for (int cb = 0; cb < kHalfCols; cb += 8) {
-        uint32_t v[8];
-        tmem_ld8(tmem + lane_base + C::kDCol + h * kHalfCols + cb, v);
-        tmem_wait_ld();
+        float sum[8];
+#pragma unroll
+        for (int ai = 0; ai < C::kAcc; ++ai) {
+          uint32_t v[8];
+          tmem_ld8(tmem + lane_base + C::kDCol + ai * C::MT + h * kHalfCols + cb, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            sum[j] = ai == 0 ? __uint_as_float(v[j]) : sum[j] + __uint_as_float(v[j]);
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int m = m_base + cb + j;
-          const float acc = __uint_as_float(v[j]);
+          const float acc = sum[j];
           if (args.splits == 1) {
             if (m < args.M && n < args.N)
               args.Y[static_cast<size_t>(m) * args.N + n] =
