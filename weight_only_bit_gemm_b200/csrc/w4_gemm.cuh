@@ -64,48 +64,52 @@ struct GemmCfg {
 __device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ __nv_bfloat162 bits_bf2(uint32_t v) {
+__device__ __forceinline__ __nv_bfloat162 bits_bf2_h(uint32_t v) {
   return *reinterpret_cast<__nv_bfloat162*>(&v);
 }
 
-// Exact INT4 dequant of one 32-bit word (8 codes) into 4 bf16 pairs:
+// Exact INT4 dequant of one 32-bit word (8 codes, see w4_prepack.cuh):
 //   w_hat = bf16_rne((q - z) * s)
-// with s (fp16) split as s_hi + s_lo, both exact in bf16 (s_lo has <= 4
-// significant bits).  q is made as the bf16 value 128 + q by OR-ing the code
-// into the mantissa of 128.0; d = (128+q) - (128+z) is exact; d*s_lo is exact
-// (<= 8 bits); and one fused multiply-add d*s_hi + d*s_lo rounds the exact
-// product d*s once to bf16.
+// with the fp16 scale s split as s_hi + s_lo, both exact in bf16 (s_lo has at
+// most 3 significant bits).  q becomes the bf16 value 128 + q by OR-ing the
+// code into the mantissa of 128.0; d = (128+q) - (128+z) is exact; d * s_lo is
+// exact (at most 7 significant bits); and one fused multiply-add
+// d * s_hi + d * s_lo rounds the exact product d * s once to bf16.
 struct Int4Dq {
   __nv_bfloat162 zm, shi, slo;
 };
 
-__device__ __forceinline__ Int4Dq int4_dq_params(uint16_t s16, uint32_t z) {
-  const float sf = __half2float(__ushort_as_half(s16));
-  const __nv_bfloat16 hi = __float2bfloat16_rn(sf);
-  const __nv_bfloat16 lo = __float2bfloat16_rn(sf - __bfloat162float(hi));
-  const __nv_bfloat16 zm = __float2bfloat16_rn(128.0f + static_cast<float>(z));
+__device__ __forceinline__ Int4Dq int4_dq_params(uint32_t s16, uint32_t z) {
+  const float sf = __half2float(__ushort_as_half(static_cast<unsigned short>(s16)));
   Int4Dq p;
-  p.zm = __halves2bfloat162(zm, zm);
-  p.shi = __halves2bfloat162(hi, hi);
-  p.slo = __halves2bfloat162(lo, lo);
+  p.shi = __floats2bfloat162_rn(sf, sf);
+  const float lo = sf - __low2float(p.shi);
+  p.slo = __floats2bfloat162_rn(lo, lo);
+  p.zm = bits_bf2_h((z * 0x00010001u) | 0x43004300u);
   return p;
 }
 
-__device__ __forceinline__ void int4_dq_word(uint32_t w, const Int4Dq& p, uint32_t* out) {
+// Pairs 0 and 1 of the word belong to row r0 (params p0), pairs 2 and 3 to
+// row r1 (params p1).
+__device__ __forceinline__ void int4_dq_word(uint32_t w, const Int4Dq& p0, const Int4Dq& p1,
+                                             uint32_t* out) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
+    const Int4Dq& p = j < 2 ? p0 : p1;
     const uint32_t t = ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
-    const __nv_bfloat162 d = __hsub2(bits_bf2(t), p.zm);
+    const __nv_bfloat162 d = __hsub2(bits_bf2_h(t), p.zm);
     const __nv_bfloat162 l = __hmul2(d, p.slo);
     out[j] = bf2_bits(__hfma2(d, p.shi, l));
   }
 }
 
-// NF4 dequant of one word: w_hat = bf16_rne(fp32(T[q] * a')), T in shared memory.
-__device__ __forceinline__ void nf4_dq_word(uint32_t w, float a, const float* __restrict__ T,
-                                            uint32_t* out) {
+// NF4 dequant of one word: w_hat = bf16_rne(fp32(T[q] * a')), T in shared
+// memory, a0 / a1 the reconstructed absmax of rows r0 / r1.
+__device__ __forceinline__ void nf4_dq_word(uint32_t w, float a0, float a1,
+                                            const float* __restrict__ T, uint32_t* out) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
+    const float a = j < 2 ? a0 : a1;
     const float f0 = __fmul_rn(T[(w >> (4 * j)) & 0xFu], a);
     const float f1 = __fmul_rn(T[(w >> (16 + 4 * j)) & 0xFu], a);
     out[j] = bf2_bits(__floats2bfloat162_rn(f0, f1));

@@ -127,11 +127,14 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     }
   } else {
     // ------------------------------------------------------------ dequant
+    // warp (quadrant q, half h) owns TMEM lanes 32q..32q+31 = row groups 2q,
+    // 2q+1, and channel blocks 4h..4h+3 of every stage
     const int dw = warp - 2;        // 0..7
     const int quad = warp & 3;      // TMEM lane quadrant this warp may access
     const int h = dw >> 2;          // 64-channel half of each stage
-    const int row = quad * 32 + lane;
+    const int row = quad * 32 + lane;  // accumulator lane owned in the epilogue
     const int n = nt * kTileRows + row;
+    const int g = lane >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     bool ok = true;
     for (int it = 0; it < nst && ok; ++it) {
@@ -143,51 +146,52 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
         break;
       }
       const uint8_t* wb = wsl + s * C::kWSlot;
-      const uint4 c0 = *reinterpret_cast<const uint4*>(wb + (2 * h) * 2048 + row * 16);
-      const uint4 c1 = *reinterpret_cast<const uint4*>(wb + (2 * h + 1) * 2048 + row * 16);
-      uint32_t out[32];
-      if constexpr (C::FMT == kFmtInt4) {
-        constexpr int gps = kStageK / C::G;
-        const uint16_t* sc = reinterpret_cast<const uint16_t*>(wb + kCodeBytes);
-        const uint8_t* zb = wb + kCodeBytes + kTileRows * gps * 2;
-        // groups of chunks 2h and 2h+1
-        const int gl0 = (2 * h * 32) / C::G;
-        const int gl1 = ((2 * h + 1) * 32) / C::G;
-        const int i0 = row * gps + gl0, i1 = row * gps + gl1;
-        const Int4Dq p0 = int4_dq_params(sc[i0], (zb[i0 >> 1] >> ((i0 & 1) * 4)) & 0xFu);
-        const Int4Dq p1 = (gl1 == gl0) ? p0
-                          : int4_dq_params(sc[i1], (zb[i1 >> 1] >> ((i1 & 1) * 4)) & 0xFu);
-        int4_dq_word(c0.x, p0, out + 0);
-        int4_dq_word(c0.y, p0, out + 4);
-        int4_dq_word(c0.z, p0, out + 8);
-        int4_dq_word(c0.w, p0, out + 12);
-        int4_dq_word(c1.x, p1, out + 16);
-        int4_dq_word(c1.y, p1, out + 20);
-        int4_dq_word(c1.z, p1, out + 24);
-        int4_dq_word(c1.w, p1, out + 28);
-      } else {
-        const int blk_in_row = (s0 + it) * 2 + h;
-        float aq = 0.0f;
-        if (n < args.N && blk_in_row * 64 < args.K) {
-          const uint32_t c = wb[kCodeBytes + row * 2 + h];
-          const long long b = static_cast<long long>(n) * (args.K / 64) + blk_in_row;
-          aq = __fmul_rn(static_cast<float>(c), __ldg(args.s2 + b / args.dq_group));
+      uint32_t out[2][16];
+#pragma unroll
+      for (int rgl = 0; rgl < 2; ++rgl) {
+        const int rg = quad * 2 + rgl;
+        const uint4 cw = *reinterpret_cast<const uint4*>(wb + code_word_offset(rg, 4 * h, lane));
+        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+        if constexpr (C::FMT == kFmtInt4) {
+          constexpr int gps = kStageK / C::G;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int gl = ((4 * h + w) * 16) / C::G;
+            const uint32_t sp = *reinterpret_cast<const uint32_t*>(wb + scale_pair_offset(rg, gl, g, gps));
+            const uint32_t zp = wb[zero_pair_offset(rg, gl, g, gps)];
+            // (the compiler merges the loads and parameter math shared by words)
+            const Int4Dq p0 = int4_dq_params(sp & 0xFFFFu, zp & 0xFu);
+            const Int4Dq p1 = int4_dq_params(sp >> 16, zp >> 4);
+            int4_dq_word(words[w], p0, p1, &out[rgl][4 * w]);
+          }
+        } else {
+          const int blk_in_row = (s0 + it) * 2 + h;
+          const uint32_t cp = *reinterpret_cast<const uint16_t*>(wb + absmax_pair_offset(rg, h, g));
+          const int r0 = nt * kTileRows + rg * 16 + g;
+          float a0 = 0.0f, a1 = 0.0f;
+          if (blk_in_row * 64 < args.K) {
+            const long long kb64 = args.K / 64;
+            if (r0 < args.N)
+              a0 = __fmul_rn(static_cast<float>(cp & 0xFFu),
+                             __ldg(args.s2 + (static_cast<long long>(r0) * kb64 + blk_in_row) / args.dq_group));
+            if (r0 + 8 < args.N)
+              a1 = __fmul_rn(static_cast<float>(cp >> 8),
+                             __ldg(args.s2 + (static_cast<long long>(r0 + 8) * kb64 + blk_in_row) / args.dq_group));
+          }
+#pragma unroll
+          for (int w = 0; w < 4; ++w) nf4_dq_word(words[w], a0, a1, Ts, &out[rgl][4 * w]);
         }
-        nf4_dq_word(c0.x, aq, Ts, out + 0);
-        nf4_dq_word(c0.y, aq, Ts, out + 4);
-        nf4_dq_word(c0.z, aq, Ts, out + 8);
-        nf4_dq_word(c0.w, aq, Ts, out + 12);
-        nf4_dq_word(c1.x, aq, Ts, out + 16);
-        nf4_dq_word(c1.y, aq, Ts, out + 20);
-        nf4_dq_word(c1.z, aq, Ts, out + 24);
-        nf4_dq_word(c1.w, aq, Ts, out + 28);
       }
       if (it >= C::kASlots &&
           !__all_sync(0xffffffffu, mbar_wait(&aempty[a], ((it / C::kASlots) - 1) & 1))) {
         ok = false;
         break;
       }
-      tmem_st32(tmem + lane_base + C::kACol + a * 64 + h * 32, out);
+#pragma unroll
+      for (int rgl = 0; rgl < 2; ++rgl)
+        tmem_st_16x256b_x4(tmem + lane_base + (static_cast<uint32_t>(16 * rgl) << 16) + C::kACol +
+                               a * 64 + h * 32,
+                           out[rgl]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

@@ -10,6 +10,7 @@
 
 #include "../../include/w4.h"
 #include "w4_gemm_kernel.cuh"
+#include "w4_gemv_kernel.cuh"
 #include "w4_prepack.cuh"
 #include "w4_quant.cuh"
 #include "w4_ptx.cuh"
@@ -127,7 +128,7 @@ w4_status w4_prepack(const uint8_t* Wq, const uint16_t* scales, const uint8_t* z
     if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
   }
   dim3 grid(ceil_div(K, kStageK), ceil_div(N, kTileRows));
-  int4_prepack_kernel<<<grid, kTileRows, 0, st>>>(Wq, scales, zeros, perm, N, K, G, Wp);
+  int4_prepack_kernel<<<grid, 256, 0, st>>>(Wq, scales, zeros, perm, N, K, G, Wp);
   return launch_status(cudaGetLastError());
 }
 
@@ -137,7 +138,7 @@ w4_status w4_unprepack(const uint8_t* Wp, int N, int K, int G, int act_order, ui
   if (!int4_shape_ok(N, K, G) || !aligned(Wp, 16)) return W4_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);
   dim3 grid(ceil_div(K, kStageK), ceil_div(N, kTileRows));
-  int4_unprepack_kernel<<<grid, kTileRows, 0, st>>>(Wp, N, K, G, Wq, scales, zeros);
+  int4_unprepack_kernel<<<grid, 256, 0, st>>>(Wp, N, K, G, Wq, scales, zeros);
   if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
   if (act_order && perm) {
     const int32_t* src = perm_region(const_cast<uint8_t*>(Wp), N, K, G);
@@ -191,7 +192,7 @@ w4_status nf4_prepack(const uint8_t* Wq, const uint8_t* absmax_q, int N, int K, 
   if (!Wq || !absmax_q || !Wp) return W4_ERR_INVALID_ARG;
   if (!nf4_shape_ok(N, K, 64, 256) || !aligned(Wp, 16)) return W4_ERR_INVALID_ARG;
   dim3 grid(ceil_div(K, kStageK), ceil_div(N, kTileRows));
-  nf4_prepack_kernel<<<grid, kTileRows, 0, as_stream(stream)>>>(Wq, absmax_q, N, K, Wp);
+  nf4_prepack_kernel<<<grid, 256, 0, as_stream(stream)>>>(Wq, absmax_q, N, K, Wp);
   return launch_status(cudaGetLastError());
 }
 
