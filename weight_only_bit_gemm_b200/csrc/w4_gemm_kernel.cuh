@@ -85,10 +85,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
           bulk_g2s(wsl + s * C::kWSlot, wsrc + static_cast<size_t>(it) * C::kWStageBytes,
                    C::kWStageBytes, &full[s], pol_w);
         }
-        const int k0 = (s0 + it) * kStageK;
-        uint8_t* xdst = xs + s * C::kXStageBytes;
-        tma_load_2d(xdst, &xmap, k0, mtile * C::MT, &full[s], pol_x);
-        tma_load_2d(xdst + C::kXBoxBytes, &xmap, k0 + 64, mtile * C::MT, &full[s], pol_x);
+        tma_load_3d(xs + s * C::kXStageBytes, &xmap, 0, mtile * C::MT, (s0 + it) * 2, &full[s],
+                    pol_x);
         ++issued;
       }
       if (issued < first) {

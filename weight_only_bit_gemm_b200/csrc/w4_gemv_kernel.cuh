@@ -31,12 +31,14 @@ struct GemvCfg {
   static constexpr int kXStageBytes = 2 * kXBoxBytes;  // 128 channels
   static constexpr int kWStageBytes = FMT == kFmtInt4 ? int4_stage_bytes(G) : nf4_stage_bytes();
   static constexpr int kWSlot = (kWStageBytes + 127) / 128 * 128;
-  static constexpr int kConsumers = 8;                 // one warp per 16-row group
+  // two warps per 16-row group, one per 64-channel half of each stage
+  static constexpr int kConsumers = 16;
   static constexpr int kThreads = 32 * (1 + kConsumers);
-  static constexpr int kNumBars = 2 * STAGES + 2;
+  static constexpr int kNumBars = 2 * STAGES + 3;
   static constexpr int kXRegion = (STAGES * kXStageBytes + 1023) / 1024 * 1024;
+  static constexpr int kRedBytes = 8 * 32 * 4 * NB * 4;  // half-sum exchange
   static constexpr int kSmemBytes =
-      1024 + kXRegion + STAGES * kWSlot + kNumBars * 8 + 16 + 64;
+      1024 + kXRegion + STAGES * kWSlot + kRedBytes + kNumBars * 8 + 16 + 64;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -57,10 +59,12 @@ __global__ void __launch_bounds__(C::kThreads)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* xs = smem;                                 // STAGES x kXStageBytes (1024-aligned)
   uint8_t* wsl = xs + C::kXRegion;                    // STAGES x kWSlot
-  uint64_t* bars = reinterpret_cast<uint64_t*>(wsl + C::STAGES * C::kWSlot);
+  float* red = reinterpret_cast<float*>(wsl + C::STAGES * C::kWSlot);  // [8][32][4 NB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + C::kRedBytes);
   uint64_t* full = bars;                              // X + W landed     (tx)
-  uint64_t* empty = full + C::STAGES;                 // 8 warps consumed
-  uint64_t* epi1 = empty + C::STAGES;                 // partials stored  (8 warps)
+  uint64_t* empty = full + C::STAGES;                 // 16 warps consumed
+  uint64_t* redb = empty + C::STAGES;                 // upper halves stored (8 warps)
+  uint64_t* epi1 = redb + 1;                          // partials stored  (8 warps)
   uint64_t* epi2 = epi1 + 1;                          // last-arrival known
   int* last_flag = reinterpret_cast<int*>(epi2 + 1);
   float* Ts = reinterpret_cast<float*>(epi2 + 1) + 4;  // NF4 levels [16]
@@ -79,7 +83,8 @@ __global__ void __launch_bounds__(C::kThreads)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], C::kConsumers);
     }
-    mbar_init(epi1, C::kConsumers);
+    mbar_init(redb, C::kConsumers / 2);
+    mbar_init(epi1, C::kConsumers / 2);
     mbar_init(epi2, 1);
     fence_barrier_init();
     grid_dep_launch();
@@ -112,10 +117,10 @@ __global__ void __launch_bounds__(C::kThreads)
           bulk_g2s(wsl + s * C::kWSlot, wsrc + static_cast<size_t>(it) * C::kWStageBytes,
                    C::kWStageBytes, &full[s], pol_w);
         }
-        const int k0 = (s0 + it) * kStageK;
-        uint8_t* xdst = xs + s * C::kXStageBytes;
-        tma_load_2d(xdst, &xmap, k0, mtile * C::MT, &full[s], pol_x);
-        tma_load_2d(xdst + C::kXBoxBytes, &xmap, k0 + 64, mtile * C::MT, &full[s], pol_x);
+        // both 64-channel boxes of the stage in one copy (X viewed as
+        // [K/64][M][64])
+        tma_load_3d(xs + s * C::kXStageBytes, &xmap, 0, mtile * C::MT, (s0 + it) * 2, &full[s],
+                    pol_x);
         ++issued;
       }
       for (int it = issued - 1; it >= 0 && it >= issued - C::STAGES; --it)
@@ -123,17 +128,20 @@ __global__ void __launch_bounds__(C::kThreads)
     }
   } else {
     // ------------------------------------------------------------ consumers
-    const int rg = warp - 1;  // 16-row group of the tile
+    const int cw = warp - 1;            // 0..15
+    const int rg = cw & 7;              // 16-row group of the tile
+    const int kq = cw >> 3;             // channel half of every stage
     const int g = lane >> 2, u = lane & 3;
     const int r0 = nt * kTileRows + rg * 16 + g;
-    float acc[C::NB][4];
+    // two accumulator sets (even / odd channel blocks) to shorten the MMA
+    // dependency chain
+    float acc[2][C::NB][4];
 #pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb)
+    for (int e = 0; e < 2; ++e)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[nb][j] = 0.0f;
-    // X fragment offsets inside a 64-channel box for token n = 8 nb + g and
-    // channels 16 (kb % 4) + 4u .. + 3 (128-byte swizzle: 16-byte chunk c of
-    // row n sits at chunk c ^ (n % 8))
+      for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[e][nb][j] = 0.0f;
     bool ok = true;
     for (int it = 0; it < nst; ++it) {
       const int s = it % C::STAGES;
@@ -142,67 +150,91 @@ __global__ void __launch_bounds__(C::kThreads)
         break;
       }
       const uint8_t* wb = wsl + s * C::kWSlot;
-      const uint8_t* xb = xs + s * C::kXStageBytes;
+      // X box of this half: token n = 8 nb + g, channels 16 w + 4u .. +3; with
+      // the 128-byte swizzle the 16-byte chunk c of row n sits at c ^ (n % 8)
+      const uint8_t* xbox = xs + s * C::kXStageBytes + kq * C::kXBoxBytes;
+      const uint4 cwd = *reinterpret_cast<const uint4*>(wb + code_word_offset(rg, 4 * kq, lane));
+      const uint32_t words[4] = {cwd.x, cwd.y, cwd.z, cwd.w};
+      Int4Dq p0[2], p1[2];
+      float a0 = 0.0f, a1 = 0.0f;
+      if constexpr (C::FMT == kFmtInt4) {
+        constexpr int gps = kStageK / C::G;
 #pragma unroll
-      for (int kq = 0; kq < 2; ++kq) {
-        const uint4 cw = *reinterpret_cast<const uint4*>(wb + code_word_offset(rg, 4 * kq, lane));
-        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-        Int4Dq p0[2], p1[2];
-        float a0 = 0.0f, a1 = 0.0f;
-        if constexpr (C::FMT == kFmtInt4) {
-          constexpr int gps = kStageK / C::G;
-#pragma unroll
-          for (int q = 0; q < (C::G == 32 ? 2 : 1); ++q) {
-            const int gl = (kq * 64 + q * 32) / C::G;
-            const uint32_t sp = *reinterpret_cast<const uint32_t*>(wb + scale_pair_offset(rg, gl, g, gps));
-            const uint32_t zp = wb[zero_pair_offset(rg, gl, g, gps)];
-            p0[q] = int4_dq_params(sp & 0xFFFFu, zp & 0xFu);
-            p1[q] = int4_dq_params(sp >> 16, zp >> 4);
-          }
-        } else {
-          const int blk_in_row = (s0 + it) * 2 + kq;
-          const uint32_t cp = *reinterpret_cast<const uint16_t*>(wb + absmax_pair_offset(rg, kq, g));
-          if (blk_in_row * 64 < args.K) {
-            const long long kb64 = args.K / 64;
-            if (r0 < args.N)
-              a0 = __fmul_rn(static_cast<float>(cp & 0xFFu),
-                             __ldg(args.s2 + (static_cast<long long>(r0) * kb64 + blk_in_row) / args.dq_group));
-            if (r0 + 8 < args.N)
-              a1 = __fmul_rn(static_cast<float>(cp >> 8),
-                             __ldg(args.s2 + (static_cast<long long>(r0 + 8) * kb64 + blk_in_row) / args.dq_group));
-          }
+        for (int q = 0; q < (C::G == 32 ? 2 : 1); ++q) {
+          const int gl = (kq * 64 + q * 32) / C::G;
+          const uint32_t sp = *reinterpret_cast<const uint32_t*>(wb + scale_pair_offset(rg, gl, g, gps));
+          const uint32_t zp = wb[zero_pair_offset(rg, gl, g, gps)];
+          p0[q] = int4_dq_params(sp & 0xFFFFu, zp & 0xFu);
+          p1[q] = int4_dq_params(sp >> 16, zp >> 4);
         }
-        const uint8_t* xbox = xb + kq * C::kXBoxBytes;
+      } else {
+        const int blk_in_row = (s0 + it) * 2 + kq;
+        const uint32_t cp = *reinterpret_cast<const uint16_t*>(wb + absmax_pair_offset(rg, kq, g));
+        if (blk_in_row * 64 < args.K) {
+          const long long kb64 = args.K / 64;
+          if (r0 < args.N)
+            a0 = __fmul_rn(static_cast<float>(cp & 0xFFu),
+                           __ldg(args.s2 + (static_cast<long long>(r0) * kb64 + blk_in_row) / args.dq_group));
+          if (r0 + 8 < args.N)
+            a1 = __fmul_rn(static_cast<float>(cp >> 8),
+                           __ldg(args.s2 + (static_cast<long long>(r0 + 8) * kb64 + blk_in_row) / args.dq_group));
+        }
+      }
+      uint2 bfr[4][C::NB];
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          uint32_t pr[4];
-          if constexpr (C::FMT == kFmtInt4) {
-            const int q = (C::G == 32) ? (w >> 1) : 0;
-            int4_dq_word(words[w], p0[q], p1[q], pr);
-          } else {
-            nf4_dq_word(words[w], a0, a1, Ts, pr);
-          }
-          const uint32_t afrag[4] = {pr[0], pr[2], pr[1], pr[3]};
+      for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int nb = 0; nb < C::NB; ++nb) {
+          const int n = nb * 8 + g;
           const int chunk = w * 2 + (u >> 1);
-#pragma unroll
-          for (int nb = 0; nb < C::NB; ++nb) {
-            const int n = nb * 8 + g;
-            const uint2 b = *reinterpret_cast<const uint2*>(
-                xbox + n * 128 + ((chunk ^ (n & 7)) << 4) + (u & 1) * 8);
-            mma_m16n8k16_bf16(acc[nb], afrag, b.x, b.y);
-          }
+          bfr[w][nb] = *reinterpret_cast<const uint2*>(xbox + n * 128 + ((chunk ^ (n & 7)) << 4) +
+                                                       (u & 1) * 8);
         }
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t pr[4];
+        if constexpr (C::FMT == kFmtInt4) {
+          const int q = (C::G == 32) ? (w >> 1) : 0;
+          int4_dq_word(words[w], p0[q], p1[q], pr);
+        } else {
+          nf4_dq_word(words[w], a0, a1, Ts, pr);
+        }
+        const uint32_t afrag[4] = {pr[0], pr[2], pr[1], pr[3]};
+#pragma unroll
+        for (int nb = 0; nb < C::NB; ++nb)
+          mma_m16n8k16_bf16(acc[w & 1][nb], afrag, bfr[w][nb].x, bfr[w][nb].y);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
 
     // ------------------------------------------------------------ epilogue
-    // acc[nb] = D[rows r0, r0+8][tokens 8nb + 2u, 8nb + 2u + 1]
-    if (ok) {
+    // the upper-half warp hands its sums to the lower-half warp of the same
+    // row group through shared memory
+    float tot[C::NB][4];
+#pragma unroll
+    for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tot[nb][j] = acc[0][nb][j] + acc[1][nb][j];
+    float* rslot = red + (rg * 32 + lane) * 4 * C::NB;
+    if (kq == 1) {
+      if (ok) {
+#pragma unroll
+        for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) rslot[nb * 4 + j] = tot[nb][j];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(redb);
+    } else if (ok && __all_sync(0xffffffffu, mbar_wait(redb, 0))) {
+#pragma unroll
+      for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tot[nb][j] += rslot[nb * 4 + j];
+      // tot[nb] = D[rows r0, r0+8][tokens 8nb + 2u, 8nb + 2u + 1]
       grid_dep_wait();
       const int tile_id = mtile * args.tiles_n + nt;
-      const int row_l = rg * 16 + g;  // row of the tile for acc[.][0..1]; +8 for [2..3]
+      const int row_l = rg * 16 + g;  // tile row of tot[.][0..1]; +8 for [2..3]
       if (args.splits == 1) {
 #pragma unroll
         for (int nb = 0; nb < C::NB; ++nb)
@@ -212,7 +244,7 @@ __global__ void __launch_bounds__(C::kThreads)
             const int nn = r0 + (j >> 1) * 8;
             if (m < args.M && nn < args.N)
               args.Y[static_cast<size_t>(m) * args.N + nn] =
-                  __bfloat16_as_ushort(__float2bfloat16_rn(acc[nb][j]));
+                  __bfloat16_as_ushort(__float2bfloat16_rn(tot[nb][j]));
           }
       } else {
         float* part = args.partial +
@@ -221,11 +253,14 @@ __global__ void __launch_bounds__(C::kThreads)
         for (int nb = 0; nb < C::NB; ++nb)
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            part[(nb * 8 + 2 * u + (j & 1)) * kTileRows + row_l + (j >> 1) * 8] = acc[nb][j];
+            part[(nb * 8 + 2 * u + (j & 1)) * kTileRows + row_l + (j >> 1) * 8] = tot[nb][j];
+        // the last CTA of this tile to arrive sums the partials in split order
+        // (mbarriers with bounded waits, not bar.sync, so that a warp that gave
+        // up earlier cannot leave the others blocked)
         __threadfence();
         __syncwarp();
         if (lane == 0) mbar_arrive(epi1);
-        if (threadIdx.x == 32) {
+        if (cw == 0 && lane == 0) {
           if (mbar_wait(epi1, 0)) {
             const unsigned prev = atomicAdd(args.counter + tile_id, 1u);
             *last_flag = (prev == static_cast<unsigned>(args.splits - 1)) ? 1 : 0;
@@ -278,7 +313,7 @@ __global__ void __launch_bounds__(C::kThreads)
                 args.Y[static_cast<size_t>(m) * args.N + nn] =
                     __bfloat16_as_ushort(__float2bfloat16_rn(sum[nb][j]));
             }
-          if (threadIdx.x == 32) args.counter[tile_id] = 0u;
+          if (cw == 0 && lane == 0) args.counter[tile_id] = 0u;
         }
       }
     }
