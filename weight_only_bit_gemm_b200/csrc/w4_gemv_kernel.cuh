@@ -53,8 +53,10 @@ struct GemvCfg {
   static constexpr int kStageBytes = FMT == kFmtInt4 ? int4_stage_bytes(G) : nf4_stage_bytes();
   static constexpr int kWarps = 8;
   static constexpr int kThreads = 32 * kWarps;
-  static constexpr int kDepth = NB <= 2 ? 8 : 4;  // units of codes in flight per lane
-  static constexpr int kNq = (FMT == kFmtInt4 && G == 32) ? 2 : 1;  // groups per unit
+  static constexpr int kMinBlocks = 2;  // CTAs per SM the register budget allows
+  static constexpr int kDepth = NB <= 2 ? 4 : 2;  // stages of codes in flight per lane
+  // groups per 128-channel stage (INT4); NF4 keeps its absmax pairs in sp[0]
+  static constexpr int kNq = FMT == kFmtInt4 ? 128 / G : 1;
 };
 
 __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t (&a)[4],
@@ -75,103 +77,64 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
-// Per-unit weight data of a lane: 4 code words and the constants of its two
-// rows (prefetched kDepth units ahead).
+// One 128-channel stage of a lane's row group: 8 code words (two 16-byte
+// loads, 512 contiguous bytes per warp each) and the constants of its two rows.
 template <class C>
-struct CodeRegs {
-  uint4 codes;
-  uint32_t sp[C::kNq];     // INT4: scale pairs (per group in the unit); NF4: absmax pair
-  uint32_t zp[C::kNq];     // INT4: zero pairs
-};
-
-// Activation fragments of one unit (fetched one unit ahead).
-template <class C>
-struct XRegs {
-  uint2 b[4][C::NB];
+struct StageRegs {
+  uint4 c0, c1;            // code words of channel blocks 0..3 and 4..7
+  uint32_t sp[C::kNq];     // INT4: scale pairs, one per group in the stage; NF4: absmax pair, block 0
+  uint32_t zp[C::kNq];     // INT4: zero pairs; NF4: absmax pair, block 1
 };
 
 template <class C>
-__device__ __forceinline__ void load_codes(const GemvArgs& a, CodeRegs<C>& r, int rgg, int unit,
-                                           int lane) {
+__device__ __forceinline__ void load_stage(const uint8_t* __restrict__ blk, StageRegs<C>& r,
+                                           int rgl, int lane) {
   const int g = lane >> 2;
-  const int tile = rgg >> 3, rgl = rgg & 7;
-  const int stage = unit >> 1, half = unit & 1;
-  const uint8_t* blk = a.Wp + (static_cast<size_t>(tile) * a.KS + stage) * C::kStageBytes;
-  r.codes = ldg_stream(blk + code_word_offset(rgl, 4 * half, lane));
+  r.c0 = ldg_stream(blk + code_word_offset(rgl, 0, lane));
+  r.c1 = ldg_stream(blk + code_word_offset(rgl, 4, lane));
   if constexpr (C::FMT == kFmtInt4) {
     constexpr int gps = kStageK / C::G;
 #pragma unroll
     for (int q = 0; q < C::kNq; ++q) {
-      const int gl = (half * 64 + q * 32) / C::G;
-      r.sp[q] = __ldg(reinterpret_cast<const uint32_t*>(blk + scale_pair_offset(rgl, gl, g, gps)));
-      r.zp[q] = __ldg(blk + zero_pair_offset(rgl, gl, g, gps));
+      r.sp[q] = __ldg(reinterpret_cast<const uint32_t*>(blk + scale_pair_offset(rgl, q, g, gps)));
+      r.zp[q] = __ldg(blk + zero_pair_offset(rgl, q, g, gps));
     }
   } else {
-    r.sp[0] = __ldg(reinterpret_cast<const uint16_t*>(blk + absmax_pair_offset(rgl, half, g)));
+    r.sp[0] = __ldg(reinterpret_cast<const uint16_t*>(blk + absmax_pair_offset(rgl, 0, g)));
+    r.zp[0] = __ldg(reinterpret_cast<const uint16_t*>(blk + absmax_pair_offset(rgl, 1, g)));
   }
 }
 
+// Dequantize one 64-channel half (4 code words) and run its MMAs.  `xrow`
+// points at X[token g][first channel of the half + 4u] (token block 0);
+// tokens_left = M - g.
 template <class C>
-__device__ __forceinline__ void load_x(const GemvArgs& a, XRegs<C>& r, int unit, int lane) {
-  const int g = lane >> 2, u = lane & 3;
-  const int k0 = unit * 64;
-#pragma unroll
-  for (int w = 0; w < 4; ++w)
-#pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb) {
-      const int n = nb * 8 + g;
-      const int k = k0 + w * 16 + 4 * u;
-      r.b[w][nb] = (n < a.M && k < a.K)
-                       ? __ldg(reinterpret_cast<const uint2*>(a.X + static_cast<size_t>(n) * a.K + k))
-                       : make_uint2(0u, 0u);
-    }
-}
-
-template <class C>
-__device__ __forceinline__ void compute_unit(const GemvArgs& a, const CodeRegs<C>& r,
-                                             const XRegs<C>& x, int rgg, int unit, int lane,
-                                             const float* __restrict__ T,
-                                             float (&acc)[2][C::NB][4]) {
-  const int g = lane >> 2;
-  const uint32_t words[4] = {r.codes.x, r.codes.y, r.codes.z, r.codes.w};
-  Int4Dq p0[C::kNq], p1[C::kNq];
-  float a0 = 0.0f, a1 = 0.0f;
-  if constexpr (C::FMT == kFmtInt4) {
-#pragma unroll
-    for (int q = 0; q < C::kNq; ++q) {
-      p0[q] = int4_dq_params(r.sp[q] & 0xFFFFu, r.zp[q] & 0xFu);
-      p1[q] = int4_dq_params(r.sp[q] >> 16, (r.zp[q] >> 4) & 0xFu);
-    }
-  } else {
-    const int r0 = rgg * 16 + g;
-    if (unit * 64 < a.K) {
-      const long long kb64 = a.K / 64;
-      if (r0 < a.N)
-        a0 = __fmul_rn(static_cast<float>(r.sp[0] & 0xFFu),
-                       __ldg(a.s2 + (static_cast<long long>(r0) * kb64 + unit) / a.dq_group));
-      if (r0 + 8 < a.N)
-        a1 = __fmul_rn(static_cast<float>((r.sp[0] >> 8) & 0xFFu),
-                       __ldg(a.s2 + (static_cast<long long>(r0 + 8) * kb64 + unit) / a.dq_group));
-    }
-  }
+__device__ __forceinline__ void mma_half(uint4 cw, const Int4Dq* p0, const Int4Dq* p1, float a0,
+                                         float a1, const float* __restrict__ T,
+                                         const uint16_t* __restrict__ xrow, size_t xnb_stride,
+                                         int tokens_left, float (&acc)[2][C::NB][4]) {
+  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     uint32_t pr[4];
     if constexpr (C::FMT == kFmtInt4) {
-      const int q = (C::kNq == 2) ? (w >> 1) : 0;
-      int4_dq_word(words[w], p0[q], p1[q], pr);
+      int4_dq_word(words[w], p0[w >> 1], p1[w >> 1], pr);
     } else {
       nf4_dq_word(words[w], a0, a1, T, pr);
     }
     const uint32_t afrag[4] = {pr[0], pr[2], pr[1], pr[3]};
 #pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb)
-      mma_m16n8k16_bf16(acc[w & 1][nb], afrag, x.b[w][nb].x, x.b[w][nb].y);
+    for (int nb = 0; nb < C::NB; ++nb) {
+      uint2 b = make_uint2(0u, 0u);
+      if (nb * 8 < tokens_left)  // token 8 nb + g exists
+        b = __ldg(reinterpret_cast<const uint2*>(xrow + nb * xnb_stride + w * 16));
+      mma_m16n8k16_bf16(acc[w & 1][nb], afrag, b.x, b.y);
+    }
   }
 }
 
 template <class C>
-__global__ void __launch_bounds__(C::kThreads) w4_gemv_kernel(const GemvArgs args) {
+__global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(const GemvArgs args) {
   __shared__ float Ts[16];
   if (C::FMT == kFmtNf4) {
     if (threadIdx.x < 16) Ts[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
@@ -182,15 +145,21 @@ __global__ void __launch_bounds__(C::kThreads) w4_gemv_kernel(const GemvArgs arg
 
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, u = lane & 3;
-  const int warp_global = blockIdx.x * C::kWarps + (threadIdx.x >> 5);
-  const int warps_total = gridDim.x * C::kWarps;
-  const int items = args.row_groups * args.segs;
+  const int rgl = threadIdx.x >> 5;  // row group inside the tile = warp index
+  const int tiles = (args.row_groups + 7) / 8;
+  const int tasks = tiles * args.segs;
+  const size_t xnb_stride = static_cast<size_t>(8) * args.K;
 
-  for (int item = warp_global; item < items; item += warps_total) {
-    const int rgg = item / args.segs;
-    const int seg = item - rgg * args.segs;
-    const int u0 = static_cast<int>(static_cast<long long>(seg) * args.units / args.segs);
-    const int u1 = static_cast<int>(static_cast<long long>(seg + 1) * args.units / args.segs);
+  // a CTA task = (tile, segment): its 8 warps take the tile's 8 row groups
+  // over the same channel range, so their activation loads share L1
+  for (int task = blockIdx.x; task < tasks; task += gridDim.x) {
+    const int tile = task / args.segs;
+    const int seg = task - tile * args.segs;
+    const int rgg = tile * 8 + rgl;
+    if (rgg >= args.row_groups) continue;
+    const int st0 = static_cast<int>(static_cast<long long>(seg) * args.KS / args.segs);
+    const int st1 = static_cast<int>(static_cast<long long>(seg + 1) * args.KS / args.segs);
+    const uint8_t* blk0 = args.Wp + (static_cast<size_t>(tile) * args.KS + st0) * C::kStageBytes;
     float acc[2][C::NB][4];
 #pragma unroll
     for (int e = 0; e < 2; ++e)
@@ -198,24 +167,60 @@ __global__ void __launch_bounds__(C::kThreads) w4_gemv_kernel(const GemvArgs arg
       for (int nb = 0; nb < C::NB; ++nb)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[e][nb][j] = 0.0f;
+    // token g of each token block; tokens >= M read nothing (zero fragments)
+    const int tokens_left = args.M - g;
+    const uint16_t* xbase = args.X + static_cast<size_t>(g) * args.K + 4 * u;
+    const int r0 = rgg * 16 + g;
 
-    // ring of kDepth units of codes in flight; activations one unit ahead
-    CodeRegs<C> cr[C::kDepth];
+    // ring of kDepth stages in flight
+    StageRegs<C> ring[C::kDepth];
 #pragma unroll
     for (int i = 0; i < C::kDepth; ++i)
-      if (u0 + i < u1) load_codes<C>(args, cr[i], rgg, u0 + i, lane);
-    XRegs<C> xa;
-    load_x<C>(args, xa, u0, lane);
-    for (int ub = u0; ub < u1; ub += C::kDepth) {
+      if (st0 + i < st1) load_stage<C>(blk0 + static_cast<size_t>(i) * C::kStageBytes, ring[i], rgl, lane);
+    for (int sb = st0; sb < st1; sb += C::kDepth) {
 #pragma unroll
       for (int i = 0; i < C::kDepth; ++i) {
-        const int un = ub + i;
-        if (un < u1) {
-          XRegs<C> xn;
-          if (un + 1 < u1) load_x<C>(args, xn, un + 1, lane);
-          compute_unit<C>(args, cr[i], xa, rgg, un, lane, Ts, acc);
-          if (un + C::kDepth < u1) load_codes<C>(args, cr[i], rgg, un + C::kDepth, lane);
-          xa = xn;
+        const int st = sb + i;
+        if (st < st1) {
+          const StageRegs<C> cur = ring[i];
+          if (st + C::kDepth < st1)
+            load_stage<C>(blk0 + static_cast<size_t>(st - st0 + C::kDepth) * C::kStageBytes,
+                          ring[i], rgl, lane);
+          Int4Dq p0[4], p1[4];  // per 32-channel quarter of the stage
+          float a0[2] = {0.0f, 0.0f}, a1[2] = {0.0f, 0.0f};
+          if constexpr (C::FMT == kFmtInt4) {
+#pragma unroll
+            for (int q = 0; q < C::kNq; ++q) {
+              const Int4Dq e0 = int4_dq_params(cur.sp[q] & 0xFFFFu, cur.zp[q] & 0xFu);
+              const Int4Dq e1 = int4_dq_params(cur.sp[q] >> 16, (cur.zp[q] >> 4) & 0xFu);
+              // group q covers quarters [q * 4 / kNq, (q + 1) * 4 / kNq)
+#pragma unroll
+              for (int t = 0; t < 4 / C::kNq; ++t) {
+                p0[q * (4 / C::kNq) + t] = e0;
+                p1[q * (4 / C::kNq) + t] = e1;
+              }
+            }
+          } else {
+            const long long kb64 = args.K / 64;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int blk = st * 2 + h;
+              if (blk < kb64) {
+                const uint32_t pair = h == 0 ? cur.sp[0] : cur.zp[0];
+                if (r0 < args.N)
+                  a0[h] = __fmul_rn(static_cast<float>(pair & 0xFFu),
+                                    __ldg(args.s2 + (static_cast<long long>(r0) * kb64 + blk) / args.dq_group));
+                if (r0 + 8 < args.N)
+                  a1[h] = __fmul_rn(static_cast<float>(pair >> 8),
+                                    __ldg(args.s2 + (static_cast<long long>(r0 + 8) * kb64 + blk) / args.dq_group));
+              }
+            }
+          }
+          const int k0 = st * kStageK;
+          mma_half<C>(cur.c0, p0, p1, a0[0], a1[0], Ts, xbase + k0, xnb_stride, tokens_left, acc);
+          if (k0 + 64 < args.K)
+            mma_half<C>(cur.c1, p0 + 2, p1 + 2, a0[1], a1[1], Ts, xbase + k0 + 64, xnb_stride,
+                        tokens_left, acc);
         }
       }
     }
@@ -226,7 +231,6 @@ __global__ void __launch_bounds__(C::kThreads) w4_gemv_kernel(const GemvArgs arg
     for (int nb = 0; nb < C::NB; ++nb)
 #pragma unroll
       for (int j = 0; j < 4; ++j) tot[nb][j] = acc[0][nb][j] + acc[1][nb][j];
-    const int r0 = rgg * 16 + g;
     bool write_y = true;
     if (args.segs > 1) {
       float* slot = args.partial +
