@@ -53,8 +53,8 @@ struct GemvCfg {
   static constexpr int kStageBytes = FMT == kFmtInt4 ? int4_stage_bytes(G) : nf4_stage_bytes();
   static constexpr int kWarps = 8;
   static constexpr int kThreads = 32 * kWarps;
-  static constexpr int kMinBlocks = 2;  // CTAs per SM the register budget allows
-  static constexpr int kDepth = NB <= 2 ? 4 : 2;  // stages of codes in flight per lane
+  static constexpr int kMinBlocks = NB == 1 ? 3 : 2;  // 85 / 128 registers
+  static constexpr int kDepth = 2;  // stages of codes in flight per lane (per-warp: 2 KB)
   // groups per 128-channel stage (INT4); NF4 keeps its absmax pairs in sp[0]
   static constexpr int kNq = FMT == kFmtInt4 ? 128 / G : 1;
 };
@@ -105,20 +105,21 @@ __device__ __forceinline__ void load_stage(const uint8_t* __restrict__ blk, Stag
   }
 }
 
-// Dequantize one 64-channel half (4 code words) and run its MMAs.  `xrow`
-// points at X[token g][first channel of the half + 4u] (token block 0);
-// tokens_left = M - g.
-template <class C>
-__device__ __forceinline__ void mma_half(uint4 cw, const Int4Dq* p0, const Int4Dq* p1, float a0,
-                                         float a1, const float* __restrict__ T,
-                                         const uint16_t* __restrict__ xrow, size_t xnb_stride,
-                                         int tokens_left, float (&acc)[2][C::NB][4]) {
-  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+// Dequantize code words [w0, w0 + nw) of one 64-channel half and run their
+// MMAs.  `xrow` points at X[token g][first channel of the half + 4u] (token
+// block 0); tokens_left = M - g; p0 / p1 are the constants of rows r0 / r1 (INT4),
+// a0 / a1 the reconstructed absmax (NF4).
+template <class C, int W0, int NW>
+__device__ __forceinline__ void mma_words(const uint32_t (&words)[4], const Int4Dq& p0,
+                                          const Int4Dq& p1, float a0, float a1,
+                                          const float* __restrict__ T,
+                                          const uint16_t* __restrict__ xrow, size_t xnb_stride,
+                                          int tokens_left, float (&acc)[2][C::NB][4]) {
 #pragma unroll
-  for (int w = 0; w < 4; ++w) {
+  for (int w = W0; w < W0 + NW; ++w) {
     uint32_t pr[4];
     if constexpr (C::FMT == kFmtInt4) {
-      int4_dq_word(words[w], p0[w >> 1], p1[w >> 1], pr);
+      int4_dq_word(words[w], p0, p1, pr);
     } else {
       nf4_dq_word(words[w], a0, a1, T, pr);
     }
@@ -186,22 +187,51 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
           if (st + C::kDepth < st1)
             load_stage<C>(blk0 + static_cast<size_t>(st - st0 + C::kDepth) * C::kStageBytes,
                           ring[i], rgl, lane);
-          Int4Dq p0[4], p1[4];  // per 32-channel quarter of the stage
-          float a0[2] = {0.0f, 0.0f}, a1[2] = {0.0f, 0.0f};
+          const int k0 = st * kStageK;
+          const uint32_t w0[4] = {cur.c0.x, cur.c0.y, cur.c0.z, cur.c0.w};
+          const uint32_t w1[4] = {cur.c1.x, cur.c1.y, cur.c1.z, cur.c1.w};
+          const bool second = k0 + 64 < args.K;
           if constexpr (C::FMT == kFmtInt4) {
+            if constexpr (C::G == 128) {
+              const Int4Dq e0 = int4_dq_params(cur.sp[0] & 0xFFFFu, cur.zp[0] & 0xFu);
+              const Int4Dq e1 = int4_dq_params(cur.sp[0] >> 16, (cur.zp[0] >> 4) & 0xFu);
+              mma_words<C, 0, 4>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
+              if (second)
+                mma_words<C, 0, 4>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
+                                   tokens_left, acc);
+            } else if constexpr (C::G == 64) {
+              {
+                const Int4Dq e0 = int4_dq_params(cur.sp[0] & 0xFFFFu, cur.zp[0] & 0xFu);
+                const Int4Dq e1 = int4_dq_params(cur.sp[0] >> 16, (cur.zp[0] >> 4) & 0xFu);
+                mma_words<C, 0, 4>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
+              }
+              if (second) {
+                const Int4Dq e0 = int4_dq_params(cur.sp[1] & 0xFFFFu, cur.zp[1] & 0xFu);
+                const Int4Dq e1 = int4_dq_params(cur.sp[1] >> 16, (cur.zp[1] >> 4) & 0xFu);
+                mma_words<C, 0, 4>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
+                                   tokens_left, acc);
+              }
+            } else {
 #pragma unroll
-            for (int q = 0; q < C::kNq; ++q) {
-              const Int4Dq e0 = int4_dq_params(cur.sp[q] & 0xFFFFu, cur.zp[q] & 0xFu);
-              const Int4Dq e1 = int4_dq_params(cur.sp[q] >> 16, (cur.zp[q] >> 4) & 0xFu);
-              // group q covers quarters [q * 4 / kNq, (q + 1) * 4 / kNq)
-#pragma unroll
-              for (int t = 0; t < 4 / C::kNq; ++t) {
-                p0[q * (4 / C::kNq) + t] = e0;
-                p1[q * (4 / C::kNq) + t] = e1;
+              for (int q = 0; q < 4; ++q) {
+                if (q >= 2 && !second) break;
+                const Int4Dq e0 = int4_dq_params(cur.sp[q] & 0xFFFFu, cur.zp[q] & 0xFu);
+                const Int4Dq e1 = int4_dq_params(cur.sp[q] >> 16, (cur.zp[q] >> 4) & 0xFu);
+                if (q == 0)
+                  mma_words<C, 0, 2>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
+                else if (q == 1)
+                  mma_words<C, 2, 2>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
+                else if (q == 2)
+                  mma_words<C, 0, 2>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
+                                     tokens_left, acc);
+                else
+                  mma_words<C, 2, 2>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
+                                     tokens_left, acc);
               }
             }
           } else {
             const long long kb64 = args.K / 64;
+            float a0[2] = {0.0f, 0.0f}, a1[2] = {0.0f, 0.0f};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int blk = st * 2 + h;
@@ -215,12 +245,13 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
                                     __ldg(args.s2 + (static_cast<long long>(r0 + 8) * kb64 + blk) / args.dq_group));
               }
             }
+            const Int4Dq none{};
+            mma_words<C, 0, 4>(w0, none, none, a0[0], a1[0], Ts, xbase + k0, xnb_stride,
+                               tokens_left, acc);
+            if (second)
+              mma_words<C, 0, 4>(w1, none, none, a0[1], a1[1], Ts, xbase + k0 + 64, xnb_stride,
+                                 tokens_left, acc);
           }
-          const int k0 = st * kStageK;
-          mma_half<C>(cur.c0, p0, p1, a0[0], a1[0], Ts, xbase + k0, xnb_stride, tokens_left, acc);
-          if (k0 + 64 < args.K)
-            mma_half<C>(cur.c1, p0 + 2, p1 + 2, a0[1], a1[1], Ts, xbase + k0 + 64, xnb_stride,
-                        tokens_left, acc);
         }
       }
     }
