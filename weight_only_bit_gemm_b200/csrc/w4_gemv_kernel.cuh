@@ -34,13 +34,13 @@ struct GemvArgs {
   const uint16_t* X;        // bf16 [M, K] (act-order: already gathered)
   const float* s2;          // NF4 second-level scales
   uint16_t* Y;              // bf16 [M, N]
-  float* partial;           // [row group][segment][32 lanes][4 NB] fp32
+  float* partial;           // [row group][slot][32 lanes][4 NB] fp32
   unsigned int* counter;    // [row group] arrivals
   int M, N, K;
   int KS;                   // stages (128 channels) per tile row
-  int units;                // 64-channel units per row = ceil(K / 64)
   int row_groups;           // ceil(N / 16)
-  int segs;                 // segments per row group
+  int max_slots;            // partial slots per row group
+  long long total;          // (row group, stage) work units = row_groups * KS
   int dq_group;             // NF4 double-quant run length
 };
 
@@ -134,6 +134,84 @@ __device__ __forceinline__ void mma_words(const uint32_t (&words)[4], const Int4
   }
 }
 
+// Warp index owning work unit u when warp w owns [floor(w U / W), floor((w+1) U / W)).
+__device__ __forceinline__ int owner_of(long long u, long long U, long long W) {
+  return static_cast<int>(((u + 1) * W + U - 1) / U) - 1;
+}
+
+// Hand a row group's accumulated sums on: write Y if this warp covered the
+// whole channel range, else store them in the warp's slot; the last
+// contributor of the row group sums the slots in order and writes Y.
+template <class C>
+__device__ __forceinline__ void flush_row_group(const GemvArgs& args, float (&acc)[2][C::NB][4],
+                                                int rgg, long long seg_start, long long seg_end,
+                                                long long U, long long W, int lane) {
+  const int g = lane >> 2, u = lane & 3;
+  const int r0 = rgg * 16 + g;
+  float tot[C::NB][4];
+#pragma unroll
+  for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      tot[nb][j] = acc[0][nb][j] + acc[1][nb][j];
+      acc[0][nb][j] = 0.0f;
+      acc[1][nb][j] = 0.0f;
+    }
+  const long long rs = static_cast<long long>(rgg) * args.KS, re = rs + args.KS;
+  bool write_y = true;
+  if (seg_start != rs || seg_end != re) {
+    const int first = owner_of(rs, U, W);
+    const int last = owner_of(re - 1, U, W);
+    const int mine = owner_of(seg_start, U, W);
+    const int contributors = last - first + 1;
+    float* slot = args.partial +
+                  ((static_cast<size_t>(rgg) * args.max_slots + (mine - first)) * 32 + lane) * 4 * C::NB;
+#pragma unroll
+    for (int nb = 0; nb < C::NB; ++nb)
+      *reinterpret_cast<float4*>(slot + nb * 4) =
+          make_float4(tot[nb][0], tot[nb][1], tot[nb][2], tot[nb][3]);
+    __threadfence();
+    __syncwarp();
+    unsigned prev = 0;
+    if (lane == 0) prev = atomicAdd(args.counter + rgg, 1u);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    write_y = prev == static_cast<unsigned>(contributors - 1);
+    if (write_y) {
+      __threadfence();
+#pragma unroll
+      for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tot[nb][j] = 0.0f;
+      const float* base =
+          args.partial + (static_cast<size_t>(rgg) * args.max_slots * 32 + lane) * 4 * C::NB;
+      for (int sp = 0; sp < contributors; ++sp) {
+#pragma unroll
+        for (int nb = 0; nb < C::NB; ++nb) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(
+              base + static_cast<size_t>(sp) * 32 * 4 * C::NB + nb * 4));
+          tot[nb][0] += v.x;
+          tot[nb][1] += v.y;
+          tot[nb][2] += v.z;
+          tot[nb][3] += v.w;
+        }
+      }
+      if (lane == 0) args.counter[rgg] = 0u;  // leave the workspace zeroed
+    }
+  }
+  if (write_y) {
+#pragma unroll
+    for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int m = nb * 8 + 2 * u + (j & 1);
+        const int nn = r0 + (j >> 1) * 8;
+        if (m < args.M && nn < args.N)
+          args.Y[static_cast<size_t>(m) * args.N + nn] =
+              __bfloat16_as_ushort(__float2bfloat16_rn(tot[nb][j]));
+      }
+  }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(const GemvArgs args) {
   __shared__ float Ts[16];
@@ -146,170 +224,126 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
 
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, u = lane & 3;
-  const int rgl = threadIdx.x >> 5;  // row group inside the tile = warp index
-  const int tiles = (args.row_groups + 7) / 8;
-  const int tasks = tiles * args.segs;
+  const long long W = static_cast<long long>(gridDim.x) * C::kWarps;
+  const long long wid = static_cast<long long>(blockIdx.x) * C::kWarps + (threadIdx.x >> 5);
+  const long long U = args.total;
+  // this warp's contiguous range of (row group, stage) units, row-group major
+  const long long ua = wid * U / W, ub = (wid + 1) * U / W;
+  if (ua >= ub) return;
+  const int KS = args.KS;
   const size_t xnb_stride = static_cast<size_t>(8) * args.K;
+  const int tokens_left = args.M - g;
+  const uint16_t* xbase = args.X + static_cast<size_t>(g) * args.K + 4 * u;
 
-  // a CTA task = (tile, segment): its 8 warps take the tile's 8 row groups
-  // over the same channel range, so their activation loads share L1
-  for (int task = blockIdx.x; task < tasks; task += gridDim.x) {
-    const int tile = task / args.segs;
-    const int seg = task - tile * args.segs;
-    const int rgg = tile * 8 + rgl;
-    if (rgg >= args.row_groups) continue;
-    const int st0 = static_cast<int>(static_cast<long long>(seg) * args.KS / args.segs);
-    const int st1 = static_cast<int>(static_cast<long long>(seg + 1) * args.KS / args.segs);
-    const uint8_t* blk0 = args.Wp + (static_cast<size_t>(tile) * args.KS + st0) * C::kStageBytes;
-    float acc[2][C::NB][4];
-#pragma unroll
-    for (int e = 0; e < 2; ++e)
-#pragma unroll
-      for (int nb = 0; nb < C::NB; ++nb)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[e][nb][j] = 0.0f;
-    // token g of each token block; tokens >= M read nothing (zero fragments)
-    const int tokens_left = args.M - g;
-    const uint16_t* xbase = args.X + static_cast<size_t>(g) * args.K + 4 * u;
-    const int r0 = rgg * 16 + g;
+  // unit -> stage block of lane's codes
+  auto blk_of = [&](long long unit) -> const uint8_t* {
+    const int rgg = static_cast<int>(unit / KS);
+    const int st = static_cast<int>(unit - static_cast<long long>(rgg) * KS);
+    return args.Wp + (static_cast<size_t>(rgg >> 3) * KS + st) * C::kStageBytes;
+  };
 
-    // ring of kDepth stages in flight
-    StageRegs<C> ring[C::kDepth];
+  StageRegs<C> ring[C::kDepth];
 #pragma unroll
-    for (int i = 0; i < C::kDepth; ++i)
-      if (st0 + i < st1) load_stage<C>(blk0 + static_cast<size_t>(i) * C::kStageBytes, ring[i], rgl, lane);
-    for (int sb = st0; sb < st1; sb += C::kDepth) {
-#pragma unroll
-      for (int i = 0; i < C::kDepth; ++i) {
-        const int st = sb + i;
-        if (st < st1) {
-          const StageRegs<C> cur = ring[i];
-          if (st + C::kDepth < st1)
-            load_stage<C>(blk0 + static_cast<size_t>(st - st0 + C::kDepth) * C::kStageBytes,
-                          ring[i], rgl, lane);
-          const int k0 = st * kStageK;
-          const uint32_t w0[4] = {cur.c0.x, cur.c0.y, cur.c0.z, cur.c0.w};
-          const uint32_t w1[4] = {cur.c1.x, cur.c1.y, cur.c1.z, cur.c1.w};
-          const bool second = k0 + 64 < args.K;
-          if constexpr (C::FMT == kFmtInt4) {
-            if constexpr (C::G == 128) {
-              const Int4Dq e0 = int4_dq_params(cur.sp[0] & 0xFFFFu, cur.zp[0] & 0xFu);
-              const Int4Dq e1 = int4_dq_params(cur.sp[0] >> 16, (cur.zp[0] >> 4) & 0xFu);
-              mma_words<C, 0, 4>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
-              if (second)
-                mma_words<C, 0, 4>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
-                                   tokens_left, acc);
-            } else if constexpr (C::G == 64) {
-              {
-                const Int4Dq e0 = int4_dq_params(cur.sp[0] & 0xFFFFu, cur.zp[0] & 0xFu);
-                const Int4Dq e1 = int4_dq_params(cur.sp[0] >> 16, (cur.zp[0] >> 4) & 0xFu);
-                mma_words<C, 0, 4>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
-              }
-              if (second) {
-                const Int4Dq e0 = int4_dq_params(cur.sp[1] & 0xFFFFu, cur.zp[1] & 0xFu);
-                const Int4Dq e1 = int4_dq_params(cur.sp[1] >> 16, (cur.zp[1] >> 4) & 0xFu);
-                mma_words<C, 0, 4>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
-                                   tokens_left, acc);
-              }
-            } else {
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                if (q >= 2 && !second) break;
-                const Int4Dq e0 = int4_dq_params(cur.sp[q] & 0xFFFFu, cur.zp[q] & 0xFu);
-                const Int4Dq e1 = int4_dq_params(cur.sp[q] >> 16, (cur.zp[q] >> 4) & 0xFu);
-                if (q == 0)
-                  mma_words<C, 0, 2>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
-                else if (q == 1)
-                  mma_words<C, 2, 2>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
-                else if (q == 2)
-                  mma_words<C, 0, 2>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
-                                     tokens_left, acc);
-                else
-                  mma_words<C, 2, 2>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
-                                     tokens_left, acc);
-              }
-            }
-          } else {
-            const long long kb64 = args.K / 64;
-            float a0[2] = {0.0f, 0.0f}, a1[2] = {0.0f, 0.0f};
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int blk = st * 2 + h;
-              if (blk < kb64) {
-                const uint32_t pair = h == 0 ? cur.sp[0] : cur.zp[0];
-                if (r0 < args.N)
-                  a0[h] = __fmul_rn(static_cast<float>(pair & 0xFFu),
-                                    __ldg(args.s2 + (static_cast<long long>(r0) * kb64 + blk) / args.dq_group));
-                if (r0 + 8 < args.N)
-                  a1[h] = __fmul_rn(static_cast<float>(pair >> 8),
-                                    __ldg(args.s2 + (static_cast<long long>(r0 + 8) * kb64 + blk) / args.dq_group));
-              }
-            }
-            const Int4Dq none{};
-            mma_words<C, 0, 4>(w0, none, none, a0[0], a1[0], Ts, xbase + k0, xnb_stride,
-                               tokens_left, acc);
-            if (second)
-              mma_words<C, 0, 4>(w1, none, none, a0[1], a1[1], Ts, xbase + k0 + 64, xnb_stride,
-                                 tokens_left, acc);
-          }
-        }
-      }
+  for (int i = 0; i < C::kDepth; ++i)
+    if (ua + i < ub) {
+      const long long un = ua + i;
+      load_stage<C>(blk_of(un), ring[i], static_cast<int>(un / KS) & 7, lane);
     }
 
-    // tot[nb] = D[rows r0, r0 + 8][tokens 8 nb + 2u, 8 nb + 2u + 1]
-    float tot[C::NB][4];
+  float acc[2][C::NB][4];
+#pragma unroll
+  for (int e = 0; e < 2; ++e)
 #pragma unroll
     for (int nb = 0; nb < C::NB; ++nb)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) tot[nb][j] = acc[0][nb][j] + acc[1][nb][j];
-    bool write_y = true;
-    if (args.segs > 1) {
-      float* slot = args.partial +
-                    ((static_cast<size_t>(rgg) * args.segs + seg) * 32 + lane) * 4 * C::NB;
+      for (int j = 0; j < 4; ++j) acc[e][nb][j] = 0.0f;
+
+  int rgg = static_cast<int>(ua / KS);
+  long long seg_start = ua;
+  for (long long base = ua; base < ub; base += C::kDepth) {
 #pragma unroll
-      for (int nb = 0; nb < C::NB; ++nb)
-        *reinterpret_cast<float4*>(slot + nb * 4) =
-            make_float4(tot[nb][0], tot[nb][1], tot[nb][2], tot[nb][3]);
-      __threadfence();
-      __syncwarp();
-      unsigned prev = 0;
-      if (lane == 0) prev = atomicAdd(args.counter + rgg, 1u);
-      prev = __shfl_sync(0xffffffffu, prev, 0);
-      write_y = prev == static_cast<unsigned>(args.segs - 1);
-      if (write_y) {
-        // last segment of this row group: sum all slots in segment order
-        __threadfence();
+    for (int i = 0; i < C::kDepth; ++i) {
+      const long long un = base + i;
+      if (un < ub) {
+        const StageRegs<C> cur = ring[i];
+        if (un + C::kDepth < ub) {
+          const long long nx = un + C::kDepth;
+          load_stage<C>(blk_of(nx), ring[i], static_cast<int>(nx / KS) & 7, lane);
+        }
+        const int st = static_cast<int>(un - static_cast<long long>(rgg) * KS);
+        const int r0 = rgg * 16 + g;
+        const int k0 = st * kStageK;
+        const uint32_t w0[4] = {cur.c0.x, cur.c0.y, cur.c0.z, cur.c0.w};
+        const uint32_t w1[4] = {cur.c1.x, cur.c1.y, cur.c1.z, cur.c1.w};
+        const bool second = k0 + 64 < args.K;
+        if constexpr (C::FMT == kFmtInt4) {
+          if constexpr (C::G == 128) {
+            const Int4Dq e0 = int4_dq_params(cur.sp[0] & 0xFFFFu, cur.zp[0] & 0xFu);
+            const Int4Dq e1 = int4_dq_params(cur.sp[0] >> 16, (cur.zp[0] >> 4) & 0xFu);
+            mma_words<C, 0, 4>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
+            if (second)
+              mma_words<C, 0, 4>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
+                                 tokens_left, acc);
+          } else if constexpr (C::G == 64) {
+            {
+              const Int4Dq e0 = int4_dq_params(cur.sp[0] & 0xFFFFu, cur.zp[0] & 0xFu);
+              const Int4Dq e1 = int4_dq_params(cur.sp[0] >> 16, (cur.zp[0] >> 4) & 0xFu);
+              mma_words<C, 0, 4>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
+            }
+            if (second) {
+              const Int4Dq e0 = int4_dq_params(cur.sp[1] & 0xFFFFu, cur.zp[1] & 0xFu);
+              const Int4Dq e1 = int4_dq_params(cur.sp[1] >> 16, (cur.zp[1] >> 4) & 0xFu);
+              mma_words<C, 0, 4>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
+                                 tokens_left, acc);
+            }
+          } else {
 #pragma unroll
-        for (int nb = 0; nb < C::NB; ++nb)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) tot[nb][j] = 0.0f;
-        const float* base =
-            args.partial + (static_cast<size_t>(rgg) * args.segs * 32 + lane) * 4 * C::NB;
-        for (int sp = 0; sp < args.segs; ++sp) {
-#pragma unroll
-          for (int nb = 0; nb < C::NB; ++nb) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                base + static_cast<size_t>(sp) * 32 * 4 * C::NB + nb * 4));
-            tot[nb][0] += v.x;
-            tot[nb][1] += v.y;
-            tot[nb][2] += v.z;
-            tot[nb][3] += v.w;
+            for (int q = 0; q < 4; ++q) {
+              if (q >= 2 && !second) break;
+              const Int4Dq e0 = int4_dq_params(cur.sp[q] & 0xFFFFu, cur.zp[q] & 0xFu);
+              const Int4Dq e1 = int4_dq_params(cur.sp[q] >> 16, (cur.zp[q] >> 4) & 0xFu);
+              if (q == 0)
+                mma_words<C, 0, 2>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
+              else if (q == 1)
+                mma_words<C, 2, 2>(w0, e0, e1, 0.f, 0.f, Ts, xbase + k0, xnb_stride, tokens_left, acc);
+              else if (q == 2)
+                mma_words<C, 0, 2>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
+                                   tokens_left, acc);
+              else
+                mma_words<C, 2, 2>(w1, e0, e1, 0.f, 0.f, Ts, xbase + k0 + 64, xnb_stride,
+                                   tokens_left, acc);
+            }
           }
+        } else {
+          const long long kb64 = args.K / 64;
+          float a0[2] = {0.0f, 0.0f}, a1[2] = {0.0f, 0.0f};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int blk = st * 2 + h;
+            if (blk < kb64) {
+              const uint32_t pair = h == 0 ? cur.sp[0] : cur.zp[0];
+              if (r0 < args.N)
+                a0[h] = __fmul_rn(static_cast<float>(pair & 0xFFu),
+                                  __ldg(args.s2 + (static_cast<long long>(r0) * kb64 + blk) / args.dq_group));
+              if (r0 + 8 < args.N)
+                a1[h] = __fmul_rn(static_cast<float>(pair >> 8),
+                                  __ldg(args.s2 + (static_cast<long long>(r0 + 8) * kb64 + blk) / args.dq_group));
+            }
+          }
+          const Int4Dq none{};
+          mma_words<C, 0, 4>(w0, none, none, a0[0], a1[0], Ts, xbase + k0, xnb_stride,
+                             tokens_left, acc);
+          if (second)
+            mma_words<C, 0, 4>(w1, none, none, a0[1], a1[1], Ts, xbase + k0 + 64, xnb_stride,
+                               tokens_left, acc);
         }
-        if (lane == 0) args.counter[rgg] = 0u;  // leave the workspace zeroed
+        // end of this row group's part of the range: flush
+        if (st == KS - 1 || un + 1 == ub) {
+          flush_row_group<C>(args, acc, rgg, seg_start, un + 1, U, W, lane);
+          ++rgg;
+          seg_start = un + 1;
+        }
       }
-    }
-    if (write_y) {
-#pragma unroll
-      for (int nb = 0; nb < C::NB; ++nb)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int m = nb * 8 + 2 * u + (j & 1);
-          const int nn = r0 + (j >> 1) * 8;
-          if (m < args.M && nn < args.N)
-            args.Y[static_cast<size_t>(m) * args.N + nn] =
-                __bfloat16_as_ushort(__float2bfloat16_rn(tot[nb][j]));
-        }
     }
   }
 }
