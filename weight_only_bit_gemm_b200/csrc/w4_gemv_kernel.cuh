@@ -235,19 +235,27 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
   const int tokens_left = args.M - g;
   const uint16_t* xbase = args.X + static_cast<size_t>(g) * args.K + 4 * u;
 
-  // unit -> stage block of lane's codes
-  auto blk_of = [&](long long unit) -> const uint8_t* {
-    const int rgg = static_cast<int>(unit / KS);
-    const int st = static_cast<int>(unit - static_cast<long long>(rgg) * KS);
-    return args.Wp + (static_cast<size_t>(rgg >> 3) * KS + st) * C::kStageBytes;
+  // prefetch cursor: (row group, stage) of the next stage to load and the
+  // address of its stage block, advanced without divisions
+  int pf_rgg = static_cast<int>(ua / KS);
+  int pf_st = static_cast<int>(ua - static_cast<long long>(pf_rgg) * KS);
+  const uint8_t* pf_ptr = args.Wp + (static_cast<size_t>(pf_rgg >> 3) * KS + pf_st) * C::kStageBytes;
+  auto advance = [&]() {
+    if (++pf_st == KS) {
+      pf_st = 0;
+      ++pf_rgg;
+      pf_ptr = args.Wp + static_cast<size_t>(pf_rgg >> 3) * KS * C::kStageBytes;
+    } else {
+      pf_ptr += C::kStageBytes;
+    }
   };
 
   StageRegs<C> ring[C::kDepth];
 #pragma unroll
   for (int i = 0; i < C::kDepth; ++i)
     if (ua + i < ub) {
-      const long long un = ua + i;
-      load_stage<C>(blk_of(un), ring[i], static_cast<int>(un / KS) & 7, lane);
+      load_stage<C>(pf_ptr, ring[i], pf_rgg & 7, lane);
+      advance();
     }
 
   float acc[2][C::NB][4];
@@ -259,6 +267,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
       for (int j = 0; j < 4; ++j) acc[e][nb][j] = 0.0f;
 
   int rgg = static_cast<int>(ua / KS);
+  int st = static_cast<int>(ua - static_cast<long long>(rgg) * KS);
   long long seg_start = ua;
   for (long long base = ua; base < ub; base += C::kDepth) {
 #pragma unroll
@@ -267,10 +276,9 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
       if (un < ub) {
         const StageRegs<C> cur = ring[i];
         if (un + C::kDepth < ub) {
-          const long long nx = un + C::kDepth;
-          load_stage<C>(blk_of(nx), ring[i], static_cast<int>(nx / KS) & 7, lane);
+          load_stage<C>(pf_ptr, ring[i], pf_rgg & 7, lane);
+          advance();
         }
-        const int st = static_cast<int>(un - static_cast<long long>(rgg) * KS);
         const int r0 = rgg * 16 + g;
         const int k0 = st * kStageK;
         const uint32_t w0[4] = {cur.c0.x, cur.c0.y, cur.c0.z, cur.c0.w};
@@ -341,7 +349,10 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
         if (st == KS - 1 || un + 1 == ub) {
           flush_row_group<C>(args, acc, rgg, seg_start, un + 1, U, W, lane);
           ++rgg;
+          st = 0;
           seg_start = un + 1;
+        } else {
+          ++st;
         }
       }
     }
