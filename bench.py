@@ -50,6 +50,33 @@ def nf4_bytes(M, N, K):
     return N * K / 2 + nb + 4 * -(-nb // 256) + 2 * M * K + 2 * M * N
 
 
+# DRAM bytes of one decode-kernel launch from an ncu capture, valid only for
+# the kernel source it was taken on (sha256 of w4_gemv_kernel.cuh).
+TRAFFIC_CAPTURE = {
+    "kernel_sha256": None,
+    "shape": {"M": 1, "N": 12288, "K": 4096, "G": 128},
+    "dram_bytes": None,
+    "profile": "profiles/w4_gemv_kernel_int4_K4096_N12288_M1.md",
+}
+
+
+def gemv_kernel_sha256():
+    import hashlib
+    path = os.path.join(ROOT, "weight_only_bit_gemm_b200", "csrc", "w4_gemv_kernel.cuh")
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()
+
+
+def traffic_per_launch(step):
+    """Measured DRAM bytes scaled to the step's mean launch (traffic tracks the
+    algorithmic bytes, so scale by their ratio); None if the kernel changed."""
+    cap = TRAFFIC_CAPTURE
+    if cap["dram_bytes"] is None or cap["kernel_sha256"] != gemv_kernel_sha256():
+        return None
+    sh = cap["shape"]
+    ratio = cap["dram_bytes"] / int4_bytes(sh["M"], sh["N"], sh["K"], sh["G"])
+    return ratio * step.step_bytes / len(step.calls)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -584,8 +611,10 @@ def main():
     if w4.device_status() != w4.W4_OK:
         raise RuntimeError("device error during the benchmark")
 
-    kern_ms = sum(per_call)
-    achieved = step.step_bytes / (kern_ms * 1e-3) / 1e9
+    # every launch in the timed step is the decode kernel: its mean duration is
+    # the step time over the launches in it
+    launch_ms = (ms / args.steps) / len(step.calls)
+    achieved = (step.step_bytes / len(step.calls)) / (launch_ms * 1e-3) / 1e9
     per_shape = {}
     for c, t in zip(step.calls, per_call):
         per_shape[f"K{c['K']}_N{c['N']}_M{c['M']}"] = {
@@ -615,9 +644,11 @@ def main():
                        "timing": "CUDA graph of one step, CUDA events on the launching stream"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "traffic": None, "peak_source": peaks["source"],
-                         "kernel": "w4_tc_gemm_kernel (per-call device time)",
-                         "per_call": per_shape},
+                         "traffic": traffic_per_launch(step), "peak_source": peaks["source"],
+                         "kernel": "w4_gemv_kernel",
+                         "launch_us": launch_ms * 1e3,
+                         "algorithmic_bytes_per_launch": step.step_bytes / len(step.calls),
+                         "per_call_isolated": per_shape},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
