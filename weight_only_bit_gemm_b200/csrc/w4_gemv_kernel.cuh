@@ -170,14 +170,14 @@ __device__ __forceinline__ void flush_row_group(const GemvArgs& args, float (&ac
     for (int nb = 0; nb < C::NB; ++nb)
       *reinterpret_cast<float4*>(slot + nb * 4) =
           make_float4(tot[nb][0], tot[nb][1], tot[nb][2], tot[nb][3]);
-    __threadfence();
+    // publish the slot with an acquire-release counter update (no full fence,
+    // which would also wait for this warp's prefetched loads)
     __syncwarp();
     unsigned prev = 0;
-    if (lane == 0) prev = atomicAdd(args.counter + rgg, 1u);
+    if (lane == 0) prev = atom_add_acq_rel_gpu(args.counter + rgg, 1u);
     prev = __shfl_sync(0xffffffffu, prev, 0);
     write_y = prev == static_cast<unsigned>(contributors - 1);
     if (write_y) {
-      __threadfence();
 #pragma unroll
       for (int nb = 0; nb < C::NB; ++nb)
 #pragma unroll
