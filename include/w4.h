@@ -54,7 +54,9 @@ enum {
   W4_ERR_UNSUPPORTED = 2, /* valid but not supported by this build           */
   W4_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed            */
   W4_ERR_TIMEOUT = 4,     /* a device pipeline wait gave up (device status)  */
-  W4_ERR_DEVICE_INPUT = 5 /* the device found bad input data (device status) */
+  W4_ERR_DEVICE_INPUT = 5, /* the device found bad input data (device status) */
+  W4_ERR_SCRATCH_LIMIT = 6 /* w4a16_gemm_static_scratch: the call needs more
+                              workspace than W4_STATIC_SCRATCH_BYTES           */
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -159,6 +161,32 @@ size_t w4_workspace_bytes(int M, int N, int K, int G, int act_order);
 w4_status w4a16_gemm(const uint16_t* X, const uint8_t* Wp, int M, int N, int K, int G,
                      int act_order, uint16_t* Y, void* workspace, size_t workspace_bytes,
                      w4_stream stream);
+
+/* ------------------------------------------------------------------------
+ * w4a16_gemm without a caller workspace.  The pages describe no such call; it
+ * computes exactly what w4a16_gemm computes, for callers that cannot allocate
+ * device memory when they call: a runtime that plans all of HBM at start-up,
+ * a caller that cannot pay cudaFree's device-wide synchronisation, or plain C
+ * code without a device allocator.  It allocates nothing (no cudaMalloc /
+ * cudaFree, no allocating library routine): its workspace is a file-scope
+ * device array of W4_STATIC_SCRATCH_BYTES (16 MiB), one copy per device.
+ *   Arguments, layouts and results as for w4a16_gemm (minus the workspace).
+ *   Limit: returns W4_ERR_SCRATCH_LIMIT, launching nothing, when
+ *          w4_workspace_bytes(M, N, K, G, act_order) > W4_STATIC_SCRATCH_BYTES
+ *          (every decode shape M <= 32 up to N * K = 28672 * 8192 fits; large
+ *          prefill shapes that split K do not: use w4a16_gemm there).
+ *   First call on a device: looks up that device's copy of the array (which
+ *          may load the module on the device) with the device current, and
+ *          returns W4_ERR_CUDA if that fails.  Make the first call on each
+ *          device before any stream capture.
+ *   Each call clears (cudaMemsetAsync on `stream`) the arrival counters it
+ *          uses before its kernel runs.
+ *   One array per device: calls whose executions can overlap on the same
+ *          device (different streams, or different host threads) race on it
+ *          and give wrong results.  Order them on one stream.              */
+#define W4_STATIC_SCRATCH_BYTES 16777216u /* 16 MiB */
+w4_status w4a16_gemm_static_scratch(const uint16_t* X, const uint8_t* Wp, int M, int N, int K,
+                                    int G, int act_order, uint16_t* Y, w4_stream stream);
 
 /* ------------------------------------------------------------------------
  * NF4 ([Survey] §6.1: 16 levels at normal-distribution quantiles, denser near

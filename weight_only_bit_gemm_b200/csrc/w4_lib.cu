@@ -44,6 +44,8 @@ const char* w4_status_string(w4_status s) {
     case W4_ERR_CUDA: return "CUDA error";
     case W4_ERR_TIMEOUT: return "device pipeline wait timed out";
     case W4_ERR_DEVICE_INPUT: return "device found invalid input data";
+    case W4_ERR_SCRATCH_LIMIT:
+      return "workspace needed exceeds the static scratch (W4_STATIC_SCRATCH_BYTES)";
     default: return "unknown status";
   }
 }

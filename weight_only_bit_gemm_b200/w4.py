@@ -39,6 +39,7 @@ _SIGS = {
     "w4_unprepack": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p, _p]),
     "w4_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "w4a16_gemm": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "w4a16_gemm_static_scratch": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p]),
     "nf4_quantize": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p]),
     "nf4_dequant": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p]),
     "nf4_levels": (None, [_p]),
@@ -54,6 +55,8 @@ for _name, (_res, _args) in _SIGS.items():
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA, W4_ERR_TIMEOUT, \
     W4_ERR_DEVICE_INPUT = range(6)
+W4_ERR_SCRATCH_LIMIT = 6
+W4_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class W4Error(RuntimeError):
@@ -184,6 +187,19 @@ def w4a16_gemm(X, Wp, N, K, G, act_order=False, out=None, workspace=None):
     ws = _ws_view(workspace if workspace is not None else _WS.get(need, X.device))
     _check(lib.w4a16_gemm(_ptr(X), _ptr(Wp), M, N, K, G, int(bool(act_order)), _ptr(out),
                           _ptr(ws), ws.numel(), _stream()), "w4a16_gemm")
+    return out
+
+
+def w4a16_gemm_static_scratch(X, Wp, N, K, G, act_order=False, out=None):
+    """w4a16_gemm with the library's static device scratch as workspace (the
+    call allocates nothing); shapes needing more than W4_STATIC_SCRATCH_BYTES
+    raise W4Error with status W4_ERR_SCRATCH_LIMIT."""
+    _cuda(X, torch.bfloat16, "X")
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _check(lib.w4a16_gemm_static_scratch(_ptr(X), _ptr(Wp), M, N, K, G, int(bool(act_order)),
+                                         _ptr(out), _stream()), "w4a16_gemm_static_scratch")
     return out
 
 
