@@ -89,8 +89,9 @@ w4_status w4_device_status(w4_stream stream);
  *   Wq       out  uint8 [N, K/2]
  *   scales   out  fp16 bits [N, K/G]
  *   zeros    out  uint8 [N, K/G]
- * Bit-exact with the CPU definition above.  |w| must be finite and below
- * 491520 (so that the fp16 scale is finite). */
+ * Bit-exact with the CPU definition above.  w must be finite and every group
+ * must have (mx - mn) / 15 < 65520, so that the fp16 scale is finite (true
+ * whenever |w| < 491000). */
 w4_status w4_quantize_rtn(const float* W, int N, int K, int G, const int32_t* g_idx,
                           uint8_t* Wq, uint16_t* scales, uint8_t* zeros,
                           w4_stream stream);
@@ -114,13 +115,16 @@ double w4_weight_bytes(int N, int K, int G);
  * B200-specific part).  Wp holds, for each tile of 128 output rows and each
  * stage of 128 input channels, one contiguous block that a single bulk copy
  * brings into shared memory:
- *   codes   8192 B: [chunk c < 4][row r < 128][16 B], chunk c covering the 32
- *           channels 32c..32c+31 of the stage; in each 32-bit word of 8
- *           channels k0..k0+7, bits 4j..4j+3 hold code k0+2j and bits
- *           16+4j..19+4j hold code k0+2j+1 (j < 4)
- *   scales  128 * (128/G) fp16, [row][group within the stage]
- *   zeros   128 * (128/G) 4-bit values, [row][group], even index in the low
- *           nibble
+ *   codes   8192 B in warp-MMA fragment order: for row group rg < 8 (16
+ *           rows), channel block kb < 8 (16 channels) and lane t < 32
+ *           (g = t / 4, u = t % 4) the 32-bit word at byte offset
+ *           (((rg * 2 + kb / 4) * 32 + t) * 4 + kb % 4) * 4 holds rows
+ *           r0 = 16 rg + g, r1 = r0 + 8 x channels c = 16 kb + 4 u .. c + 3
+ *           as four pairs j: bits 4j..4j+3 and 16+4j..19+4j hold
+ *           (r0, c, c+1), (r0, c+2, c+3), (r1, c, c+1), (r1, c+2, c+3)
+ *   scales  fp16 [rg][group within the stage][g][2] (rows r0, r1)
+ *   zeros   uint8 [rg][group][g] = z(r0) | z(r1) << 4
+ *           (stage block: 8512 / 8832 / 9472 B for G = 128 / 64 / 32)
  * Rows >= N and channels >= K are padding (code 0, scale 0, zero 0).  With
  * act_order, the channels are taken in the order that makes each group
  * contiguous (a stable sort of k by g_idx[k]) and that permutation, int32
@@ -213,8 +217,9 @@ w4_status nf4_dequant(const uint8_t* Wq, const uint8_t* absmax_q, const float* s
 void nf4_levels(float out[16]);
 
 /* NF4 pre-shuffled layout: as for INT4 (same codes block per 128 rows x 128
- * channels) followed by the absmax codes [row][2] (two 64-blocks per stage).
- * s2 stays in its canonical array. */
+ * channels) followed by the absmax codes uint8 [rg][64-block in stage (2)]
+ * [g][2] (rows r0, r1); stage block 8448 B.  s2 stays in its canonical
+ * array. */
 size_t nf4_prepacked_bytes(int N, int K);
 w4_status nf4_prepack(const uint8_t* Wq, const uint8_t* absmax_q, int N, int K,
                       uint8_t* Wp, w4_stream stream);
