@@ -61,11 +61,27 @@ struct GemmCfg {
   static_assert(kColsNeeded <= 512, "tensor memory");
 };
 
-__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) {
-  return *reinterpret_cast<uint32_t*>(&v);
+// bf16x2 arithmetic on 32-bit registers (low half = first element).
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
-__device__ __forceinline__ __nv_bfloat162 bits_bf2_h(uint32_t v) {
-  return *reinterpret_cast<__nv_bfloat162*>(&v);
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// (lo, hi) fp32 -> bf16x2, round to nearest even
+__device__ __forceinline__ uint32_t bf2_from_f32(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
 }
 
 // Exact INT4 dequant of one 32-bit word (8 codes, see w4_prepack.cuh):
@@ -75,17 +91,18 @@ __device__ __forceinline__ __nv_bfloat162 bits_bf2_h(uint32_t v) {
 // code into the mantissa of 128.0; d = (128+q) - (128+z) is exact; d * s_lo is
 // exact (at most 7 significant bits); and one fused multiply-add
 // d * s_hi + d * s_lo rounds the exact product d * s once to bf16.
+// The three constants are bf16x2 bit patterns with equal halves.
 struct Int4Dq {
-  __nv_bfloat162 zm, shi, slo;
+  uint32_t zm, shi, slo;
 };
 
 __device__ __forceinline__ Int4Dq int4_dq_params(uint32_t s16, uint32_t z) {
   const float sf = __half2float(__ushort_as_half(static_cast<unsigned short>(s16)));
   Int4Dq p;
-  p.shi = __floats2bfloat162_rn(sf, sf);
-  const float lo = sf - __low2float(p.shi);
-  p.slo = __floats2bfloat162_rn(lo, lo);
-  p.zm = bits_bf2_h((z * 0x00010001u) | 0x43004300u);
+  p.shi = bf2_from_f32(sf, sf);
+  const float lo = sf - __uint_as_float(p.shi << 16);  // exact
+  p.slo = bf2_from_f32(lo, lo);
+  p.zm = (z * 0x00010001u) | 0x43004300u;
   return p;
 }
 
@@ -97,9 +114,8 @@ __device__ __forceinline__ void int4_dq_word(uint32_t w, const Int4Dq& p0, const
   for (int j = 0; j < 4; ++j) {
     const Int4Dq& p = j < 2 ? p0 : p1;
     const uint32_t t = ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
-    const __nv_bfloat162 d = __hsub2(bits_bf2_h(t), p.zm);
-    const __nv_bfloat162 l = __hmul2(d, p.slo);
-    out[j] = bf2_bits(__hfma2(d, p.shi, l));
+    const uint32_t d = bf2_sub(t, p.zm);
+    out[j] = bf2_fma(d, p.shi, bf2_mul(d, p.slo));
   }
 }
 
@@ -112,7 +128,7 @@ __device__ __forceinline__ void nf4_dq_word(uint32_t w, float a0, float a1,
     const float a = j < 2 ? a0 : a1;
     const float f0 = __fmul_rn(T[(w >> (4 * j)) & 0xFu], a);
     const float f1 = __fmul_rn(T[(w >> (16 + 4 * j)) & 0xFu], a);
-    out[j] = bf2_bits(__floats2bfloat162_rn(f0, f1));
+    out[j] = bf2_from_f32(f0, f1);
   }
 }
 
@@ -126,7 +142,7 @@ struct GemmArgs {
   int KS;                 // stages per tile row = ceil(K / 128)
   int tiles_n;
   int splits;
-  int dq_group;           // NF4 double-quant run length
+  FastDiv64 by_dq;        // NF4: 64-block index -> s2 index (double-quant run)
 };
 
 }  // namespace w4

@@ -171,10 +171,10 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
             const long long kb64 = args.K / 64;
             if (r0 < args.N)
               a0 = __fmul_rn(static_cast<float>(cp & 0xFFu),
-                             __ldg(args.s2 + (static_cast<long long>(r0) * kb64 + blk_in_row) / args.dq_group));
+                             __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0) * kb64 + blk_in_row, args.by_dq)));
             if (r0 + 8 < args.N)
               a1 = __fmul_rn(static_cast<float>(cp >> 8),
-                             __ldg(args.s2 + (static_cast<long long>(r0 + 8) * kb64 + blk_in_row) / args.dq_group));
+                             __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0 + 8) * kb64 + blk_in_row, args.by_dq)));
           }
 #pragma unroll
           for (int w = 0; w < 4; ++w) nf4_dq_word(words[w], a0, a1, Ts, &out[rgl][4 * w]);

@@ -219,6 +219,40 @@ __device__ __forceinline__ void grid_dep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Division by a divisor fixed for the launch, by multiplication (Granlund and
+// Montgomery, "Division by invariant integers using multiplication", 1994):
+// with l = ceil(log2 d) and m = floor(2^B (2^l - d) / d) + 1,
+//   n / d = (mulhi(n, m) + n) >> l   for every n < 2^(B-1)  (B = 32 or 64).
+struct FastDiv32 {
+  uint32_t m, l;
+};
+struct FastDiv64 {
+  unsigned long long m;
+  uint32_t l;
+};
+
+inline FastDiv32 make_fast_div32(uint32_t d) {
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  const unsigned long long m = (((1ull << 32) * ((1ull << l) - d)) / d) + 1;
+  return FastDiv32{static_cast<uint32_t>(m), l};
+}
+inline FastDiv64 make_fast_div64(unsigned long long d) {
+  uint32_t l = 0;
+  while (l < 63 && (1ull << l) < d) ++l;
+  const unsigned __int128 m =
+      ((static_cast<unsigned __int128>(1) << 64) * ((static_cast<unsigned __int128>(1) << l) - d)) /
+          d + 1;
+  return FastDiv64{static_cast<unsigned long long>(m), l};
+}
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, FastDiv32 f) {
+  return (__umulhi(n, f.m) + n) >> f.l;
+}
+__device__ __forceinline__ unsigned long long fast_div(unsigned long long n, FastDiv64 f) {
+  return (__umul64hi(n, f.m) + n) >> f.l;
+}
+
 // Atomic add with acquire-release semantics at GPU scope: publishes this
 // thread's earlier writes (and, through a preceding warp barrier, those of its
 // warp) and makes later reads see what the previous releasers published.
