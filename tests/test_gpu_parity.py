@@ -187,6 +187,12 @@ GEMM_CASES = [
     (1, 1024, 5120, 32, True),
     (16, 512, 13824, 32, True),
     (256, 256, 2048, 32, True),
+    # decode work-split edge cases
+    (1, 16, 64, 64, False),          # one unit: a single warp does everything
+    (2, 1, 128, 128, False),         # one output row
+    (8, 77, 320, 32, False),         # last stage has no second half, ragged N
+    (32, 1000, 4096, 128, False),    # four token blocks, ragged N
+    (5, 4096, 4160, 64, False),      # K = 32.5 stages: last stage half, G = 64
 ]
 
 
@@ -227,7 +233,7 @@ def test_nf4_gemm_unit_vectors_exact(w4):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 512, 4096), (8, 384, 1024), (32, 200, 1536),
-                                   (300, 256, 512)])
+                                   (300, 256, 512), (1, 40, 64), (3, 4096, 14336)])
 def test_nf4_gemm_tolerance(w4, M, N, K):
     W = S.draw_w(N, K, 0.02, seed=M, tag=3)
     Wq_r, c_r, s2_r = O.nf4_quantize(W)

@@ -107,16 +107,34 @@ __device__ __forceinline__ Int4Dq int4_dq_params(uint32_t s16, uint32_t z) {
 }
 
 // Pairs 0 and 1 of the word belong to row r0 (params p0), pairs 2 and 3 to
-// row r1 (params p1).
+// row r1 (params p1).  One asm block, so that each pair costs exactly one
+// LOP3 (plus one shift for pairs 1..3) and three bf16x2 instructions.
 __device__ __forceinline__ void int4_dq_word(uint32_t w, const Int4Dq& p0, const Int4Dq& p1,
                                              uint32_t* out) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const Int4Dq& p = j < 2 ? p0 : p1;
-    const uint32_t t = ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
-    const uint32_t d = bf2_sub(t, p.zm);
-    out[j] = bf2_fma(d, p.shi, bf2_mul(d, p.slo));
-  }
+  const uint32_t mask = 0x000F000Fu, magic = 0x43004300u;
+  asm("{\n\t.reg .b32 t0, t1, t2, t3, d0, d1, d2, d3, l0, l1, l2, l3;\n\t"
+      "lop3.b32 t0, %4, %5, %6, 0xEA;\n\t"
+      "shr.b32 t1, %4, 4;\n\t"
+      "lop3.b32 t1, t1, %5, %6, 0xEA;\n\t"
+      "shr.b32 t2, %4, 8;\n\t"
+      "lop3.b32 t2, t2, %5, %6, 0xEA;\n\t"
+      "shr.b32 t3, %4, 12;\n\t"
+      "lop3.b32 t3, t3, %5, %6, 0xEA;\n\t"
+      "sub.rn.bf16x2 d0, t0, %7;\n\t"
+      "sub.rn.bf16x2 d1, t1, %7;\n\t"
+      "sub.rn.bf16x2 d2, t2, %10;\n\t"
+      "sub.rn.bf16x2 d3, t3, %10;\n\t"
+      "mul.rn.bf16x2 l0, d0, %9;\n\t"
+      "mul.rn.bf16x2 l1, d1, %9;\n\t"
+      "mul.rn.bf16x2 l2, d2, %12;\n\t"
+      "mul.rn.bf16x2 l3, d3, %12;\n\t"
+      "fma.rn.bf16x2 %0, d0, %8, l0;\n\t"
+      "fma.rn.bf16x2 %1, d1, %8, l1;\n\t"
+      "fma.rn.bf16x2 %2, d2, %11, l2;\n\t"
+      "fma.rn.bf16x2 %3, d3, %11, l3;\n\t}"
+      : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
+      : "r"(w), "r"(mask), "r"(magic), "r"(p0.zm), "r"(p0.shi), "r"(p0.slo), "r"(p1.zm),
+        "r"(p1.shi), "r"(p1.slo));
 }
 
 // NF4 dequant of one word: w_hat = bf16_rne(fp32(T[q] * a')), T in shared
