@@ -148,11 +148,16 @@ w4_status w4_unprepack(const uint8_t* Wp, int N, int K, int G, int act_order,
 
 /* ------------------------------------------------------------------------
  * W4A16 linear: Y = X . w_hat^T with w_hat as in w4_dequant, bf16 products,
- * fp32 accumulation, bf16 (round to nearest even) output.  One kernel path:
- * tcgen05 tensor-core MMAs with the dequantized weight tile in tensor memory
- * (the swapped product Y^T = W_hat . X^T), M split into tiles of 16..256
- * tokens; the decode shapes (M <= 16) stream the packed weights once
- * ([Survey] §4.3: AWQ "GEMV" for single requests, "GEMM" for batches).
+ * fp32 accumulation, bf16 (round to nearest even) output.  Two kernels,
+ * chosen by M ([Survey] §4.3: AWQ ships a "GEMV" kernel for single requests
+ * and a "GEMM" kernel for batches): M <= 32 streams the packed weights once
+ * through warp-level MMAs; M > 32 runs tcgen05 tensor-core MMAs with the
+ * dequantized weight tile in tensor memory (Y^T = W_hat . X^T), M in tiles
+ * of 64..256 tokens.  The kernels use programmatic dependent launch and
+ * start reading Wp before the kernel before them on the stream has
+ * finished: Wp is constant model state and must not be written by that
+ * kernel (this library's prepack kernels make their writes visible before
+ * they exit, so prepack followed by a GEMM is fine).
  *   X          in   bf16 [M, K], 16-byte aligned, K % 64 == 0
  *   Wp         in   from w4_prepack (act_order must match)
  *   M, N, K, G M >= 1, N >= 1

@@ -1,30 +1,36 @@
 // w4_gemv_kernel.cuh -- decode path (M <= 32 tokens).
 //
 // Every warp is an independent streaming worker.  The work units are
-// (16-row group, 128-channel stage) pairs, numbered row-group major; warp w
-// owns the contiguous range of q + (w < r) units that starts at
-// w q + min(w, r) (U = q W + r units, W warps).  A lane loads each unit's
-// packed codes (two 16-byte vectors, 512 contiguous bytes per warp each) and
-// its row pair's constants straight into registers two units ahead,
-// dequantizes into the A fragments of warp-level m16n8k16 bf16 MMAs and
-// accumulates in fp32 registers.  No shared memory ring, no producer, no
-// barriers between warps: the only synchronisation is the deterministic
-// reduction over the warps that share a row group (partials in a fixed slot
-// per warp; the last one to arrive sums them in slot order).
+// (32-row pair of row groups, 128-channel stage) pairs, numbered row-pair
+// major; warp w owns the contiguous range of q + (w < r) units that starts at
+// w q + min(w, r) (U = q W + r units, W warps).  Each lane copies its share
+// of a unit's packed codes (four 16-byte vectors: 1 KB per row group per warp)
+// and a few lanes the row groups' scale and zero bytes into the warp's own
+// shared-memory ring with cp.async, three units ahead; the warp then reads the
+// unit back into registers, dequantizes into the A fragments of warp-level
+// m16n8k16 bf16 MMAs (one activation fragment serves both row groups) and
+// accumulates in fp32 registers.  No producer warp and no barriers between
+// warps: the only synchronisation is the deterministic reduction over the
+// warps that share a row pair (partials in a fixed slot per warp; the last
+// one to arrive sums them in slot order).
 //
 // Why not tcgen05 here: a tcgen05.mma of kind::f16 occupies the SM's tensor
 // core for ~200 cycles whatever its N (measured on B200 for N = 16..256), so a
 // 16-token tile consumes only 128 x 16 weights per 200 cycles per SM (about
-// 1.4 TB/s of 4-bit weights on 148 SMs).  Plain 16-byte loads from many
-// independent warps reach the HBM rate without a copy pipeline.
+// 1.4 TB/s of 4-bit weights on 148 SMs).
 //
 // Instruction economy matters more than anything else here: the SM issues
 // one warp instruction per cycle per sub-partition, and most of the integer
 // and bf16x2 instructions this loop needs run at half rate on B200.  So all
-// per-launch divisions are by multiplication with host-made constants, the
-// loop counters are 32-bit, the register ring rotates without copies, and
+// per-launch divisions are by multiplication with host-made constants, loop
+// counters are 32-bit, two row groups share each activation load, and
 // activations are loaded without predicates (rows past M are clamped to row
 // M - 1; the MMA columns they feed are never stored).
+//
+// The first units' weights are requested before the launch dependency on
+// the previous kernel resolves (weights are constant model state; X, Y and
+// the workspace are touched only after it), so a chain of these kernels keeps
+// HBM busy across kernel boundaries.
 //
 // Channel order: inside each 16-channel block, lane (g, u) holds channels
 // 4u..4u+3 (see w4_prepack.cuh) in the MMA's k slots {2u, 2u+1, 2u+8, 2u+9};
@@ -51,6 +57,10 @@ struct GemvArgs {
   FastDiv64 by_dq;          // NF4: 64-block index -> s2 index
 };
 
+// Row groups (16 rows each) per decode work unit: two share each activation
+// fragment; with four token blocks one, so that the accumulators fit.
+__host__ __device__ constexpr int gemv_row_groups(int NB) { return NB >= 4 ? 1 : 2; }
+
 template <int NB_, int FMT_, int G_>
 struct GemvCfg {
   static constexpr int NB = NB_;   // token blocks of 8
@@ -60,11 +70,15 @@ struct GemvCfg {
   static constexpr int kStageBytes = FMT == kFmtInt4 ? int4_stage_bytes(G) : nf4_stage_bytes();
   static constexpr int kWarps = 8;
   static constexpr int kThreads = 32 * kWarps;
-  // resident CTAs per SM (80 or 128 registers a thread): 3 where the
-  // register ring fits in 80 without spilling
-  static constexpr int kMinBlocks = NB == 1 && FMT_ == kFmtInt4 && G_ >= 64 ? 3 : 2;
+  static constexpr int kMinBlocks = 2;  // resident CTAs per SM (128 registers a thread)
   // groups per 128-channel stage (INT4); NF4 keeps its absmax pairs in sp[0] / zp[0]
   static constexpr int kNq = FMT == kFmtInt4 ? 128 / G : 1;
+  static constexpr int kDepth = 4;  // per-warp ring slots (3 units in flight)
+  static constexpr int kScaleBytes = FMT == kFmtInt4 ? 32 * kNq : 32;  // NF4: absmax pairs
+  static constexpr int kZeroBytes = FMT == kFmtInt4 ? 8 * kNq : 0;
+  static constexpr int kRG = gemv_row_groups(NB);  // row groups per work unit
+  static constexpr int kSlot = kRG * 1024 + (kRG * (kScaleBytes + kZeroBytes) + 15) / 16 * 16;
+  static constexpr int kSmemBytes = kWarps * kDepth * kSlot;
 };
 
 __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t (&a)[4],
@@ -76,66 +90,99 @@ __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Streaming 16-byte load: read once, no L1 allocation.
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// One 128-channel stage of a lane's row group: 8 code words (two 16-byte
-// loads, 512 contiguous bytes per warp each) and the constants of its two rows.
+// One 128-channel stage of a lane's R row groups in registers.
 template <class C>
 struct StageRegs {
-  uint4 c0, c1;            // code words of channel blocks 0..3 and 4..7
-  uint32_t sp[C::kNq];     // INT4: scale pairs, one per group in the stage; NF4: absmax pair, block 0
-  uint32_t zp[C::kNq];     // INT4: zero pairs; NF4: absmax pair, block 1
+  uint4 c[C::kRG][2];           // code words of channel blocks 0..3 and 4..7
+  uint32_t sp[C::kRG][C::kNq];  // INT4: scale pairs per group; NF4: absmax pair, block 0
+  uint32_t zp[C::kRG][C::kNq];  // INT4: zero pairs; NF4: absmax pair, block 1
 };
 
 template <class C>
-__device__ __forceinline__ void load_stage(const uint8_t* __restrict__ blk, StageRegs<C>& r,
-                                           int rgl, int lane) {
-  const int g = lane >> 2;
-  r.c0 = ldg_stream(blk + code_word_offset(rgl, 0, lane));
-  r.c1 = ldg_stream(blk + code_word_offset(rgl, 4, lane));
-  if constexpr (C::FMT == kFmtInt4) {
-    constexpr int gps = kStageK / C::G;
+__device__ __forceinline__ void issue_stage(const uint8_t* __restrict__ blk, uint32_t slot, int rpl,
+                                            int lane) {
+  constexpr int R = C::kRG;
+  const int rgl0 = rpl * R;
+  const uint8_t* cb = blk + rgl0 * 1024 + lane * 16;
 #pragma unroll
-    for (int q = 0; q < C::kNq; ++q) {
-      r.sp[q] = __ldg(reinterpret_cast<const uint32_t*>(blk + scale_pair_offset(rgl, q, g, gps)));
-      r.zp[q] = __ldg(blk + zero_pair_offset(rgl, q, g, gps));
+  for (int i = 0; i < 2 * R; ++i) cp_async16(slot + i * 512 + lane * 16, cb + i * 512);
+  constexpr int sbytes = R * C::kScaleBytes;
+  constexpr int sl = sbytes / 16;
+  if constexpr (C::FMT == kFmtInt4) {
+    constexpr int gps = C::kNq;
+    const uint8_t* sc = blk + kCodeBytes + rgl0 * C::kScaleBytes;
+    const uint8_t* zc = blk + kCodeBytes + kTileRows * gps * 2 + rgl0 * C::kZeroBytes;
+    if (lane < sl) cp_async16(slot + R * 1024 + lane * 16, sc + lane * 16);
+    constexpr int zbytes = R * C::kZeroBytes;
+    if constexpr (zbytes == 8) {
+      if (lane == sl) cp_async8(slot + R * 1024 + sbytes, zc);
+    } else {
+      const int zl = lane - sl;
+      if (zl >= 0 && zl < zbytes / 16) cp_async16(slot + R * 1024 + sbytes + zl * 16, zc + zl * 16);
     }
   } else {
-    r.sp[0] = __ldg(reinterpret_cast<const uint16_t*>(blk + absmax_pair_offset(rgl, 0, g)));
-    r.zp[0] = __ldg(reinterpret_cast<const uint16_t*>(blk + absmax_pair_offset(rgl, 1, g)));
+    if (lane < sl) cp_async16(slot + R * 1024 + lane * 16, blk + kCodeBytes + rgl0 * 32 + lane * 16);
   }
 }
 
-// Dequantize code words [W0, W0 + NW) of one 64-channel half and run their
-// MMAs.  xs[nb] points at X[token row of block nb][first channel of the
-// half + 4u]; p0 / p1 are the constants of rows r0 / r1 (INT4), a0 / a1 the
-// reconstructed absmax (NF4).
+template <class C>
+__device__ __forceinline__ void read_stage(const uint8_t* slot, StageRegs<C>& r, int lane) {
+  constexpr int R = C::kRG;
+  const int g = lane >> 2;
+#pragma unroll
+  for (int rr = 0; rr < R; ++rr) {
+    r.c[rr][0] = *reinterpret_cast<const uint4*>(slot + rr * 1024 + lane * 16);
+    r.c[rr][1] = *reinterpret_cast<const uint4*>(slot + rr * 1024 + 512 + lane * 16);
+    if constexpr (C::FMT == kFmtInt4) {
+#pragma unroll
+      for (int q = 0; q < C::kNq; ++q) {
+        r.sp[rr][q] = *reinterpret_cast<const uint32_t*>(slot + R * 1024 + rr * C::kScaleBytes + (q * 8 + g) * 4);
+        r.zp[rr][q] = slot[R * 1024 + R * C::kScaleBytes + rr * C::kZeroBytes + q * 8 + g];
+      }
+    } else {
+      r.sp[rr][0] = *reinterpret_cast<const uint16_t*>(slot + R * 1024 + rr * 32 + g * 2);
+      r.zp[rr][0] = *reinterpret_cast<const uint16_t*>(slot + R * 1024 + rr * 32 + (8 + g) * 2);
+    }
+  }
+}
+
+// Words [W0, W0 + NW) of one 64-channel half for the R row groups: one
+// activation fragment per word index serves every row group.
 template <class C, int W0, int NW>
-__device__ __forceinline__ void mma_words(const uint32_t (&words)[4], const Int4Dq& p0,
-                                          const Int4Dq& p1, float a0, float a1,
+__device__ __forceinline__ void mma_words(const uint32_t (&words)[C::kRG][4],
+                                          const Int4Dq (&p0)[C::kRG], const Int4Dq (&p1)[C::kRG],
+                                          const float (&a0)[C::kRG], const float (&a1)[C::kRG],
                                           const float* __restrict__ T,
                                           const uint16_t* const (&xs)[C::NB],
-                                          float (&acc)[2][C::NB][4]) {
+                                          float (&acc)[C::kRG][2][C::NB][4]) {
 #pragma unroll
   for (int w = W0; w < W0 + NW; ++w) {
-    uint32_t pr[4];
-    if constexpr (C::FMT == kFmtInt4) {
-      int4_dq_word(words[w], p0, p1, pr);
-    } else {
-      nf4_dq_word(words[w], a0, a1, T, pr);
-    }
-    const uint32_t afrag[4] = {pr[0], pr[2], pr[1], pr[3]};
+    uint2 b[C::NB];
 #pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb) {
-      const uint2 b = __ldg(reinterpret_cast<const uint2*>(xs[nb] + w * 16));
-      mma_m16n8k16_bf16(acc[w & 1][nb], afrag, b.x, b.y);
+    for (int nb = 0; nb < C::NB; ++nb) b[nb] = __ldg(reinterpret_cast<const uint2*>(xs[nb] + w * 16));
+#pragma unroll
+    for (int rr = 0; rr < C::kRG; ++rr) {
+      uint32_t pr[4];
+      if constexpr (C::FMT == kFmtInt4) {
+        int4_dq_word(words[rr][w], p0[rr], p1[rr], pr);
+      } else {
+        nf4_dq_word(words[rr][w], a0[rr], a1[rr], T, pr);
+      }
+      const uint32_t afrag[4] = {pr[0], pr[2], pr[1], pr[3]};
+#pragma unroll
+      for (int nb = 0; nb < C::NB; ++nb) mma_m16n8k16_bf16(acc[rr][w & 1][nb], afrag, b[nb].x, b[nb].y);
     }
   }
 }
@@ -146,86 +193,91 @@ __device__ __forceinline__ uint32_t owner_of(uint32_t u, const GemvArgs& a) {
   return u < big ? fast_div(u, a.by_q1) : a.r + fast_div(u - big, a.by_q);
 }
 
-// Hand a row group's accumulated sums on: write Y if this warp covered the
-// whole channel range (units [seg0, seg1) == the row group's), else store
-// them in the warp's slot; the last contributor of the row group sums the
-// slots in order and writes Y.
 template <class C>
-__device__ __forceinline__ void flush_row_group(const GemvArgs& args, float (&acc)[2][C::NB][4],
-                                                int rgg, uint32_t seg0, uint32_t seg1,
-                                                uint32_t wid, int lane) {
+__device__ __forceinline__ void flush_row_group(const GemvArgs& args,
+                                                float (&acc)[C::kRG][2][C::NB][4], int rpg,
+                                                uint32_t seg0, uint32_t seg1, uint32_t wid, int lane) {
+  constexpr int R = C::kRG;
+  constexpr int V = R * C::NB * 4;  // floats per lane
   const int g = lane >> 2, u = lane & 3;
-  const int r0 = rgg * 16 + g;
-  float tot[C::NB][4];
+  float tot[R][C::NB][4];
 #pragma unroll
-  for (int nb = 0; nb < C::NB; ++nb)
+  for (int rr = 0; rr < R; ++rr)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      tot[nb][j] = acc[0][nb][j] + acc[1][nb][j];
-      acc[0][nb][j] = 0.0f;
-      acc[1][nb][j] = 0.0f;
-    }
-  const uint32_t rs = static_cast<uint32_t>(rgg) * static_cast<uint32_t>(args.KS);
+    for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        tot[rr][nb][j] = acc[rr][0][nb][j] + acc[rr][1][nb][j];
+        acc[rr][0][nb][j] = 0.0f;
+        acc[rr][1][nb][j] = 0.0f;
+      }
+  const uint32_t rs = static_cast<uint32_t>(rpg) * static_cast<uint32_t>(args.KS);
   const uint32_t re = rs + static_cast<uint32_t>(args.KS);
   bool write_y = true;
   if (seg0 != rs || seg1 != re) {
     const uint32_t first = owner_of(rs, args);
     const uint32_t contributors = owner_of(re - 1, args) - first + 1;
-    float* slot = args.partial +
-                  ((static_cast<size_t>(rgg) * args.max_slots + (wid - first)) * 32 + lane) * 4 * C::NB;
+    float* slot = args.partial + ((static_cast<size_t>(rpg) * args.max_slots + (wid - first)) * 32 + lane) * V;
 #pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb)
-      *reinterpret_cast<float4*>(slot + nb * 4) =
-          make_float4(tot[nb][0], tot[nb][1], tot[nb][2], tot[nb][3]);
-    // publish the slot with an acquire-release counter update (no full fence,
-    // which would also wait for this warp's prefetched loads)
+    for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+      for (int nb = 0; nb < C::NB; ++nb)
+        *reinterpret_cast<float4*>(slot + (rr * C::NB + nb) * 4) =
+            make_float4(tot[rr][nb][0], tot[rr][nb][1], tot[rr][nb][2], tot[rr][nb][3]);
     __syncwarp();
     unsigned prev = 0;
-    if (lane == 0) prev = atom_add_acq_rel_gpu(args.counter + rgg, 1u);
+    if (lane == 0) prev = atom_add_acq_rel_gpu(args.counter + rpg, 1u);
     prev = __shfl_sync(0xffffffffu, prev, 0);
     write_y = prev == contributors - 1;
     if (write_y) {
 #pragma unroll
-      for (int nb = 0; nb < C::NB; ++nb)
+      for (int rr = 0; rr < R; ++rr)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tot[nb][j] = 0.0f;
-      const float* base =
-          args.partial + (static_cast<size_t>(rgg) * args.max_slots * 32 + lane) * 4 * C::NB;
+        for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) tot[rr][nb][j] = 0.0f;
+      const float* base = args.partial + (static_cast<size_t>(rpg) * args.max_slots * 32 + lane) * V;
       for (uint32_t sp = 0; sp < contributors; ++sp) {
 #pragma unroll
-        for (int nb = 0; nb < C::NB; ++nb) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(
-              base + static_cast<size_t>(sp) * 32 * 4 * C::NB + nb * 4));
-          tot[nb][0] += v.x;
-          tot[nb][1] += v.y;
-          tot[nb][2] += v.z;
-          tot[nb][3] += v.w;
-        }
+        for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+          for (int nb = 0; nb < C::NB; ++nb) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                base + static_cast<size_t>(sp) * 32 * V + (rr * C::NB + nb) * 4));
+            tot[rr][nb][0] += v.x;
+            tot[rr][nb][1] += v.y;
+            tot[rr][nb][2] += v.z;
+            tot[rr][nb][3] += v.w;
+          }
       }
-      if (lane == 0) args.counter[rgg] = 0u;  // leave the workspace zeroed
+      if (lane == 0) args.counter[rpg] = 0u;
     }
   }
   if (write_y) {
 #pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb)
+    for (int rr = 0; rr < R; ++rr) {
+      const int r0 = (rpg * R + rr) * 16 + g;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int m = nb * 8 + 2 * u + (j & 1);
-        const int nn = r0 + (j >> 1) * 8;
-        if (m < args.M && nn < args.N)
-          args.Y[static_cast<size_t>(m) * args.N + nn] =
-              __bfloat16_as_ushort(__float2bfloat16_rn(tot[nb][j]));
-      }
+      for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = nb * 8 + 2 * u + (j & 1);
+          const int nn = r0 + (j >> 1) * 8;
+          if (m < args.M && nn < args.N)
+            args.Y[static_cast<size_t>(m) * args.N + nn] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(tot[rr][nb][j]));
+        }
+    }
   }
 }
 
-// Dequantize and multiply one 128-channel stage of row group rgg.
 template <class C>
 __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageRegs<C>& cur,
-                                              int rgg, int st, int g,
+                                              int rpg, int st, int g,
                                               const uint16_t* const (&xrow)[C::NB],
                                               const float* __restrict__ Ts,
-                                              float (&acc)[2][C::NB][4]) {
+                                              float (&acc)[C::kRG][2][C::NB][4]) {
+  constexpr int R = C::kRG;
   const int k0 = st * kStageK;
   const uint16_t* xa[C::NB];
   const uint16_t* xb[C::NB];
@@ -234,63 +286,60 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
     xa[nb] = xrow[nb] + k0;
     xb[nb] = xa[nb] + 64;
   }
-  const uint32_t w0[4] = {cur.c0.x, cur.c0.y, cur.c0.z, cur.c0.w};
-  const uint32_t w1[4] = {cur.c1.x, cur.c1.y, cur.c1.z, cur.c1.w};
-  const bool second = k0 + 64 < args.K;  // K % 64 == 0: the second half exists or not
-  if constexpr (C::FMT == kFmtInt4) {
-    if constexpr (C::G == 128) {
-      const Int4Dq e0 = int4_dq_params(cur.sp[0] & 0xFFFFu, cur.zp[0] & 0xFu);
-      const Int4Dq e1 = int4_dq_params(cur.sp[0] >> 16, (cur.zp[0] >> 4) & 0xFu);
-      mma_words<C, 0, 4>(w0, e0, e1, 0.f, 0.f, Ts, xa, acc);
-      if (second) mma_words<C, 0, 4>(w1, e0, e1, 0.f, 0.f, Ts, xb, acc);
-    } else if constexpr (C::G == 64) {
-      {
-        const Int4Dq e0 = int4_dq_params(cur.sp[0] & 0xFFFFu, cur.zp[0] & 0xFu);
-        const Int4Dq e1 = int4_dq_params(cur.sp[0] >> 16, (cur.zp[0] >> 4) & 0xFu);
-        mma_words<C, 0, 4>(w0, e0, e1, 0.f, 0.f, Ts, xa, acc);
-      }
-      if (second) {
-        const Int4Dq e0 = int4_dq_params(cur.sp[1] & 0xFFFFu, cur.zp[1] & 0xFu);
-        const Int4Dq e1 = int4_dq_params(cur.sp[1] >> 16, (cur.zp[1] >> 4) & 0xFu);
-        mma_words<C, 0, 4>(w1, e0, e1, 0.f, 0.f, Ts, xb, acc);
-      }
-    } else {
+  uint32_t w0[R][4], w1[R][4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (q >= 2 && !second) break;
-        const Int4Dq e0 = int4_dq_params(cur.sp[q] & 0xFFFFu, cur.zp[q] & 0xFu);
-        const Int4Dq e1 = int4_dq_params(cur.sp[q] >> 16, (cur.zp[q] >> 4) & 0xFu);
-        if (q == 0)
-          mma_words<C, 0, 2>(w0, e0, e1, 0.f, 0.f, Ts, xa, acc);
-        else if (q == 1)
-          mma_words<C, 2, 2>(w0, e0, e1, 0.f, 0.f, Ts, xa, acc);
-        else if (q == 2)
-          mma_words<C, 0, 2>(w1, e0, e1, 0.f, 0.f, Ts, xb, acc);
-        else
-          mma_words<C, 2, 2>(w1, e0, e1, 0.f, 0.f, Ts, xb, acc);
+  for (int rr = 0; rr < R; ++rr) {
+    w0[rr][0] = cur.c[rr][0].x; w0[rr][1] = cur.c[rr][0].y; w0[rr][2] = cur.c[rr][0].z; w0[rr][3] = cur.c[rr][0].w;
+    w1[rr][0] = cur.c[rr][1].x; w1[rr][1] = cur.c[rr][1].y; w1[rr][2] = cur.c[rr][1].z; w1[rr][3] = cur.c[rr][1].w;
+  }
+  const bool second = k0 + 64 < args.K;
+  const float fz[R] = {};
+  if constexpr (C::FMT == kFmtInt4) {
+#pragma unroll
+    for (int q = 0; q < C::kNq; ++q) {
+      if (q >= C::kNq / 2 && C::kNq > 1 && !second) break;
+      Int4Dq e0[R], e1[R];
+#pragma unroll
+      for (int rr = 0; rr < R; ++rr) {
+        e0[rr] = int4_dq_params(cur.sp[rr][q] & 0xFFFFu, cur.zp[rr][q] & 0xFu);
+        e1[rr] = int4_dq_params(cur.sp[rr][q] >> 16, (cur.zp[rr][q] >> 4) & 0xFu);
+      }
+      if constexpr (C::G == 128) {
+        mma_words<C, 0, 4>(w0, e0, e1, fz, fz, Ts, xa, acc);
+        if (second) mma_words<C, 0, 4>(w1, e0, e1, fz, fz, Ts, xb, acc);
+      } else if constexpr (C::G == 64) {
+        if (q == 0) mma_words<C, 0, 4>(w0, e0, e1, fz, fz, Ts, xa, acc);
+        else mma_words<C, 0, 4>(w1, e0, e1, fz, fz, Ts, xb, acc);
+      } else {
+        if (q == 0) mma_words<C, 0, 2>(w0, e0, e1, fz, fz, Ts, xa, acc);
+        else if (q == 1) mma_words<C, 2, 2>(w0, e0, e1, fz, fz, Ts, xa, acc);
+        else if (q == 2) mma_words<C, 0, 2>(w1, e0, e1, fz, fz, Ts, xb, acc);
+        else mma_words<C, 2, 2>(w1, e0, e1, fz, fz, Ts, xb, acc);
       }
     }
   } else {
-    // NF4: a' = code * s2[block index / dq_group] per (row, 64-block)
     const unsigned long long kb64 = static_cast<unsigned long long>(args.K / 64);
-    const int r0 = rgg * 16 + g;
-    float a0[2] = {0.0f, 0.0f}, a1[2] = {0.0f, 0.0f};
+    float a0[2][R], a1[2][R];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const unsigned long long blk = static_cast<unsigned long long>(st) * 2 + h;
-      if (blk < kb64) {
-        const uint32_t pair = h == 0 ? cur.sp[0] : cur.zp[0];
-        if (r0 < args.N)
-          a0[h] = __fmul_rn(static_cast<float>(pair & 0xFFu),
-                            __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0) * kb64 + blk,
-                                                     args.by_dq)));
-        if (r0 + 8 < args.N)
-          a1[h] = __fmul_rn(static_cast<float>(pair >> 8),
-                            __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0 + 8) * kb64 + blk,
-                                                     args.by_dq)));
+#pragma unroll
+      for (int rr = 0; rr < R; ++rr) {
+        a0[h][rr] = 0.0f;
+        a1[h][rr] = 0.0f;
+        const int r0 = (rpg * R + rr) * 16 + g;
+        if (blk < kb64) {
+          const uint32_t pair = h == 0 ? cur.sp[rr][0] : cur.zp[rr][0];
+          if (r0 < args.N)
+            a0[h][rr] = __fmul_rn(static_cast<float>(pair & 0xFFu),
+                                  __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0) * kb64 + blk, args.by_dq)));
+          if (r0 + 8 < args.N)
+            a1[h][rr] = __fmul_rn(static_cast<float>(pair >> 8),
+                                  __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0 + 8) * kb64 + blk, args.by_dq)));
+        }
       }
     }
-    const Int4Dq none{};
+    Int4Dq none[R] = {};
     mma_words<C, 0, 4>(w0, none, none, a0[0], a1[0], Ts, xa, acc);
     if (second) mma_words<C, 0, 4>(w1, none, none, a0[1], a1[1], Ts, xb, acc);
   }
@@ -298,25 +347,23 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
 
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(const GemvArgs args) {
+  constexpr int R = C::kRG;
   __shared__ float Ts[16];
   if (C::FMT == kFmtNf4) {
     if (threadIdx.x < 16) Ts[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
     __syncthreads();
   }
   grid_dep_launch();
-  grid_dep_wait();  // X, Y and the workspace may belong to the previous kernel
 
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, u = lane & 3;
   const uint32_t wid = blockIdx.x * C::kWarps + (threadIdx.x >> 5);
-  // this warp's contiguous range of (row group, stage) units, row-group major
   const uint32_t ua = wid * args.q + (wid < args.r ? wid : args.r);
   const int left = static_cast<int>(args.q) + (wid < args.r ? 1 : 0);
   if (left == 0) return;
   const int KS = args.KS;
+  constexpr int kPairsPerTile = 8 / R;
 
-  // activation rows of this lane's token columns; rows past M read row M - 1
-  // (those accumulator columns are never stored)
   const uint16_t* xrow[C::NB];
 #pragma unroll
   for (int nb = 0; nb < C::NB; ++nb) {
@@ -324,63 +371,68 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
     xrow[nb] = args.X + static_cast<size_t>(row) * args.K + 4 * u;
   }
 
-  // prefetch cursor: (row group, stage) of the next stage to load and the
-  // address of its stage block
-  const int rgg0 = static_cast<int>(fast_div(ua, args.by_ks));
-  const int st0 = static_cast<int>(ua) - rgg0 * KS;
-  int pf_rgg = rgg0, pf_st = st0;
+  const int rpg0 = static_cast<int>(fast_div(ua, args.by_ks));
+  const int st0 = static_cast<int>(ua) - rpg0 * KS;
+  int pf_rpg = rpg0, pf_st = st0;
   const uint8_t* pf_ptr =
-      args.Wp + (static_cast<size_t>(pf_rgg >> 3) * KS + pf_st) * C::kStageBytes;
+      args.Wp + (static_cast<size_t>(pf_rpg / kPairsPerTile) * KS + pf_st) * C::kStageBytes;
   auto advance = [&]() {
     if (++pf_st == KS) {
       pf_st = 0;
-      ++pf_rgg;
-      pf_ptr = args.Wp + static_cast<size_t>(pf_rgg >> 3) * KS * C::kStageBytes;
+      ++pf_rpg;
+      pf_ptr = args.Wp + static_cast<size_t>(pf_rpg / kPairsPerTile) * KS * C::kStageBytes;
     } else {
       pf_ptr += C::kStageBytes;
     }
   };
 
-  // three register sets, two stages in flight: set (i + 2) % 3 is refilled
-  // while set i is consumed, so the ring rotates without copies
-  StageRegs<C> ring[3];
+  extern __shared__ __align__(16) uint8_t w4_gemv_smem[];
+  uint8_t* ring = w4_gemv_smem + (threadIdx.x >> 5) * (C::kDepth * C::kSlot);
+  const uint32_t ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < C::kDepth - 1; ++i) {
     if (i < left) {
-      load_stage<C>(pf_ptr, ring[i], pf_rgg & 7, lane);
+      issue_stage<C>(pf_ptr, ring_s + i * C::kSlot, pf_rpg % kPairsPerTile, lane);
       advance();
     }
+    cp_async_commit();
+  }
+  grid_dep_wait();  // X, Y and the workspace may belong to the previous kernel
 
-  float acc[2][C::NB][4];
+  float acc[R][2][C::NB][4];
 #pragma unroll
-  for (int e = 0; e < 2; ++e)
+  for (int rr = 0; rr < R; ++rr)
 #pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb)
+    for (int e = 0; e < 2; ++e)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[e][nb][j] = 0.0f;
+      for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[rr][e][nb][j] = 0.0f;
 
-  int rgg = rgg0, st = st0;
-  uint32_t seg0 = ua;  // first unit of this warp's part of row group rgg
-  int n = 0;
-  for (;;) {
-#pragma unroll
-    for (int i = 0; i < 3; ++i) {
-      if (n == left) return;
-      if (n + 2 < left) {
-        load_stage<C>(pf_ptr, ring[(i + 2) % 3], pf_rgg & 7, lane);
-        advance();
-      }
-      stage_compute<C>(args, ring[i], rgg, st, g, xrow, Ts, acc);
-      if (st == KS - 1 || n + 1 == left) {
-        const uint32_t seg1 = ua + static_cast<uint32_t>(n) + 1;
-        flush_row_group<C>(args, acc, rgg, seg0, seg1, wid, lane);
-        ++rgg;
-        st = 0;
-        seg0 = seg1;
-      } else {
-        ++st;
-      }
-      ++n;
+  int rpg = rpg0, st = st0;
+  uint32_t seg0 = ua;
+  int cs = 0;
+  for (int n = 0; n < left; ++n) {
+    cp_async_wait<C::kDepth - 2>();
+    __syncwarp();
+    StageRegs<C> cur;
+    read_stage<C>(ring + cs * C::kSlot, cur, lane);
+    if (n + C::kDepth - 1 < left) {
+      const int is = cs == 0 ? C::kDepth - 1 : cs - 1;
+      issue_stage<C>(pf_ptr, ring_s + is * C::kSlot, pf_rpg % kPairsPerTile, lane);
+      advance();
+    }
+    cp_async_commit();
+    cs = cs + 1 == C::kDepth ? 0 : cs + 1;
+    stage_compute<C>(args, cur, rpg, st, g, xrow, Ts, acc);
+    if (st == KS - 1 || n + 1 == left) {
+      const uint32_t seg1 = ua + static_cast<uint32_t>(n) + 1;
+      flush_row_group<C>(args, acc, rpg, seg0, seg1, wid, lane);
+      ++rpg;
+      st = 0;
+      seg0 = seg1;
+    } else {
+      ++st;
     }
   }
 }

@@ -121,6 +121,9 @@ __global__ void int4_prepack_kernel(const uint8_t* __restrict__ Wq,
       blk[zero_pair_offset(rg, gl, g, gps)] = static_cast<uint8_t>(z0 | (z1 << 4));
     }
   }
+  // The GEMM kernels start streaming Wp before their launch dependency on
+  // the previous kernel resolves: make every write visible before exiting.
+  __threadfence();
 }
 
 // grid (stages, tiles), block 256.
@@ -148,6 +151,7 @@ __global__ void nf4_prepack_kernel(const uint8_t* __restrict__ Wq,
       }
     }
   }
+  __threadfence();  // as in int4_prepack_kernel
 }
 
 // Act-order channel permutation: a stable sort of k by g_idx[k] when every
@@ -181,6 +185,7 @@ __global__ void act_order_perm_kernel(const int32_t* __restrict__ g_idx, int K, 
     if (threadIdx.x == 0) set_dev_error(W4_DEV_ERR_INPUT);
     for (int k = threadIdx.x; k < K; k += blockDim.x) perm[k] = k;
   }
+  __threadfence();  // as in int4_prepack_kernel
 }
 
 // Inverse of int4_prepack_kernel in prepacked channel order.  grid (stages,
