@@ -171,20 +171,22 @@ def barrier(pg):
         pg.barrier()
 
 
-def max_over_ranks(pg, v: float) -> float:
-    if pg is None:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+def _reduce(pg, v: float, op) -> float:
+    # NCCL reduces device tensors; gloo (the CPU tests of this logic) host ones
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(pg, v: float) -> float:
+    """The slowest rank's time: the job is done when the last rank is."""
+    return v if pg is None else _reduce(pg, v, pg.ReduceOp.MAX)
 
 
 def sum_over_ranks(pg, v: float) -> float:
-    if pg is None:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    pg.all_reduce(t, op=pg.ReduceOp.SUM)
-    return float(t.item())
+    """Whole-job totals (bytes processed by all ranks)."""
+    return v if pg is None else _reduce(pg, v, pg.ReduceOp.SUM)
 
 
 def bf16_dev(bits):
