@@ -54,7 +54,8 @@ struct GemmCfg {
   static constexpr int kThreads = 64 + kDqWarps * 32;
   static constexpr int kNumBars = 2 * STAGES + 2 * kASlots + 3;
   static constexpr int kSmemBytes =
-      1024 /* alignment slack */ + STAGES * (kXStageBytes + kWSlot) + kNumBars * 8 + 16 + 64;
+      1024 /* alignment slack */ + STAGES * (kXStageBytes + kWSlot) + kNumBars * 8 + 16 + 64 +
+      64 /* NF4 level table alignment */;
   static constexpr int kMinBlocks = kTmemCols <= 256 && kSmemBytes <= 113 * 1024 ? 2 : 1;
   static_assert(MT % 16 == 0 && MT >= 16 && MT <= 256, "MMA N for M=128 is 16..256 step 16");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -137,17 +138,39 @@ __device__ __forceinline__ void int4_dq_word(uint32_t w, const Int4Dq& p0, const
         "r"(p1.shi), "r"(p1.slo));
 }
 
-// NF4 dequant of one word: w_hat = bf16_rne(fp32(T[q] * a')), T in shared
-// memory, a0 / a1 the reconstructed absmax of rows r0 / r1.
-__device__ __forceinline__ void nf4_dq_word(uint32_t w, float a0, float a1,
-                                            const float* __restrict__ T, uint32_t* out) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float a = j < 2 ? a0 : a1;
-    const float f0 = __fmul_rn(T[(w >> (4 * j)) & 0xFu], a);
-    const float f1 = __fmul_rn(T[(w >> (16 + 4 * j)) & 0xFu], a);
-    out[j] = bf2_from_f32(f0, f1);
-  }
+// NF4 dequant of one word: w_hat = bf16_rne(fp32(T[q] * a')), with the 16
+// levels T in shared memory at the 64-byte-aligned shared address tb (so that
+// a level's address is tb | 4q), a0 / a1 the reconstructed absmax of rows
+// r0 / r1.  One asm block: per code one shift and one LOP3 for the address,
+// one shared load, one fp32 multiply; one conversion per pair.
+__device__ __forceinline__ void nf4_dq_word(uint32_t w, float a0, float a1, uint32_t tb,
+                                            uint32_t* out) {
+  const uint32_t m = 0x3Cu;
+  asm("{\n\t.reg .b32 o0, o1, o2, o3, o4, o5, o6, o7;\n\t"
+      ".reg .f32 v0, v1, v2, v3, v4, v5, v6, v7;\n\t"
+      "shl.b32 o0, %4, 2;\n\t  lop3.b32 o0, o0, %7, %8, 0xEA;\n\t"
+      "shr.b32 o1, %4, 14;\n\t lop3.b32 o1, o1, %7, %8, 0xEA;\n\t"
+      "shr.b32 o2, %4, 2;\n\t  lop3.b32 o2, o2, %7, %8, 0xEA;\n\t"
+      "shr.b32 o3, %4, 18;\n\t lop3.b32 o3, o3, %7, %8, 0xEA;\n\t"
+      "shr.b32 o4, %4, 6;\n\t  lop3.b32 o4, o4, %7, %8, 0xEA;\n\t"
+      "shr.b32 o5, %4, 22;\n\t lop3.b32 o5, o5, %7, %8, 0xEA;\n\t"
+      "shr.b32 o6, %4, 10;\n\t lop3.b32 o6, o6, %7, %8, 0xEA;\n\t"
+      "shr.b32 o7, %4, 26;\n\t lop3.b32 o7, o7, %7, %8, 0xEA;\n\t"
+      "ld.shared.f32 v0, [o0];\n\t ld.shared.f32 v1, [o1];\n\t"
+      "ld.shared.f32 v2, [o2];\n\t ld.shared.f32 v3, [o3];\n\t"
+      "ld.shared.f32 v4, [o4];\n\t ld.shared.f32 v5, [o5];\n\t"
+      "ld.shared.f32 v6, [o6];\n\t ld.shared.f32 v7, [o7];\n\t"
+      "mul.rn.f32 v0, v0, %5;\n\t mul.rn.f32 v1, v1, %5;\n\t"
+      "mul.rn.f32 v2, v2, %5;\n\t mul.rn.f32 v3, v3, %5;\n\t"
+      "mul.rn.f32 v4, v4, %6;\n\t mul.rn.f32 v5, v5, %6;\n\t"
+      "mul.rn.f32 v6, v6, %6;\n\t mul.rn.f32 v7, v7, %6;\n\t"
+      "cvt.rn.bf16x2.f32 %0, v1, v0;\n\t"
+      "cvt.rn.bf16x2.f32 %1, v3, v2;\n\t"
+      "cvt.rn.bf16x2.f32 %2, v5, v4;\n\t"
+      "cvt.rn.bf16x2.f32 %3, v7, v6;\n\t}"
+      : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
+      : "r"(w), "f"(a0), "f"(a1), "r"(m), "r"(tb)
+      : "memory");
 }
 
 struct GemmArgs {

@@ -23,7 +23,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
   uint64_t* epi2 = epi1 + 1;                            // last-arrival known (1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi2 + 1);
   int* last_flag = reinterpret_cast<int*>(tmem_holder + 1);
-  float* Ts = reinterpret_cast<float*>(tmem_holder + 4);  // NF4 levels [16]
+  float* Ts = reinterpret_cast<float*>(                   // NF4 levels [16], 64-byte aligned
+      (reinterpret_cast<uintptr_t>(tmem_holder + 4) + 63) & ~static_cast<uintptr_t>(63));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
                              __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0 + 8) * kb64 + blk_in_row, args.by_dq)));
           }
 #pragma unroll
-          for (int w = 0; w < 4; ++w) nf4_dq_word(words[w], a0, a1, Ts, &out[rgl][4 * w]);
+          for (int w = 0; w < 4; ++w) nf4_dq_word(words[w], a0, a1, smem_u32(Ts), &out[rgl][4 * w]);
         }
       }
       if (it >= C::kASlots &&
@@ -254,16 +255,30 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
           __threadfence();
           const float* base =
               args.partial + static_cast<size_t>(tile_id) * args.splits * C::MT * kTileRows;
+          // kCb columns at a time, so that kCb loads per split are in flight
+          // (one column at a time leaves the reduction L2-latency bound)
+          constexpr int kCb = kHalfCols < 16 ? kHalfCols : 16;
 #pragma unroll 1
-          for (int c = 0; c < kHalfCols; ++c) {
-            const int ml = h * kHalfCols + c;
-            const int m = mtile * C::MT + ml;
-            float acc = 0.0f;
-            for (int sp = 0; sp < args.splits; ++sp)
-              acc += __ldcg(base + (static_cast<size_t>(sp) * C::MT + ml) * kTileRows + row);
-            if (m < args.M && n < args.N)
-              args.Y[static_cast<size_t>(m) * args.N + n] =
-                  __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+          for (int c0 = 0; c0 < kHalfCols; c0 += kCb) {
+            const int ml0 = h * kHalfCols + c0;
+            float acc[kCb];
+#pragma unroll
+            for (int j = 0; j < kCb; ++j) acc[j] = 0.0f;
+            for (int sp = 0; sp < args.splits; ++sp) {
+              const float* src = base + (static_cast<size_t>(sp) * C::MT + ml0) * kTileRows + row;
+              float v[kCb];
+#pragma unroll
+              for (int j = 0; j < kCb; ++j) v[j] = __ldcg(src + j * kTileRows);
+#pragma unroll
+              for (int j = 0; j < kCb; ++j) acc[j] += v[j];
+            }
+#pragma unroll
+            for (int j = 0; j < kCb; ++j) {
+              const int m = mtile * C::MT + ml0 + j;
+              if (m < args.M && n < args.N)
+                args.Y[static_cast<size_t>(m) * args.N + n] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+            }
           }
           if (threadIdx.x == 64) args.counter[tile_id] = 0u;  // leave the workspace zeroed
         }

@@ -164,7 +164,7 @@ template <class C, int W0, int NW>
 __device__ __forceinline__ void mma_words(const uint32_t (&words)[C::kRG][4],
                                           const Int4Dq (&p0)[C::kRG], const Int4Dq (&p1)[C::kRG],
                                           const float (&a0)[C::kRG], const float (&a1)[C::kRG],
-                                          const float* __restrict__ T,
+                                          uint32_t tb,
                                           const uint16_t* const (&xs)[C::NB],
                                           float (&acc)[C::kRG][2][C::NB][4]) {
 #pragma unroll
@@ -178,7 +178,7 @@ __device__ __forceinline__ void mma_words(const uint32_t (&words)[C::kRG][4],
       if constexpr (C::FMT == kFmtInt4) {
         int4_dq_word(words[rr][w], p0[rr], p1[rr], pr);
       } else {
-        nf4_dq_word(words[rr][w], a0[rr], a1[rr], T, pr);
+        nf4_dq_word(words[rr][w], a0[rr], a1[rr], tb, pr);
       }
       const uint32_t afrag[4] = {pr[0], pr[2], pr[1], pr[3]};
 #pragma unroll
@@ -275,7 +275,7 @@ template <class C>
 __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageRegs<C>& cur,
                                               int rpg, int st, int g,
                                               const uint16_t* const (&xrow)[C::NB],
-                                              const float* __restrict__ Ts,
+                                              uint32_t tb,
                                               float (&acc)[C::kRG][2][C::NB][4]) {
   constexpr int R = C::kRG;
   const int k0 = st * kStageK;
@@ -305,16 +305,16 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
         e1[rr] = int4_dq_params(cur.sp[rr][q] >> 16, (cur.zp[rr][q] >> 4) & 0xFu);
       }
       if constexpr (C::G == 128) {
-        mma_words<C, 0, 4>(w0, e0, e1, fz, fz, Ts, xa, acc);
-        if (second) mma_words<C, 0, 4>(w1, e0, e1, fz, fz, Ts, xb, acc);
+        mma_words<C, 0, 4>(w0, e0, e1, fz, fz, tb, xa, acc);
+        if (second) mma_words<C, 0, 4>(w1, e0, e1, fz, fz, tb, xb, acc);
       } else if constexpr (C::G == 64) {
-        if (q == 0) mma_words<C, 0, 4>(w0, e0, e1, fz, fz, Ts, xa, acc);
-        else mma_words<C, 0, 4>(w1, e0, e1, fz, fz, Ts, xb, acc);
+        if (q == 0) mma_words<C, 0, 4>(w0, e0, e1, fz, fz, tb, xa, acc);
+        else mma_words<C, 0, 4>(w1, e0, e1, fz, fz, tb, xb, acc);
       } else {
-        if (q == 0) mma_words<C, 0, 2>(w0, e0, e1, fz, fz, Ts, xa, acc);
-        else if (q == 1) mma_words<C, 2, 2>(w0, e0, e1, fz, fz, Ts, xa, acc);
-        else if (q == 2) mma_words<C, 0, 2>(w1, e0, e1, fz, fz, Ts, xb, acc);
-        else mma_words<C, 2, 2>(w1, e0, e1, fz, fz, Ts, xb, acc);
+        if (q == 0) mma_words<C, 0, 2>(w0, e0, e1, fz, fz, tb, xa, acc);
+        else if (q == 1) mma_words<C, 2, 2>(w0, e0, e1, fz, fz, tb, xa, acc);
+        else if (q == 2) mma_words<C, 0, 2>(w1, e0, e1, fz, fz, tb, xb, acc);
+        else mma_words<C, 2, 2>(w1, e0, e1, fz, fz, tb, xb, acc);
       }
     }
   } else {
@@ -340,15 +340,15 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
       }
     }
     Int4Dq none[R] = {};
-    mma_words<C, 0, 4>(w0, none, none, a0[0], a1[0], Ts, xa, acc);
-    if (second) mma_words<C, 0, 4>(w1, none, none, a0[1], a1[1], Ts, xb, acc);
+    mma_words<C, 0, 4>(w0, none, none, a0[0], a1[0], tb, xa, acc);
+    if (second) mma_words<C, 0, 4>(w1, none, none, a0[1], a1[1], tb, xb, acc);
   }
 }
 
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(const GemvArgs args) {
   constexpr int R = C::kRG;
-  __shared__ float Ts[16];
+  __shared__ __align__(64) float Ts[16];  // NF4 levels
   if (C::FMT == kFmtNf4) {
     if (threadIdx.x < 16) Ts[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
     __syncthreads();
@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
     }
     cp_async_commit();
     cs = cs + 1 == C::kDepth ? 0 : cs + 1;
-    stage_compute<C>(args, cur, rpg, st, g, xrow, Ts, acc);
+    stage_compute<C>(args, cur, rpg, st, g, xrow, smem_u32(Ts), acc);
     if (st == KS - 1 || n + 1 == left) {
       const uint32_t seg1 = ua + static_cast<uint32_t>(n) + 1;
       flush_row_group<C>(args, acc, rpg, seg0, seg1, wid, lane);
