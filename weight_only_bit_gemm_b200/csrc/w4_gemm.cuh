@@ -97,14 +97,23 @@ struct Int4Dq {
   uint32_t zm, shi, slo;
 };
 
-__device__ __forceinline__ Int4Dq int4_dq_params(uint32_t s16, uint32_t z) {
-  const float sf = __half2float(__ushort_as_half(static_cast<unsigned short>(s16)));
-  Int4Dq p;
-  p.shi = bf2_from_f32(sf, sf);
-  const float lo = sf - __uint_as_float(p.shi << 16);  // exact
-  p.slo = bf2_from_f32(lo, lo);
-  p.zm = (z * 0x00010001u) | 0x43004300u;
-  return p;
+// The constants of both rows of a lane at once, from the packed fp16 scale
+// pair sp = s(r0) | s(r1) << 16 and the zero byte zp = z(r0) | z(r1) << 4.
+__device__ __forceinline__ void int4_dq_params2(uint32_t sp, uint32_t zp, Int4Dq& p0, Int4Dq& p1) {
+  float s0, s1;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
+      : "=f"(s0), "=f"(s1)
+      : "r"(sp));
+  p0.shi = bf2_from_f32(s0, s0);
+  p1.shi = bf2_from_f32(s1, s1);
+  const float l0 = s0 - __uint_as_float(p0.shi << 16);  // exact
+  const float l1 = s1 - __uint_as_float(p1.shi << 16);
+  p0.slo = bf2_from_f32(l0, l0);
+  p1.slo = bf2_from_f32(l1, l1);
+  const uint32_t t = zp * 0x00010001u;  // z(r0) at bits 0 and 16, z(r1) at 4 and 20
+  p0.zm = (t & 0x000F000Fu) | 0x43004300u;
+  p1.zm = ((t >> 4) & 0x000F000Fu) | 0x43004300u;
 }
 
 // Pairs 0 and 1 of the word belong to row r0 (params p0), pairs 2 and 3 to
@@ -183,7 +192,7 @@ struct GemmArgs {
   int KS;                 // stages per tile row = ceil(K / 128)
   int tiles_n;
   int splits;
-  FastDiv64 by_dq;        // NF4: 64-block index -> s2 index (double-quant run)
+  FastDivIdx by_dq;        // NF4: 64-block index -> s2 index (double-quant run)
 };
 
 }  // namespace w4

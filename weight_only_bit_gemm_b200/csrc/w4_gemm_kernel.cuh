@@ -159,8 +159,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
             const uint32_t sp = *reinterpret_cast<const uint32_t*>(wb + scale_pair_offset(rg, gl, g, gps));
             const uint32_t zp = wb[zero_pair_offset(rg, gl, g, gps)];
             // (the compiler merges the loads and parameter math shared by words)
-            const Int4Dq p0 = int4_dq_params(sp & 0xFFFFu, zp & 0xFu);
-            const Int4Dq p1 = int4_dq_params(sp >> 16, zp >> 4);
+            Int4Dq p0, p1;
+            int4_dq_params2(sp, zp, p0, p1);
             int4_dq_word(words[w], p0, p1, &out[rgl][4 * w]);
           }
         } else {

@@ -54,7 +54,7 @@ struct GemvArgs {
   int max_slots;            // partial slots per row group
   uint32_t q, r;            // units per warp: q + (w < r)
   FastDiv32 by_ks, by_q, by_q1;
-  FastDiv64 by_dq;          // NF4: 64-block index -> s2 index
+  FastDivIdx by_dq;          // NF4: 64-block index -> s2 index
 };
 
 // Row groups (16 rows each) per decode work unit: two share each activation
@@ -300,10 +300,7 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
       if (q >= C::kNq / 2 && C::kNq > 1 && !second) break;
       Int4Dq e0[R], e1[R];
 #pragma unroll
-      for (int rr = 0; rr < R; ++rr) {
-        e0[rr] = int4_dq_params(cur.sp[rr][q] & 0xFFFFu, cur.zp[rr][q] & 0xFu);
-        e1[rr] = int4_dq_params(cur.sp[rr][q] >> 16, (cur.zp[rr][q] >> 4) & 0xFu);
-      }
+      for (int rr = 0; rr < R; ++rr) int4_dq_params2(cur.sp[rr][q], cur.zp[rr][q], e0[rr], e1[rr]);
       if constexpr (C::G == 128) {
         mma_words<C, 0, 4>(w0, e0, e1, fz, fz, tb, xa, acc);
         if (second) mma_words<C, 0, 4>(w1, e0, e1, fz, fz, tb, xb, acc);

@@ -253,6 +253,24 @@ __device__ __forceinline__ unsigned long long fast_div(unsigned long long n, Fas
   return (__umul64hi(n, f.m) + n) >> f.l;
 }
 
+// Division by a launch constant for indices that may or may not fit in 31
+// bits: the 32-bit form when the host saw that every index does.
+struct FastDivIdx {
+  FastDiv64 d64;
+  FastDiv32 d32;
+  int narrow;  // every index < 2^31
+};
+inline FastDivIdx make_fast_div_idx(unsigned long long d, unsigned long long max_index) {
+  FastDivIdx f;
+  f.d64 = make_fast_div64(d);
+  f.narrow = max_index < (1ull << 31) && d < (1ull << 31) ? 1 : 0;
+  f.d32 = make_fast_div32(f.narrow ? static_cast<uint32_t>(d) : 1u);
+  return f;
+}
+__device__ __forceinline__ unsigned long long fast_div(unsigned long long n, const FastDivIdx& f) {
+  return f.narrow ? fast_div(static_cast<uint32_t>(n), f.d32) : fast_div(n, f.d64);
+}
+
 // Atomic add with acquire-release semantics at GPU scope: publishes this
 // thread's earlier writes (and, through a preceding warp barrier, those of its
 // warp) and makes later reads see what the previous releasers published.
