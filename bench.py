@@ -319,46 +319,80 @@ def measure_decode(step, args, pg, local):
 
 
 def measure_e2e(step, args, pg):
-    """Same step through the public API with host buffers: pinned-host X ->
-    device, the 12 calls, device Y -> pinned host, all inside the timed region."""
-    hx = [c["X"].cpu().pin_memory() for c in step.calls]
-    hy = [torch.empty(c["Y"].shape, dtype=torch.bfloat16).pin_memory() for c in step.calls]
-    dx = [torch.empty_like(c["X"]) for c in step.calls]
-    dy = [torch.empty_like(c["Y"]) for c in step.calls]
-    stream = torch.cuda.Stream()
+    """Same step through the public API with host buffers: every step copies
+    its 12 activation inputs from pinned host memory to the device, runs the
+    12 calls, and reads the 12 outputs back into pinned host memory, all
+    inside the timed region.  Copies run on their own streams and are double
+    buffered, so that step k's outputs travel back and step k+1's inputs
+    travel in while the calls of another step run."""
+    n_calls = len(step.calls)
+    x_sizes = [c["X"].numel() for c in step.calls]
+    y_sizes = [c["Y"].numel() for c in step.calls]
+    hx = torch.cat([c["X"].reshape(-1).cpu() for c in step.calls]).pin_memory()
+    hy = torch.empty(sum(y_sizes), dtype=torch.bfloat16).pin_memory()
 
-    def e2e_step():
-        for d, h in zip(dx, hx):
-            d.copy_(h, non_blocking=True)
-        step.run(X_override=dx, Y_override=dy)
-        for h, d in zip(hy, dy):
-            h.copy_(d, non_blocking=True)
+    def views(buf, sizes, shapes):
+        out, o = [], 0
+        for n, sh in zip(sizes, shapes):
+            out.append(buf[o:o + n].view(sh))
+            o += n
+        return out
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            e2e_step()
-    stream.synchronize()
-    g = capture(e2e_step, stream)
-    n = max(1, min(args.steps, 2000))
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            g.replay()
-    stream.synchronize()
+    dx = [torch.empty_like(hx, device="cuda") for _ in range(2)]
+    dy = [torch.empty(hy.shape, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    xv = [views(dx[b], x_sizes, [c["X"].shape for c in step.calls]) for b in range(2)]
+    yv = [views(dy[b], y_sizes, [c["Y"].shape for c in step.calls]) for b in range(2)]
+    cs, xs, ys = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    graphs = []
+    for b in range(2):
+        with torch.cuda.stream(cs):
+            step.run(X_override=xv[b], Y_override=yv[b])
+        cs.synchronize()
+        graphs.append(capture(lambda b=b: step.run(X_override=xv[b], Y_override=yv[b]), cs))
+    x_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    y_free = [torch.cuda.Event() for _ in range(2)]
+
+    def one_step(k):
+        b = k % 2
+        if k >= 2:
+            xs.wait_event(done[b])        # the calls of step k-2 have read dx[b]
+        with torch.cuda.stream(xs):
+            dx[b].copy_(hx, non_blocking=True)
+        x_ready[b].record(xs)
+        cs.wait_event(x_ready[b])
+        if k >= 2:
+            cs.wait_event(y_free[b])      # step k-2's outputs have left dy[b]
+        with torch.cuda.stream(cs):
+            graphs[b].replay()
+        done[b].record(cs)
+        ys.wait_event(done[b])
+        with torch.cuda.stream(ys):
+            hy.copy_(dy[b], non_blocking=True)
+        y_free[b].record(ys)
+
+    n = max(2, min(args.steps, 2000))
+    for k in range(args.warmup):
+        one_step(k)
+    torch.cuda.synchronize()
     barrier(pg)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record()
-        for _ in range(n):
-            g.replay()
-        end.record()
+    start.record(xs)
+    cs.wait_event(start)
+    ys.wait_event(start)
+    for k in range(n):
+        one_step(k)
+    cs.wait_event(y_free[(n - 1) % 2])
+    end.record(cs)
     end.synchronize()
     ms = max_over_ranks(pg, start.elapsed_time(end))
-    # results really arrived on the host
-    assert torch.equal(hy[0], dy[0].cpu())
-    h2d = sum(t.numel() * 2 for t in hx)
-    d2h = sum(t.numel() * 2 for t in hy)
-    del g
+    # the outputs really arrived on the host: the last step's buffer
+    assert torch.equal(hy, dy[(n - 1) % 2].cpu())
+    for g in graphs:
+        del g
+    h2d = hx.numel() * 2
+    d2h = hy.numel() * 2
     return ms, n, h2d, d2h
 
 
