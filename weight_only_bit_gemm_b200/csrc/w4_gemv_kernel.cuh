@@ -58,8 +58,12 @@ struct GemvArgs {
 };
 
 // Row groups (16 rows each) per decode work unit: two share each activation
-// fragment; with four token blocks one, so that the accumulators fit.
-__host__ __device__ constexpr int gemv_row_groups(int NB) { return NB >= 4 ? 1 : 2; }
+// fragment.  Accumulator sets per (row group, token block): two alternate
+// between consecutive words so that MMAs do not wait on each other; with four
+// token blocks the blocks themselves give that independence, and one set keeps
+// the registers within budget.
+__host__ __device__ constexpr int gemv_row_groups(int) { return 2; }
+__host__ __device__ constexpr int gemv_acc_split(int NB) { return NB >= 4 ? 1 : 2; }
 
 template <int NB_, int FMT_, int G_>
 struct GemvCfg {
@@ -77,6 +81,7 @@ struct GemvCfg {
   static constexpr int kScaleBytes = FMT == kFmtInt4 ? 32 * kNq : 32;  // NF4: absmax pairs
   static constexpr int kZeroBytes = FMT == kFmtInt4 ? 8 * kNq : 0;
   static constexpr int kRG = gemv_row_groups(NB);  // row groups per work unit
+  static constexpr int kAS = gemv_acc_split(NB);  // accumulators per (row group, token block)
   static constexpr int kSlot = kRG * 1024 + (kRG * (kScaleBytes + kZeroBytes) + 15) / 16 * 16;
   static constexpr int kSmemBytes = kWarps * kDepth * kSlot;
 };
@@ -166,7 +171,7 @@ __device__ __forceinline__ void mma_words(const uint32_t (&words)[C::kRG][4],
                                           const float (&a0)[C::kRG], const float (&a1)[C::kRG],
                                           uint32_t tb,
                                           const uint16_t* const (&xs)[C::NB],
-                                          float (&acc)[C::kRG][2][C::NB][4]) {
+                                          float (&acc)[C::kRG][C::kAS][C::NB][4]) {
 #pragma unroll
   for (int w = W0; w < W0 + NW; ++w) {
     uint2 b[C::NB];
@@ -182,7 +187,7 @@ __device__ __forceinline__ void mma_words(const uint32_t (&words)[C::kRG][4],
       }
       const uint32_t afrag[4] = {pr[0], pr[2], pr[1], pr[3]};
 #pragma unroll
-      for (int nb = 0; nb < C::NB; ++nb) mma_m16n8k16_bf16(acc[rr][w & 1][nb], afrag, b[nb].x, b[nb].y);
+      for (int nb = 0; nb < C::NB; ++nb) mma_m16n8k16_bf16(acc[rr][w % C::kAS][nb], afrag, b[nb].x, b[nb].y);
     }
   }
 }
@@ -195,7 +200,7 @@ __device__ __forceinline__ uint32_t owner_of(uint32_t u, const GemvArgs& a) {
 
 template <class C>
 __device__ __forceinline__ void flush_row_group(const GemvArgs& args,
-                                                float (&acc)[C::kRG][2][C::NB][4], int rpg,
+                                                float (&acc)[C::kRG][C::kAS][C::NB][4], int rpg,
                                                 uint32_t seg0, uint32_t seg1, uint32_t wid, int lane) {
   constexpr int R = C::kRG;
   constexpr int V = R * C::NB * 4;  // floats per lane
@@ -207,9 +212,9 @@ __device__ __forceinline__ void flush_row_group(const GemvArgs& args,
     for (int nb = 0; nb < C::NB; ++nb)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        tot[rr][nb][j] = acc[rr][0][nb][j] + acc[rr][1][nb][j];
+        tot[rr][nb][j] = C::kAS == 2 ? acc[rr][0][nb][j] + acc[rr][C::kAS - 1][nb][j] : acc[rr][0][nb][j];
         acc[rr][0][nb][j] = 0.0f;
-        acc[rr][1][nb][j] = 0.0f;
+        acc[rr][C::kAS - 1][nb][j] = 0.0f;
       }
   const uint32_t rs = static_cast<uint32_t>(rpg) * static_cast<uint32_t>(args.KS);
   const uint32_t re = rs + static_cast<uint32_t>(args.KS);
@@ -276,7 +281,7 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
                                               int rpg, int st, int g,
                                               const uint16_t* const (&xrow)[C::NB],
                                               uint32_t tb,
-                                              float (&acc)[C::kRG][2][C::NB][4]) {
+                                              float (&acc)[C::kRG][C::kAS][C::NB][4]) {
   constexpr int R = C::kRG;
   const int k0 = st * kStageK;
   const uint16_t* xa[C::NB];
@@ -396,11 +401,11 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
   }
   grid_dep_wait();  // X, Y and the workspace may belong to the previous kernel
 
-  float acc[R][2][C::NB][4];
+  float acc[R][C::kAS][C::NB][4];
 #pragma unroll
   for (int rr = 0; rr < R; ++rr)
 #pragma unroll
-    for (int e = 0; e < 2; ++e)
+    for (int e = 0; e < C::kAS; ++e)
 #pragma unroll
       for (int nb = 0; nb < C::NB; ++nb)
 #pragma unroll
