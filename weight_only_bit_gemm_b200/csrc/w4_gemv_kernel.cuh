@@ -58,12 +58,12 @@ struct GemvArgs {
 };
 
 // Row groups (16 rows each) per decode work unit: two share each activation
-// fragment.  Accumulator sets per (row group, token block): two alternate
-// between consecutive words so that MMAs do not wait on each other; with four
-// token blocks the blocks themselves give that independence, and one set keeps
-// the registers within budget.
+// fragment.  Accumulator sets per (row group, token block): with one token
+// block two alternate between consecutive words so that MMAs do not wait on
+// each other; with two or four token blocks the blocks themselves give that
+// independence, and one set keeps the registers within budget.
 __host__ __device__ constexpr int gemv_row_groups(int) { return 2; }
-__host__ __device__ constexpr int gemv_acc_split(int NB) { return NB >= 4 ? 1 : 2; }
+__host__ __device__ constexpr int gemv_acc_split(int NB) { return NB >= 2 ? 1 : 2; }
 
 template <int NB_, int FMT_, int G_>
 struct GemvCfg {
