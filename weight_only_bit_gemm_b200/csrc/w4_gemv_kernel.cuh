@@ -55,6 +55,7 @@ struct GemvArgs {
   uint32_t q, r;            // units per warp: q + (w < r)
   FastDiv32 by_ks, by_q, by_q1;
   FastDivIdx by_dq;          // NF4: 64-block index -> s2 index
+  int dq_group;             // NF4: 64-blocks per second-level scale
 };
 
 // Row groups (16 rows each) per decode work unit: two share each activation
@@ -276,11 +277,23 @@ __device__ __forceinline__ void flush_row_group(const GemvArgs& args,
   }
 }
 
+// NF4: per row of the lane, the second-level scale it last looked up and the
+// run of 64-blocks (relative to the row's first block) that scale covers.
+// Consecutive stages of a row stay in one run for up to dq_group blocks, so a
+// scale is loaded once per run instead of once per stage, off the critical
+// path of every other stage.
+template <class C>
+struct S2Cache {
+  int rpg = -1;
+  int lo[C::kRG][2], hi[C::kRG][2];
+  float v[C::kRG][2];
+};
+
 template <class C>
 __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageRegs<C>& cur,
                                               int rpg, int st, int g,
                                               const uint16_t* const (&xrow)[C::NB],
-                                              uint32_t tb,
+                                              uint32_t tb, S2Cache<C>& sc,
                                               float (&acc)[C::kRG][C::kAS][C::NB][4]) {
   constexpr int R = C::kRG;
   const int k0 = st * kStageK;
@@ -320,24 +333,42 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
       }
     }
   } else {
-    const unsigned long long kb64 = static_cast<unsigned long long>(args.K / 64);
+    const int kb64 = args.K / 64;
+    if (sc.rpg != rpg) {  // a new row group unit: forget the runs
+      sc.rpg = rpg;
+#pragma unroll
+      for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          sc.lo[rr][hf] = 0;
+          sc.hi[rr][hf] = 0;
+          sc.v[rr][hf] = 0.0f;
+        }
+    }
     float a0[2][R], a1[2][R];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const unsigned long long blk = static_cast<unsigned long long>(st) * 2 + h;
+      const int blk = st * 2 + h;
 #pragma unroll
       for (int rr = 0; rr < R; ++rr) {
-        a0[h][rr] = 0.0f;
-        a1[h][rr] = 0.0f;
-        const int r0 = (rpg * R + rr) * 16 + g;
-        if (blk < kb64) {
-          const uint32_t pair = h == 0 ? cur.sp[rr][0] : cur.zp[rr][0];
-          if (r0 < args.N)
-            a0[h][rr] = __fmul_rn(static_cast<float>(pair & 0xFFu),
-                                  __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0) * kb64 + blk, args.by_dq)));
-          if (r0 + 8 < args.N)
-            a1[h][rr] = __fmul_rn(static_cast<float>(pair >> 8),
-                                  __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0 + 8) * kb64 + blk, args.by_dq)));
+        const uint32_t pair = h == 0 ? cur.sp[rr][0] : cur.zp[rr][0];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int r = (rpg * R + rr) * 16 + g + 8 * hf;
+          float a = 0.0f;
+          if (blk < kb64 && r < args.N) {
+            if (blk < sc.lo[rr][hf] || blk >= sc.hi[rr][hf]) {
+              const unsigned long long rowb = static_cast<unsigned long long>(r) * kb64;
+              const unsigned long long idx = fast_div(rowb + static_cast<unsigned long long>(blk), args.by_dq);
+              sc.v[rr][hf] = __ldg(args.s2 + idx);
+              const long long lo = static_cast<long long>(idx * static_cast<unsigned long long>(args.dq_group)) -
+                                   static_cast<long long>(rowb);
+              sc.lo[rr][hf] = static_cast<int>(lo);
+              sc.hi[rr][hf] = static_cast<int>(lo + args.dq_group);
+            }
+            a = __fmul_rn(static_cast<float>(hf == 0 ? (pair & 0xFFu) : (pair >> 8)), sc.v[rr][hf]);
+          }
+          if (hf == 0) a0[h][rr] = a; else a1[h][rr] = a;
         }
       }
     }
@@ -411,6 +442,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[rr][e][nb][j] = 0.0f;
 
+  S2Cache<C> s2c;  // NF4 only (unused, and removed, for INT4)
   int rpg = rpg0, st = st0;
   uint32_t seg0 = ua;
   int cs = 0;
@@ -426,7 +458,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
     }
     cp_async_commit();
     cs = cs + 1 == C::kDepth ? 0 : cs + 1;
-    stage_compute<C>(args, cur, rpg, st, g, xrow, smem_u32(Ts), acc);
+    stage_compute<C>(args, cur, rpg, st, g, xrow, smem_u32(Ts), s2c, acc);
     if (st == KS - 1 || n + 1 == left) {
       const uint32_t seg1 = ua + static_cast<uint32_t>(n) + 1;
       flush_row_group<C>(args, acc, rpg, seg0, seg1, wid, lane);
