@@ -99,17 +99,6 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint3
       : "memory");
 }
 
-// 2-D tiled tensor copy global -> shared (no multicast).  c0 is the inner
-// (contiguous) coordinate in elements, c1 the row.
-__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c0,
-                                            int c1, uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-
 // 3-D tiled tensor copy global -> shared (no multicast).
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int c0,
                                             int c1, int c2, uint64_t* bar, uint64_t policy) {
@@ -167,19 +156,6 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
-// Each thread of the warp stores 32 consecutive 32-bit columns of its lane.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
-      "%29, %30, %31, %32};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
-      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
-      "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
-}
 // 16 lanes x 256 bits, repeated 4 times along the columns: thread (g = t/4,
 // u = t%4) writes lanes base+g and base+g+8, columns 8r+2u and 8r+2u+1 of
 // repetition r, from v[4r+0..1] (lane g) and v[4r+2..3] (lane g+8).
@@ -278,11 +254,6 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned int* p, unsign
   unsigned int old;
   asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
-}
-
-// Named barrier among a subset of warps.
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ------------------------------------------------------ UMMA descriptors
