@@ -33,6 +33,11 @@ R9  NF4 dequant is ``bf16(fp32(T[q] * absmax'))``.
 
 All floating-point steps are numpy float32 operations (IEEE, round to nearest
 even) unless stated as fp64; the matmul accumulates in fp64.
+
+Parity unpinned: the exact NF4 level values.  The pages print no table; the
+tests pin what they do fix (16 levels, strictly increasing, an exact zero,
+-1 and +1 at the ends, spacing smallest near zero), not the digits of R6's
+construction, so agreement with any other NF4 table is not claimed.
 """
 from __future__ import annotations
 
