@@ -294,9 +294,12 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
   }
 }
 
-// act-order: X'[m, j] = X[m, perm[j]]
+// act-order: X'[m, j] = X[m, perm[j]].  The GEMM launched after it may start
+// at once (programmatic dependent launch) and stream its weights while this
+// runs; it reads X' only after its dependency wait.
 __global__ void gather_x_kernel(const uint16_t* __restrict__ X, const int32_t* __restrict__ perm,
                                 int M, int K, uint16_t* __restrict__ Xp) {
+  grid_dep_launch();
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   const int m = blockIdx.y;
   if (j < K && m < M) Xp[static_cast<size_t>(m) * K + j] = X[static_cast<size_t>(m) * K + perm[j]];
