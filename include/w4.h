@@ -70,6 +70,13 @@ int w4_version(void);
  * W4_ERR_DEVICE_INPUT (or W4_ERR_CUDA if the synchronisation itself failed). */
 w4_status w4_device_status(w4_stream stream);
 
+/* Failure-path check (no counterpart on the pages): launches one thread that
+ * runs this library's bounded pipeline wait on a barrier nothing arrives on,
+ * with a limit of about 1 ms instead of the kernels' 2 s.  The wait gives up,
+ * sets the device error word and returns; the next w4_device_status(stream)
+ * returns W4_ERR_TIMEOUT and the context stays usable.  Nothing faults. */
+w4_status w4_selftest_wait_timeout(w4_stream stream);
+
 /* ------------------------------------------------------------------------
  * INT4 asymmetric round-to-nearest quantization, group-wise along K.
  * [Comparison] §2.3: scale = (max - min) / (2^b - 1), zero_point =

@@ -261,3 +261,16 @@ def test_workspace_shared_across_shapes(w4):
             _check(y, xb, what)
     # the counter region is left zeroed
     assert int(ws[: 65536 * 4].count_nonzero()) == 0
+
+
+def test_bounded_wait_times_out_and_context_survives(w4):
+    # a pipeline wait on a barrier that nothing arrives on gives up, reports
+    # W4_ERR_TIMEOUT through the device error word, and leaves the context usable
+    w4.selftest_wait_timeout()
+    assert w4.device_status() == w4.W4_ERR_TIMEOUT
+    assert w4.device_status() == w4.W4_OK          # the word was cleared
+    what, Wp = _int4_layer(w4, 256, 512, 128, False, seed=4)
+    xb = S.draw_x(4, 512, seed=4, tag=2, N=256)
+    y = w4.w4a16_gemm(x_dev(xb), Wp, 256, 512, 128)
+    status_ok(w4)
+    _check(y, xb, what)

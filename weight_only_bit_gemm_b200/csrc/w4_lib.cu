@@ -32,6 +32,21 @@ bool int4_shape_ok(int N, int K, int G) {
          static_cast<long long>(N) * K <= (1LL << 40);
 }
 
+// Failure-path check: one bounded wait on an mbarrier that nothing arrives
+// on, with a short limit (about 1 ms): it must give up, set the device error
+// word and return, leaving the context usable.
+constexpr long long kSelftestWaitCycles = 2000000;
+
+__global__ void wait_timeout_probe_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, limit);
+}
+
 }  // namespace
 
 extern "C" {
@@ -63,6 +78,11 @@ w4_status w4_device_status(w4_stream stream) {
   if (v & W4_DEV_ERR_TIMEOUT) return W4_ERR_TIMEOUT;
   if (v & W4_DEV_ERR_INPUT) return W4_ERR_DEVICE_INPUT;
   return W4_OK;
+}
+
+w4_status w4_selftest_wait_timeout(w4_stream stream) {
+  wait_timeout_probe_kernel<<<1, 32, 0, as_stream(stream)>>>(kSelftestWaitCycles);
+  return launch_status(cudaGetLastError());
 }
 
 double w4_weight_bytes(int N, int K, int G) {

@@ -31,6 +31,7 @@ _SIGS = {
     "w4_status_string": (ctypes.c_char_p, [_i]),
     "w4_version": (_i, []),
     "w4_device_status": (_i, [_p]),
+    "w4_selftest_wait_timeout": (_i, [_p]),
     "w4_weight_bytes": (ctypes.c_double, [_i, _i, _i]),
     "w4_quantize_rtn": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p]),
     "w4_dequant": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
@@ -94,6 +95,12 @@ def _cuda(t, dtype, name):
 def device_status() -> int:
     """Synchronise the current stream and return/clear the device error word."""
     return lib.w4_device_status(_stream())
+
+
+def selftest_wait_timeout() -> None:
+    """Run the bounded-wait failure path once (see w4.h); device_status() then
+    reports W4_ERR_TIMEOUT."""
+    _check(lib.w4_selftest_wait_timeout(_stream()), "w4_selftest_wait_timeout")
 
 
 # ----------------------------------------------------------------- INT4 RTN
