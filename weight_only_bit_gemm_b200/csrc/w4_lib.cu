@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -26,6 +27,20 @@ inline bool aligned(const void* p, uintptr_t a) {
 inline bool valid_group(int G) { return G == 32 || G == 64 || G == 128; }
 inline w4_status launch_status(cudaError_t e) { return e == cudaSuccess ? W4_OK : W4_ERR_CUDA; }
 inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+// A kernel's dynamic shared-memory limit is a per-device setting: raise it
+// once on each device the kernel runs on (`done` holds one bit per device).
+template <class Kernel>
+cudaError_t ensure_smem_limit(Kernel* kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 bool int4_shape_ok(int N, int K, int G) {
   return N >= 1 && K >= 1 && valid_group(G) && K >= G && K % G == 0 && K % 2 == 0 &&
@@ -101,11 +116,11 @@ w4_status w4_quantize_rtn(const float* W, int N, int K, int G, const int32_t* g_
   const int ng = K / G;
   const size_t smem = static_cast<size_t>(ng) * 16;
   if (smem > 200 * 1024) return W4_ERR_UNSUPPORTED;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(rtn_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         200 * 1024);
-  });
+  static std::atomic<uint64_t> smem_set{0};
+  if (ensure_smem_limit(rtn_quantize_kernel, 200 * 1024, smem_set) != cudaSuccess) {
+    cudaGetLastError();
+    return W4_ERR_CUDA;
+  }
   rtn_quantize_kernel<<<N, 256, smem, as_stream(stream)>>>(W, N, K, G, g_idx, Wq, scales, zeros);
   return launch_status(cudaGetLastError());
 }
