@@ -1,5 +1,6 @@
-"""Oracle: group-wise INT4 (asymmetric, RTN) and NF4 (double-quantized) weight
-quantization, packing, dequantization and the fp64 matmul reference.
+"""Oracle: group-wise INT4 (asymmetric and symmetric RTN) and NF4
+(double-quantized) weight quantization, the AWQ per-input-channel factor,
+packing, dequantization and the fp64 matmul reference.
 
 TEST INFRASTRUCTURE ONLY -- see the package docstring for who may import it.
 
@@ -29,7 +30,12 @@ R7  an NF4 value on a midpoint takes the lower code;
 R8  double quantization: per run of 256 consecutive blocks,
     ``s2 = max(absmax) / 255``, ``c = rint(absmax / s2)`` in [0, 255],
     ``absmax' = c * s2`` in fp32; codes are chosen with the unquantized absmax;
-R9  NF4 dequant is ``bf16(fp32(T[q] * absmax'))``.
+R9  NF4 dequant is ``bf16(fp32(T[q] * absmax'))``;
+R10 symmetric INT4: ``scale = fp16(max|w| / 7)``, codes ``rint(w / scale)``
+    clamped to [-7, 7] and stored + 8 (zero point 8, code 0 unused);
+R11 AWQ: the factor s is an input (found offline); weights enter
+    quantization as the fp32 product ``w * s_k``, activations the GEMM as
+    ``bf16(fp32(x / s_k))``.
 
 All floating-point steps are numpy float32 operations (IEEE, round to nearest
 even) unless stated as fp64; the matmul accumulates in fp64.
@@ -54,6 +60,7 @@ __all__ = [
     "nf4_codes", "nf4_double_quant", "nf4_quantize", "nf4_dequant", "matmul_ref",
     "matmul_exact_small", "ulp_bf16", "tolerance", "check_matmul",
     "weight_bytes", "code_bytes", "nf4_weight_bytes",
+    "sym_params", "quantize_sym", "awq_scale_weights", "awq_scale_activations",
 ]
 
 F32 = np.float32
@@ -155,6 +162,67 @@ def quantize_rtn(W: np.ndarray, G: int, g_idx: np.ndarray | None = None):
     zk = zp.astype(F32)[:, gk]
     q = np.clip(np.rint(W / sk) + zk, 0, 15)
     return q.astype(np.uint8), s16, zp
+
+
+# ---------------------------------------------------------------------------
+# Symmetric (absmax) quantization.  [Comparison] §2.3 gives the symmetric form
+# for 8 bits: scale = max|w| / 127, values in [-127, 127]; [Survey] §1's worked
+# example divides a maximum of 80 by 127.  With b bits the levels are
+# [-(2^(b-1) - 1), 2^(b-1) - 1].  For b = 4 the code stored is q + 8 in
+# [1, 15] with zero point 8, the same canonical format as asymmetric RTN, so
+# dequant and the GEMM take it unchanged.  Readings: the scale is stored in
+# fp16 like the asymmetric one (R2), a zero scale becomes 1.0, round half to
+# even (R3).
+# ---------------------------------------------------------------------------
+
+def sym_params(W: np.ndarray, G: int, g_idx: np.ndarray | None = None, bits: int = 4):
+    """Per (row, group) fp32 scale max|w| / (2^(bits-1) - 1) and its fp16 value.
+
+    Returns (scale_fp32 [N, K/G], scale_fp16 [N, K/G])."""
+    W = np.ascontiguousarray(W, dtype=F32)
+    N, K = W.shape
+    gk = group_index(K, G, g_idx)
+    mn, mx = _group_minmax(W, G, gk, g_idx is None)
+    amax = np.maximum(np.abs(mn), np.abs(mx))
+    qmax = F32(2 ** (bits - 1) - 1)
+    s32 = amax / qmax
+    s16 = s32.astype(np.float16)
+    s16[s16 == 0] = np.float16(1.0)
+    return s32, s16
+
+
+def quantize_sym(W: np.ndarray, G: int, g_idx: np.ndarray | None = None):
+    """4-bit symmetric codes: q = clamp(round(w / scale), -7, 7), stored q + 8.
+
+    Returns (codes uint8 [N, K] in [1, 15], scale fp16 [N, K/G], zero uint8
+    [N, K/G] = 8)."""
+    W = np.ascontiguousarray(W, dtype=F32)
+    N, K = W.shape
+    gk = group_index(K, G, g_idx)
+    _, s16 = sym_params(W, G, g_idx, 4)
+    sk = s16.astype(F32)[:, gk]
+    q = np.clip(np.rint(W / sk), -7, 7) + 8
+    return q.astype(np.uint8), s16, np.full(s16.shape, 8, np.uint8)
+
+
+# ---------------------------------------------------------------------------
+# AWQ per-input-channel factor.  [Survey] §4.1 and [Comparison] §4.1: the
+# weights are quantized as W * s (a factor s_k > 0 per input channel, found
+# offline) and the activations enter as X / s, so (X / s)(W s)^T = X W^T
+# before quantization; the runtime is the same W4A16 GEMM.  Readings: W * s is
+# an fp32 product, X / s an fp32 division of the bf16 value, each rounded to
+# nearest even (the latter then to bf16).
+# ---------------------------------------------------------------------------
+
+def awq_scale_weights(W: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """W[n, k] * s[k] in fp32."""
+    return (np.asarray(W, dtype=F32) * np.asarray(s, dtype=F32)[None, :]).astype(F32)
+
+
+def awq_scale_activations(x_bits: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """bf16 bits of fp32(x[m, k] / s[k])."""
+    x = bf16_bits_to_f32(x_bits)
+    return bf16_round_bits((x / np.asarray(s, dtype=F32)[None, :]).astype(F32))
 
 
 def pack_nibbles(codes: np.ndarray) -> np.ndarray:

@@ -221,6 +221,129 @@ def test_g_idx_validation():
         O.quantize_rtn(W, 32, np.full(64, -1, np.int32))
 
 
+# ---------------------------------------------------------------- symmetric INT4
+
+SYM_WORKED = _parse_worked(os.path.join(GOLDEN, "int4_sym_worked.txt"))
+
+
+def test_sym_page_worked_example():
+    # [Survey] §1: a largest magnitude of 80 gives an 8-bit symmetric scale of
+    # 80/127, about 0.63; the sign of the extreme does not matter (absmax)
+    for ext in (80.0, -80.0):
+        w = np.array([[ext, 3.0, -1.0, 0.5]], np.float32)
+        s32, _ = O.sym_params(w, 4, bits=8)
+        assert abs(float(s32[0, 0]) - 0.63) < 0.005
+        assert float(s32[0, 0]) == float(np.float32(80.0) / np.float32(127.0))
+
+
+@pytest.mark.parametrize("case", SYM_WORKED, ids=lambda c: c["name"])
+def test_sym_worked_examples(case):
+    G = int(case["G"][0])
+    w = np.array([float(v) for v in case["w"]], np.float32)[None, :]
+    codes, s16, zp = O.quantize_sym(w, G)
+    assert s16.view(np.uint16)[0, 0] == int(case["scale_f16_bits"][0], 16)
+    assert np.all(zp == 8)
+    assert codes[0].tolist() == [int(v) for v in case["codes"]]
+    packed = O.pack_nibbles(codes)
+    assert packed[0].tolist() == [int(v, 16) for v in case["packed_hex"]]
+    what = O.bf16_bits_to_f32(O.dequant_rtn(packed, s16, zp, G))
+    assert what[0].tolist() == [float(v) for v in case["what"]]
+
+
+@pytest.mark.parametrize("G", [32, 128])
+def test_sym_bound_symmetry_and_nearest_level(G):
+    W = _rand_w(48, 512, 40 + G)
+    W[2, :G] = 0.0
+    q, s16, zp = O.quantize_sym(W, G)
+    assert q.min() >= 1 and q.max() <= 15 and np.all(zp == 8)
+    gk = np.arange(W.shape[1]) // G
+    sf = s16.astype(np.float64)[:, gk]
+    # max|w| of each group lands on code 1 or 15; every weight is within half
+    # a step (fp16 rounding of the scale moves the ends by at most 7 * 2^-11)
+    what = O.dequant_rtn_f32(O.pack_nibbles(q), s16, zp, G)
+    err = np.abs(W.astype(np.float64) - what)
+    assert np.all(err <= sf * (0.5 + 7 * 2.0 ** -11))
+    Wg, qg = W.reshape(48, -1, G), q.reshape(48, -1, G)
+    amax_at = np.abs(Wg).argmax(-1)[..., None]
+    qa = np.take_along_axis(qg, amax_at, -1)[..., 0]
+    nz = np.abs(Wg).max(-1) > 0
+    assert np.all((qa[nz] == 1) | (qa[nz] == 15))
+    # zero group -> scale 1.0 and every code 8
+    assert s16[2, 0] == np.float16(1.0) and np.all(q[2, :G] == 8)
+    # negating W mirrors every code about the zero point: rint(-t) = -rint(t)
+    qn, sn, _ = O.quantize_sym(-W, G)
+    assert np.array_equal(sn, s16) and np.array_equal(qn.astype(int), 16 - q.astype(int))
+    # brute force on a slice: the code is a nearest of the 15 levels in units
+    # of the scale, ties to the even integer
+    for n in range(4):
+        for k in range(0, 512, 7):
+            t = float(np.float32(W[n, k]) / np.float32(sf[n, k]))
+            dist = [abs(t - (lv - 8)) for lv in range(1, 16)]
+            best = min(dist)
+            cands = [lv for lv, d in zip(range(1, 16), dist) if abs(d - best) < 1e-12]
+            pick = cands[0] if len(cands) == 1 else [c for c in cands if (c - 8) % 2 == 0][0]
+            assert int(q[n, k]) == pick
+
+
+def test_sym_act_order_equals_permuted_contiguous():
+    K, G = 256, 64
+    W = _rand_w(10, K, 41)
+    perm = S.draw_perm(K, seed=2, tag=5, N=10)
+    g_idx = S.act_order_g_idx(perm, G)
+    q, s, z = O.quantize_sym(W, G, g_idx)
+    qp, sp, zpp = O.quantize_sym(W[:, perm], G)
+    assert np.array_equal(q[:, perm], qp)
+    assert np.array_equal(s, sp) and np.array_equal(z, zpp)
+
+
+# ---------------------------------------------------------------- AWQ factor
+
+def test_awq_identity_and_powers_of_two():
+    W = _rand_w(8, 256, 42)
+    xb = S.draw_x(4, 256, seed=3)
+    one = np.ones(256, np.float32)
+    assert np.array_equal(O.awq_scale_weights(W, one), W)
+    assert np.array_equal(O.awq_scale_activations(xb, one), xb)
+    # a power of two changes only the exponent: exact on both sides
+    s = np.where(np.arange(256) % 3 == 0, 2.0, 0.5).astype(np.float32)
+    ws = O.awq_scale_weights(W, s)
+    assert np.array_equal(ws, W * s[None, :])
+    xs = O.bf16_bits_to_f32(O.awq_scale_activations(xb, s))
+    assert np.array_equal(xs, O.bf16_bits_to_f32(xb) / s[None, :])
+
+
+def test_awq_product_invariance():
+    # [Survey] §4.1: (W s)(X / s) leaves the product unchanged; with bf16
+    # activations the only change is one bf16 rounding of each x / s
+    rng = np.random.default_rng(7)
+    M, N, K = 3, 5, 192
+    W = _rand_w(N, K, 43)
+    s = rng.uniform(0.5, 2.0, K).astype(np.float32)   # not a power of two
+    xb = S.draw_x(M, K, seed=4)
+    x = O.bf16_bits_to_f32(xb).astype(np.float64)
+    xs = O.bf16_bits_to_f32(O.awq_scale_activations(xb, s)).astype(np.float64)
+    ws = O.awq_scale_weights(W, s).astype(np.float64)
+    y0 = x @ W.astype(np.float64).T
+    y1 = xs @ ws.T
+    bound = (np.abs(x) @ np.abs(W.astype(np.float64)).T) * (2.0 ** -8 + 2.0 ** -22)
+    assert np.all(np.abs(y1 - y0) <= bound)
+
+
+def test_awq_effective_weight_follows_page_formula():
+    # [Comparison] §4.1: the weight X sees is round(W s / scale) scale / s,
+    # so its error is at most half a step of the scaled group, divided by s_k
+    rng = np.random.default_rng(8)
+    N, K, G = 16, 256, 64
+    W = _rand_w(N, K, 44)
+    s = rng.uniform(0.95, 1.05, K).astype(np.float32)
+    q, s16, zp = O.quantize_rtn(O.awq_scale_weights(W, s), G)
+    f = O.dequant_rtn_f32(O.pack_nibbles(q), s16, zp, G)
+    eff = f / s[None, :].astype(np.float64)
+    step = s16.astype(np.float64)[:, np.arange(K) // G]
+    bound = step * (0.5 + 15 * 2.0 ** -11) / s[None, :] + np.abs(W) * 2.0 ** -22
+    assert np.all(np.abs(eff - W.astype(np.float64)) <= bound)
+
+
 # ---------------------------------------------------------------- NF4
 
 def test_nf4_table_invariants():
@@ -436,3 +559,66 @@ def test_planted_mistakes(monkeypatch):
         return np.floor(a / s).astype(np.uint8), s2
     assert _pins_fail(monkeypatch, "nf4_double_quant", dq_truncating)
     monkeypatch.undo()
+
+
+def test_planted_mistakes_sym_and_awq(monkeypatch):
+    import oracle.w4_oracle as M
+
+    def caught(name, fn, checks):
+        monkeypatch.setattr(M, name, fn)
+        monkeypatch.setattr(O, name, fn)
+        try:
+            for chk in checks:
+                try:
+                    chk()
+                except AssertionError:
+                    return True
+            return False
+        finally:
+            monkeypatch.undo()
+
+    sym_checks = [
+        lambda: [test_sym_worked_examples(c) for c in SYM_WORKED],
+        lambda: test_sym_bound_symmetry_and_nearest_level(32),
+        test_sym_page_worked_example,
+    ]
+    orig_params = M.sym_params
+
+    def over_eight(W, G, g_idx=None, bits=4):      # 2^(b-1) instead of 2^(b-1) - 1
+        s32, _ = orig_params(W, G, g_idx, bits)
+        q = 2.0 ** (bits - 1)
+        s32 = (s32 * np.float32(2 ** (bits - 1) - 1) / np.float32(q)).astype(np.float32)
+        s16 = s32.astype(np.float16)
+        s16[s16 == 0] = np.float16(1.0)
+        return s32, s16
+    assert caught("sym_params", over_eight, sym_checks)
+
+    def signed_max(W, G, g_idx=None, bits=4):      # max(w) instead of max|w|
+        W = np.ascontiguousarray(W, np.float32)
+        gk = M.group_index(W.shape[1], G, g_idx)
+        _, mx = M._group_minmax(W, G, gk, g_idx is None)
+        s32 = (mx / np.float32(2 ** (bits - 1) - 1)).astype(np.float32)
+        s16 = s32.astype(np.float16)
+        s16[s16 == 0] = np.float16(1.0)
+        return s32, s16
+    assert caught("sym_params", signed_max, sym_checks)
+
+    def sym_floor(W, G, g_idx=None):
+        W = np.ascontiguousarray(W, np.float32)
+        gk = M.group_index(W.shape[1], G, g_idx)
+        _, s16 = M.sym_params(W, G, g_idx, 4)
+        q = np.clip(np.floor(W / s16.astype(np.float32)[:, gk] + np.float32(0.5)), -7, 7) + 8
+        return q.astype(np.uint8), s16, np.full(s16.shape, 8, np.uint8)
+    assert caught("quantize_sym", sym_floor, sym_checks)
+
+    awq_checks = [test_awq_identity_and_powers_of_two, test_awq_product_invariance,
+                  test_awq_effective_weight_follows_page_formula]
+
+    def x_times_s(x_bits, s):
+        x = M.bf16_bits_to_f32(x_bits)
+        return M.bf16_round_bits((x * np.asarray(s, np.float32)[None, :]).astype(np.float32))
+    assert caught("awq_scale_activations", x_times_s, awq_checks)
+
+    def w_over_s(W, s):
+        return (np.asarray(W, np.float32) / np.asarray(s, np.float32)[None, :]).astype(np.float32)
+    assert caught("awq_scale_weights", w_over_s, awq_checks)
