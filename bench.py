@@ -476,6 +476,43 @@ def measure_rows(w4, peaks):
     ts = time_calls(big_calls, reps=5)
     rows["act_order_m256"] = {"configs": "M=256, G=32", "TFLOP/s": sum(big_flops) / sum(ts) / 1e9}
 
+    # NEXT row: symmetric INT4 after the AWQ factor (decode shapes of Llama-7B)
+    aw = S.AWQ_SYM_DECODE
+    awq_calls, plain_calls, awq_bytes = [], [], []
+    for (K, N) in aw["shapes"]:
+        G = aw["G"]
+        W = torch.from_numpy(S.layer_w(aw, K, N)).cuda()
+        sd = torch.from_numpy(S.layer_awq_s(aw, K, N)).cuda()
+        Ws = w4.awq_scale_weights(W, sd)
+        Wq, sc, zr = w4.quantize_sym(Ws, G)
+        if (K, N) == (4096, 22016):
+            t = time_calls([lambda: w4.awq_scale_weights(W, sd, out=Ws)], reps=5)[0]
+            b = 2 * N * K * 4 + K * 4
+            rows["awq_scale_weights"] = {"shape": [N, K], "ms": t, "GB/s": b / t / 1e6,
+                                         "frac_of_hbm": b / t / 1e6 / hbm}
+            t = time_calls([lambda: w4.quantize_sym(Ws, G)], reps=5)[0]
+            qb = N * K * 4 + N * K / 2 + N * (K // G) * 3
+            rows["quantize_sym"] = {"shape": [N, K], "G": G, "ms": t, "GB/s": qb / t / 1e6,
+                                    "frac_of_hbm": qb / t / 1e6 / hbm}
+        wp = w4.prepack(Wq, sc, zr, G)
+        reps = [wp] + [wp.clone() for _ in range(_replicas_for(wp.numel(), l2) - 1)]
+        for M in aw["Ms"]:
+            X = bf16_dev(S.layer_x(aw, M, K, N))
+            for r in reps:
+                awq_calls.append(lambda X=X, r=r, N=N, K=K, G=G, sd=sd:
+                                 w4.w4a16_awq_gemm(X, sd, r, N, K, G))
+                plain_calls.append(lambda X=X, r=r, N=N, K=K, G=G: w4.w4a16_gemm(X, r, N, K, G))
+                awq_bytes.append(int4_bytes(M, N, K, G) + 4 * K)
+        del W, Ws, Wq, sc, zr
+    ts = time_calls(awq_calls, reps=5)
+    tp = time_calls(plain_calls, reps=5)
+    rows["awq_sym_decode"] = {
+        "configs": "(K,N) in {(4096,12288),(4096,4096),(4096,22016),(11008,4096)} x M in {1,4,16}, "
+                   "G=128, symmetric codes, AWQ factor on X",
+        "TB/s": sum(awq_bytes) / sum(ts) / 1e9,
+        "frac_of_hbm": sum(awq_bytes) / sum(ts) / 1e6 / hbm,
+        "same_weights_without_factor_TB/s": sum(awq_bytes) / sum(tp) / 1e9}
+
     # a8: prefill tensor-core GEMM (70B MLP shapes)
     pf = S.PREFILL_70B
     out = {}
@@ -590,6 +627,16 @@ def run_single(w4, args):
         X = bf16_dev(S.layer_x(S.NF4_DECODE, M, K, N))
         f = (lambda: w4.nf4_gemm(X, wp, s2, N, K))
         nbytes, flops = nf4_bytes(M, N, K), 2.0 * M * N * K
+    elif fmt == "awq":
+        aw = S.AWQ_SYM_DECODE
+        G = aw["G"]
+        W = torch.from_numpy(S.layer_w(aw, K, N)).cuda()
+        sd = torch.from_numpy(S.layer_awq_s(aw, K, N)).cuda()
+        Wq, sc, zr = w4.quantize_sym(w4.awq_scale_weights(W, sd), G)
+        wp = w4.prepack(Wq, sc, zr, G)
+        X = bf16_dev(S.layer_x(aw, M, K, N))
+        f = (lambda: w4.w4a16_awq_gemm(X, sd, wp, N, K, G))
+        nbytes, flops = int4_bytes(M, N, K, G) + 4 * K, 2.0 * M * N * K
     else:
         G = WL["G"]
         W = torch.from_numpy(S.layer_w(WL, K, N)).cuda()
@@ -615,7 +662,7 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the other-row measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--single", nargs=4, metavar=("FMT", "K", "N", "M"),
-                    help="profiling aid: run one layer call (FMT int4|nf4) warmup+steps times "
+                    help="profiling aid: run one layer call (FMT int4|nf4|awq) warmup+steps times "
                          "eagerly and print its mean device time")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -103,6 +103,40 @@ w4_status w4_quantize_rtn(const float* W, int N, int K, int G, const int32_t* g_
                           uint8_t* Wq, uint16_t* scales, uint8_t* zeros,
                           w4_stream stream);
 
+/* INT4 symmetric (absmax) quantization, group-wise along K, in the same
+ * canonical format as w4_quantize_rtn (so w4_dequant, w4_prepack and
+ * w4a16_gemm take it unchanged).  [Comparison] §2.3: symmetric scale =
+ * max|w| / (2^(b-1) - 1), values in [-(2^(b-1) - 1), 2^(b-1) - 1] (printed
+ * for b = 8: /127; [Survey] §1 works 80 / 127 = 0.63); here b = 4:
+ *   scale = fp16(max_k |w_k| / 7), or 1.0 if that is 0
+ *   q_k = clamp(rint(w_k / scale), -7, 7) + 8      (codes 1..15; 0 unused)
+ *   zero point = 8 for every group
+ * Arguments, group definition (g_idx), error behaviour and preconditions as
+ * for w4_quantize_rtn, with max|w| / 7 < 65520 in every group. */
+w4_status w4_quantize_sym(const float* W, int N, int K, int G, const int32_t* g_idx,
+                          uint8_t* Wq, uint16_t* scales, uint8_t* zeros,
+                          w4_stream stream);
+
+/* AWQ per-input-channel factor ([Survey] §4.1, [Comparison] §4.1): the
+ * weights of input channel k are quantized as w * s_k and the activations
+ * enter the product as x / s_k, so (X / s)(W s)^T = X W^T before
+ * quantization; the effective weight is round(W s / scale) scale / s.  s is
+ * an input (found offline by the calibration search the pages describe).
+ *   W      in   fp32 [N, K]
+ *   s      in   fp32 [K], finite and nonzero (not checked)
+ *   W_out  out  fp32 [N, K] = fp32(W[n, k] * s[k]) (round to nearest even);
+ *               may be W itself
+ * Quantize W_out with w4_quantize_rtn or w4_quantize_sym, then prepack. */
+w4_status w4_awq_scale_weights(const float* W, const float* s, int N, int K, float* W_out,
+                               w4_stream stream);
+
+/* X_out[m, k] = bf16_rne(fp32(X[m, k]) / s[k]) (IEEE division): the
+ * activation side of the AWQ factor, as w4a16_awq_gemm applies it.
+ *   X, X_out  bf16 [M, K], 16-byte aligned, K % 8 == 0; X_out may be X
+ *   s         fp32 [K], 16-byte aligned                                    */
+w4_status w4_awq_scale_activations(const uint16_t* X, const float* s, int M, int K,
+                                   uint16_t* X_out, w4_stream stream);
+
 /* Dequantization to the bf16 compute dtype ([Survey] §6.2, [Primer] §七):
  *   w_hat[n,k] = bf16_rne( float(q - zp) * float(scale) )
  * (the fp32 product is exact, so there is exactly one rounding).
@@ -177,6 +211,21 @@ size_t w4_workspace_bytes(int M, int N, int K, int G, int act_order);
 w4_status w4a16_gemm(const uint16_t* X, const uint8_t* Wp, int M, int N, int K, int G,
                      int act_order, uint16_t* Y, void* workspace, size_t workspace_bytes,
                      w4_stream stream);
+
+/* ------------------------------------------------------------------------
+ * W4A16 linear for AWQ weights: Y = (X / s) . w_hat^T, with w_hat from
+ * weights quantized as W s (w4_awq_scale_weights).  The division is done
+ * once, by a prologue kernel that writes bf16(x / s_k) into the workspace
+ * (the same pass that applies the act-order permutation), and the weight
+ * stream and GEMM kernels are w4a16_gemm's; the result is identical to
+ * w4_awq_scale_activations followed by w4a16_gemm.
+ *   s          in   fp32 [K], 16-byte aligned, finite and nonzero
+ *   workspace  at least w4_awq_workspace_bytes(M, N, K, G, act_order)
+ *   all other arguments as for w4a16_gemm                                  */
+size_t w4_awq_workspace_bytes(int M, int N, int K, int G, int act_order);
+w4_status w4a16_awq_gemm(const uint16_t* X, const float* s, const uint8_t* Wp, int M, int N,
+                         int K, int G, int act_order, uint16_t* Y, void* workspace,
+                         size_t workspace_bytes, w4_stream stream);
 
 /* ------------------------------------------------------------------------
  * w4a16_gemm without a caller workspace.  The pages describe no such call; it

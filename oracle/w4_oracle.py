@@ -31,9 +31,9 @@ R8  double quantization: per run of 256 consecutive blocks,
     ``s2 = max(absmax) / 255``, ``c = rint(absmax / s2)`` in [0, 255],
     ``absmax' = c * s2`` in fp32; codes are chosen with the unquantized absmax;
 R9  NF4 dequant is ``bf16(fp32(T[q] * absmax'))``;
-R10 symmetric INT4: ``scale = fp16(max|w| / 7)``, codes ``rint(w / scale)``
+R14 symmetric INT4: ``scale = fp16(max|w| / 7)``, codes ``rint(w / scale)``
     clamped to [-7, 7] and stored + 8 (zero point 8, code 0 unused);
-R11 AWQ: the factor s is an input (found offline); weights enter
+R15 AWQ: the factor s is an input (found offline); weights enter
     quantization as the fp32 product ``w * s_k``, activations the GEMM as
     ``bf16(fp32(x / s_k))``.
 

@@ -128,3 +128,31 @@ def test_fullsize_nf4_decode(w4, K, N):
         assert w4.device_status() == w4.W4_OK
         _check(Y, xb, what, rows)
         del X, Y
+
+
+@pytest.mark.parametrize("K,N", S.AWQ_SYM_DECODE["shapes"])
+def test_fullsize_awq_sym_decode(w4, K, N):
+    wl = S.AWQ_SYM_DECODE
+    G = wl["G"]
+    W = S.layer_w(wl, K, N)
+    s = S.layer_awq_s(wl, K, N)
+    sd = torch.from_numpy(s).cuda()
+    Wsd = w4.awq_scale_weights(torch.from_numpy(W).cuda(), sd)
+    Wq, sc, zr = w4.quantize_sym(Wsd, G)
+    del Wsd
+    Wp = w4.prepack(Wq, sc, zr, G)
+    rows = _sample_rows(N, 48, K)
+    q, sr, z = O.quantize_sym(O.awq_scale_weights(W[rows], s), G)
+    Wq_r = O.pack_nibbles(q)
+    assert np.array_equal(Wq.cpu().numpy()[rows], Wq_r)
+    assert np.array_equal(_host_u16(sc)[rows], sr.view(np.uint16))
+    assert np.array_equal(zr.cpu().numpy()[rows], z)
+    what = O.dequant_rtn(Wq_r, sr, z, G)
+    del W
+    for M in wl["Ms"]:
+        xb = S.layer_x(wl, M, K, N)
+        X = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+        Y = w4.w4a16_awq_gemm(X, sd, Wp, N, K, G)
+        assert w4.device_status() == w4.W4_OK
+        _check(Y, O.awq_scale_activations(xb, s), what, rows)
+        del X, Y

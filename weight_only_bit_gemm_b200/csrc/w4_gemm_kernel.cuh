@@ -294,15 +294,68 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
   }
 }
 
-// act-order: X'[m, j] = X[m, perm[j]].  The GEMM launched after it may start
-// at once (programmatic dependent launch) and stream its weights while this
-// runs; it reads X' only after its dependency wait.
-__global__ void gather_x_kernel(const uint16_t* __restrict__ X, const int32_t* __restrict__ perm,
-                                int M, int K, uint16_t* __restrict__ Xp) {
+// The activation prologue, run before a GEMM whose X needs rewriting:
+//   X'[m, j] = X[m, c],  c = perm[j] with act-order, else c = j,
+// and with the AWQ factor s ("大模型量化选型：五种主流方案对比与实战" §4.1:
+// the weights are quantized as W s, the activations enter as X / s)
+//   X'[m, j] = bf16_rne(fp32(X[m, c]) / s[c])        (IEEE division).
+// 8 consecutive outputs per thread (one 16-byte store); K % 8 == 0, X and X'
+// 16-byte aligned, s 16-byte aligned.  Without PERM each thread reads only
+// the 8 inputs it writes, so X' may be X itself.  The GEMM launched after it
+// may start at once (programmatic dependent launch) and stream its weights
+// while this runs; it reads X' only after its dependency wait.
+template <bool PERM, bool SCALE>
+__global__ void __launch_bounds__(256) x_prologue_kernel(const uint16_t* X,
+                                                         const int32_t* __restrict__ perm,
+                                                         const float* __restrict__ s, int M,
+                                                         int K, uint16_t* Xp) {
   grid_dep_launch();
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  const int m = blockIdx.y;
-  if (j < K && m < M) Xp[static_cast<size_t>(m) * K + j] = X[static_cast<size_t>(m) * K + perm[j]];
+  const size_t k8 = static_cast<size_t>(K) / 8;
+  const size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<size_t>(M) * k8) return;
+  const size_t m = t / k8;
+  const int j0 = static_cast<int>(t - m * k8) * 8;
+  const uint16_t* xr = X + m * K;
+  uint32_t v[8];
+  int c[8];
+  if (PERM) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      c[e] = perm[j0 + e];
+      v[e] = xr[c[e]];
+    }
+  } else {
+    const uint4 w = *reinterpret_cast<const uint4*>(xr + j0);
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      c[e] = j0 + e;
+      v[e] = (wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+    }
+  }
+  if (SCALE) {
+    float sv[8];
+    if (PERM) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sv[e] = s[c[e]];
+    } else {
+      const float4 a = *reinterpret_cast<const float4*>(s + j0);
+      const float4 b = *reinterpret_cast<const float4*>(s + j0 + 4);
+      sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w;
+      sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float q = __fdiv_rn(__uint_as_float(v[e] << 16), sv[e]);
+      v[e] = __bfloat16_as_ushort(__float2bfloat16_rn(q));
+    }
+  }
+  uint4 o;
+  o.x = v[0] | (v[1] << 16);
+  o.y = v[2] | (v[3] << 16);
+  o.z = v[4] | (v[5] << 16);
+  o.w = v[6] | (v[7] << 16);
+  *reinterpret_cast<uint4*>(Xp + m * K + j0) = o;
 }
 
 }  // namespace w4

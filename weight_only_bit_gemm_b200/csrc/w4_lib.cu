@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -27,6 +28,7 @@ inline bool aligned(const void* p, uintptr_t a) {
 inline bool valid_group(int G) { return G == 32 || G == 64 || G == 128; }
 inline w4_status launch_status(cudaError_t e) { return e == cudaSuccess ? W4_OK : W4_ERR_CUDA; }
 inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+int sm_count();  // the current device's SMs (defined with the GEMM host code)
 
 // A kernel's dynamic shared-memory limit is a per-device setting: raise it
 // once on each device the kernel runs on (`done` holds one bit per device).
@@ -107,8 +109,13 @@ double w4_weight_bytes(int N, int K, int G) {
 }
 
 // ---------------------------------------------------------------- INT4 RTN
-w4_status w4_quantize_rtn(const float* W, int N, int K, int G, const int32_t* g_idx,
-                          uint8_t* Wq, uint16_t* scales, uint8_t* zeros, w4_stream stream) {
+}  // extern "C"
+
+namespace {
+
+template <bool SYM>
+w4_status quantize_int4(const float* W, int N, int K, int G, const int32_t* g_idx, uint8_t* Wq,
+                        uint16_t* scales, uint8_t* zeros, w4_stream stream) {
   if (!W || !Wq || !scales || !zeros) return W4_ERR_INVALID_ARG;
   if (!int4_shape_ok(N, K, G)) return W4_ERR_INVALID_ARG;
   if (!aligned(W, 4) || !aligned(scales, 2) || (g_idx && !aligned(g_idx, 4)))
@@ -117,11 +124,39 @@ w4_status w4_quantize_rtn(const float* W, int N, int K, int G, const int32_t* g_
   const size_t smem = static_cast<size_t>(ng) * 16;
   if (smem > 200 * 1024) return W4_ERR_UNSUPPORTED;
   static std::atomic<uint64_t> smem_set{0};
-  if (ensure_smem_limit(rtn_quantize_kernel, 200 * 1024, smem_set) != cudaSuccess) {
+  if (ensure_smem_limit(rtn_quantize_kernel<SYM>, 200 * 1024, smem_set) != cudaSuccess) {
     cudaGetLastError();
     return W4_ERR_CUDA;
   }
-  rtn_quantize_kernel<<<N, 256, smem, as_stream(stream)>>>(W, N, K, G, g_idx, Wq, scales, zeros);
+  rtn_quantize_kernel<SYM>
+      <<<N, 256, smem, as_stream(stream)>>>(W, N, K, G, g_idx, Wq, scales, zeros);
+  return launch_status(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+w4_status w4_quantize_rtn(const float* W, int N, int K, int G, const int32_t* g_idx,
+                          uint8_t* Wq, uint16_t* scales, uint8_t* zeros, w4_stream stream) {
+  return quantize_int4<false>(W, N, K, G, g_idx, Wq, scales, zeros, stream);
+}
+
+w4_status w4_quantize_sym(const float* W, int N, int K, int G, const int32_t* g_idx,
+                          uint8_t* Wq, uint16_t* scales, uint8_t* zeros, w4_stream stream) {
+  return quantize_int4<true>(W, N, K, G, g_idx, Wq, scales, zeros, stream);
+}
+
+w4_status w4_awq_scale_weights(const float* W, const float* s, int N, int K, float* W_out,
+                               w4_stream stream) {
+  if (!W || !s || !W_out) return W4_ERR_INVALID_ARG;
+  if (N < 1 || K < 1) return W4_ERR_INVALID_ARG;
+  if (!aligned(W, 4) || !aligned(s, 4) || !aligned(W_out, 4)) return W4_ERR_INVALID_ARG;
+  const size_t total = static_cast<size_t>(N) * K;
+  const size_t blocks =
+      std::min<size_t>((total + 255) / 256, static_cast<size_t>(sm_count()) * 16);
+  awq_scale_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(
+      W, s, N, K, W_out);
   return launch_status(cudaGetLastError());
 }
 

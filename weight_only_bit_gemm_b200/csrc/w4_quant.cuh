@@ -18,6 +18,7 @@ namespace w4 {
 struct RtnParam {
   float sf;   // fp16 scale widened to fp32
   float zp;   // zero point 0..15
+  float lo;   // lowest code: 0 (asymmetric) or 1 (symmetric, levels -7..7)
   uint16_t s16;
 };
 
@@ -33,18 +34,37 @@ __device__ __forceinline__ RtnParam rtn_param(float mx, float nx) {
   p.sf = __half2float(s16);
   float z = rintf(__fdiv_rn(nx, p.sf));
   p.zp = fminf(fmaxf(z, 0.0f), 15.0f);
+  p.lo = 0.0f;
   return p;
 }
 
+// Symmetric (absmax) form of the same section: scale = max|w| / (2^(b-1) - 1)
+// = max|w| / 7 for b = 4, levels -7..7 stored with zero point 8.
+__device__ __forceinline__ RtnParam sym_param(float mx, float nx) {
+  const float s32 = __fdiv_rn(fmaxf(mx, nx), 7.0f);
+  __half s16 = __float2half_rn(s32);
+  if (__half2float(s16) == 0.0f) s16 = __float2half_rn(1.0f);
+  RtnParam p;
+  p.s16 = __half_as_ushort(s16);
+  p.sf = __half2float(s16);
+  p.zp = 8.0f;
+  p.lo = 1.0f;
+  return p;
+}
+
+// rint(w / scale) + zp clamped to [lo, 15]; for the symmetric form that is
+// clamp(rint(w / scale), -7, 7) + 8 (all values are small integers in fp32).
 __device__ __forceinline__ uint32_t rtn_code(float w, const RtnParam& p) {
   float q = __fadd_rn(rintf(__fdiv_rn(w, p.sf)), p.zp);
-  q = fminf(fmaxf(q, 0.0f), 15.0f);
+  q = fminf(fmaxf(q, p.lo), 15.0f);
   return static_cast<uint32_t>(q);
 }
 
 // One CTA per output row.  Shared memory: per-group max(w,0) and max(-w,0)
 // as ordered non-negative float bit patterns (so integer max is float max).
 // Dynamic shared memory: 2 * ngroups * 4 bytes + 2 * ngroups * 4 bytes.
+// SYM selects the symmetric scale and zero point 8.
+template <bool SYM>
 __global__ void __launch_bounds__(256) rtn_quantize_kernel(
     const float* __restrict__ W, int N, int K, int G, const int32_t* __restrict__ g_idx,
     uint8_t* __restrict__ Wq, uint16_t* __restrict__ scales, uint8_t* __restrict__ zeros) {
@@ -100,7 +120,8 @@ __global__ void __launch_bounds__(256) rtn_quantize_kernel(
   __syncthreads();
 
   for (int g = threadIdx.x; g < ng; g += blockDim.x) {
-    const RtnParam p = rtn_param(__uint_as_float(pos_bits[g]), __uint_as_float(neg_bits[g]));
+    const float mx = __uint_as_float(pos_bits[g]), nx = __uint_as_float(neg_bits[g]);
+    const RtnParam p = SYM ? sym_param(mx, nx) : rtn_param(mx, nx);
     sf_s[g] = p.sf;
     zp_s[g] = p.zp;
     scales[static_cast<size_t>(n) * ng + g] = p.s16;
@@ -122,6 +143,7 @@ __global__ void __launch_bounds__(256) rtn_quantize_kernel(
       RtnParam p;
       p.sf = sf_s[g];
       p.zp = zp_s[g];
+      p.lo = SYM ? 1.0f : 0.0f;
       code[e] = rtn_code(row[k], p);
     }
     out[b] = static_cast<uint8_t>(code[0] | (code[1] << 4));
@@ -163,6 +185,18 @@ __global__ void rtn_dequant_kernel(const uint8_t* __restrict__ Wq,
   }
   *reinterpret_cast<uint4*>(out + static_cast<size_t>(n) * K + k0) =
       make_uint4(res[0], res[1], res[2], res[3]);
+}
+
+// ---------------------------------------------------------------- AWQ factor
+// "大模型量化选型：五种主流方案对比与实战" §4.1: the weights of input channel k
+// are multiplied by s_k before quantization (the activations are divided by
+// it at run time).  W_out[n, k] = fp32(W[n, k] * s_k); W_out may be W.
+__global__ void awq_scale_weights_kernel(const float* W, const float* __restrict__ s, int N,
+                                         int K, float* W_out) {
+  const size_t total = static_cast<size_t>(N) * K;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    W_out[i] = __fmul_rn(W[i], s[i % static_cast<size_t>(K)]);
 }
 
 // ---------------------------------------------------------------- NF4

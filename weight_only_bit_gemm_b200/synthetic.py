@@ -18,11 +18,16 @@ distributions the workloads name:
   pattern in a ``uint16`` array.
 * ``g_idx``: the act-order group map ``g_idx[perm[j]] = j // G`` for a seeded
   permutation ``perm`` of ``range(K)``.
+* ``s``: the AWQ per-input-channel factor, fp32 ``[K]`` uniform in
+  ``[lo, hi]`` (default 0.95..1.05, the range
+  "【推理与部署篇05】模型量化部署深度对比" §4.1 gives for important and
+  secondary channels); the search that finds it offline is not run here.
 
 Generators (``numpy.random.default_rng`` keyed by integer lists):
 ``[seed, tag, K, N]`` for W (draw order: W, then the outlier columns),
 ``[seed, tag, K, N, M]`` for X (X, then its outlier channels) and
-``[seed, tag, K, N, 7]`` for the act-order permutation.
+``[seed, tag, K, N, 7]`` for the act-order permutation and
+``[seed, tag, K, N, 11]`` for the AWQ factor.
 """
 from __future__ import annotations
 
@@ -51,6 +56,12 @@ def draw_w(N: int, K: int, sigma: float = 0.02, *, seed: int = 0, tag: int = 0,
 def draw_perm(K: int, *, seed: int = 0, tag: int = 0, N: int = 0) -> np.ndarray:
     """Seeded permutation of ``range(K)`` (its own generator stream)."""
     return _rng(seed, tag, K, N, 7).permutation(K).astype(np.int64)
+
+
+def draw_awq_s(K: int, *, seed: int = 0, tag: int = 0, N: int = 0, lo: float = 0.95,
+               hi: float = 1.05) -> np.ndarray:
+    """fp32 per-input-channel factor ``[K]`` uniform in ``[lo, hi]``."""
+    return _rng(seed, tag, K, N, 11).uniform(lo, hi, K).astype(np.float32)
 
 
 def act_order_g_idx(perm: np.ndarray, G: int) -> np.ndarray:
@@ -103,7 +114,15 @@ PREFILL_70B = dict(name="70B MLP prefill", tag=4, shapes=[(8192, 28672), (28672,
 ACT_ORDER_13B = dict(name="13B MLP act-order", tag=5, shapes=[(5120, 13824), (13824, 5120)],
                      Ms=[1, 16, 256], G=32, G_sweep=[64, 128], sigma=0.02)
 
-WORKLOADS = [TINY, LLAMA7B_DECODE, NF4_DECODE, PREFILL_70B, ACT_ORDER_13B]
+# Symmetric INT4 weights quantized after the AWQ factor (W s), activations
+# divided by it: the Llama-7B decode shapes, with the activation outliers
+# that motivate AWQ.
+AWQ_SYM_DECODE = dict(name="Llama-7B decode GEMV, AWQ factor + symmetric INT4", tag=6,
+                      shapes=[(4096, 12288), (4096, 4096), (4096, 22016), (11008, 4096)],
+                      Ms=[1, 4, 16], G=128, sigma=0.02,
+                      x_outlier_frac=0.001, x_outlier_scale=50.0, awq_lo=0.95, awq_hi=1.05)
+
+WORKLOADS = [TINY, LLAMA7B_DECODE, NF4_DECODE, PREFILL_70B, ACT_ORDER_13B, AWQ_SYM_DECODE]
 
 
 def layer_w(wl: dict, K: int, N: int, seed: int = 0) -> np.ndarray:
@@ -116,3 +135,8 @@ def layer_x(wl: dict, M: int, K: int, N: int, seed: int = 0) -> np.ndarray:
     return draw_x(M, K, seed=seed, tag=wl["tag"], N=N,
                   outlier_frac=wl.get("x_outlier_frac", 0.0),
                   outlier_scale=wl.get("x_outlier_scale", 1.0))
+
+
+def layer_awq_s(wl: dict, K: int, N: int, seed: int = 0) -> np.ndarray:
+    return draw_awq_s(K, seed=seed, tag=wl["tag"], N=N, lo=wl.get("awq_lo", 0.95),
+                      hi=wl.get("awq_hi", 1.05))

@@ -34,6 +34,9 @@ _SIGS = {
     "w4_selftest_wait_timeout": (_i, [_p]),
     "w4_weight_bytes": (ctypes.c_double, [_i, _i, _i]),
     "w4_quantize_rtn": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p]),
+    "w4_quantize_sym": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p]),
+    "w4_awq_scale_weights": (_i, [_p, _p, _i, _i, _p, _p]),
+    "w4_awq_scale_activations": (_i, [_p, _p, _i, _i, _p, _p]),
     "w4_dequant": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "w4_prepacked_bytes": (_sz, [_i, _i, _i, _i]),
     "w4_prepack": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
@@ -41,6 +44,8 @@ _SIGS = {
     "w4_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "w4a16_gemm": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),
     "w4a16_gemm_static_scratch": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p]),
+    "w4_awq_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "w4a16_awq_gemm": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),
     "nf4_quantize": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p]),
     "nf4_dequant": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p]),
     "nf4_levels": (None, [_p]),
@@ -105,8 +110,7 @@ def selftest_wait_timeout() -> None:
 
 # ----------------------------------------------------------------- INT4 RTN
 
-def quantize_rtn(W, G, g_idx=None):
-    """fp32 W [N, K] -> (Wq uint8 [N, K/2], scales fp16 [N, K/G], zeros uint8 [N, K/G])."""
+def _quantize_int4(fn, name, W, G, g_idx):
     _cuda(W, torch.float32, "W")
     N, K = W.shape
     dev = W.device
@@ -115,9 +119,42 @@ def quantize_rtn(W, G, g_idx=None):
     zr = torch.empty((N, K // G), dtype=torch.uint8, device=dev)
     if g_idx is not None:
         _cuda(g_idx, torch.int32, "g_idx")
-    _check(lib.w4_quantize_rtn(_ptr(W), N, K, G, _ptr(g_idx), _ptr(Wq), _ptr(sc), _ptr(zr),
-                               _stream()), "w4_quantize_rtn")
+    _check(fn(_ptr(W), N, K, G, _ptr(g_idx), _ptr(Wq), _ptr(sc), _ptr(zr), _stream()), name)
     return Wq, sc, zr
+
+
+def quantize_rtn(W, G, g_idx=None):
+    """fp32 W [N, K] -> (Wq uint8 [N, K/2], scales fp16 [N, K/G], zeros uint8 [N, K/G])."""
+    return _quantize_int4(lib.w4_quantize_rtn, "w4_quantize_rtn", W, G, g_idx)
+
+
+def quantize_sym(W, G, g_idx=None):
+    """Symmetric INT4 (scale max|w|/7, zero point 8), same outputs as quantize_rtn."""
+    return _quantize_int4(lib.w4_quantize_sym, "w4_quantize_sym", W, G, g_idx)
+
+
+def awq_scale_weights(W, s, out=None):
+    """fp32 W [N, K] * s [K] (per input channel) in fp32."""
+    _cuda(W, torch.float32, "W")
+    _cuda(s, torch.float32, "s")
+    N, K = W.shape
+    if out is None:
+        out = torch.empty_like(W)
+    _check(lib.w4_awq_scale_weights(_ptr(W), _ptr(s), N, K, _ptr(out), _stream()),
+           "w4_awq_scale_weights")
+    return out
+
+
+def awq_scale_activations(X, s, out=None):
+    """bf16 X [M, K] / s [K] per input channel, rounded to bf16."""
+    _cuda(X, torch.bfloat16, "X")
+    _cuda(s, torch.float32, "s")
+    M, K = X.shape
+    if out is None:
+        out = torch.empty_like(X)
+    _check(lib.w4_awq_scale_activations(_ptr(X), _ptr(s), M, K, _ptr(out), _stream()),
+           "w4_awq_scale_activations")
+    return out
 
 
 def dequant(Wq, scales, zeros, G, g_idx=None):
@@ -207,6 +244,25 @@ def w4a16_gemm_static_scratch(X, Wp, N, K, G, act_order=False, out=None):
         out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
     _check(lib.w4a16_gemm_static_scratch(_ptr(X), _ptr(Wp), M, N, K, G, int(bool(act_order)),
                                          _ptr(out), _stream()), "w4a16_gemm_static_scratch")
+    return out
+
+
+def awq_workspace_bytes(M, N, K, G, act_order=False) -> int:
+    return lib.w4_awq_workspace_bytes(M, N, K, G, int(bool(act_order)))
+
+
+def w4a16_awq_gemm(X, s, Wp, N, K, G, act_order=False, out=None, workspace=None):
+    """Y[M, N] = (X / s) . dequant(W s)^T for bf16 X [M, K], the AWQ factor
+    s [K] and prepacked Wp of weights quantized after awq_scale_weights."""
+    _cuda(X, torch.bfloat16, "X")
+    _cuda(s, torch.float32, "s")
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    need = awq_workspace_bytes(M, N, K, G, act_order)
+    ws = _ws_view(workspace if workspace is not None else _WS.get(need, X.device))
+    _check(lib.w4a16_awq_gemm(_ptr(X), _ptr(s), _ptr(Wp), M, N, K, G, int(bool(act_order)),
+                              _ptr(out), _ptr(ws), ws.numel(), _stream()), "w4a16_awq_gemm")
     return out
 
 
