@@ -1,5 +1,5 @@
-"""Oracle: group-wise INT4 (asymmetric and symmetric RTN) and NF4
-(double-quantized) weight quantization, the AWQ per-input-channel factor,
+"""Oracle: group-wise INT4 (asymmetric and symmetric RTN) and NF4 / FP4
+(block-wise, double-quantized) weight quantization, the AWQ per-input-channel factor,
 packing, dequantization and the fp64 matmul reference.
 
 TEST INFRASTRUCTURE ONLY -- see the package docstring for who may import it.
@@ -35,7 +35,11 @@ R14 symmetric INT4: ``scale = fp16(max|w| / 7)``, codes ``rint(w / scale)``
     clamped to [-7, 7] and stored + 8 (zero point 8, code 0 unused);
 R15 AWQ: the factor s is an input (found offline); weights enter
     quantization as the fp32 product ``w * s_k``, activations the GEMM as
-    ``bf16(fp32(x / s_k))``.
+    ``bf16(fp32(x / s_k))``;
+R17 FP4: E2M1 codes (sign bit 3, exponent bits 2..1, mantissa bit 0) with
+    magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 divided by 6; nearest magnitude,
+    the lower on a midpoint; sign bit only for a nonzero magnitude; blocks,
+    double quantization and dequantization as NF4.
 
 All floating-point steps are numpy float32 operations (IEEE, round to nearest
 even) unless stated as fp64; the matmul accumulates in fp64.
@@ -61,6 +65,7 @@ __all__ = [
     "matmul_exact_small", "ulp_bf16", "tolerance", "check_matmul",
     "weight_bytes", "code_bytes", "nf4_weight_bytes",
     "sym_params", "quantize_sym", "awq_scale_weights", "awq_scale_activations",
+    "fp4_table", "fp4_midpoints", "fp4_codes", "fp4_quantize", "fp4_dequant",
 ]
 
 F32 = np.float32
@@ -349,6 +354,73 @@ def nf4_dequant(Wq: np.ndarray, absmax_q: np.ndarray, s2: np.ndarray,
     s = np.asarray(s2, dtype=F32)[np.arange(nb) // dq_group]
     a_dq = c * s                                              # fp32 product
     vals = nf4_table()[qb] * a_dq[:, None]                    # fp32 product
+    return bf16_round_bits(vals.reshape(shape))
+
+
+# ---------------------------------------------------------------------------
+# FP4: the other 4-bit type of the same block-wise scheme.  [Survey] §6.3
+# names NF4 and FP4 as the two 4-bit formats of that scheme; [Survey] §6.1
+# says plain FP4 keeps three significant bits with uneven spacing;
+# [Comparison] §7.2 gives the 4-bit float layout [S:1][E:2][M:1] (E2M1).
+# Readings (R17): code bit 3 is the sign, bits 2..1 the exponent e, bit 0
+# the mantissa m; magnitude m/2 for e = 0, else 2^(e-1) (1 + m/2), i.e.
+# 0, 0.5, 1, 1.5, 2, 3, 4, 6 for codes 0..7; the table is divided by 6 so
+# that it spans [-1, 1] like NF4's and the block absmax maps to code 7.  A
+# value takes the nearest magnitude (the lower one on a midpoint) and the
+# sign bit only when that magnitude is not zero.  Blocks, double
+# quantization and dequantization are NF4's (R8, R9) with this table.
+# ---------------------------------------------------------------------------
+
+def fp4_table() -> np.ndarray:
+    """16 FP4 levels, fp32: code c -> sign * magnitude(e, m) / 6 (R17), each
+    the single fp32 rounding of an exact quotient."""
+    out = np.empty(16, dtype=F32)
+    for c in range(16):
+        e, m = (c >> 1) & 3, c & 1
+        mag = 0.5 * m if e == 0 else 2.0 ** (e - 1) * (1.0 + 0.5 * m)   # exact in fp32
+        v = F32(mag) / F32(6.0)
+        out[c] = -v if c & 8 else v
+    return out
+
+
+def fp4_midpoints() -> np.ndarray:
+    """Magnitude thresholds t_i = fp32((T[i] + T[i+1]) / 2), i = 0..6, over
+    the ascending positive levels T[0..7]."""
+    T = fp4_table()[:8].astype(np.float64)
+    return ((T[:-1] + T[1:]) / 2.0).astype(F32)
+
+
+def fp4_codes(W: np.ndarray, blocksize: int = 64) -> np.ndarray:
+    """Code of each weight: v = w / absmax (fp32; 0 if absmax is 0),
+    magnitude code = number of thresholds below |v|, plus 8 when v < 0 and
+    that magnitude is not zero.  Returns uint8 [N, K]."""
+    B = _blocks(W, blocksize)
+    a = np.abs(B).max(axis=1)
+    safe = np.where(a > 0, a, F32(1.0)).astype(F32)
+    v = np.where(a[:, None] > 0, B / safe[:, None], F32(0.0)).astype(F32)
+    mag = np.searchsorted(fp4_midpoints(), np.abs(v), side="left")
+    q = np.where((v < 0) & (mag > 0), mag + 8, mag)
+    return q.astype(np.uint8).reshape(np.shape(W))
+
+
+def fp4_quantize(W: np.ndarray, blocksize: int = 64, dq_group: int = 256):
+    """As nf4_quantize with the FP4 codes: (packed codes, absmax codes, s2)."""
+    q = fp4_codes(W, blocksize)
+    c, s2 = nf4_double_quant(nf4_absmax(W, blocksize), dq_group)
+    return pack_nibbles(q), c, s2
+
+
+def fp4_dequant(Wq: np.ndarray, absmax_q: np.ndarray, s2: np.ndarray,
+                blocksize: int = 64, dq_group: int = 256) -> np.ndarray:
+    """bf16 bits [N, K] of fp32(T_fp4[q] * absmax'), absmax' = fp32(c * s2)."""
+    q = unpack_nibbles(Wq)
+    shape = q.shape
+    qb = q.reshape(-1, blocksize)
+    nb = qb.shape[0]
+    c = np.asarray(absmax_q, dtype=np.uint8)[:nb].astype(F32)
+    s = np.asarray(s2, dtype=F32)[np.arange(nb) // dq_group]
+    a_dq = c * s                                              # fp32 product
+    vals = fp4_table()[qb] * a_dq[:, None]                    # fp32 product
     return bf16_round_bits(vals.reshape(shape))
 
 

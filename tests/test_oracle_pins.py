@@ -495,6 +495,135 @@ def test_tolerance_ulp():
 
 # ---------------------------------------------------------------- planted mistakes
 
+# ---------------------------------------------------------------- FP4 (E2M1)
+
+FP4_WORKED = _parse_worked(os.path.join(GOLDEN, "fp4_worked.txt"))
+
+
+def test_fp4_table_is_e2m1():
+    # the E2M1 magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6 (one sign, two
+    # exponent, one mantissa bit); the table is them over 6, sign in bit 3
+    T = O.fp4_table()
+    assert T.dtype == np.float32 and T.shape == (16,)
+    e2m1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for c in range(8):
+        exact = Fraction(e2m1[c]) / 6
+        assert abs(Fraction(float(T[c])) - exact) <= exact * Fraction(1, 2 ** 24)
+        assert T[c + 8] == -T[c]
+    assert np.signbit(T[8]) and T[8] == 0
+    assert T[7] == 1.0 and T[15] == -1.0
+    assert np.all(np.diff(T[:8]) > 0)
+    # spacing doubles with each exponent step above the subnormal pair
+    gaps = np.diff(T[:8].astype(np.float64)) * 6
+    assert np.allclose(gaps, [0.5, 0.5, 0.5, 0.5, 1, 1, 2])
+
+
+@pytest.mark.parametrize("case", FP4_WORKED, ids=lambda c: c["name"])
+def test_fp4_worked_example(case):
+    w = np.zeros((1, 64), np.float32)
+    vals = [float(v) for v in case["w"]]
+    w[0, :len(vals)] = vals
+    Wq, c, s2 = O.fp4_quantize(w)
+    codes = O.unpack_nibbles(Wq)[0]
+    assert codes[:len(vals)].tolist() == [int(v) for v in case["codes"]]
+    assert np.all(codes[len(vals):] == 0)
+    assert Wq[0, :4].tolist() == [int(v, 16) for v in case["packed_hex"]]
+    assert np.all(Wq[0, 4:] == 0)
+    assert int(c[0]) == int(case["absmax_code"][0])
+    what = O.bf16_bits_to_f32(O.fp4_dequant(Wq, c, s2))[0]
+    assert what[:len(vals)].tolist() == [float(v) for v in case["what"]]
+
+
+def test_fp4_brute_force_nearest_and_sign():
+    W = _rand_w(16, 256, 45, sigma=1.0)
+    W[0, :64] = 0.0                                   # zero block -> all code 0
+    W[1, 1:64] = np.linspace(-1, 1, 63, dtype=np.float32) * np.float32(0.9)
+    W[1, 0] = 1.0                                     # absmax 1: v = w exactly
+    q = O.fp4_codes(W)
+    assert np.all(q[0, :64] == 0)
+    T = O.fp4_table().astype(np.float64)
+    B = W.reshape(-1, 64)
+    a = np.abs(B).max(axis=1)
+    qb = q.reshape(-1, 64)
+    for b in range(B.shape[0]):
+        for k in range(64):
+            if a[b] == 0:
+                continue
+            v = float(np.float32(B[b, k]) / np.float32(a[b]))
+            dist = [abs(abs(v) - T[m]) for m in range(8)]
+            best = min(dist)
+            mag = min(m for m in range(8) if dist[m] - best <= 1e-15)   # lower on a tie
+            want = mag + 8 if (v < 0 and mag > 0) else mag
+            assert int(qb[b, k]) == want
+    # negating W flips the sign bit of every nonzero magnitude
+    qn = O.fp4_codes(-W)
+    nz = (q & 7) > 0
+    assert np.array_equal(qn[nz], q[nz] ^ 8) and np.array_equal(qn[~nz], q[~nz])
+
+
+def test_fp4_dequant_error_bound():
+    W = _rand_w(32, 512, 46)
+    Wq, c, s2 = O.fp4_quantize(W)
+    what = O.bf16_bits_to_f32(O.fp4_dequant(Wq, c, s2)).astype(np.float64)
+    B = W.reshape(-1, 64).astype(np.float64)
+    a = np.abs(B).max(axis=1, keepdims=True)
+    s = s2.astype(np.float64)[np.arange(B.shape[0]) // 256][:, None]
+    # largest half-gap of the table is (6 - 4) / 2 / 6 = 1/6 of the absmax;
+    # the 8-bit absmax adds at most s2 / 2; bf16 rounding 2^-9 relative
+    err = np.abs(what.reshape(B.shape) - B)
+    assert np.all(err <= a / 6 + s / 2 + np.abs(B) * 2.0 ** -8 + 1e-12)
+    # a weight at +-absmax comes back within the absmax quantization step
+    top = np.abs(B).argmax(axis=1)
+    wt = what.reshape(B.shape)[np.arange(B.shape[0]), top]
+    bt = B[np.arange(B.shape[0]), top]
+    assert np.all(np.abs(wt - bt) <= s[:, 0] / 2 + np.abs(bt) * 2.0 ** -8)
+
+
+def test_planted_mistakes_fp4(monkeypatch):
+    import oracle.w4_oracle as M
+    checks = [test_fp4_table_is_e2m1, lambda: [test_fp4_worked_example(c) for c in FP4_WORKED],
+              test_fp4_brute_force_nearest_and_sign]
+
+    def caught(name, fn):
+        monkeypatch.setattr(M, name, fn)
+        monkeypatch.setattr(O, name, fn)
+        try:
+            for chk in checks:
+                try:
+                    chk()
+                except AssertionError:
+                    return True
+            return False
+        finally:
+            monkeypatch.undo()
+
+    orig_table = M.fp4_table
+
+    def bias_off_by_one():                 # 2^e instead of 2^(e-1)
+        T = orig_table() * np.float32(6)
+        T = np.where(np.abs(T) >= 1, T * 2, T).astype(np.float32)
+        return (T / np.float32(12)).astype(np.float32)
+    assert caught("fp4_table", bias_off_by_one)
+
+    orig_codes = M.fp4_codes
+
+    def negative_zero_code(W, blocksize=64):  # sign bit set on zero magnitudes
+        q = orig_codes(W, blocksize)
+        neg = np.asarray(W, np.float32) < 0
+        return np.where(neg, q | 8, q).astype(np.uint8)
+    assert caught("fp4_codes", negative_zero_code)
+
+    def ties_up(W, blocksize=64):             # upper magnitude on a midpoint
+        B = M._blocks(W, blocksize)
+        a = np.abs(B).max(axis=1)
+        safe = np.where(a > 0, a, np.float32(1.0)).astype(np.float32)
+        v = np.where(a[:, None] > 0, B / safe[:, None], np.float32(0.0)).astype(np.float32)
+        mag = np.searchsorted(M.fp4_midpoints(), np.abs(v), side="right")
+        q = np.where((v < 0) & (mag > 0), mag + 8, mag)
+        return q.astype(np.uint8).reshape(np.shape(W))
+    assert caught("fp4_codes", ties_up)
+
+
 def _pins_fail(monkeypatch, name, fn):
     """Replace one oracle function by a mutated copy and report whether any
     of the core pins catches it."""
