@@ -39,7 +39,12 @@ R15 AWQ: the factor s is an input (found offline); weights enter
 R17 FP4: E2M1 codes (sign bit 3, exponent bits 2..1, mantissa bit 0) with
     magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 divided by 6; nearest magnitude,
     the lower on a midpoint; sign bit only for a nonzero magnitude; blocks,
-    double quantization and dequantization as NF4.
+    double quantization and dequantization as NF4;
+R18 GPTQ: H = 2 X^T X (fp64); dead channels H_kk = 0 -> 1 and w_k = 0;
+    act-order = stable sort by decreasing H_kk; damping 0.01 * mean(diag H);
+    the update uses the inverse Hessian of the remaining columns, eliminated
+    one column at a time; group parameters from the compensated weights at
+    the group's first column; codes decided in fp32.
 
 All floating-point steps are numpy float32 operations (IEEE, round to nearest
 even) unless stated as fp64; the matmul accumulates in fp64.
@@ -66,6 +71,7 @@ __all__ = [
     "weight_bytes", "code_bytes", "nf4_weight_bytes",
     "sym_params", "quantize_sym", "awq_scale_weights", "awq_scale_activations",
     "fp4_table", "fp4_midpoints", "fp4_codes", "fp4_quantize", "fp4_dequant",
+    "gptq_hessian", "gptq_prepare", "gptq_eliminate", "gptq_quantize", "gptq_loss",
 ]
 
 F32 = np.float32
@@ -422,6 +428,106 @@ def fp4_dequant(Wq: np.ndarray, absmax_q: np.ndarray, s2: np.ndarray,
     a_dq = c * s                                              # fp32 product
     vals = fp4_table()[qb] * a_dq[:, None]                    # fp32 product
     return bf16_round_bits(vals.reshape(shape))
+
+
+# ---------------------------------------------------------------------------
+# GPTQ error compensation at quantization time.  [Comparison] §3.1: per layer,
+# H = 2 X X^T from calibration activations; Q = W; for each column in turn
+# (by importance): quantize it, take the error, spread it over the columns not
+# yet quantized through the (inverse) Hessian, "remaining -= err / H_diag *
+# H_row".  [Survey] §3 (GPTQ): this is the Optimal Brain Surgeon update, it
+# needs the inverse of H, and a small damping (percdamp, 0.01) is added to
+# H's diagonal so that it stays invertible.  [Survey] §3.2: desc_act orders
+# the columns by activation size; group_size 128 shares one scale and zero
+# point per group.  Readings (R18):
+#   H = 2 X^T X in fp64 for X [n, K] (rows = calibration tokens);
+#   a channel with H_kk = 0 (never activated) gets H_kk = 1 and w_k = 0;
+#   act-order = a stable sort of the channels by decreasing H_kk;
+#   damping H += lambda I, lambda = 0.01 * mean(diag H);
+#   "H_diag" and "H_row" are those of the inverse Hessian of the columns not
+#   yet quantized: Hi = H^-1, and after column j, Hi loses row and column j
+#   by Gaussian elimination (Hi_F <- Hi_F - Hi_Fj Hi_jF / Hi_jj, which is
+#   the inverse of H restricted to the remaining columns);
+#   a group's scale and zero point come from its (already compensated)
+#   weights when its first column is reached, by the RTN rule (R1-R3) on
+#   their fp32 values; codes are decided in fp32; the error uses the fp32
+#   dequantized value (q - z) * scale; the compensation runs in fp64.
+# ---------------------------------------------------------------------------
+
+def gptq_hessian(x_bits: np.ndarray) -> np.ndarray:
+    """H = 2 X^T X in fp64 for bf16 calibration activations X [n, K]."""
+    x = bf16_bits_to_f64(x_bits)
+    return 2.0 * (x.T @ x)
+
+
+def gptq_prepare(H: np.ndarray, act_order: bool, damp: float = 0.01):
+    """Dead channels, order and damping (R18).  Returns (H' fp64 in the
+    processing order, perm int64 [K] = processing position -> channel, dead
+    bool [K])."""
+    H = np.array(H, dtype=np.float64, copy=True)
+    K = H.shape[0]
+    d = np.diag(H).copy()
+    dead = d == 0
+    H[dead, dead] = 1.0
+    d[dead] = 1.0
+    perm = np.argsort(-d, kind="stable") if act_order else np.arange(K)
+    H = H[np.ix_(perm, perm)]
+    H[np.diag_indices(K)] += damp * float(np.mean(np.diag(H)))
+    return H, perm.astype(np.int64), dead
+
+
+def gptq_eliminate(Hi: np.ndarray, j: int) -> np.ndarray:
+    """Remove column j from the inverse Hessian of the columns j.. : returns
+    the inverse Hessian of the columns j+1.. (Gaussian elimination)."""
+    r = Hi[j, j + 1:]
+    return Hi[j + 1:, j + 1:] - np.outer(Hi[j + 1:, j], r) / Hi[j, j]
+
+
+def gptq_quantize(W: np.ndarray, H: np.ndarray, G: int, act_order: bool = False,
+                  damp: float = 0.01):
+    """INT4 codes with GPTQ error compensation (R18).
+
+    Returns (codes uint8 [N, K], scale fp16 [N, K/G], zero uint8 [N, K/G],
+    g_idx int32 [K] or None): the canonical format of ``quantize_rtn``; with
+    act-order the channel processed j-th belongs to group j // G."""
+    W = np.array(W, dtype=np.float64, copy=True)
+    N, K = W.shape
+    if K % G:
+        raise ValueError("K must be a multiple of G")
+    Hp, perm, dead = gptq_prepare(H, act_order, damp)
+    W[:, dead] = 0.0
+    Q = W[:, perm]                                  # working copy, processing order
+    Hi = np.linalg.inv(Hp)
+    codes = np.zeros((N, K), dtype=np.uint8)
+    s16 = np.zeros((N, K // G), dtype=np.float16)
+    zp = np.zeros((N, K // G), dtype=np.uint8)
+    for j in range(K):
+        g = j // G
+        if j % G == 0:                              # group parameters, compensated weights
+            s16[:, g:g + 1], zp[:, g:g + 1] = rtn_params(Q[:, j:j + G].astype(F32), G)
+        sf = s16[:, g].astype(F32)
+        zf = zp[:, g].astype(F32)
+        w32 = Q[:, j].astype(F32)
+        q = np.clip(np.rint(w32 / sf) + zf, 0, 15)  # decided in fp32
+        codes[:, j] = q.astype(np.uint8)
+        deq = ((q - zf) * sf).astype(F32).astype(np.float64)
+        err = (Q[:, j] - deq) / Hi[0, 0]
+        Q[:, j + 1:] -= np.outer(err, Hi[0, 1:])    # spread over the remaining columns
+        Hi = gptq_eliminate(Hi, 0)
+    out = np.zeros_like(codes)
+    out[:, perm] = codes
+    if act_order:
+        g_idx = np.empty(K, dtype=np.int32)
+        g_idx[perm] = (np.arange(K) // G).astype(np.int32)
+        return out, s16, zp, g_idx
+    return out, s16, zp, None
+
+
+def gptq_loss(W: np.ndarray, what_bits: np.ndarray, H: np.ndarray) -> float:
+    """Layer output error tr((W - W_hat) H (W - W_hat)^T) in fp64 (the
+    quantity the compensation lowers; H undamped)."""
+    D = np.asarray(W, dtype=np.float64) - bf16_bits_to_f64(what_bits)
+    return float(np.einsum("nk,kl,nl->", D, np.asarray(H, np.float64), D))
 
 
 # ---------------------------------------------------------------------------

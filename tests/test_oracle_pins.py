@@ -624,6 +624,131 @@ def test_planted_mistakes_fp4(monkeypatch):
     assert caught("fp4_codes", ties_up)
 
 
+# ---------------------------------------------------------------- GPTQ
+
+def _calib_h(K, n, seed, rank=4):
+    # correlated synthetic calibration activations: noise plus a few shared factors
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((n, K)) + rng.standard_normal((n, rank)) @ rng.standard_normal((rank, K))
+    return O.gptq_hessian(S.to_bf16_bits(x.astype(np.float32)))
+
+
+def _rtn_code(w, s, z):
+    return int(np.clip(np.rint(np.float32(w) / np.float32(s)) + z, 0, 15))
+
+
+@pytest.mark.parametrize("act", [False, True])
+def test_gptq_identity_hessian_is_rtn(act):
+    # H = c I: the inverse Hessian has no off-diagonal entries, nothing is
+    # spread, and (equal diagonal) act-order keeps the natural order
+    W = _rand_w(24, 256, 47)
+    q, s, z, gi = O.gptq_quantize(W, 3.5 * np.eye(256), 64, act)
+    qr, sr, zr = O.quantize_rtn(W, 64)
+    assert np.array_equal(q, qr) and np.array_equal(s, sr) and np.array_equal(z, zr)
+    if act:
+        assert np.array_equal(gi, np.arange(256) // 64)
+
+
+def test_gptq_two_columns_closed_form():
+    # K = 2, one group: column 0 is quantized as RTN; column 1 then carries
+    # the value u minimising the 2x2 quadratic (e0, w1 - u) H' (e0, w1 - u)^T,
+    # u = w1 + e0 * b' / c' for H' = [[a', b'], [b', c']] (damped), and is
+    # quantized with the group's RTN parameters
+    rng = np.random.default_rng(48)
+    changed = 0
+    for _ in range(200):
+        w = rng.uniform(-1, 1, 2).astype(np.float32)
+        a, c = rng.uniform(0.5, 2.0, 2)
+        b = rng.uniform(-0.9, 0.9) * np.sqrt(a * c)
+        H = np.array([[a, b], [b, c]])
+        q, s, z, _ = O.gptq_quantize(w[None, :], H, 2)
+        sr_, zr_ = O.rtn_params(w[None, :], 2)
+        sf, zf = float(sr_[0, 0]), int(zr_[0, 0])
+        assert s[0, 0] == sr_[0, 0] and z[0, 0] == zf
+        q0 = _rtn_code(w[0], sf, zf)
+        e0 = float(w[0]) - float(np.float32((q0 - zf) * np.float32(sf)))
+        lam = 0.01 * (a + c) / 2
+        u = float(w[1]) + e0 * b / (c + lam)
+        assert q[0, 0] == q0 and q[0, 1] == _rtn_code(u, sf, zf)
+        changed += q[0, 1] != _rtn_code(w[1], sf, zf)
+    assert changed > 3           # the compensation does move codes
+
+
+def test_gptq_elimination_is_inverse_of_remaining_block():
+    rng = np.random.default_rng(49)
+    A = rng.standard_normal((12, 12))
+    H = A @ A.T + 12 * np.eye(12)
+    Hi = np.linalg.inv(H)
+    for j in range(3):
+        Hi = O.gptq_eliminate(Hi, 0)
+        assert np.allclose(Hi, np.linalg.inv(H[j + 1:, j + 1:]), rtol=1e-10, atol=1e-12)
+
+
+def test_gptq_lowers_layer_error_and_handles_dead_channels():
+    K, N, G = 256, 32, 32
+    H = _calib_h(K, 384, 50)
+    H[7, :] = 0.0
+    H[:, 7] = 0.0                       # channel 7 never activated
+    W = _rand_w(N, K, 51)
+    for act in (False, True):
+        q, s, z, gi = O.gptq_quantize(W, H, G, act)
+        gk = O.group_index(K, G, gi)
+        assert q.max() <= 15
+        # dead channel: weight treated as 0 -> code = zero point -> w_hat = 0
+        assert np.array_equal(q[:, 7], z[np.arange(N), gk[7]])
+        what = O.dequant_rtn(O.pack_nibbles(q), s, z, G, gi)
+        assert np.all(what[:, 7] == 0)
+        qr, sr, zr = O.quantize_rtn(W, G)
+        Wl = W.copy()
+        Wl[:, 7] = 0.0
+        l_g = O.gptq_loss(Wl, what, H)
+        l_r = O.gptq_loss(Wl, O.dequant_rtn(O.pack_nibbles(qr), sr, zr, G), H)
+        assert l_g < 0.5 * l_r
+        if act:
+            # processing order: decreasing diag(H), each group exactly G channels
+            d = np.diag(H).copy()
+            d[7] = 1.0
+            ng = K // G
+            assert all(d[gi == g].min() >= d[gi == g + 1].max() for g in range(ng - 1))
+            assert np.all(np.bincount(gi) == G)
+
+
+def test_planted_mistakes_gptq(monkeypatch):
+    import oracle.w4_oracle as M
+    checks = [test_gptq_two_columns_closed_form,
+              test_gptq_lowers_layer_error_and_handles_dead_channels,
+              test_gptq_elimination_is_inverse_of_remaining_block]
+
+    def caught(name, fn):
+        monkeypatch.setattr(M, name, fn)
+        monkeypatch.setattr(O, name, fn)
+        try:
+            for chk in checks:
+                try:
+                    chk()
+                except (AssertionError, np.linalg.LinAlgError):
+                    return True
+            return False
+        finally:
+            monkeypatch.undo()
+
+    def no_elimination(Hi, j):                # keep the first inverse: drop the row/col only
+        return Hi[j + 1:, j + 1:].copy()
+    assert caught("gptq_eliminate", no_elimination)
+
+    def elim_sign(Hi, j):                     # + instead of -
+        r = Hi[j, j + 1:]
+        return Hi[j + 1:, j + 1:] + np.outer(Hi[j + 1:, j], r) / Hi[j, j]
+    assert caught("gptq_eliminate", elim_sign)
+
+    orig_prep = M.gptq_prepare
+
+    def undamped_as_hessian(H, act_order, damp=0.01):   # H where H^-1 belongs
+        Hp, perm, dead = orig_prep(H, act_order, damp)
+        return np.linalg.inv(Hp), perm, dead
+    assert caught("gptq_prepare", undamped_as_hessian)
+
+
 def _pins_fail(monkeypatch, name, fn):
     """Replace one oracle function by a mutated copy and report whether any
     of the core pins catches it."""
