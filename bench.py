@@ -53,7 +53,7 @@ def nf4_bytes(M, N, K):
 # DRAM bytes of one decode-kernel launch from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of w4_gemv_kernel.cuh).
 TRAFFIC_CAPTURE = {
-    "kernel_sha256": "32df8ca0b3ba32910c6d9bac3bb804b7a0e496f3a7fe4dc58e2fe2d020c47471",
+    "kernel_sha256": "148e452dbe957e51ca200f80df3791137d4985face69a418263765501ea4843a",
     "shape": {"M": 1, "N": 12288, "K": 4096, "G": 128},
     "dram_bytes": 26178048,
     "profile": "profiles/w4_gemv_kernel_int4_K4096_N12288_M1.md",
@@ -448,6 +448,29 @@ def measure_rows(w4, peaks):
                                "TB/s": sum(nbytes) / sum(ts) / 1e9,
                                "frac_of_hbm": sum(nbytes) / sum(ts) / 1e6 / hbm}
 
+    # NEXT row: FP4 (E2M1) table in the NF4 kernels, same shapes
+    f4 = S.FP4_DECODE
+    calls, nbytes = [], []
+    for (K, N) in f4["shapes"]:
+        W = torch.from_numpy(S.layer_w(f4, K, N)).cuda()
+        q4, c4, s24 = w4.fp4_quantize(W)
+        if (K, N) == f4["shapes"][0]:
+            t = time_calls([lambda: w4.fp4_quantize(W)], reps=5)[0]
+            b = N * K * 4 + N * K / 2 + N * K / 64
+            rows["fp4_quantize"] = {"shape": [N, K], "ms": t, "GB/s": b / t / 1e6}
+        wp = w4.nf4_prepack(q4, c4)
+        reps = [wp] + [wp.clone() for _ in range(_replicas_for(wp.numel(), l2) - 1)]
+        for M in f4["Ms"]:
+            X = bf16_dev(S.layer_x(f4, M, K, N))
+            for r in reps:
+                calls.append(lambda X=X, r=r, s=s24, N=N, K=K: w4.fp4_gemm(X, r, s, N, K))
+                nbytes.append(nf4_bytes(M, N, K))
+        del W
+    ts = time_calls(calls, reps=5)
+    rows["fp4_gemm_decode"] = {"configs": "(K,N) in {(4096,14336),(14336,4096)} x M in {1,8,32}",
+                               "TB/s": sum(nbytes) / sum(ts) / 1e9,
+                               "frac_of_hbm": sum(nbytes) / sum(ts) / 1e6 / hbm}
+
     # a3: act-order (g_idx) decode and M=256, group 32
     ao = S.ACT_ORDER_13B
     dec_calls, dec_bytes, big_calls, big_flops = [], [], [], []
@@ -620,12 +643,14 @@ def run_reference(args, world, rank):
 
 def run_single(w4, args):
     fmt, K, N, M = args.single[0], *map(int, args.single[1:])
-    if fmt == "nf4":
-        W = torch.from_numpy(S.layer_w(S.NF4_DECODE, K, N)).cuda()
-        q, c, s2 = w4.nf4_quantize(W)
+    if fmt in ("nf4", "fp4"):
+        wl = S.NF4_DECODE if fmt == "nf4" else S.FP4_DECODE
+        W = torch.from_numpy(S.layer_w(wl, K, N)).cuda()
+        q, c, s2 = (w4.nf4_quantize if fmt == "nf4" else w4.fp4_quantize)(W)
         wp = w4.nf4_prepack(q, c)
-        X = bf16_dev(S.layer_x(S.NF4_DECODE, M, K, N))
-        f = (lambda: w4.nf4_gemm(X, wp, s2, N, K))
+        X = bf16_dev(S.layer_x(wl, M, K, N))
+        gemm = w4.nf4_gemm if fmt == "nf4" else w4.fp4_gemm
+        f = (lambda: gemm(X, wp, s2, N, K))
         nbytes, flops = nf4_bytes(M, N, K), 2.0 * M * N * K
     elif fmt == "awq":
         aw = S.AWQ_SYM_DECODE
@@ -662,7 +687,7 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the other-row measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--single", nargs=4, metavar=("FMT", "K", "N", "M"),
-                    help="profiling aid: run one layer call (FMT int4|nf4|awq) warmup+steps times "
+                    help="profiling aid: run one layer call (FMT int4|nf4|fp4|awq) warmup+steps times "
                          "eagerly and print its mean device time")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -292,6 +292,36 @@ w4_status nf4_gemm(const uint16_t* X, const uint8_t* Wp, const float* s2, int M,
                    int K, int dq_group, uint16_t* Y, void* workspace,
                    size_t workspace_bytes, w4_stream stream);
 
+/* ------------------------------------------------------------------------
+ * FP4: the second 4-bit type of the block-wise scheme ([Survey] §6.3: the
+ * library offers NF4 and FP4; [Survey] §6.1: plain FP4 has three significant
+ * bits and uneven spacing), with the 4-bit float layout [S:1][E:2][M:1]
+ * ([Comparison] §7.2).  Code bit 3 = sign, bits 2..1 = exponent e, bit 0 =
+ * mantissa m; magnitude m/2 (e = 0) or 2^(e-1)(1 + m/2), i.e. 0, 0.5, 1, 1.5,
+ * 2, 3, 4, 6 for codes 0..7; table T = magnitude / 6 (fp32), so T spans
+ * [-1, 1] and a block's absmax maps to code 7.
+ *   v = w / a as for NF4; magnitude code = #{ i < 7 : |v| > t_i },
+ *   t_i = fp32((T[i] + T[i+1]) / 2) (the lower magnitude on a midpoint);
+ *   q = magnitude code + 8 if v < 0 and that code is not 0, else the code.
+ * Blocks, double quantization, dequantization (w_hat = bf16(fp32(T[q] a'))),
+ * arguments, layouts and errors are those of nf4_quantize / nf4_dequant.
+ * The prepacked layout is NF4's: prepack with nf4_prepack
+ * (nf4_prepacked_bytes), size the workspace with nf4_workspace_bytes.      */
+w4_status fp4_quantize(const float* W, int N, int K, int blocksize, int dq_group,
+                       uint8_t* Wq, uint8_t* absmax_q, float* s2, w4_stream stream);
+w4_status fp4_dequant(const uint8_t* Wq, const uint8_t* absmax_q, const float* s2, int N,
+                      int K, int blocksize, int dq_group, uint16_t* W_out,
+                      w4_stream stream);
+
+/* The 16 FP4 levels this library uses (host memory, fp32). */
+void fp4_levels(float out[16]);
+
+/* Y = X . w_hat^T for FP4 weights: the NF4 kernels with the FP4 table.
+ *   Arguments as for nf4_gemm; Wp from nf4_prepack of fp4_quantize output. */
+w4_status fp4_gemm(const uint16_t* X, const uint8_t* Wp, const float* s2, int M, int N,
+                   int K, int dq_group, uint16_t* Y, void* workspace,
+                   size_t workspace_bytes, w4_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

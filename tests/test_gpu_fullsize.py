@@ -156,3 +156,37 @@ def test_fullsize_awq_sym_decode(w4, K, N):
         assert w4.device_status() == w4.W4_OK
         _check(Y, O.awq_scale_activations(xb, s), what, rows)
         del X, Y
+
+
+@pytest.mark.parametrize("K,N", S.FP4_DECODE["shapes"])
+def test_fullsize_fp4_decode(w4, K, N):
+    wl = S.FP4_DECODE
+    dq = wl["dq_group"]
+    W = S.layer_w(wl, K, N)
+    Wq, c, s2 = w4.fp4_quantize(torch.from_numpy(W).cuda(), 64, dq)
+    Wp = w4.nf4_prepack(Wq, c)
+    kb64 = K // 64
+    step = dq // math.gcd(kb64, dq)
+    rows = _sample_rows(N, 24, K)
+    Wq_h, c_h, s2_h = Wq.cpu().numpy(), c.cpu().numpy(), s2.cpu().numpy()
+    what_rows = []
+    for r in rows:
+        r0 = (r // step) * step
+        r1 = min(N, r0 + step)
+        wq_w, c_w, s2_w = O.fp4_quantize(W[r0:r1], 64, dq)
+        if r1 - r0 == step:
+            b0, b1 = r0 * kb64, r1 * kb64
+            assert np.array_equal(Wq_h[r0:r1], wq_w)
+            assert np.array_equal(c_h[b0:b1], c_w)
+            assert np.array_equal(s2_h[b0 // dq:b0 // dq + s2_w.size].view(np.uint32),
+                                  s2_w.view(np.uint32))
+        what_rows.append(O.fp4_dequant(wq_w, c_w, s2_w, 64, dq)[r - r0])
+    what = np.stack(what_rows)
+    del W
+    for M in wl["Ms"]:
+        xb = S.layer_x(wl, M, K, N)
+        X = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+        Y = w4.fp4_gemm(X, Wp, s2, N, K, dq)
+        assert w4.device_status() == w4.W4_OK
+        _check(Y, xb, what, rows)
+        del X, Y

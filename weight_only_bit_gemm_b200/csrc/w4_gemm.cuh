@@ -193,6 +193,7 @@ struct GemmArgs {
   int tiles_n;
   int splits;
   FastDivIdx by_dq;        // NF4: 64-block index -> s2 index (double-quant run)
+  int table;              // NF4 layout: level table (kTableNf4 / kTableFp4)
 };
 
 }  // namespace w4

@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     fence_barrier_init();
     grid_dep_launch();  // the next kernel on the stream may start its prologue
   }
-  if (C::FMT == kFmtNf4 && threadIdx.x < 16) Ts[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
+  if (C::FMT == kFmtNf4 && threadIdx.x < 16) Ts[threadIdx.x] = level_value(args.table, threadIdx.x);
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::kTmemCols);
     tmem_relinquish();

@@ -56,6 +56,7 @@ struct GemvArgs {
   FastDiv32 by_ks, by_q, by_q1;
   FastDivIdx by_dq;          // NF4: 64-block index -> s2 index
   int dq_group;             // NF4: 64-blocks per second-level scale
+  int table;                // NF4 layout: level table (kTableNf4 / kTableFp4)
 };
 
 // Row groups (16 rows each) per decode work unit: two share each activation
@@ -381,9 +382,9 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(const GemvArgs args) {
   constexpr int R = C::kRG;
-  __shared__ __align__(64) float Ts[16];  // NF4 levels
+  __shared__ __align__(64) float Ts[16];  // NF4 / FP4 levels
   if (C::FMT == kFmtNf4) {
-    if (threadIdx.x < 16) Ts[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
+    if (threadIdx.x < 16) Ts[threadIdx.x] = level_value(args.table, threadIdx.x);
     __syncthreads();
   }
   grid_dep_launch();

@@ -226,8 +226,48 @@ __device__ __forceinline__ uint32_t nf4_code(float v) {
   return q;
 }
 
+// FP4 in the same block-wise scheme ("大模型量化选型" §6.3 names NF4 and FP4
+// as its two 4-bit types; "【推理与部署篇05】模型量化部署深度对比" §7.2 gives
+// the 4-bit float layout [S:1][E:2][M:1]).  Code bit 3 = sign, bits 2..1 =
+// exponent e, bit 0 = mantissa m; magnitude m/2 (e = 0) or 2^(e-1)(1 + m/2):
+// 0, 0.5, 1, 1.5, 2, 3, 4, 6, divided by 6 so that the table spans [-1, 1].
+__constant__ float kFp4Levels[16] = {
+    0.0f,  0.5f / 6.0f,  1.0f / 6.0f,  1.5f / 6.0f,  2.0f / 6.0f,  3.0f / 6.0f,  4.0f / 6.0f,  1.0f,
+    -0.0f, -0.5f / 6.0f, -1.0f / 6.0f, -1.5f / 6.0f, -2.0f / 6.0f, -3.0f / 6.0f, -4.0f / 6.0f, -1.0f};
+
+static const float kFp4LevelsHost[16] = {
+    0.0f,  0.5f / 6.0f,  1.0f / 6.0f,  1.5f / 6.0f,  2.0f / 6.0f,  3.0f / 6.0f,  4.0f / 6.0f,  1.0f,
+    -0.0f, -0.5f / 6.0f, -1.0f / 6.0f, -1.5f / 6.0f, -2.0f / 6.0f, -3.0f / 6.0f, -4.0f / 6.0f, -1.0f};
+
+// Which 16-entry level table a block-wise (NF4-layout) weight uses.
+enum LevelTable : int { kTableNf4 = 0, kTableFp4 = 1 };
+
+__device__ __forceinline__ float level_value(int table, int i) {
+  return table == kTableFp4 ? kFp4Levels[i] : __uint_as_float(kNf4LevelBits[i]);
+}
+
+// Nearest magnitude among levels 0..7 (the lower one on a midpoint; the
+// midpoints are the fp32 averages of neighbours), sign bit only when the
+// magnitude is not zero.
+struct Fp4Mids {
+  float t[7];
+  __device__ __forceinline__ Fp4Mids() {
+#pragma unroll
+    for (int i = 0; i < 7; ++i) t[i] = __fmul_rn(__fadd_rn(kFp4Levels[i], kFp4Levels[i + 1]), 0.5f);
+  }
+  __device__ __forceinline__ uint32_t code(float v) const {
+    const float av = fabsf(v);
+    uint32_t mag = 0;
+#pragma unroll
+    for (int i = 0; i < 7; ++i) mag += (av > t[i]) ? 1u : 0u;
+    return (v < 0.0f && mag != 0u) ? (mag | 8u) : mag;
+  }
+};
+
 // One thread per 64-block, one CTA per run of dq_group blocks
 // (blockDim.x == dq_group).  Writes packed codes, absmax codes and s2.
+// TABLE selects the NF4 or the FP4 codes; everything else is shared.
+template <int TABLE>
 __global__ void nf4_quantize_kernel(const float* __restrict__ W, long long nblocks, int dq_group,
                                     uint8_t* __restrict__ Wq, uint8_t* __restrict__ absmax_q,
                                     float* __restrict__ s2) {
@@ -265,13 +305,14 @@ __global__ void nf4_quantize_kernel(const float* __restrict__ W, long long nbloc
   const float c = fminf(fmaxf(rintf(__fdiv_rn(a, sc)), 0.0f), 255.0f);
   absmax_q[b] = static_cast<uint8_t>(c);
   uint32_t packed[8];
+  const Fp4Mids fp4;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     uint32_t word = 0;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float v = (a > 0.0f) ? __fdiv_rn(w[8 * i + e], a) : 0.0f;
-      word |= nf4_code(v) << (4 * e);
+      word |= (TABLE == kTableFp4 ? fp4.code(v) : nf4_code(v)) << (4 * e);
     }
     packed[i] = word;
   }
@@ -284,9 +325,9 @@ __global__ void nf4_quantize_kernel(const float* __restrict__ W, long long nbloc
 __global__ void nf4_dequant_kernel(const uint8_t* __restrict__ Wq,
                                    const uint8_t* __restrict__ absmax_q,
                                    const float* __restrict__ s2, long long total8,
-                                   int dq_group, uint16_t* __restrict__ out) {
+                                   int dq_group, int table, uint16_t* __restrict__ out) {
   __shared__ float T[16];
-  if (threadIdx.x < 16) T[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
+  if (threadIdx.x < 16) T[threadIdx.x] = level_value(table, threadIdx.x);
   __syncthreads();
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= total8) return;

@@ -122,7 +122,13 @@ AWQ_SYM_DECODE = dict(name="Llama-7B decode GEMV, AWQ factor + symmetric INT4", 
                       Ms=[1, 4, 16], G=128, sigma=0.02,
                       x_outlier_frac=0.001, x_outlier_scale=50.0, awq_lo=0.95, awq_hi=1.05)
 
-WORKLOADS = [TINY, LLAMA7B_DECODE, NF4_DECODE, PREFILL_70B, ACT_ORDER_13B, AWQ_SYM_DECODE]
+# FP4 (E2M1) weights in the NF4 block-wise layout, on the NF4 decode shapes.
+FP4_DECODE = dict(name="FP4 decode/small batch", tag=7,
+                  shapes=[(4096, 14336), (14336, 4096)], Ms=[1, 8, 32],
+                  blocksize=64, dq_group=256, sigma=0.02)
+
+WORKLOADS = [TINY, LLAMA7B_DECODE, NF4_DECODE, PREFILL_70B, ACT_ORDER_13B, AWQ_SYM_DECODE,
+             FP4_DECODE]
 
 
 def layer_w(wl: dict, K: int, N: int, seed: int = 0) -> np.ndarray:

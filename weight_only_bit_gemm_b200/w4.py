@@ -53,6 +53,10 @@ _SIGS = {
     "nf4_prepack": (_i, [_p, _p, _i, _i, _p, _p]),
     "nf4_workspace_bytes": (_sz, [_i, _i, _i]),
     "nf4_gemm": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "fp4_quantize": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p]),
+    "fp4_dequant": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p]),
+    "fp4_levels": (None, [_p]),
+    "fp4_gemm": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -268,13 +272,21 @@ def w4a16_awq_gemm(X, s, Wp, N, K, G, act_order=False, out=None, workspace=None)
 
 # ----------------------------------------------------------------- NF4
 
-def nf4_levels():
+def _levels(fn):
     buf = (ctypes.c_float * 16)()
-    lib.nf4_levels(ctypes.cast(buf, ctypes.c_void_p))
+    fn(ctypes.cast(buf, ctypes.c_void_p))
     return list(buf)
 
 
-def nf4_quantize(W, blocksize=64, dq_group=256):
+def nf4_levels():
+    return _levels(lib.nf4_levels)
+
+
+def fp4_levels():
+    return _levels(lib.fp4_levels)
+
+
+def _blockwise_quantize(fn, name, W, blocksize, dq_group):
     _cuda(W, torch.float32, "W")
     N, K = W.shape
     dev = W.device
@@ -282,20 +294,39 @@ def nf4_quantize(W, blocksize=64, dq_group=256):
     Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
     aq = torch.empty(nb, dtype=torch.uint8, device=dev)
     s2 = torch.empty((nb + dq_group - 1) // dq_group, dtype=torch.float32, device=dev)
-    _check(lib.nf4_quantize(_ptr(W), N, K, blocksize, dq_group, _ptr(Wq), _ptr(aq), _ptr(s2),
-                            _stream()), "nf4_quantize")
+    _check(fn(_ptr(W), N, K, blocksize, dq_group, _ptr(Wq), _ptr(aq), _ptr(s2), _stream()), name)
     return Wq, aq, s2
 
 
-def nf4_dequant(Wq, absmax_q, s2, dq_group=256, blocksize=64):
+def _blockwise_dequant(fn, name, Wq, absmax_q, s2, dq_group, blocksize):
     N, K = Wq.shape[0], Wq.shape[1] * 2
     out = torch.empty((N, K), dtype=torch.bfloat16, device=Wq.device)
-    _check(lib.nf4_dequant(_ptr(Wq), _ptr(absmax_q), _ptr(s2), N, K, blocksize, dq_group,
-                           _ptr(out), _stream()), "nf4_dequant")
+    _check(fn(_ptr(Wq), _ptr(absmax_q), _ptr(s2), N, K, blocksize, dq_group, _ptr(out),
+              _stream()), name)
     return out
 
 
+def nf4_quantize(W, blocksize=64, dq_group=256):
+    return _blockwise_quantize(lib.nf4_quantize, "nf4_quantize", W, blocksize, dq_group)
+
+
+def nf4_dequant(Wq, absmax_q, s2, dq_group=256, blocksize=64):
+    return _blockwise_dequant(lib.nf4_dequant, "nf4_dequant", Wq, absmax_q, s2, dq_group,
+                              blocksize)
+
+
+def fp4_quantize(W, blocksize=64, dq_group=256):
+    """FP4 (E2M1 / 6) codes in the NF4 block-wise layout: (Wq, absmax codes, s2)."""
+    return _blockwise_quantize(lib.fp4_quantize, "fp4_quantize", W, blocksize, dq_group)
+
+
+def fp4_dequant(Wq, absmax_q, s2, dq_group=256, blocksize=64):
+    return _blockwise_dequant(lib.fp4_dequant, "fp4_dequant", Wq, absmax_q, s2, dq_group,
+                              blocksize)
+
+
 def nf4_prepack(Wq, absmax_q):
+    """Prepack NF4 or FP4 codes (the layout is shared)."""
     N, K = Wq.shape[0], Wq.shape[1] * 2
     nbytes = lib.nf4_prepacked_bytes(N, K)
     if nbytes == 0:
@@ -309,13 +340,22 @@ def nf4_workspace_bytes(M, N, K) -> int:
     return lib.nf4_workspace_bytes(M, N, K)
 
 
-def nf4_gemm(X, Wp, s2, N, K, dq_group=256, out=None, workspace=None):
+def _blockwise_gemm(fn, name, X, Wp, s2, N, K, dq_group, out, workspace):
     _cuda(X, torch.bfloat16, "X")
     M = X.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
     need = nf4_workspace_bytes(M, N, K)
     ws = _ws_view(workspace if workspace is not None else _WS.get(need, X.device))
-    _check(lib.nf4_gemm(_ptr(X), _ptr(Wp), _ptr(s2), M, N, K, dq_group, _ptr(out), _ptr(ws),
-                        ws.numel(), _stream()), "nf4_gemm")
+    _check(fn(_ptr(X), _ptr(Wp), _ptr(s2), M, N, K, dq_group, _ptr(out), _ptr(ws), ws.numel(),
+              _stream()), name)
     return out
+
+
+def nf4_gemm(X, Wp, s2, N, K, dq_group=256, out=None, workspace=None):
+    return _blockwise_gemm(lib.nf4_gemm, "nf4_gemm", X, Wp, s2, N, K, dq_group, out, workspace)
+
+
+def fp4_gemm(X, Wp, s2, N, K, dq_group=256, out=None, workspace=None):
+    """Y = X . w_hat^T for FP4 weights prepacked with nf4_prepack."""
+    return _blockwise_gemm(lib.fp4_gemm, "fp4_gemm", X, Wp, s2, N, K, dq_group, out, workspace)
