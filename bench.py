@@ -536,6 +536,22 @@ def measure_rows(w4, peaks):
         "frac_of_hbm": sum(awq_bytes) / sum(ts) / 1e6 / hbm,
         "same_weights_without_factor_TB/s": sum(awq_bytes) / sum(tp) / 1e9}
 
+    # NEXT row: GPTQ at quantization time (13B MLP up-projection, act-order, G = 32,
+    # 512 calibration tokens): Hessian, then the compensated quantization
+    K, N, G, ncal = 5120, 13824, ao["G"], 512
+    W = torch.from_numpy(S.layer_w(ao, K, N)).cuda()
+    xc = bf16_dev(S.draw_calib_x(ncal, K, tag=ao["tag"]))
+    t_h = time_calls([lambda: w4.gptq_hessian(xc)], reps=3)[0]
+    H = w4.gptq_hessian(xc)
+    t_q = time_calls([lambda: w4.gptq_quantize(W, H, G, True)], reps=2, warm=1)[0]
+    fl_h = 2.0 * ncal * K * K
+    fl_q = 2.0 * K ** 3 / 3 + 1.0 * N * K * K   # factor + inverse, column updates
+    rows["gptq"] = {"shape": [N, K], "G": G, "act_order": True, "calib_tokens": ncal,
+                    "hessian_ms": t_h, "hessian_TFLOP/s": fl_h / t_h / 1e9,
+                    "quantize_ms": t_q, "quantize_TFLOP/s": fl_q / t_q / 1e9}
+    del W, xc, H
+    torch.cuda.empty_cache()
+
     # a8: prefill tensor-core GEMM (70B MLP shapes)
     pf = S.PREFILL_70B
     out = {}
@@ -652,6 +668,14 @@ def run_single(w4, args):
         gemm = w4.nf4_gemm if fmt == "nf4" else w4.fp4_gemm
         f = (lambda: gemm(X, wp, s2, N, K))
         nbytes, flops = nf4_bytes(M, N, K), 2.0 * M * N * K
+    elif fmt == "gptq":
+        # M = calibration tokens; act-order, G = 32 (the 13B act-order family)
+        G = S.ACT_ORDER_13B["G"]
+        W = torch.from_numpy(S.layer_w(S.ACT_ORDER_13B, K, N)).cuda()
+        xc = bf16_dev(S.draw_calib_x(M, K, tag=S.ACT_ORDER_13B["tag"]))
+        H = w4.gptq_hessian(xc)
+        f = (lambda W=W, H=H: w4.gptq_quantize(W, H, G, True))
+        nbytes, flops = N * K * 4, 2.0 * K ** 3 / 3 + 1.0 * N * K * K
     elif fmt == "awq":
         aw = S.AWQ_SYM_DECODE
         G = aw["G"]
@@ -687,7 +711,7 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the other-row measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--single", nargs=4, metavar=("FMT", "K", "N", "M"),
-                    help="profiling aid: run one layer call (FMT int4|nf4|fp4|awq) warmup+steps times "
+                    help="profiling aid: run one layer call (FMT int4|nf4|fp4|awq|gptq) warmup+steps times "
                          "eagerly and print its mean device time")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -137,6 +137,46 @@ w4_status w4_awq_scale_weights(const float* W, const float* s, int N, int K, flo
 w4_status w4_awq_scale_activations(const uint16_t* X, const float* s, int M, int K,
                                    uint16_t* X_out, w4_stream stream);
 
+/* GPTQ error compensation at quantization time ([Comparison] §3.1; [Survey]
+ * §3, §3.2).  The layer's columns are quantized one at a time (INT4, the
+ * asymmetric RTN rule of w4_quantize_rtn per group) and each column's error
+ * is spread over the columns not yet quantized through the inverse of the
+ * damped Hessian H' = H + lambda I, lambda = damp * mean(diag H):
+ *   Hi = H'^-1 over the remaining columns; for column j:
+ *     q_j = quantize(w_j);  e = (w_j - dq(q_j)) / Hi_jj
+ *     w_k -= e * Hi_jk for every later k;  Hi loses row/column j (Gaussian
+ *     elimination, i.e. Hi becomes the inverse of H' without column j).
+ * A group's scale and zero point are taken from its current (compensated)
+ * weights when its first column is reached.  A channel with H_kk = 0 gets
+ * H_kk = 1 and weight 0.  With act_order the columns are taken in the order
+ * of decreasing H_kk (stable), group g holds the channels processed in
+ * positions [gG, (g+1)G), and g_idx receives that map (the act-order format
+ * of w4_quantize_rtn / w4_prepack).  The device computes Hi's upper Cholesky
+ * factor once in fp64 and runs the column updates in fp32; the result agrees
+ * with an fp64 evaluation of the steps above up to rounding (a weight near a
+ * rounding boundary may take the neighbouring code).
+ *   W         in   fp32 [N, K]
+ *   H         in   fp32 [K, K], symmetric positive semi-definite (e.g. from
+ *                  w4_gptq_hessian); a negative or non-finite diagonal entry
+ *                  or a non-positive pivot is reported as W4_ERR_DEVICE_INPUT
+ *   G         32, 64 or 128; K % G == 0, K % 32 == 0, K <= 65536
+ *   damp      >= 0 (the pages use 0.01)
+ *   Wq, scales, zeros  out, as w4_quantize_rtn
+ *   g_idx     out  int32 [K]; required with act_order, else may be NULL
+ *                  (then receives k / G)
+ *   workspace device memory of w4_gptq_workspace_bytes(N, K, G) bytes,
+ *             256-byte aligned, contents irrelevant (about 20 K^2 + 9 N K B) */
+size_t w4_gptq_workspace_bytes(int N, int K, int G);
+w4_status w4_gptq_quantize(const float* W, const float* H, int N, int K, int G, int act_order,
+                           float damp, uint8_t* Wq, uint16_t* scales, uint8_t* zeros,
+                           int32_t* g_idx, void* workspace, size_t workspace_bytes,
+                           w4_stream stream);
+
+/* H = 2 X^T X ([Comparison] §3.1: H = 2 X X^T with X the calibration
+ * activations as columns), fp32 accumulation.
+ *   X  in   bf16 [n, K] (n calibration tokens);  H  out  fp32 [K, K]     */
+w4_status w4_gptq_hessian(const uint16_t* X, int n, int K, float* H, w4_stream stream);
+
 /* Dequantization to the bf16 compute dtype ([Survey] §6.2, [Primer] §七):
  *   w_hat[n,k] = bf16_rne( float(q - zp) * float(scale) )
  * (the fp32 product is exact, so there is exactly one rounding).

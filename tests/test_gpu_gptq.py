@@ -1,0 +1,144 @@
+"""GPU parity for GPTQ error compensation, through the C ABI, against the CPU
+oracle on the same seeded inputs.
+
+The device factorizes the inverse Hessian once in fp64 and runs the column
+updates in fp32, the oracle eliminates in fp64, so a weight near a rounding
+boundary may take the neighbouring code on one side and the difference then
+propagates along its row.  Checked exactly: the Hessian's symmetry, the
+identity-Hessian case (equal to plain RTN), the first group's scales and
+zero points, the act-order map, dead channels.  Checked by property: code
+agreement with the oracle, the layer error tr((W - W_hat) H (W - W_hat)^T)
+against the oracle's and RTN's, and a GEMM on the result."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from weight_only_bit_gemm_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def w4():
+    from weight_only_bit_gemm_b200 import build
+    build.build()
+    from weight_only_bit_gemm_b200 import w4 as mod
+    return mod
+
+
+def dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.view(dtype)
+    return t.cuda()
+
+
+def host_u16(t):
+    return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def status_ok(w4):
+    assert w4.device_status() == w4.W4_OK
+
+
+@pytest.mark.parametrize("n,K", [(384, 256), (100, 1000), (512, 1024)])
+def test_gptq_hessian(w4, n, K):
+    xb = S.draw_calib_x(n, K, seed=1, tag=40)
+    H = w4.gptq_hessian(dev(xb.view(np.int16), torch.bfloat16))
+    status_ok(w4)
+    h = H.cpu().numpy().astype(np.float64)
+    assert np.array_equal(h, h.T)
+    ref = O.gptq_hessian(xb)
+    xa = np.abs(O.bf16_bits_to_f64(xb))
+    bound = 2.0 * (xa.T @ xa) * (n * 2.0 ** -23) + 1e-30
+    assert np.all(np.abs(h - ref) <= bound)
+
+
+@pytest.mark.parametrize("act", [False, True])
+def test_gptq_identity_hessian_is_rtn(w4, act):
+    N, K, G = 96, 512, 64
+    W = S.draw_w(N, K, 0.02, seed=2, tag=41)
+    H = (3.0 * np.eye(K)).astype(np.float32)
+    Wq, sc, zr, gi = w4.gptq_quantize(dev(W), dev(H), G, act)
+    status_ok(w4)
+    q, s, z = O.quantize_rtn(W, G)
+    assert np.array_equal(Wq.cpu().numpy(), O.pack_nibbles(q))
+    assert np.array_equal(host_u16(sc), s.view(np.uint16))
+    assert np.array_equal(zr.cpu().numpy(), z)
+    if act:
+        assert np.array_equal(gi.cpu().numpy(), np.arange(K) // G)
+
+
+GPTQ_CASES = [
+    # (N, K, G, act, n)
+    (64, 256, 32, False, 384),
+    (300, 1024, 128, False, 512),
+    (200, 768, 64, True, 384),
+    (130, 1024, 32, True, 512),
+]
+
+
+@pytest.mark.parametrize("N,K,G,act,n", GPTQ_CASES)
+def test_gptq_against_oracle(w4, N, K, G, act, n):
+    xb = S.draw_calib_x(n, K, seed=3, tag=42)
+    H = O.gptq_hessian(xb).astype(np.float32)
+    H[11, :] = 0.0
+    H[:, 11] = 0.0                          # a channel never activated
+    W = S.draw_w(N, K, 0.02, seed=3, tag=42)
+    Wq, sc, zr, gi = w4.gptq_quantize(dev(W), dev(H), G, act)
+    status_ok(w4)
+    qo, so, zo, go = O.gptq_quantize(W, H.astype(np.float64), G, act)
+    q = O.unpack_nibbles(Wq.cpu().numpy())
+    s = host_u16(sc).view(np.float16)
+    z = zr.cpu().numpy()
+    g = gi.cpu().numpy() if act else None
+    if act:
+        assert np.array_equal(g, go)
+    # first group of the processing order: nothing compensated yet -> exact
+    assert np.array_equal(s[:, 0].view(np.uint16), so[:, 0].view(np.uint16))
+    assert np.array_equal(z[:, 0], zo[:, 0])
+    gk = O.group_index(K, G, g)
+    assert np.array_equal(q[:, 11], z[np.arange(N), gk[11]])
+    agree = float(np.mean(q == qo))
+    assert agree >= 0.98, agree
+    Wl = W.copy()
+    Wl[:, 11] = 0.0
+    l_dev = O.gptq_loss(Wl, O.dequant_rtn(O.pack_nibbles(q), s, z, G, g), H)
+    l_ora = O.gptq_loss(Wl, O.dequant_rtn(O.pack_nibbles(qo), so, zo, G, go), H)
+    qr, sr, zr_ = O.quantize_rtn(W, G)
+    l_rtn = O.gptq_loss(Wl, O.dequant_rtn(O.pack_nibbles(qr), sr, zr_, G), H)
+    assert l_dev <= 1.02 * l_ora, (l_dev, l_ora)
+    assert l_dev < 0.5 * l_rtn, (l_dev, l_rtn)
+
+
+def test_gptq_output_feeds_the_gemm(w4):
+    N, K, G, M = 256, 1024, 32, 8
+    xb = S.draw_calib_x(384, K, seed=4, tag=43)
+    Hd = w4.gptq_hessian(dev(xb.view(np.int16), torch.bfloat16))
+    W = S.draw_w(N, K, 0.02, seed=4, tag=43)
+    Wq, sc, zr, gi = w4.gptq_quantize(dev(W), Hd, G, True)
+    Wp = w4.prepack(Wq, sc, zr, G, gi)
+    x = S.draw_x(M, K, seed=4, tag=43, N=N)
+    y = w4.w4a16_gemm(dev(x.view(np.int16), torch.bfloat16), Wp, N, K, G, True)
+    status_ok(w4)
+    what = O.dequant_rtn(Wq.cpu().numpy(), host_u16(sc).view(np.float16), zr.cpu().numpy(), G,
+                         gi.cpu().numpy())
+    y_ref, ab = O.matmul_ref(x, what)
+    ok, ratio = O.check_matmul(host_u16(y), y_ref, ab)
+    assert ok, ratio
+
+
+def test_gptq_bad_hessian_reported(w4):
+    N, K, G = 16, 128, 32
+    W = S.draw_w(N, K, 0.02, seed=5, tag=44)
+    H = np.eye(K, dtype=np.float32)
+    H[3, 3] = -1.0                          # not a Hessian
+    w4.gptq_quantize(dev(W), dev(H), G)
+    assert w4.device_status() == w4.W4_ERR_DEVICE_INPUT
+    status_ok(w4)                           # cleared; the context is usable
+    H[3, 3] = 1.0
+    Wq, _, _, _ = w4.gptq_quantize(dev(W), dev(H), G)
+    status_ok(w4)
+    q, _, _ = O.quantize_rtn(W, G)
+    assert np.array_equal(Wq.cpu().numpy(), O.pack_nibbles(q))

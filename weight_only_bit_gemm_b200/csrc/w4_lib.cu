@@ -13,6 +13,7 @@
 #include "../../include/w4.h"
 #include "w4_gemm_kernel.cuh"
 #include "w4_gemv_kernel.cuh"
+#include "w4_gptq.cuh"
 #include "w4_prepack.cuh"
 #include "w4_quant.cuh"
 #include "w4_ptx.cuh"
@@ -157,6 +158,127 @@ w4_status w4_awq_scale_weights(const float* W, const float* s, int N, int K, flo
       std::min<size_t>((total + 255) / 256, static_cast<size_t>(sm_count()) * 16);
   awq_scale_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(
       W, s, N, K, W_out);
+  return launch_status(cudaGetLastError());
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// GPTQ: workspace regions (each 256-byte aligned).
+namespace {
+
+struct GptqLayout {
+  size_t A, T, U, Q, E, codes, d, lambda, dead, perm, pos, total;
+};
+
+GptqLayout gptq_layout(int N, int K) {
+  auto r = [](size_t v) { return (v + 255) / 256 * 256; };
+  const size_t kk = static_cast<size_t>(K) * K, nk = static_cast<size_t>(N) * K;
+  GptqLayout l{};
+  size_t o = 0;
+  l.A = o;      o += r(kk * 8);
+  l.T = o;      o += r(kk * 8);
+  l.U = o;      o += r(kk * 4);
+  l.Q = o;      o += r(nk * 4);
+  l.E = o;      o += r(static_cast<size_t>(kGptqB) * N * 4);
+  l.codes = o;  o += r(nk);
+  l.d = o;      o += r(static_cast<size_t>(K) * 8);
+  l.lambda = o; o += 256;
+  l.dead = o;   o += r(static_cast<size_t>(K));
+  l.perm = o;   o += r(static_cast<size_t>(K) * 4);
+  l.pos = o;    o += r(static_cast<size_t>(K) * 4);
+  l.total = o;
+  return l;
+}
+
+bool gptq_shape_ok(int N, int K, int G) {
+  return int4_shape_ok(N, K, G) && K % kChol == 0 && K <= 65536;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t w4_gptq_workspace_bytes(int N, int K, int G) {
+  if (!gptq_shape_ok(N, K, G)) return 0;
+  return gptq_layout(N, K).total;
+}
+
+w4_status w4_gptq_hessian(const uint16_t* X, int n, int K, float* H, w4_stream stream) {
+  if (!X || !H || n < 1 || K < 1 || K > 65536) return W4_ERR_INVALID_ARG;
+  if (!aligned(X, 2) || !aligned(H, 4)) return W4_ERR_INVALID_ARG;
+  const int t = ceil_div(K, 64);
+  gptq_hessian_kernel<<<dim3(t, t), 256, 0, as_stream(stream)>>>(X, n, K, H);
+  return launch_status(cudaGetLastError());
+}
+
+w4_status w4_gptq_quantize(const float* W, const float* H, int N, int K, int G, int act_order,
+                           float damp, uint8_t* Wq, uint16_t* scales, uint8_t* zeros,
+                           int32_t* g_idx, void* workspace, size_t workspace_bytes,
+                           w4_stream stream) {
+  if (!W || !H || !Wq || !scales || !zeros || !workspace) return W4_ERR_INVALID_ARG;
+  if (act_order && !g_idx) return W4_ERR_INVALID_ARG;
+  if (!gptq_shape_ok(N, K, G) || !(damp >= 0.0f)) return W4_ERR_INVALID_ARG;
+  if (!aligned(W, 4) || !aligned(H, 4) || !aligned(scales, 2) || !aligned(workspace, 256) ||
+      (g_idx && !aligned(g_idx, 4)))
+    return W4_ERR_INVALID_ARG;
+  const GptqLayout l = gptq_layout(N, K);
+  if (workspace_bytes < l.total) return W4_ERR_INVALID_ARG;
+  static std::atomic<uint64_t> smem_set{0};
+  if (ensure_smem_limit(gptq_block_kernel, static_cast<int>(kGptqBlockSmem), smem_set) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return W4_ERR_CUDA;
+  }
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* A = reinterpret_cast<double*>(ws + l.A);
+  double* T = reinterpret_cast<double*>(ws + l.T);
+  float* U = reinterpret_cast<float*>(ws + l.U);
+  float* Q = reinterpret_cast<float*>(ws + l.Q);
+  float* E = reinterpret_cast<float*>(ws + l.E);
+  uint8_t* codes = ws + l.codes;
+  double* d = reinterpret_cast<double*>(ws + l.d);
+  double* lambda = reinterpret_cast<double*>(ws + l.lambda);
+  uint8_t* dead = ws + l.dead;
+  int32_t* perm = reinterpret_cast<int32_t*>(ws + l.perm);
+  int32_t* pos = reinterpret_cast<int32_t*>(ws + l.pos);
+
+  // prepare: diagonal, order, damping, A = J P^T H P J + lambda I, Q = W P
+  gptq_diag_kernel<<<ceil_div(K, 256), 256, 0, st>>>(H, K, d, dead);
+  gptq_order_kernel<<<ceil_div(K, 256), 256, 0, st>>>(d, K, act_order ? 1 : 0, perm, pos);
+  gptq_damp_kernel<<<1, 256, 0, st>>>(d, K, static_cast<double>(damp), lambda);
+  gptq_build_kernel<<<dim3(ceil_div(K, 32), ceil_div(K, 8)), 256, 0, st>>>(H, d, perm, lambda,
+                                                                            K, A);
+  const size_t nk = static_cast<size_t>(N) * K;
+  gptq_gather_w_kernel<<<static_cast<unsigned>((nk + 255) / 256), 256, 0, st>>>(W, perm, dead, N,
+                                                                               K, Q);
+  // factor: A = L' L'^T (lower, in place), T = L'^-1, U = J T J
+  const int nb = K / kChol;
+  for (int jb = 0; jb < nb; ++jb) {
+    chol_diag_kernel<<<1, kChol * kChol, 0, st>>>(A, K, jb);
+    const int rest = nb - jb - 1;
+    if (rest > 0) {
+      chol_panel_kernel<<<rest, kChol, 0, st>>>(A, K, jb);
+      chol_update_kernel<<<dim3(rest, rest), kChol * kChol, 0, st>>>(A, K, jb);
+    }
+  }
+  trinv_diag_kernel<<<nb, kChol, 0, st>>>(A, K, T);
+  for (int ib = 1; ib < nb; ++ib) trinv_row_kernel<<<ib, kChol * kChol, 0, st>>>(A, K, ib, T);
+  gptq_u_kernel<<<dim3(ceil_div(K, 32), ceil_div(K, 8)), 256, 0, st>>>(T, K, U);
+  // quantize: lazy blocks of kGptqB columns
+  for (int j0 = 0; j0 < K; j0 += kGptqB) {
+    const int bw = std::min(kGptqB, K - j0);
+    gptq_block_kernel<<<ceil_div(N, kGptqRows), kGptqRows, kGptqBlockSmem, st>>>(
+        Q, U, N, K, G, j0, bw, E, codes, scales, zeros);
+    if (j0 + bw < K)
+      gptq_trailing_kernel<<<dim3(ceil_div(K - j0 - bw, 64), ceil_div(N, 64)), 256, 0, st>>>(
+          Q, U, E, N, K, j0, bw);
+  }
+  const size_t half = nk / 2;
+  gptq_pack_kernel<<<static_cast<unsigned>((half + 255) / 256), 256, 0, st>>>(codes, pos, N, K,
+                                                                              Wq);
+  if (g_idx) gptq_gidx_kernel<<<ceil_div(K, 256), 256, 0, st>>>(pos, K, G, g_idx);
   return launch_status(cudaGetLastError());
 }
 

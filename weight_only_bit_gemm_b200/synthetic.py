@@ -18,6 +18,10 @@ distributions the workloads name:
   pattern in a ``uint16`` array.
 * ``g_idx``: the act-order group map ``g_idx[perm[j]] = j // G`` for a seeded
   permutation ``perm`` of ``range(K)``.
+* calibration activations for GPTQ's Hessian: fp32 ``standard_normal`` ``[n, K]``
+  plus ``rank`` shared factors (``standard_normal [n, rank] @ standard_normal
+  [rank, K]``), so that channels are correlated as real activations are,
+  rounded to bf16;
 * ``s``: the AWQ per-input-channel factor, fp32 ``[K]`` uniform in
   ``[lo, hi]`` (default 0.95..1.05, the range
   "【推理与部署篇05】模型量化部署深度对比" §4.1 gives for important and
@@ -27,7 +31,8 @@ Generators (``numpy.random.default_rng`` keyed by integer lists):
 ``[seed, tag, K, N]`` for W (draw order: W, then the outlier columns),
 ``[seed, tag, K, N, M]`` for X (X, then its outlier channels) and
 ``[seed, tag, K, N, 7]`` for the act-order permutation and
-``[seed, tag, K, N, 11]`` for the AWQ factor.
+``[seed, tag, K, N, 11]`` for the AWQ factor and ``[seed, tag, K, n, 13]`` for the
+calibration activations.
 """
 from __future__ import annotations
 
@@ -62,6 +67,17 @@ def draw_awq_s(K: int, *, seed: int = 0, tag: int = 0, N: int = 0, lo: float = 0
                hi: float = 1.05) -> np.ndarray:
     """fp32 per-input-channel factor ``[K]`` uniform in ``[lo, hi]``."""
     return _rng(seed, tag, K, N, 11).uniform(lo, hi, K).astype(np.float32)
+
+
+def draw_calib_x(n: int, K: int, *, seed: int = 0, tag: int = 0, rank: int = 4) -> np.ndarray:
+    """bf16 calibration activations ``[n, K]`` (uint16 bits) with ``rank``
+    shared factors."""
+    rng = _rng(seed, tag, K, n, 13)
+    x = rng.standard_normal((n, K), dtype=np.float32)
+    if rank > 0:
+        x += rng.standard_normal((n, rank), dtype=np.float32) @ \
+            rng.standard_normal((rank, K), dtype=np.float32)
+    return to_bf16_bits(x)
 
 
 def act_order_g_idx(perm: np.ndarray, G: int) -> np.ndarray:

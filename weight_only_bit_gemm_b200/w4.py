@@ -37,6 +37,10 @@ _SIGS = {
     "w4_quantize_sym": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p]),
     "w4_awq_scale_weights": (_i, [_p, _p, _i, _i, _p, _p]),
     "w4_awq_scale_activations": (_i, [_p, _p, _i, _i, _p, _p]),
+    "w4_gptq_workspace_bytes": (_sz, [_i, _i, _i]),
+    "w4_gptq_quantize": (_i, [_p, _p, _i, _i, _i, _i, ctypes.c_float, _p, _p, _p, _p, _p, _sz,
+                              _p]),
+    "w4_gptq_hessian": (_i, [_p, _i, _i, _p, _p]),
     "w4_dequant": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "w4_prepacked_bytes": (_sz, [_i, _i, _i, _i]),
     "w4_prepack": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
@@ -159,6 +163,36 @@ def awq_scale_activations(X, s, out=None):
     _check(lib.w4_awq_scale_activations(_ptr(X), _ptr(s), M, K, _ptr(out), _stream()),
            "w4_awq_scale_activations")
     return out
+
+
+def gptq_hessian(X):
+    """H = 2 X^T X (fp32 [K, K]) for bf16 calibration activations X [n, K]."""
+    _cuda(X, torch.bfloat16, "X")
+    n, K = X.shape
+    H = torch.empty((K, K), dtype=torch.float32, device=X.device)
+    _check(lib.w4_gptq_hessian(_ptr(X), n, K, _ptr(H), _stream()), "w4_gptq_hessian")
+    return H
+
+
+def gptq_quantize(W, H, G, act_order=False, damp=0.01):
+    """INT4 codes with GPTQ error compensation: (Wq, scales, zeros, g_idx)
+    in the format of quantize_rtn (g_idx None without act-order)."""
+    _cuda(W, torch.float32, "W")
+    _cuda(H, torch.float32, "H")
+    N, K = W.shape
+    dev = W.device
+    need = lib.w4_gptq_workspace_bytes(N, K, G)
+    if need == 0:
+        raise W4Error(W4_ERR_INVALID_ARG, "w4_gptq_workspace_bytes")
+    ws = _ws_view(torch.empty(need + 256, dtype=torch.uint8, device=dev))
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    sc = torch.empty((N, K // G), dtype=torch.float16, device=dev)
+    zr = torch.empty((N, K // G), dtype=torch.uint8, device=dev)
+    gi = torch.empty(K, dtype=torch.int32, device=dev) if act_order else None
+    _check(lib.w4_gptq_quantize(_ptr(W), _ptr(H), N, K, G, int(bool(act_order)), float(damp),
+                                _ptr(Wq), _ptr(sc), _ptr(zr), _ptr(gi), _ptr(ws), ws.numel(),
+                                _stream()), "w4_gptq_quantize")
+    return Wq, sc, zr, gi
 
 
 def dequant(Wq, scales, zeros, G, g_idx=None):
