@@ -1,5 +1,6 @@
-"""Oracle: group-wise INT4 (asymmetric and symmetric RTN) and NF4 / FP4
-(block-wise, double-quantized) weight quantization, the AWQ per-input-channel factor,
+"""Oracle: group-wise INT4 (asymmetric and symmetric RTN, GPTQ) and NF4 / FP4
+(block-wise, double-quantized) weight quantization, the LLM.int8 mixed
+decomposition, the AWQ per-input-channel factor,
 packing, dequantization and the fp64 matmul reference.
 
 TEST INFRASTRUCTURE ONLY -- see the package docstring for who may import it.
@@ -44,7 +45,11 @@ R18 GPTQ: H = 2 X^T X (fp64); dead channels H_kk = 0 -> 1 and w_k = 0;
     act-order = stable sort by decreasing H_kk; damping 0.01 * mean(diag H);
     the update uses the inverse Hessian of the remaining columns, eliminated
     one column at a time; group parameters from the compensated weights at
-    the group's first column; codes decided in fp32.
+    the group's first column; codes decided in fp32;
+R19 LLM.int8: per-row weight absmax/127, outlier channels |x| > 6.0 in any
+    token of the call, per-token activation absmax/127 over the other
+    channels, exact INT8 sum scaled by s_x s_w plus the outlier channels'
+    product with bf16 dequantized INT8 weights.
 
 All floating-point steps are numpy float32 operations (IEEE, round to nearest
 even) unless stated as fp64; the matmul accumulates in fp64.
@@ -72,6 +77,7 @@ __all__ = [
     "sym_params", "quantize_sym", "awq_scale_weights", "awq_scale_activations",
     "fp4_table", "fp4_midpoints", "fp4_codes", "fp4_quantize", "fp4_dequant",
     "gptq_hessian", "gptq_prepare", "gptq_eliminate", "gptq_quantize", "gptq_loss",
+    "int8_quantize_weights", "int8_outliers", "int8_quantize_activations", "int8_mixed_ref",
 ]
 
 F32 = np.float32
@@ -528,6 +534,65 @@ def gptq_loss(W: np.ndarray, what_bits: np.ndarray, H: np.ndarray) -> float:
     quantity the compensation lowers; H undamped)."""
     D = np.asarray(W, dtype=np.float64) - bf16_bits_to_f64(what_bits)
     return float(np.einsum("nk,kl,nl->", D, np.asarray(H, np.float64), D))
+
+
+# ---------------------------------------------------------------------------
+# LLM.int8 mixed decomposition.  [Survey] §2.1: vector-wise quantization (one
+# scale per column of the weight matrix, i.e. per output feature: row n of
+# W [N, K] here) and mixed-precision decomposition (the feature dimensions
+# where the activations exceed 6.0 in magnitude go through a 16-bit matmul,
+# the rest through INT8, and the two results are added).  [Comparison] §6.1:
+# llm_int8_threshold = 6.0 and no 16-bit copy of the weights is kept.
+# Readings (R19):
+#   s_w[n] = max_k |w| / 127 (fp32; 1 if 0), q_w = clamp(rint(w / s_w), +-127);
+#   O = {k : |x[m, k]| > threshold for some token m of the call};
+#   s_x[m] = max_{k not in O} |x[m, k]| / 127 (1 if 0);
+#   q_x = clamp(rint(x / s_x), +-127) outside O and 0 inside O;
+#   y[m, n] = (sum_k q_x q_w) s_x[m] s_w[n] + sum_{k in O} x[m, k] w16[n, k],
+#   w16 = bf16(fp32(q_w s_w)) (the 16-bit weights of the outlier channels are
+#   the dequantized INT8 ones); the INT8 sum is exact (int64 here).
+# ---------------------------------------------------------------------------
+
+def int8_quantize_weights(W: np.ndarray):
+    """Per output row: (q_w int8 [N, K], s_w fp32 [N])."""
+    W = np.ascontiguousarray(W, dtype=F32)
+    s = (np.abs(W).max(axis=1) / F32(127.0)).astype(F32)
+    s[s == 0] = F32(1.0)
+    q = np.clip(np.rint(W / s[:, None]), -127, 127).astype(np.int8)
+    return q, s
+
+
+def int8_outliers(x_bits: np.ndarray, threshold: float = 6.0) -> np.ndarray:
+    """Outlier channels of a call: bool [K], |x| > threshold for some token."""
+    x = bf16_bits_to_f32(x_bits)
+    return np.any(np.abs(x) > F32(threshold), axis=0)
+
+
+def int8_quantize_activations(x_bits: np.ndarray, outliers: np.ndarray):
+    """Per token over the non-outlier channels: (q_x int8 [M, K], s_x fp32 [M])."""
+    x = bf16_bits_to_f32(x_bits)
+    keep = ~np.asarray(outliers, dtype=bool)
+    a = np.where(keep[None, :], np.abs(x), F32(0)).max(axis=1)
+    s = (a / F32(127.0)).astype(F32)
+    s[s == 0] = F32(1.0)
+    q = np.clip(np.rint(x / s[:, None]), -127, 127)
+    q = np.where(keep[None, :], q, 0).astype(np.int8)
+    return q, s
+
+
+def int8_mixed_ref(x_bits: np.ndarray, q_w: np.ndarray, s_w: np.ndarray,
+                   threshold: float = 6.0):
+    """(y_ref fp64 [M, N], abs_ref fp64 [M, N]) of the decomposed product."""
+    O_ = int8_outliers(x_bits, threshold)
+    q_x, s_x = int8_quantize_activations(x_bits, O_)
+    acc = q_x.astype(np.int64) @ q_w.astype(np.int64).T                 # exact
+    sx = s_x.astype(np.float64)[:, None]
+    sw = s_w.astype(np.float64)[None, :]
+    y_int = acc.astype(np.float64) * sx * sw
+    a_int = (np.abs(q_x).astype(np.int64) @ np.abs(q_w).astype(np.int64).T) * sx * sw
+    w16 = bf16_bits_to_f64(bf16_round_bits((q_w[:, O_].astype(F32) * s_w[:, None]).astype(F32)))
+    x = bf16_bits_to_f64(x_bits)[:, O_]
+    return y_int + x @ w16.T, a_int + np.abs(x) @ np.abs(w16).T
 
 
 # ---------------------------------------------------------------------------

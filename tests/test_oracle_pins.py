@@ -749,6 +749,99 @@ def test_planted_mistakes_gptq(monkeypatch):
     assert caught("gptq_prepare", undamped_as_hessian)
 
 
+# ---------------------------------------------------------------- LLM.int8
+
+INT8_WORKED = _parse_worked(os.path.join(GOLDEN, "int8_mixed_worked.txt"))
+
+
+@pytest.mark.parametrize("case", INT8_WORKED, ids=lambda c: c["name"])
+def test_int8_worked_example(case):
+    f = lambda key: np.array([float(v) for v in case[key]], np.float32)
+    xb = S.to_bf16_bits(f("x")[None, :])
+    W = np.stack([f("w0"), f("w1")])
+    qw, sw = O.int8_quantize_weights(W)
+    assert qw[0].tolist() == [int(v) for v in case["qw0"]] and np.all(qw[1] == 0)
+    assert sw.tolist() == [float(v) for v in case["sw"]]
+    Ol = O.int8_outliers(xb)
+    assert np.flatnonzero(Ol).tolist() == [int(v) for v in case["outliers"]]
+    qx, sx = O.int8_quantize_activations(xb, Ol)
+    assert qx[0].tolist() == [int(v) for v in case["qx"]]
+    assert sx.tolist() == [float(v) for v in case["sx"]]
+    y, _ = O.int8_mixed_ref(xb, qw, sw)
+    assert y[0].tolist() == [float(v) for v in case["y"]]
+
+
+def test_int8_threshold_is_strict_and_all_outliers_is_16bit():
+    xb = S.to_bf16_bits(np.array([[6.0, -6.0, 6.03125, 1.0]], np.float32))
+    assert np.flatnonzero(O.int8_outliers(xb)).tolist() == [2]
+    # every channel an outlier: the INT8 part vanishes, y = x . bf16(q_w s_w)
+    W = _rand_w(8, 64, 52)
+    xb = S.draw_x(3, 64, seed=5)
+    qw, sw = O.int8_quantize_weights(W)
+    y, _ = O.int8_mixed_ref(xb, qw, sw, threshold=0.0)
+    w16 = O.bf16_bits_to_f64(O.bf16_round_bits((qw.astype(np.float32) * sw[:, None]).astype(np.float32)))
+    assert np.allclose(y, O.bf16_bits_to_f64(xb) @ w16.T, rtol=1e-12, atol=0)
+
+
+def test_int8_error_bound_against_exact_product():
+    # |y - x W| <= sum_k |x| s_w / 2 + |w| s_x / 2 + s_x s_w / 4 over the INT8
+    # channels, plus the outlier channels' bf16 weight rounding
+    W = _rand_w(32, 1024, 53)
+    xb = S.draw_x(5, 1024, seed=6, outlier_frac=0.005, outlier_scale=40.0)
+    qw, sw = O.int8_quantize_weights(W)
+    y, _ = O.int8_mixed_ref(xb, qw, sw)
+    x = O.bf16_bits_to_f64(xb)
+    Ol = O.int8_outliers(xb)
+    assert Ol.sum() >= 3
+    _, sx = O.int8_quantize_activations(xb, Ol)
+    Wd = W.astype(np.float64)
+    keep = ~Ol
+    b = (np.abs(x[:, keep]) @ np.ones((keep.sum(), 1))) * sw[None, :] / 2 \
+        + sx[:, None].astype(np.float64) * (np.abs(Wd[:, keep]).sum(axis=1)[None, :] / 2) \
+        + keep.sum() * sx[:, None] * sw[None, :] / 4
+    b += np.abs(x[:, Ol]) @ (np.abs(Wd[:, Ol]).T * (2.0 ** -8) + sw[None, :] / 2)
+    assert np.all(np.abs(y - x @ Wd.T) <= b * 1.0001)
+
+
+def test_planted_mistakes_int8(monkeypatch):
+    import oracle.w4_oracle as M
+    checks = [lambda: [test_int8_worked_example(c) for c in INT8_WORKED],
+              test_int8_threshold_is_strict_and_all_outliers_is_16bit,
+              test_int8_error_bound_against_exact_product]
+
+    def caught(name, fn):
+        monkeypatch.setattr(M, name, fn)
+        monkeypatch.setattr(O, name, fn)
+        try:
+            for chk in checks:
+                try:
+                    chk()
+                except AssertionError:
+                    return True
+            return False
+        finally:
+            monkeypatch.undo()
+
+    def per_column_scale(W):                  # one scale per input channel
+        W = np.ascontiguousarray(W, np.float32)
+        s = (np.abs(W).max(axis=0) / np.float32(127.0)).astype(np.float32)
+        s[s == 0] = np.float32(1.0)
+        q = np.clip(np.rint(W / s[None, :]), -127, 127).astype(np.int8)
+        return q, np.ones(W.shape[0], np.float32) * s.mean()
+    assert caught("int8_quantize_weights", per_column_scale)
+
+    def inclusive(x_bits, threshold=6.0):    # >= instead of >
+        return np.any(np.abs(M.bf16_bits_to_f32(x_bits)) >= np.float32(threshold), axis=0)
+    assert caught("int8_outliers", inclusive)
+
+    orig_qa = M.int8_quantize_activations
+
+    def outliers_counted_twice(x_bits, outliers):
+        q, s = orig_qa(x_bits, np.zeros_like(np.asarray(outliers, bool)))
+        return q, s
+    assert caught("int8_quantize_activations", outliers_counted_twice)
+
+
 def _pins_fail(monkeypatch, name, fn):
     """Replace one oracle function by a mutated copy and report whether any
     of the core pins catches it."""
