@@ -536,6 +536,30 @@ def measure_rows(w4, peaks):
         "frac_of_hbm": sum(awq_bytes) / sum(ts) / 1e6 / hbm,
         "same_weights_without_factor_TB/s": sum(awq_bytes) / sum(tp) / 1e9}
 
+    # NEXT row: LLM.int8 mixed decomposition on the Llama-7B decode inputs
+    # (0.1% of channels x50, i.e. outliers above the 6.0 threshold)
+    i8_calls, i8_bytes = [], []
+    for (K, N) in WL["shapes"]:
+        W = torch.from_numpy(S.layer_w(WL, K, N)).cuda()
+        qw, sw = w4.llm_int8_quantize_weights(W)
+        if (K, N) == (4096, 22016):
+            t = time_calls([lambda: w4.llm_int8_quantize_weights(W)], reps=5)[0]
+            b = N * K * 4 + N * K + 4 * N
+            rows["llm_int8_quantize"] = {"shape": [N, K], "ms": t, "GB/s": b / t / 1e6}
+        reps = [qw] + [qw.clone() for _ in range(_replicas_for(qw.numel(), l2) - 1)]
+        for M in WL["Ms"]:
+            X = bf16_dev(S.layer_x(WL, M, K, N))
+            for r in reps:
+                i8_calls.append(lambda X=X, r=r, sw=sw: w4.llm_int8_gemm(X, r, sw))
+                i8_bytes.append(N * K + 4 * N + 2 * M * K + 2 * M * N)
+        del W
+    ts = time_calls(i8_calls, reps=5)
+    rows["llm_int8_decode"] = {
+        "configs": "(K,N) in {(4096,12288),(4096,4096),(4096,22016),(11008,4096)} x M in {1,4,16}, "
+                   "threshold 6.0",
+        "TB/s": sum(i8_bytes) / sum(ts) / 1e9,
+        "frac_of_hbm": sum(i8_bytes) / sum(ts) / 1e6 / hbm}
+
     # NEXT row: GPTQ at quantization time (13B MLP up-projection, act-order, G = 32,
     # 512 calibration tokens): Hessian, then the compensated quantization
     K, N, G, ncal = 5120, 13824, ao["G"], 512
@@ -676,6 +700,12 @@ def run_single(w4, args):
         H = w4.gptq_hessian(xc)
         f = (lambda W=W, H=H: w4.gptq_quantize(W, H, G, True))
         nbytes, flops = N * K * 4, 2.0 * K ** 3 / 3 + 1.0 * N * K * K
+    elif fmt == "int8":
+        W = torch.from_numpy(S.layer_w(WL, K, N)).cuda()
+        qw, sw = w4.llm_int8_quantize_weights(W)
+        X = bf16_dev(S.layer_x(WL, M, K, N))
+        f = (lambda: w4.llm_int8_gemm(X, qw, sw))
+        nbytes, flops = N * K + 4 * N + 2 * M * K + 2 * M * N, 2.0 * M * N * K
     elif fmt == "awq":
         aw = S.AWQ_SYM_DECODE
         G = aw["G"]
@@ -711,7 +741,7 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the other-row measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--single", nargs=4, metavar=("FMT", "K", "N", "M"),
-                    help="profiling aid: run one layer call (FMT int4|nf4|fp4|awq|gptq) warmup+steps times "
+                    help="profiling aid: run one layer call (FMT int4|nf4|fp4|awq|gptq|int8) warmup+steps times "
                          "eagerly and print its mean device time")
     args = ap.parse_args()
     if args.warmup < 3:

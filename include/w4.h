@@ -177,6 +177,32 @@ w4_status w4_gptq_quantize(const float* W, const float* H, int N, int K, int G, 
  *   X  in   bf16 [n, K] (n calibration tokens);  H  out  fp32 [K, K]     */
 w4_status w4_gptq_hessian(const uint16_t* X, int n, int K, float* H, w4_stream stream);
 
+/* LLM.int8 mixed decomposition ([Survey] §2.1: one weight scale per output
+ * feature; input channels whose activation exceeds the threshold in magnitude
+ * go through a 16-bit product, the others through INT8, and the results are
+ * added; [Comparison] §6.1: threshold 6.0, no 16-bit weight copy kept).
+ *   llm_int8_quantize_weights:  s_w[n] = max_k |w[n,k]| / 127 (1 if 0),
+ *     q_w = clamp(rint(w / s_w), -127, 127)
+ *     W in fp32 [N, K];  qw out int8 [N, K];  sw out fp32 [N]
+ *   llm_int8_gemm, per call:
+ *     O = {k : |x[m,k]| > threshold for some m}
+ *     s_x[m] = max over k not in O of |x[m,k]| / 127 (1 if 0)
+ *     q_x = clamp(rint(x / s_x), -127, 127) outside O, 0 on O
+ *     y[m,n] = (sum_k q_x q_w) s_x[m] s_w[n]             (exact int32 sum)
+ *            + sum_{k in O} x[m,k] bf16(q_w[n,k] s_w[n])  (fp32)
+ *     X bf16 [M, K]; qw 16-byte aligned; K % 64 == 0, K <= 65536;
+ *     Y bf16 [M, N]; threshold >= 0 (the pages use 6.0);
+ *     workspace of llm_int8_workspace_bytes(M, N, K) bytes, 256-byte aligned,
+ *     contents irrelevant; the call leaves it dirty, so it must not be the
+ *     workspace of w4a16_gemm / nf4_gemm (which must stay zeroed).  The INT8
+ *     product uses warp-level s8 MMAs.                                      */
+w4_status llm_int8_quantize_weights(const float* W, int N, int K, int8_t* qw, float* sw,
+                                    w4_stream stream);
+size_t llm_int8_workspace_bytes(int M, int N, int K);
+w4_status llm_int8_gemm(const uint16_t* X, const int8_t* qw, const float* sw, int M, int N, int K,
+                        float threshold, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                        w4_stream stream);
+
 /* Dequantization to the bf16 compute dtype ([Survey] §6.2, [Primer] §七):
  *   w_hat[n,k] = bf16_rne( float(q - zp) * float(scale) )
  * (the fp32 product is exact, so there is exactly one rounding).

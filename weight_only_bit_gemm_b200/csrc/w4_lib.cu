@@ -14,6 +14,7 @@
 #include "w4_gemm_kernel.cuh"
 #include "w4_gemv_kernel.cuh"
 #include "w4_gptq.cuh"
+#include "w4_int8.cuh"
 #include "w4_prepack.cuh"
 #include "w4_quant.cuh"
 #include "w4_ptx.cuh"
@@ -279,6 +280,92 @@ w4_status w4_gptq_quantize(const float* W, const float* H, int N, int K, int G, 
   gptq_pack_kernel<<<static_cast<unsigned>((half + 255) / 256), 256, 0, st>>>(codes, pos, N, K,
                                                                               Wq);
   if (g_idx) gptq_gidx_kernel<<<ceil_div(K, 256), 256, 0, st>>>(pos, K, G, g_idx);
+  return launch_status(cudaGetLastError());
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// LLM.int8: workspace regions (each 256-byte aligned).
+namespace {
+
+struct Int8Layout {
+  size_t flag, list, count, qx, sx, acc, total;
+};
+
+Int8Layout int8_layout(int M, int N, int K) {
+  auto r = [](size_t v) { return (v + 255) / 256 * 256; };
+  Int8Layout l{};
+  size_t o = 0;
+  l.flag = o;  o += r(static_cast<size_t>(K));
+  l.list = o;  o += r(static_cast<size_t>(K) * 4);
+  l.count = o; o += 256;
+  l.qx = o;    o += r(static_cast<size_t>(M) * K);
+  l.sx = o;    o += r(static_cast<size_t>(M) * 4);
+  l.acc = o;   o += r(static_cast<size_t>(M) * N * 4);
+  l.total = o;
+  return l;
+}
+
+bool int8_shape_ok(int M, int N, int K) {
+  return M >= 1 && N >= 1 && K >= 64 && K % 64 == 0 && K <= 65536 &&
+         static_cast<long long>(M) * N <= (1LL << 31) && static_cast<long long>(N) * K <= (1LL << 40);
+}
+
+}  // namespace
+
+extern "C" {
+
+w4_status llm_int8_quantize_weights(const float* W, int N, int K, int8_t* qw, float* sw,
+                                    w4_stream stream) {
+  if (!W || !qw || !sw || N < 1 || K < 1) return W4_ERR_INVALID_ARG;
+  if (!aligned(W, 4) || !aligned(sw, 4)) return W4_ERR_INVALID_ARG;
+  int8_quantize_weights_kernel<<<N, 256, 0, as_stream(stream)>>>(W, N, K, qw, sw);
+  return launch_status(cudaGetLastError());
+}
+
+size_t llm_int8_workspace_bytes(int M, int N, int K) {
+  if (!int8_shape_ok(M, N, K)) return 0;
+  return int8_layout(M, N, K).total;
+}
+
+w4_status llm_int8_gemm(const uint16_t* X, const int8_t* qw, const float* sw, int M, int N, int K,
+                        float threshold, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                        w4_stream stream) {
+  if (!X || !qw || !sw || !Y || !workspace) return W4_ERR_INVALID_ARG;
+  if (!int8_shape_ok(M, N, K) || !(threshold >= 0.0f)) return W4_ERR_INVALID_ARG;
+  if (!aligned(X, 2) || !aligned(qw, 16) || !aligned(sw, 4) || !aligned(Y, 2) ||
+      !aligned(workspace, 256))
+    return W4_ERR_INVALID_ARG;
+  const Int8Layout l = int8_layout(M, N, K);
+  if (workspace_bytes < l.total) return W4_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* flag = ws + l.flag;
+  int32_t* list = reinterpret_cast<int32_t*>(ws + l.list);
+  int32_t* count = reinterpret_cast<int32_t*>(ws + l.count);
+  int8_t* qx = reinterpret_cast<int8_t*>(ws + l.qx);
+  float* sx = reinterpret_cast<float*>(ws + l.sx);
+  int* acc = reinterpret_cast<int*>(ws + l.acc);
+  int8_outliers_kernel<<<1, 1024, 0, st>>>(X, M, K, threshold, flag, list, count);
+  int8_quantize_x_kernel<<<M, 256, 0, st>>>(X, flag, K, qx, sx);
+  if (cudaMemsetAsync(acc, 0, static_cast<size_t>(M) * N * 4, st) != cudaSuccess) {
+    cudaGetLastError();
+    return W4_ERR_CUDA;
+  }
+  // work items: (16-row tile, K slice), about 24 warps per SM
+  const int row_tiles = ceil_div(N, 16);
+  const int steps_total = K / 64;
+  const int target = sm_count() * 24;
+  int slices = std::min(steps_total, std::max(1, ceil_div(target, row_tiles)));
+  const int steps = ceil_div(steps_total, slices);
+  slices = ceil_div(steps_total, steps);
+  const long long items = static_cast<long long>(row_tiles) * slices;
+  int8_product_kernel<<<static_cast<unsigned>((items + kInt8Warps - 1) / kInt8Warps),
+                        kInt8Warps * 32, 0, st>>>(qw, qx, M, N, K, row_tiles, slices, steps, acc);
+  const size_t outs = static_cast<size_t>(M) * N;
+  int8_epilogue_kernel<<<static_cast<unsigned>((outs + 255) / 256), 256, 0, st>>>(
+      acc, sx, sw, X, qw, list, count, M, N, K, Y);
   return launch_status(cudaGetLastError());
 }
 

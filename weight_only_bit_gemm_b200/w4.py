@@ -41,6 +41,9 @@ _SIGS = {
     "w4_gptq_quantize": (_i, [_p, _p, _i, _i, _i, _i, ctypes.c_float, _p, _p, _p, _p, _p, _sz,
                               _p]),
     "w4_gptq_hessian": (_i, [_p, _i, _i, _p, _p]),
+    "llm_int8_quantize_weights": (_i, [_p, _i, _i, _p, _p, _p]),
+    "llm_int8_workspace_bytes": (_sz, [_i, _i, _i]),
+    "llm_int8_gemm": (_i, [_p, _p, _p, _i, _i, _i, ctypes.c_float, _p, _p, _sz, _p]),
     "w4_dequant": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "w4_prepacked_bytes": (_sz, [_i, _i, _i, _i]),
     "w4_prepack": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
@@ -195,6 +198,33 @@ def gptq_quantize(W, H, G, act_order=False, damp=0.01):
     return Wq, sc, zr, gi
 
 
+def llm_int8_quantize_weights(W):
+    """fp32 W [N, K] -> (q_w int8 [N, K], s_w fp32 [N]), one scale per output row."""
+    _cuda(W, torch.float32, "W")
+    N, K = W.shape
+    qw = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    sw = torch.empty(N, dtype=torch.float32, device=W.device)
+    _check(lib.llm_int8_quantize_weights(_ptr(W), N, K, _ptr(qw), _ptr(sw), _stream()),
+           "llm_int8_quantize_weights")
+    return qw, sw
+
+
+def llm_int8_gemm(X, qw, sw, threshold=6.0, out=None, workspace=None):
+    """Y = X . W^T by the LLM.int8 mixed decomposition (outliers |x| > threshold)."""
+    _cuda(X, torch.bfloat16, "X")
+    M, K = X.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    need = lib.llm_int8_workspace_bytes(M, N, K)
+    if need == 0:
+        raise W4Error(W4_ERR_INVALID_ARG, "llm_int8_workspace_bytes")
+    ws = _ws_view(workspace if workspace is not None else _WS_SCRATCH.get(need, X.device))
+    _check(lib.llm_int8_gemm(_ptr(X), _ptr(qw), _ptr(sw), M, N, K, float(threshold), _ptr(out),
+                             _ptr(ws), ws.numel(), _stream()), "llm_int8_gemm")
+    return out
+
+
 def dequant(Wq, scales, zeros, G, g_idx=None):
     N, K = Wq.shape[0], Wq.shape[1] * 2
     out = torch.empty((N, K), dtype=torch.bfloat16, device=Wq.device)
@@ -248,6 +278,9 @@ class Workspace:
 
 
 _WS = Workspace()
+# scratch whose contents the library does not keep zeroed (LLM.int8): never
+# the zero-kept workspace of the W4A16 / NF4 GEMMs
+_WS_SCRATCH = Workspace()
 
 
 def _ws_view(buf):
