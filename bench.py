@@ -53,9 +53,9 @@ def nf4_bytes(M, N, K):
 # DRAM bytes of one decode-kernel launch from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of w4_gemv_kernel.cuh).
 TRAFFIC_CAPTURE = {
-    "kernel_sha256": "148e452dbe957e51ca200f80df3791137d4985face69a418263765501ea4843a",
+    "kernel_sha256": "4218176cac61511b085dca981eb0bef8f64c9445de3552d5b0ceea6ab48dec90",
     "shape": {"M": 1, "N": 12288, "K": 4096, "G": 128},
-    "dram_bytes": 26178048,
+    "dram_bytes": 26178304,
     "profile": "profiles/w4_gemv_kernel_int4_K4096_N12288_M1.md",
 }
 

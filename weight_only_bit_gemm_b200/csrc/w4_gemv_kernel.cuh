@@ -167,18 +167,34 @@ __device__ __forceinline__ void read_stage(const uint8_t* slot, StageRegs<C>& r,
 
 // Words [W0, W0 + NW) of one 64-channel half for the R row groups: one
 // activation fragment per word index serves every row group.
+// Activation fragments of one 64-channel half: either loaded word by word
+// as the MMAs need them (XHalf::ptr) or held in registers, loaded ahead
+// (XHalf::reg).  Lane: 8 bytes per word and token block.
+template <class C>
+struct XHalf {
+  const uint16_t* ptr[C::NB];
+  uint2 reg[4][C::NB];
+};
+
+// Whether a decode configuration holds the next stage's activation fragments
+// in registers (loaded while the current stage computes).  Measured on B200:
+// faster with one token block, not with two; four would spill.
+template <class C>
+__host__ __device__ constexpr bool gemv_x_ahead() { return C::NB == 1; }
+
 template <class C, int W0, int NW>
 __device__ __forceinline__ void mma_words(const uint32_t (&words)[C::kRG][4],
                                           const Int4Dq (&p0)[C::kRG], const Int4Dq (&p1)[C::kRG],
                                           const float (&a0)[C::kRG], const float (&a1)[C::kRG],
-                                          uint32_t tb,
-                                          const uint16_t* const (&xs)[C::NB],
+                                          uint32_t tb, const XHalf<C>& xs,
                                           float (&acc)[C::kRG][C::kAS][C::NB][4]) {
 #pragma unroll
   for (int w = W0; w < W0 + NW; ++w) {
     uint2 b[C::NB];
 #pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb) b[nb] = __ldg(reinterpret_cast<const uint2*>(xs[nb] + w * 16));
+    for (int nb = 0; nb < C::NB; ++nb)
+      b[nb] = gemv_x_ahead<C>() ? xs.reg[w][nb]
+                                : __ldg(reinterpret_cast<const uint2*>(xs.ptr[nb] + w * 16));
 #pragma unroll
     for (int rr = 0; rr < C::kRG; ++rr) {
       uint32_t pr[4];
@@ -290,21 +306,44 @@ struct S2Cache {
   float v[C::kRG][2];
 };
 
+// Registers of half h of stage st <- its activation fragments.
+template <class C>
+__device__ __forceinline__ void load_x_half(const uint16_t* const (&xrow)[C::NB], int st, int h,
+                                            XHalf<C>& xh) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w)
+#pragma unroll
+    for (int nb = 0; nb < C::NB; ++nb)
+      xh.reg[w][nb] = __ldg(reinterpret_cast<const uint2*>(xrow[nb] + st * kStageK + h * 64 + w * 16));
+}
+
+// One stage of a lane's row groups.  With gemv_x_ahead, xf holds this
+// stage's activation fragments on entry and, as each half is done with, that
+// half of the next stage `nst` (if has_next) is loaded in its place.
 template <class C>
 __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageRegs<C>& cur,
                                               int rpg, int st, int g,
-                                              const uint16_t* const (&xrow)[C::NB],
-                                              uint32_t tb, S2Cache<C>& sc,
+                                              const uint16_t* const (&xrow)[C::NB], int nst,
+                                              bool has_next, XHalf<C> (&xf)[2], uint32_t tb,
+                                              S2Cache<C>& sc,
                                               float (&acc)[C::kRG][C::kAS][C::NB][4]) {
   constexpr int R = C::kRG;
   const int k0 = st * kStageK;
-  const uint16_t* xa[C::NB];
-  const uint16_t* xb[C::NB];
+  if constexpr (!gemv_x_ahead<C>()) {
 #pragma unroll
-  for (int nb = 0; nb < C::NB; ++nb) {
-    xa[nb] = xrow[nb] + k0;
-    xb[nb] = xa[nb] + 64;
+    for (int nb = 0; nb < C::NB; ++nb) {
+      xf[0].ptr[nb] = xrow[nb] + k0;
+      xf[1].ptr[nb] = xrow[nb] + k0 + 64;
+    }
   }
+  const bool nsecond = has_next && nst * kStageK + 64 < args.K;
+  auto reload = [&](int h) {
+    if constexpr (gemv_x_ahead<C>()) {
+      if (h == 0 ? has_next : nsecond) load_x_half<C>(xrow, nst, h, xf[h]);
+    }
+  };
+  const XHalf<C>& xa = xf[0];
+  const XHalf<C>& xb = xf[1];
   uint32_t w0[R][4], w1[R][4];
 #pragma unroll
   for (int rr = 0; rr < R; ++rr) {
@@ -322,17 +361,29 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
       for (int rr = 0; rr < R; ++rr) int4_dq_params2(cur.sp[rr][q], cur.zp[rr][q], e0[rr], e1[rr]);
       if constexpr (C::G == 128) {
         mma_words<C, 0, 4>(w0, e0, e1, fz, fz, tb, xa, acc);
+        reload(0);
         if (second) mma_words<C, 0, 4>(w1, e0, e1, fz, fz, tb, xb, acc);
       } else if constexpr (C::G == 64) {
-        if (q == 0) mma_words<C, 0, 4>(w0, e0, e1, fz, fz, tb, xa, acc);
-        else mma_words<C, 0, 4>(w1, e0, e1, fz, fz, tb, xb, acc);
+        if (q == 0) {
+          mma_words<C, 0, 4>(w0, e0, e1, fz, fz, tb, xa, acc);
+          reload(0);
+        } else {
+          mma_words<C, 0, 4>(w1, e0, e1, fz, fz, tb, xb, acc);
+        }
       } else {
-        if (q == 0) mma_words<C, 0, 2>(w0, e0, e1, fz, fz, tb, xa, acc);
-        else if (q == 1) mma_words<C, 2, 2>(w0, e0, e1, fz, fz, tb, xa, acc);
-        else if (q == 2) mma_words<C, 0, 2>(w1, e0, e1, fz, fz, tb, xb, acc);
-        else mma_words<C, 2, 2>(w1, e0, e1, fz, fz, tb, xb, acc);
+        if (q == 0) {
+          mma_words<C, 0, 2>(w0, e0, e1, fz, fz, tb, xa, acc);
+        } else if (q == 1) {
+          mma_words<C, 2, 2>(w0, e0, e1, fz, fz, tb, xa, acc);
+          reload(0);
+        } else if (q == 2) {
+          mma_words<C, 0, 2>(w1, e0, e1, fz, fz, tb, xb, acc);
+        } else {
+          mma_words<C, 2, 2>(w1, e0, e1, fz, fz, tb, xb, acc);
+        }
       }
     }
+    reload(1);
   } else {
     const int kb64 = args.K / 64;
     if (sc.rpg != rpg) {  // a new row group unit: forget the runs
@@ -375,7 +426,9 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
     }
     Int4Dq none[R] = {};
     mma_words<C, 0, 4>(w0, none, none, a0[0], a1[0], tb, xa, acc);
+    reload(0);
     if (second) mma_words<C, 0, 4>(w1, none, none, a0[1], a1[1], tb, xb, acc);
+    reload(1);
   }
 }
 
@@ -443,6 +496,13 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[rr][e][nb][j] = 0.0f;
 
+  // activation fragments of the first stage (X is read only after the wait)
+  XHalf<C> xf[2];
+  if constexpr (gemv_x_ahead<C>()) {
+    load_x_half<C>(xrow, st0, 0, xf[0]);
+    if (st0 * kStageK + 64 < args.K) load_x_half<C>(xrow, st0, 1, xf[1]);
+  }
+
   S2Cache<C> s2c;  // NF4 only (unused, and removed, for INT4)
   int rpg = rpg0, st = st0;
   uint32_t seg0 = ua;
@@ -459,7 +519,9 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
     }
     cp_async_commit();
     cs = cs + 1 == C::kDepth ? 0 : cs + 1;
-    stage_compute<C>(args, cur, rpg, st, g, xrow, smem_u32(Ts), s2c, acc);
+    const int nst = st == KS - 1 ? 0 : st + 1;
+    stage_compute<C>(args, cur, rpg, st, g, xrow, nst, n + 1 < left, xf, smem_u32(Ts), s2c,
+                     acc);
     if (st == KS - 1 || n + 1 == left) {
       const uint32_t seg1 = ua + static_cast<uint32_t>(n) + 1;
       flush_row_group<C>(args, acc, rpg, seg0, seg1, wid, lane);
