@@ -21,9 +21,10 @@
 //             act-order permutation (stable, decreasing H_kk), damping
 //             lambda = damp * mean(diag H), A = J P^T H P J + lambda I (fp64);
 //   factor    blocked lower Cholesky of A (32 x 32 tiles: diagonal factor,
-//             panel solve, trailing update), then the blocked inverse T = L'^-1
-//             (diagonal tiles inverted in parallel, then one block row at a
-//             time), then U = J T J in fp32;
+//             panel solve, trailing update), then the inverse T = L'^-1
+//             (diagonal tiles inverted in parallel, then the off-diagonal
+//             blocks by doubling: log2(K / 32) levels of two tile GEMMs), then
+//             U = J T J in fp32;
 //   quantize  lazy blocks of 128 columns: one thread per weight row applies
 //             the in-block updates column by column in shared memory (and
 //             decides codes, group scales and zero points there); a tiled
@@ -265,32 +266,56 @@ __global__ void __launch_bounds__(kChol) trinv_diag_kernel(const double* __restr
   for (int r = 0; r < kChol; ++r) T[(o + r) * K + o + c] = X[r][c];
 }
 
-// Block row ib of T = L^-1 (tiles j < ib, one CTA each):
-//   T[ib][j] = -T[ib][ib] * sum_{k = j}^{ib - 1} L[ib][k] T[k][j].
-__global__ void __launch_bounds__(1024) trinv_row_kernel(const double* __restrict__ L, int K,
-                                                         int ib, double* __restrict__ T) {
+// The off-diagonal tiles of T = L^-1 by doubling.  At level s (in tiles),
+// pair b joins the first block F = [2bs, 2bs + s) and the second block
+// S = [2bs + s, min(2bs + 2s, nb)), whose inverses are complete; then
+//   T[S][F] = -T[S][S] L[S][F] T[F][F],
+// in two tile-GEMM launches over every pair of the level (grid: tile column
+// j < s, tile row i < |S|, pair b).  P = L[S][F] T[F][F] goes to scratch, at
+// tile (b s + i) s + j (only the last pair can have |S| < s).
+__global__ void __launch_bounds__(1024) trinv_level_p_kernel(const double* __restrict__ L,
+                                                             const double* __restrict__ T, int K,
+                                                             int nb, int s,
+                                                             double* __restrict__ P) {
+  const int j = blockIdx.x, i = blockIdx.y, b = blockIdx.z;
+  const int F0 = 2 * b * s, S0 = F0 + s;
+  if (i >= min(s, nb - S0)) return;
   __shared__ double Lt[kChol][kChol + 1], Tt[kChol][kChol + 1];
-  const int j = blockIdx.x;
   const int r = threadIdx.x >> 5, c = threadIdx.x & 31;
-  const size_t oi = static_cast<size_t>(ib) * kChol, oj = static_cast<size_t>(j) * kChol;
-  double s = 0.0;
-  for (int kb = j; kb < ib; ++kb) {
-    const size_t ok = static_cast<size_t>(kb) * kChol;
+  const size_t oi = static_cast<size_t>(S0 + i) * kChol, oj = static_cast<size_t>(F0 + j) * kChol;
+  double acc = 0.0;
+  for (int k = j; k < s; ++k) {  // T[F][F] is lower triangular in tiles
+    const size_t ok = static_cast<size_t>(F0 + k) * kChol;
     __syncthreads();
     Lt[r][c] = L[(oi + r) * K + ok + c];
     Tt[r][c] = T[(ok + r) * K + oj + c];
     __syncthreads();
 #pragma unroll 8
-    for (int m = 0; m < kChol; ++m) s += Lt[r][m] * Tt[m][c];
+    for (int m = 0; m < kChol; ++m) acc += Lt[r][m] * Tt[m][c];
   }
-  __syncthreads();
-  Tt[r][c] = s;                                        // S
-  Lt[r][c] = T[(oi + r) * K + oi + c];                 // T[ib][ib]
-  __syncthreads();
-  double v = 0.0;
+  P[((static_cast<size_t>(b) * s + i) * s + j) * (kChol * kChol) + r * kChol + c] = acc;
+}
+
+__global__ void __launch_bounds__(1024) trinv_level_t_kernel(const double* __restrict__ P, int K,
+                                                             int nb, int s,
+                                                             double* __restrict__ T) {
+  const int j = blockIdx.x, i = blockIdx.y, b = blockIdx.z;
+  const int F0 = 2 * b * s, S0 = F0 + s;
+  if (i >= min(s, nb - S0)) return;
+  __shared__ double At[kChol][kChol + 1], Pt[kChol][kChol + 1];
+  const int r = threadIdx.x >> 5, c = threadIdx.x & 31;
+  const size_t oi = static_cast<size_t>(S0 + i) * kChol;
+  double acc = 0.0;
+  for (int k = 0; k <= i; ++k) {  // T[S][S] is lower triangular in tiles
+    const size_t ok = static_cast<size_t>(S0 + k) * kChol;
+    __syncthreads();
+    At[r][c] = T[(oi + r) * K + ok + c];
+    Pt[r][c] = P[((static_cast<size_t>(b) * s + k) * s + j) * (kChol * kChol) + r * kChol + c];
+    __syncthreads();
 #pragma unroll 8
-  for (int m = 0; m < kChol; ++m) v -= Lt[r][m] * Tt[m][c];
-  T[(oi + r) * K + oj + c] = v;
+    for (int m = 0; m < kChol; ++m) acc -= At[r][m] * Pt[m][c];
+  }
+  T[(oi + r) * K + static_cast<size_t>(F0 + j) * kChol + c] = acc;
 }
 
 // U[a][b] = T[K-1-a][K-1-b] for b >= a (fp32): the upper Cholesky factor of

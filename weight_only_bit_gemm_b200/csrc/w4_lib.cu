@@ -265,7 +265,14 @@ w4_status w4_gptq_quantize(const float* W, const float* H, int N, int K, int G, 
     }
   }
   trinv_diag_kernel<<<nb, kChol, 0, st>>>(A, K, T);
-  for (int ib = 1; ib < nb; ++ib) trinv_row_kernel<<<ib, kChol * kChol, 0, st>>>(A, K, ib, T);
+  // off-diagonal blocks by doubling; P (at most K^2 / 4 doubles) borrows U's
+  // region, which is written only after T is complete
+  double* P = reinterpret_cast<double*>(U);
+  for (int s = 1; s < nb; s *= 2) {
+    const dim3 grid(s, s, ceil_div(nb, 2 * s));
+    trinv_level_p_kernel<<<grid, kChol * kChol, 0, st>>>(A, T, K, nb, s, P);
+    trinv_level_t_kernel<<<grid, kChol * kChol, 0, st>>>(P, K, nb, s, T);
+  }
   gptq_u_kernel<<<dim3(ceil_div(K, 32), ceil_div(K, 8)), 256, 0, st>>>(T, K, U);
   // quantize: lazy blocks of kGptqB columns
   for (int j0 = 0; j0 < K; j0 += kGptqB) {
