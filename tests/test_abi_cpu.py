@@ -78,3 +78,75 @@ def test_bad_shapes_rejected_on_host():
     odd = ctypes.c_void_p((1 << 20) + 2)
     assert w4.lib.w4a16_gemm(odd, fake, 1, 4, 128, 128, 0, fake, fake, 1 << 20, None) == \
         w4.W4_ERR_INVALID_ARG
+
+
+def test_fp4_levels_equal_oracle_table():
+    got = w4.fp4_levels()
+    want = O.fp4_table()
+    import numpy as np
+    assert np.array_equal(np.array(got, np.float32).view(np.uint32), want.view(np.uint32))
+
+
+def test_workspace_sizes_of_the_variants():
+    r256 = lambda v: (v + 255) // 256 * 256
+    # the AWQ call adds the rewritten activations, M x K bf16, to the plain plan
+    for (M, N, K) in [(1, 4096, 4096), (16, 12288, 4096), (512, 8192, 28672)]:
+        plain = w4.workspace_bytes(M, N, K, 128)
+        assert w4.awq_workspace_bytes(M, N, K, 128) == plain + r256(2 * M * K)
+        assert w4.awq_workspace_bytes(M, N, K, 128, True) == w4.workspace_bytes(M, N, K, 128, True)
+    # GPTQ: two fp64 and one fp32 K x K matrices, the fp32 working weights, the
+    # block errors, the codes and per-channel vectors
+    N, K = 13824, 5120
+    got = w4.lib.w4_gptq_workspace_bytes(N, K, 32)
+    floor = 20 * K * K + 4 * N * K + 4 * 128 * N + N * K + 17 * K
+    assert floor <= got <= floor + 12 * 256
+    assert w4.lib.w4_gptq_workspace_bytes(N, 5120 + 16, 16) == 0   # unsupported group
+    assert w4.lib.w4_gptq_workspace_bytes(N, 131072, 128) == 0     # K above 65536
+    # LLM.int8: flags, list, count, q_x, s_x, int32 accumulator
+    M, N, K = 16, 22016, 4096
+    got = w4.lib.llm_int8_workspace_bytes(M, N, K)
+    assert M * K + 4 * M * N <= got <= M * K + 4 * M * N + 5 * K + 6 * 256
+    assert w4.lib.llm_int8_workspace_bytes(M, N, 4000) == 0         # K % 64 != 0
+
+
+@pytest.mark.parametrize("call", [
+    lambda: w4.lib.w4_quantize_sym(None, 4, 128, 128, None, None, None, None, None),
+    lambda: w4.lib.w4_awq_scale_weights(None, None, 4, 128, None, None),
+    lambda: w4.lib.w4_awq_scale_activations(None, None, 1, 128, None, None),
+    lambda: w4.lib.w4a16_awq_gemm(None, None, None, 1, 4, 128, 128, 0, None, None, 0, None),
+    lambda: w4.lib.fp4_quantize(None, 4, 128, 64, 256, None, None, None, None),
+    lambda: w4.lib.fp4_dequant(None, None, None, 4, 128, 64, 256, None, None),
+    lambda: w4.lib.fp4_gemm(None, None, None, 1, 4, 128, 256, None, None, 0, None),
+    lambda: w4.lib.w4_gptq_hessian(None, 16, 128, None, None),
+    lambda: w4.lib.w4_gptq_quantize(None, None, 4, 128, 32, 0, 0.01, None, None, None, None,
+                                    None, 0, None),
+    lambda: w4.lib.llm_int8_quantize_weights(None, 4, 128, None, None, None),
+    lambda: w4.lib.llm_int8_gemm(None, None, None, 1, 4, 128, 6.0, None, None, 0, None),
+])
+def test_null_pointers_rejected_on_host_variants(call):
+    assert call() == w4.W4_ERR_INVALID_ARG
+
+
+def test_variant_bad_arguments_rejected_on_host():
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: argument checks come first
+    # act-order GPTQ needs somewhere to put g_idx
+    assert w4.lib.w4_gptq_quantize(fake, fake, 4, 128, 32, 1, 0.01, fake, fake, fake, None,
+                                   fake, 1 << 30, None) == w4.W4_ERR_INVALID_ARG
+    # negative damping, too small a workspace
+    assert w4.lib.w4_gptq_quantize(fake, fake, 4, 128, 32, 0, -1.0, fake, fake, fake, None,
+                                   fake, 1 << 30, None) == w4.W4_ERR_INVALID_ARG
+    assert w4.lib.w4_gptq_quantize(fake, fake, 4, 128, 32, 0, 0.01, fake, fake, fake, None,
+                                   fake, 256, None) == w4.W4_ERR_INVALID_ARG
+    # LLM.int8: K % 64, negative threshold, weights not 16-byte aligned
+    assert w4.lib.llm_int8_gemm(fake, fake, fake, 1, 4, 96, 6.0, fake, fake, 1 << 30, None) == \
+        w4.W4_ERR_INVALID_ARG
+    assert w4.lib.llm_int8_gemm(fake, fake, fake, 1, 4, 128, -1.0, fake, fake, 1 << 30, None) == \
+        w4.W4_ERR_INVALID_ARG
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert w4.lib.llm_int8_gemm(fake, odd, fake, 1, 4, 128, 6.0, fake, fake, 1 << 30, None) == \
+        w4.W4_ERR_INVALID_ARG
+    # AWQ: the factor must be 16-byte aligned; activations need K % 8 == 0
+    assert w4.lib.w4a16_awq_gemm(fake, odd, fake, 1, 4, 128, 128, 0, fake, fake, 1 << 30,
+                                 None) == w4.W4_ERR_INVALID_ARG
+    assert w4.lib.w4_awq_scale_activations(fake, fake, 1, 12, fake, None) == \
+        w4.W4_ERR_INVALID_ARG
