@@ -51,7 +51,7 @@ typedef void* w4_stream; /* a cudaStream_t */
 enum {
   W4_OK = 0,
   W4_ERR_INVALID_ARG = 1, /* null/misaligned pointer, size out of range      */
-  W4_ERR_UNSUPPORTED = 2, /* valid but not supported by this build           */
+  W4_ERR_UNSUPPORTED = 2, /* valid but not supported by this library         */
   W4_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed            */
   W4_ERR_TIMEOUT = 4,     /* a device pipeline wait gave up (device status)  */
   W4_ERR_DEVICE_INPUT = 5, /* the device found bad input data (device status) */
