@@ -54,10 +54,12 @@ R19 LLM.int8: per-row weight absmax/127, outlier channels |x| > 6.0 in any
 All floating-point steps are numpy float32 operations (IEEE, round to nearest
 even) unless stated as fp64; the matmul accumulates in fp64.
 
-Parity unpinned: the exact NF4 level values.  The pages print no table; the
-tests pin what they do fix (16 levels, strictly increasing, an exact zero,
--1 and +1 at the ends, spacing smallest near zero), not the digits of R6's
-construction, so agreement with any other NF4 table is not claimed.
+NF4 levels: the pages print no table.  The tests pin what the pages fix (16
+levels, strictly increasing, an exact zero, -1 and +1 at the ends, spacing
+smallest near zero) and, to one fp32 ulp, the digits of R6's construction
+against an independent fp64 evaluation of it (bisection on the normal CDF
+written through erfc, not the library inverse CDF used here).  Agreement
+with any NF4 table published elsewhere is not claimed.
 """
 from __future__ import annotations
 

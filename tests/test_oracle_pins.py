@@ -376,6 +376,77 @@ def _erfinv_pos(y):
     return 0.5 * (lo + hi)
 
 
+def _normal_quantile_bisect(p):
+    """x with Phi(x) = p, Phi(x) = erfc(-x / sqrt 2) / 2, by 300 bisection
+    steps in fp64 (converges to the last bit; no library inverse CDF)."""
+    lo, hi = -12.0, 12.0
+    for _ in range(300):
+        mid = 0.5 * (lo + hi)
+        if 0.5 * math.erfc(-mid / math.sqrt(2.0)) < p:
+            lo = mid
+        else:
+            hi = mid
+    return 0.5 * (lo + hi)
+
+
+def _nf4_levels_independent():
+    """The R6 construction evaluated independently of the oracle: the QLoRA
+    offset delta = 1 - (1/30 + 1/32)/2; quantiles at the first 8 of 9 equally
+    spaced probabilities from delta down to 1/2 (positive side) and the first
+    7 of 8 (negative side, mirrored); an exact zero; all divided by the
+    largest quantile; fp64 throughout, one rounding to fp32 at the end
+    ([Survey] §6.1: levels are normal quantiles, denser near zero, with an
+    exact zero; §6.2 and [Primer] §七: NF4 spans [-1, 1] under the absmax)."""
+    delta = 1.0 - (Fraction(1, 30) + Fraction(1, 32)) / 2
+    steps_p = [delta + (Fraction(1, 2) - delta) * i / 8 for i in range(8)]
+    steps_n = [delta + (Fraction(1, 2) - delta) * i / 7 for i in range(7)]
+    top = _normal_quantile_bisect(float(delta))
+    vals = [_normal_quantile_bisect(float(p)) / top for p in steps_p]
+    vals += [-_normal_quantile_bisect(float(p)) / top for p in steps_n]
+    vals.append(0.0)
+    return np.array(sorted(vals), np.float64).astype(np.float32)
+
+
+def test_nf4_table_digits_pinned():
+    # every level within one fp32 ulp of the independent evaluation (they
+    # agree bit for bit on this machine); a wrong delta, a wrong split of the
+    # quantiles between the two signs or a wrong normaliser moves several
+    # levels by thousands of ulps
+    T = O.nf4_table()
+    ref = _nf4_levels_independent()
+    assert T.dtype == np.float32 and T.shape == (16,)
+    assert np.all(np.abs(T.view(np.int32).astype(np.int64) - ref.view(np.int32)) <= 1)
+
+
+def test_planted_mistakes_nf4_table(monkeypatch):
+    import statistics
+    import oracle.w4_oracle as M
+    nd = statistics.NormalDist()
+
+    def built(delta, n_pos_steps, n_neg_steps, n_pos, n_neg, norm="top"):
+        pos = [nd.inv_cdf(delta + (0.5 - delta) * i / n_pos_steps) for i in range(n_pos)]
+        neg = [-nd.inv_cdf(delta + (0.5 - delta) * i / n_neg_steps) for i in range(n_neg)]
+        lv = sorted(neg + [0.0] + pos)
+        d = nd.inv_cdf(delta) if norm == "top" else max(abs(v) for v in lv[1:-1])
+        return np.array([v / d for v in lv], np.float64).astype(np.float32)
+
+    good = 1.0 - 0.5 * (1 / 30 + 1 / 32)
+    mistakes = {
+        "delta from 1/30 only": built(1.0 - 0.5 * (2 / 30), 8, 7, 8, 7),
+        "delta from 1/32 only": built(1.0 - 0.5 * (2 / 32), 8, 7, 8, 7),
+        "negatives on the positive grid": built(good, 8, 8, 8, 7),
+        "positives on the negative grid": built(good, 7, 7, 8, 7),
+        "normalised by the second level": built(good, 8, 7, 8, 7, norm="second"),
+    }
+    for name, table in mistakes.items():
+        monkeypatch.setattr(M, "nf4_table", lambda t=table: t)
+        monkeypatch.setattr(O, "nf4_table", lambda t=table: t)
+        with pytest.raises(AssertionError):
+            test_nf4_table_digits_pinned()
+        monkeypatch.undo()
+    test_nf4_table_digits_pinned()
+
+
 def test_nf4_codes_brute_force_nearest():
     rng = np.random.default_rng(8)
     W = (rng.standard_normal((6, 128)) * 0.02).astype(np.float32)
