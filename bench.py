@@ -56,7 +56,6 @@ TRAFFIC_CAPTURE = {
     "kernel_sha256": "4218176cac61511b085dca981eb0bef8f64c9445de3552d5b0ceea6ab48dec90",
     "shape": {"M": 1, "N": 12288, "K": 4096, "G": 128},
     "dram_bytes": 26178304,
-    "profile": "profiles/w4_gemv_kernel_int4_K4096_N12288_M1.md",
 }
 
 
@@ -283,6 +282,38 @@ def time_calls(calls, reps: int, warm: int = 2):
     return [t / reps for t in tot]
 
 
+def time_graph(calls, reps: int = 5, warm: int = 2):
+    """Device time (ms) of one pass over `calls` (closures, run in order on the
+    current stream) captured as one CUDA graph, averaged over `reps` replays;
+    the calls are run once eagerly first so that nothing allocates during the
+    capture.  Comparable with the graph-timed decode step: launch latency is
+    hidden and consecutive kernels overlap through programmatic dependent
+    launch."""
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for f in calls:
+            f()
+    stream.synchronize()
+
+    def run_all():
+        for f in calls:
+            f()
+    g = capture(run_all, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            g.replay()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+    b.synchronize()
+    del g
+    return a.elapsed_time(b) / reps
+
+
 def measure_decode(step, args, pg, local):
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
@@ -443,10 +474,13 @@ def measure_rows(w4, peaks):
                 calls.append(lambda X=X, r=r, s=s24, N=N, K=K: w4.nf4_gemm(X, r, s, N, K))
                 nbytes.append(nf4_bytes(M, N, K))
         del W
+    tg = time_graph(calls)
     ts = time_calls(calls, reps=5)
     rows["nf4_gemm_decode"] = {"configs": "(K,N) in {(4096,14336),(14336,4096)} x M in {1,8,32}",
-                               "TB/s": sum(nbytes) / sum(ts) / 1e9,
-                               "frac_of_hbm": sum(nbytes) / sum(ts) / 1e6 / hbm}
+                               "timing": "CUDA graph of all calls",
+                               "TB/s": sum(nbytes) / tg / 1e9,
+                               "frac_of_hbm": sum(nbytes) / tg / 1e6 / hbm,
+                               "eager_TB/s": sum(nbytes) / sum(ts) / 1e9}
 
     # NEXT row: FP4 (E2M1) table in the NF4 kernels, same shapes
     f4 = S.FP4_DECODE
@@ -466,38 +500,51 @@ def measure_rows(w4, peaks):
                 calls.append(lambda X=X, r=r, s=s24, N=N, K=K: w4.fp4_gemm(X, r, s, N, K))
                 nbytes.append(nf4_bytes(M, N, K))
         del W
+    tg = time_graph(calls)
     ts = time_calls(calls, reps=5)
     rows["fp4_gemm_decode"] = {"configs": "(K,N) in {(4096,14336),(14336,4096)} x M in {1,8,32}",
-                               "TB/s": sum(nbytes) / sum(ts) / 1e9,
-                               "frac_of_hbm": sum(nbytes) / sum(ts) / 1e6 / hbm}
+                               "timing": "CUDA graph of all calls",
+                               "TB/s": sum(nbytes) / tg / 1e9,
+                               "frac_of_hbm": sum(nbytes) / tg / 1e6 / hbm,
+                               "eager_TB/s": sum(nbytes) / sum(ts) / 1e9}
 
-    # a3: act-order (g_idx) decode and M=256, group 32
+    # a3: act-order (g_idx) decode and M=256, group 32 and the 64 / 128 sweep
     ao = S.ACT_ORDER_13B
-    dec_calls, dec_bytes, big_calls, big_flops = [], [], [], []
-    for (K, N) in ao["shapes"]:
-        G = ao["G"]
-        W = torch.from_numpy(S.layer_w(ao, K, N)).cuda()
-        g_idx = torch.from_numpy(S.act_order_g_idx(S.draw_perm(K, tag=ao["tag"], N=N), G)).cuda()
-        Wq, sc, zr = w4.quantize_rtn(W, G, g_idx)
-        wp = w4.prepack(Wq, sc, zr, G, g_idx)
-        reps = [wp] + [wp.clone() for _ in range(_replicas_for(wp.numel(), l2) - 1)]
-        for M in ao["Ms"]:
-            X = bf16_dev(S.layer_x(ao, M, K, N))
-            for r in reps:
-                f = (lambda X=X, r=r, N=N, K=K, G=G: w4.w4a16_gemm(X, r, N, K, G, True))
-                if M <= 16:
-                    dec_calls.append(f)
-                    dec_bytes.append(int4_bytes(M, N, K, G) + 4 * K)
-                else:
-                    big_calls.append(f)
-                    big_flops.append(2.0 * M * N * K)
-        del W, Wq, sc, zr
-    ts = time_calls(dec_calls, reps=5)
-    rows["act_order_decode"] = {"configs": "(K,N) in {(5120,13824),(13824,5120)} x M in {1,16}, G=32",
-                                "TB/s": sum(dec_bytes) / sum(ts) / 1e9,
-                                "frac_of_hbm": sum(dec_bytes) / sum(ts) / 1e6 / hbm}
-    ts = time_calls(big_calls, reps=5)
-    rows["act_order_m256"] = {"configs": "M=256, G=32", "TFLOP/s": sum(big_flops) / sum(ts) / 1e9}
+    sweep = {}
+    for G in [ao["G"], *ao["G_sweep"]]:
+        dec_calls, dec_bytes, big_calls, big_flops = [], [], [], []
+        for (K, N) in ao["shapes"]:
+            W = torch.from_numpy(S.layer_w(ao, K, N)).cuda()
+            g_idx = torch.from_numpy(
+                S.act_order_g_idx(S.draw_perm(K, tag=ao["tag"], N=N), G)).cuda()
+            Wq, sc, zr = w4.quantize_rtn(W, G, g_idx)
+            wp = w4.prepack(Wq, sc, zr, G, g_idx)
+            reps = [wp] + [wp.clone() for _ in range(_replicas_for(wp.numel(), l2) - 1)]
+            for M in ao["Ms"]:
+                X = bf16_dev(S.layer_x(ao, M, K, N))
+                for r in reps:
+                    f = (lambda X=X, r=r, N=N, K=K, G=G: w4.w4a16_gemm(X, r, N, K, G, True))
+                    if M <= 16:
+                        dec_calls.append(f)
+                        dec_bytes.append(int4_bytes(M, N, K, G) + 4 * K)
+                    else:
+                        big_calls.append(f)
+                        big_flops.append(2.0 * M * N * K)
+            del W, Wq, sc, zr
+        tg = time_graph(dec_calls)
+        te = sum(time_calls(dec_calls, reps=5))
+        tb = time_graph(big_calls)
+        sweep[f"G{G}"] = {"decode_TB/s": sum(dec_bytes) / tg / 1e9,
+                          "decode_frac_of_hbm": sum(dec_bytes) / tg / 1e6 / hbm,
+                          "decode_eager_TB/s": sum(dec_bytes) / te / 1e9,
+                          "m256_TFLOP/s": sum(big_flops) / tb / 1e9,
+                          "m256_frac_of_bf16_peak": sum(big_flops) / tb / 1e9 / peaks["bf16_tflops"]}
+        del dec_calls, big_calls, reps, wp
+        torch.cuda.empty_cache()
+    rows["act_order"] = {"configs": "(K,N) in {(5120,13824),(13824,5120)}; decode M in {1,16}, "
+                                    "prefill M=256; g_idx from a seeded permutation",
+                         "timing": "CUDA graph of all calls of a group size",
+                         "per_G": sweep}
 
     # NEXT row: symmetric INT4 after the AWQ factor (decode shapes of Llama-7B)
     aw = S.AWQ_SYM_DECODE
@@ -527,14 +574,17 @@ def measure_rows(w4, peaks):
                 plain_calls.append(lambda X=X, r=r, N=N, K=K, G=G: w4.w4a16_gemm(X, r, N, K, G))
                 awq_bytes.append(int4_bytes(M, N, K, G) + 4 * K)
         del W, Ws, Wq, sc, zr
+    tg = time_graph(awq_calls)
+    tpg = time_graph(plain_calls)
     ts = time_calls(awq_calls, reps=5)
-    tp = time_calls(plain_calls, reps=5)
     rows["awq_sym_decode"] = {
         "configs": "(K,N) in {(4096,12288),(4096,4096),(4096,22016),(11008,4096)} x M in {1,4,16}, "
                    "G=128, symmetric codes, AWQ factor on X",
-        "TB/s": sum(awq_bytes) / sum(ts) / 1e9,
-        "frac_of_hbm": sum(awq_bytes) / sum(ts) / 1e6 / hbm,
-        "same_weights_without_factor_TB/s": sum(awq_bytes) / sum(tp) / 1e9}
+        "timing": "CUDA graph of all calls",
+        "TB/s": sum(awq_bytes) / tg / 1e9,
+        "frac_of_hbm": sum(awq_bytes) / tg / 1e6 / hbm,
+        "same_weights_without_factor_TB/s": sum(awq_bytes) / tpg / 1e9,
+        "eager_TB/s": sum(awq_bytes) / sum(ts) / 1e9}
 
     # NEXT row: LLM.int8 mixed decomposition on the Llama-7B decode inputs
     # (0.1% of channels x50, i.e. outliers above the 6.0 threshold)
@@ -553,12 +603,15 @@ def measure_rows(w4, peaks):
                 i8_calls.append(lambda X=X, r=r, sw=sw: w4.llm_int8_gemm(X, r, sw))
                 i8_bytes.append(N * K + 4 * N + 2 * M * K + 2 * M * N)
         del W
+    tg = time_graph(i8_calls)
     ts = time_calls(i8_calls, reps=5)
     rows["llm_int8_decode"] = {
         "configs": "(K,N) in {(4096,12288),(4096,4096),(4096,22016),(11008,4096)} x M in {1,4,16}, "
                    "threshold 6.0",
-        "TB/s": sum(i8_bytes) / sum(ts) / 1e9,
-        "frac_of_hbm": sum(i8_bytes) / sum(ts) / 1e6 / hbm}
+        "timing": "CUDA graph of all calls",
+        "TB/s": sum(i8_bytes) / tg / 1e9,
+        "frac_of_hbm": sum(i8_bytes) / tg / 1e6 / hbm,
+        "eager_TB/s": sum(i8_bytes) / sum(ts) / 1e9}
 
     # NEXT row: GPTQ at quantization time (13B MLP up-projection, act-order, G = 32,
     # 512 calibration tokens): Hessian, then the compensated quantization
@@ -621,22 +674,47 @@ def _oracle_call(Wq, s, z, xb):
     O.matmul_ref(xb, O.dequant_rtn(Wq, s, z, WL["G"]))
 
 
+def blas_threads() -> int:
+    """Threads NumPy's BLAS runs the oracle's fp64 product on (its default:
+    every core this process may use)."""
+    from threadpoolctl import threadpool_info
+    n = [int(i.get("num_threads", 1)) for i in threadpool_info() if i.get("user_api") == "blas"]
+    return max(n) if n else 1
+
+
 def oracle_sample(rows=4096):
     """Time the CPU oracle (dequant + fp64 matmul) on the decode workload: the
-    first `rows` output rows of each of the 4 layer shapes at M = 1, BLAS
-    limited to one thread.  Returns (bytes, seconds, description)."""
-    from threadpoolctl import threadpool_limits
+    first `rows` output rows of each of the 4 layer shapes at M = 1, on the
+    host's cores (BLAS default threads).  Returns (bytes, seconds, description)."""
     tot_b, tot_s = 0.0, 0.0
-    with threadpool_limits(limits=1):
-        for (K, N) in WL["shapes"]:
-            r = min(rows, N)
-            Wq, s, z, xb = _oracle_layer(K, N, r)
-            t0 = time.perf_counter()
-            _oracle_call(Wq, s, z, xb)
-            tot_s += time.perf_counter() - t0
-            tot_b += int4_bytes(1, r, K, WL["G"])
+    for (K, N) in WL["shapes"]:
+        r = min(rows, N)
+        Wq, s, z, xb = _oracle_layer(K, N, r)
+        t0 = time.perf_counter()
+        _oracle_call(Wq, s, z, xb)
+        tot_s += time.perf_counter() - t0
+        tot_b += int4_bytes(1, r, K, WL["G"])
     return tot_b, tot_s, (f"first {rows} output rows of each of the 4 layer shapes at M=1: "
-                          "numpy dequant + fp64 matmul, 1 thread")
+                          f"numpy dequant + fp64 matmul, BLAS on {blas_threads()} threads")
+
+
+def oracle_prefill_sample(tokens=256, rows=4096):
+    """The oracle on a bounded prefill sample: tokens 0..tokens-1 of the 70B
+    M = 512 activations against the first `rows` output rows of the
+    K = 8192, N = 28672 layer.  Returns (flops, seconds, description)."""
+    import oracle as O
+    pf = S.PREFILL_70B
+    K, N = pf["shapes"][0]
+    W = S.layer_w(pf, K, N)[:rows]
+    q, s, z = O.quantize_rtn(W, pf["G"])                # offline step, not timed
+    Wq = O.pack_nibbles(q)
+    xb = S.layer_x(pf, pf["Ms"][0], K, N)[:tokens]
+    t0 = time.perf_counter()
+    O.matmul_ref(xb, O.dequant_rtn(Wq, s, z, pf["G"]))
+    sec = time.perf_counter() - t0
+    return (2.0 * tokens * rows * K, sec,
+            f"tokens 0..{tokens - 1} of the M={pf['Ms'][0]} input x first {rows} output rows of "
+            f"K={K}, N={N}: numpy dequant + fp64 matmul, BLAS on {blas_threads()} threads")
 
 
 def run_reference(args, world, rank):
@@ -646,36 +724,35 @@ def run_reference(args, world, rank):
     takes about two minutes."""
     if rank != 0:
         return
-    from threadpoolctl import threadpool_limits
     n_total = args.warmup + args.steps
     budget = max(0.002, 90.0 / n_total)             # seconds per step
-    with threadpool_limits(limits=1):
-        # calibrate seconds per row on a 1024-row slice of the deepest layer
-        Wq, s, z, xb = _oracle_layer(11008, 4096, 1024)
-        _oracle_call(Wq, s, z, xb)
+    # calibrate seconds per row on a 1024-row slice of the deepest layer
+    Wq, s, z, xb = _oracle_layer(11008, 4096, 1024)
+    _oracle_call(Wq, s, z, xb)
+    t0 = time.perf_counter()
+    _oracle_call(Wq, s, z, xb)
+    per_row = 1.5 * (time.perf_counter() - t0) / 1024
+    rows = int(max(8, min(4096, budget / max(per_row, 1e-9))))
+    prepared = [(K, N, *_oracle_layer(K, N, min(rows, N))) for (K, N) in WL["shapes"]]
+    tot_b, tot_s = 0.0, 0.0
+    for i in range(n_total):
+        K, N, Wq, s, z, xb = prepared[i % len(prepared)]
         t0 = time.perf_counter()
         _oracle_call(Wq, s, z, xb)
-        per_row = 1.5 * (time.perf_counter() - t0) / 1024
-        rows = int(max(8, min(4096, budget / max(per_row, 1e-9))))
-        prepared = [(K, N, *_oracle_layer(K, N, min(rows, N))) for (K, N) in WL["shapes"]]
-        tot_b, tot_s = 0.0, 0.0
-        for i in range(n_total):
-            K, N, Wq, s, z, xb = prepared[i % len(prepared)]
-            t0 = time.perf_counter()
-            _oracle_call(Wq, s, z, xb)
-            dt = time.perf_counter() - t0
-            if i >= args.warmup:
-                tot_s += dt
-                tot_b += int4_bytes(1, Wq.shape[0], K, WL["G"])
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            tot_s += dt
+            tot_b += int4_bytes(1, Wq.shape[0], K, WL["G"])
     v = tot_b / tot_s / 1e12
+    cores = blas_threads()
     sample = (f"one M=1 decode call per step on the first {rows} output rows of a layer, "
-              "4 layer shapes rotating; numpy dequant + fp64 matmul, 1 thread")
+              f"4 layer shapes rotating; numpy dequant + fp64 matmul, BLAS on {cores} threads")
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": tot_s * 1e3 / max(1, args.steps), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "sample": sample},
-            "cpu_baseline": {"value": v, "unit": "TB/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": v, "unit": "TB/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -789,8 +866,11 @@ def main():
             rows = measure_rows(w4, peaks)
         if not args.no_cpu:
             b, sec, desc = oracle_sample()
-            cpu = {"value": b / sec / 1e12, "unit": "TB/s", "cores": 1, "kind": "oracle",
-                   "sample": desc, "seconds": sec}
+            fl, psec, pdesc = oracle_prefill_sample()
+            cpu = {"value": b / sec / 1e12, "unit": "TB/s", "cores": blas_threads(),
+                   "kind": "oracle", "sample": desc, "seconds": sec,
+                   "prefill": {"value": fl / psec / 1e12, "unit": "TFLOP/s", "sample": pdesc,
+                               "seconds": psec}}
 
     if rank == 0:
         line = {

@@ -267,12 +267,16 @@ w4_status w4_unprepack(const uint8_t* Wp, int N, int K, int G, int act_order,
  * they exit, so prepack followed by a GEMM is fine).
  *   X          in   bf16 [M, K], 16-byte aligned, K % 64 == 0
  *   Wp         in   from w4_prepack (act_order must match)
- *   M, N, K, G M >= 1, N >= 1
+ *   M, N, K, G M >= 1, N >= 1; with M <= 32 (the decode kernel) N is at most
+ *              2097152 (65536 groups of 32 rows, one arrival counter each):
+ *              larger N returns W4_ERR_UNSUPPORTED, launching nothing
  *   Y          out  bf16 [M, N]
  *   workspace  device scratch of at least w4_workspace_bytes(M,N,K,G,act_order)
  *              bytes, 256-byte aligned, ZEROED ONCE before its first use; the
  *              library leaves it zeroed after every call (split-K counters).
- *              Calls that share a workspace must be ordered on one stream.  */
+ *              Calls that share a workspace must be ordered on one stream.
+ *              w4_workspace_bytes returns 0 for an invalid or unsupported
+ *              shape.                                                       */
 size_t w4_workspace_bytes(int M, int N, int K, int G, int act_order);
 w4_status w4a16_gemm(const uint16_t* X, const uint8_t* Wp, int M, int N, int K, int G,
                      int act_order, uint16_t* Y, void* workspace, size_t workspace_bytes,
@@ -309,7 +313,11 @@ w4_status w4a16_awq_gemm(const uint16_t* X, const float* s, const uint8_t* Wp, i
  *   First call on a device: looks up that device's copy of the array (which
  *          may load the module on the device) with the device current, and
  *          returns W4_ERR_CUDA if that fails.  Make the first call on each
- *          device before any stream capture.
+ *          device before any stream capture.  The address is cached per
+ *          device together with the context it was found in; a call that
+ *          finds another context current (after cudaDeviceReset, or after
+ *          the primary context was released and created again) looks it up
+ *          again, so that call too should come before any capture.
  *   Each call clears (cudaMemsetAsync on `stream`) the arrival counters it
  *          uses before its kernel runs.
  *   One array per device: calls whose executions can overlap on the same
@@ -352,7 +360,9 @@ w4_status nf4_prepack(const uint8_t* Wq, const uint8_t* absmax_q, int N, int K,
                       uint8_t* Wp, w4_stream stream);
 
 /* Y = X . w_hat^T for NF4 weights (same kernel family as w4a16_gemm).
- *   X bf16 [M,K]; Wp from nf4_prepack; s2 as from nf4_quantize; Y bf16 [M,N]. */
+ *   X bf16 [M,K]; Wp from nf4_prepack; s2 as from nf4_quantize; Y bf16 [M,N].
+ *   Workspace rules, the decode limit N <= 2097152 at M <= 32 and the 0 that
+ *   nf4_workspace_bytes returns for an unsupported shape are w4a16_gemm's. */
 size_t nf4_workspace_bytes(int M, int N, int K);
 w4_status nf4_gemm(const uint16_t* X, const uint8_t* Wp, const float* s2, int M, int N,
                    int K, int dq_group, uint16_t* Y, void* workspace,

@@ -150,3 +150,26 @@ def test_variant_bad_arguments_rejected_on_host():
                                  None) == w4.W4_ERR_INVALID_ARG
     assert w4.lib.w4_awq_scale_activations(fake, fake, 1, 12, fake, None) == \
         w4.W4_ERR_INVALID_ARG
+
+
+def test_decode_row_limit_rejected_on_host():
+    # the decode kernel keeps one arrival counter per 32-row group in a fixed
+    # region of 65536 counters: N = 2097152 is the largest decode N; one row
+    # more is reported unsupported (workspace size 0, the call refused before
+    # any launch, so fake device pointers do) instead of aliasing the counters
+    limit = 65536 * 32
+    for M in (1, 16, 32):
+        assert w4.lib.w4_workspace_bytes(M, limit, 256, 128, 0) > 0
+        assert w4.lib.w4_workspace_bytes(M, limit + 1, 256, 128, 0) == 0
+        assert w4.lib.w4_awq_workspace_bytes(M, limit + 1, 256, 128, 0) == 0
+        assert w4.lib.nf4_workspace_bytes(M, limit + 1, 256) == 0
+    # above the decode range the tensor-core kernel has no such limit
+    assert w4.lib.w4_workspace_bytes(33, limit + 1, 256, 128, 0) > 0
+    fake = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 24)
+    st = w4.lib.w4a16_gemm(fake, fake, 1, limit + 32, 256, 128, 0, fake, ws, 1 << 30, None)
+    assert st == w4.W4_ERR_UNSUPPORTED
+    st = w4.lib.nf4_gemm(fake, fake, fake, 4, limit + 32, 256, 256, fake, ws, 1 << 30, None)
+    assert st == w4.W4_ERR_UNSUPPORTED
+    st = w4.lib.w4a16_gemm_static_scratch(fake, fake, 1, limit + 32, 256, 128, 0, fake, None)
+    assert st == w4.W4_ERR_UNSUPPORTED

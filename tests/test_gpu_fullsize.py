@@ -83,9 +83,12 @@ def test_fullsize_llama7b_decode(w4, K, N):
     _int4_case(w4, S.LLAMA7B_DECODE, K, N, S.LLAMA7B_DECODE["Ms"], False)
 
 
+@pytest.mark.parametrize("G", [S.ACT_ORDER_13B["G"], *S.ACT_ORDER_13B["G_sweep"]])
 @pytest.mark.parametrize("K,N", S.ACT_ORDER_13B["shapes"])
-def test_fullsize_act_order_13b(w4, K, N):
-    _int4_case(w4, S.ACT_ORDER_13B, K, N, S.ACT_ORDER_13B["Ms"], True, n_tokens=24)
+def test_fullsize_act_order_13b(w4, K, N, G):
+    # group 32 and the 64 / 128 sweep, each with its own g_idx of the same
+    # seeded permutation
+    _int4_case(w4, dict(S.ACT_ORDER_13B, G=G), K, N, S.ACT_ORDER_13B["Ms"], True, n_tokens=24)
 
 
 @pytest.mark.parametrize("K,N", S.PREFILL_70B["shapes"])

@@ -159,7 +159,8 @@ def _check(y_dev, xbits, what, rows=None):
     return ratio
 
 
-@pytest.mark.parametrize("G,act", [(128, False), (64, False), (32, False), (32, True)])
+@pytest.mark.parametrize("G,act", [(128, False), (64, False), (32, False), (32, True),
+                                   (64, True), (128, True)])
 def test_gemm_unit_vectors_exact(w4, G, act):
     # X rows are unit vectors e_k: Y[m, :] = w_hat[:, k_m] exactly
     N, K = 256, 1024
@@ -187,6 +188,14 @@ GEMM_CASES = [
     (1, 1024, 5120, 32, True),
     (16, 512, 13824, 32, True),
     (256, 256, 2048, 32, True),
+    # act-order group-size sweep ([Survey] §3.2 desc_act with group 64 / 128)
+    (1, 300, 1280, 64, True),        # ragged N, K = 10 stages
+    (7, 77, 768, 128, True),
+    (16, 512, 5120, 64, True),
+    (24, 200, 2560, 128, True),      # three token blocks
+    (33, 128, 1024, 64, True),       # just over the decode range: tensor-core path
+    (256, 384, 2048, 128, True),
+    (300, 256, 1536, 64, True),      # ragged M tile
     # decode work-split edge cases
     (1, 16, 64, 64, False),          # one unit: a single warp does everything
     (2, 1, 128, 128, False),         # one output row

@@ -1,6 +1,7 @@
 """w4a16_gemm_static_scratch: the GEMM with the library's static device
 scratch as workspace, called through the C ABI, against the existing
-w4a16_gemm entry point on the same inputs.
+w4a16_gemm entry point on the same inputs and against the oracle's fp64
+product, both within the matmul tolerance.
 
 Collected last (file name), so it runs after every other test has used the
 library, and it passes alone too.  Two calls in a row per case: the second
@@ -71,14 +72,17 @@ def test_static_scratch_matches_w4a16_gemm(M, N, K, G, act):
     X = _dev(xb.view(np.int16), torch.bfloat16)
     y_entry = w4.w4a16_gemm(X, Wp, N, K, G, act)
     assert w4.device_status() == w4.W4_OK
-    y_ref = O.bf16_bits_to_f64(_host_u16(y_entry))
-    _, abs_ref = O.matmul_ref(xb, what)
+    y_via_entry = O.bf16_bits_to_f64(_host_u16(y_entry))
+    y_oracle, abs_ref = O.matmul_ref(xb, what)
     for _ in range(2):
         y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         w4.w4a16_gemm_static_scratch(X, Wp, N, K, G, act, out=y)
         assert w4.device_status() == w4.W4_OK
-        ok, ratio = O.check_matmul(_host_u16(y), y_ref, abs_ref)
-        assert ok, f"worst difference / tolerance = {ratio}"
+        yh = _host_u16(y)
+        ok, ratio = O.check_matmul(yh, y_via_entry, abs_ref)
+        assert ok, f"against w4a16_gemm: worst difference / tolerance = {ratio}"
+        ok, ratio = O.check_matmul(yh, y_oracle, abs_ref)
+        assert ok, f"against the oracle: worst error / tolerance = {ratio}"
 
 
 @pytest.mark.gpu

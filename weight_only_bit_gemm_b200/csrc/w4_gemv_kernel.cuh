@@ -251,6 +251,9 @@ __device__ __forceinline__ void flush_row_group(const GemvArgs& args,
     unsigned prev = 0;
     if (lane == 0) prev = atom_add_acq_rel_gpu(args.counter + rpg, 1u);
     prev = __shfl_sync(0xffffffffu, prev, 0);
+    // the shuffle carries lane 0's acquire to the other lanes as a value
+    // only; the warp barrier orders their partial loads after it
+    __syncwarp();
     write_y = prev == contributors - 1;
     if (write_y) {
 #pragma unroll
