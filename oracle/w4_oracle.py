@@ -32,6 +32,10 @@ R8  double quantization: per run of 256 consecutive blocks,
     ``s2 = max(absmax) / 255``, ``c = rint(absmax / s2)`` in [0, 255],
     ``absmax' = c * s2`` in fp32; codes are chosen with the unquantized absmax;
 R9  NF4 dequant is ``bf16(fp32(T[q] * absmax'))``;
+R20 mean-offset double quantization (the variant of R8): per run, the mean
+    of the constants (fp64 sum in block order, one rounding to fp32) is
+    subtracted and the residuals take the symmetric 8-bit formula
+    (``max|d| / 127``, codes in [-127, 127]); ``absmax' = fp32(c * s2) + mean``;
 R14 symmetric INT4: ``scale = fp16(max|w| / 7)``, codes ``rint(w / scale)``
     clamped to [-7, 7] and stored + 8 (zero point 8, code 0 unused);
 R15 AWQ: the factor s is an input (found offline); weights enter
@@ -74,6 +78,8 @@ __all__ = [
     "group_index", "rtn_params", "quantize_rtn", "pack_nibbles", "unpack_nibbles",
     "dequant_rtn_f32", "dequant_rtn", "nf4_table", "nf4_midpoints", "nf4_absmax",
     "nf4_codes", "nf4_double_quant", "nf4_quantize", "nf4_dequant", "matmul_ref",
+    "nf4_double_quant_mean", "nf4_absmax_mean_dequant", "nf4_quantize_meandq",
+    "nf4_dequant_meandq",
     "matmul_exact_small", "ulp_bf16", "tolerance", "check_matmul",
     "weight_bytes", "code_bytes", "nf4_weight_bytes",
     "sym_params", "quantize_sym", "awq_scale_weights", "awq_scale_activations",
@@ -367,6 +373,80 @@ def nf4_dequant(Wq: np.ndarray, absmax_q: np.ndarray, s2: np.ndarray,
     c = np.asarray(absmax_q, dtype=np.uint8)[:nb].astype(F32)
     s = np.asarray(s2, dtype=F32)[np.arange(nb) // dq_group]
     a_dq = c * s                                              # fp32 product
+    vals = nf4_table()[qb] * a_dq[:, None]                    # fp32 product
+    return bf16_round_bits(vals.reshape(shape))
+
+
+# ---------------------------------------------------------------------------
+# R20: mean-offset double quantization of the NF4 block constants.
+# [Survey] §6.2 and [Primer] §七: the per-block absmax constants are
+# quantized a second time to save memory; [Comparison] §6 names the switch
+# (bnb_4bit_use_double_quant).  The pages do not say how.  This variant
+# centres each run of dq_group constants on the run's mean before the second
+# quantization, so that the 8 bits cover the spread of the constants rather
+# than their whole range, and stores the residuals with the pages' own
+# symmetric 8-bit formula ([Comparison] §2.3: scale = max|x| / 127,
+# q = round(x / scale) in [-127, 127]).  Per run the mean and the scale are
+# kept in fp32.  Codes of the weights are still chosen with the unquantized
+# absmax (as in R8).
+# ---------------------------------------------------------------------------
+
+def nf4_double_quant_mean(absmax: np.ndarray, dq_group: int = 256):
+    """R20: returns (c int8 [nblocks], mean fp32 [runs], s2 fp32 [runs]).
+
+    Per run of dq_group consecutive blocks (the last run may be shorter):
+      mean = fp32(S / n), S the fp64 sum of the run's fp32 constants added
+             in block order, n the number of blocks in the run;
+      d    = fp32(a - mean);
+      s2   = fp32(max |d| / 127), 1 if that is 0;
+      c    = clamp(rint(d / s2), -127, 127) (fp32 divide)."""
+    a = np.asarray(absmax, dtype=F32)
+    nb = a.size
+    nruns = (nb + dq_group - 1) // dq_group
+    c = np.empty(nb, np.int8)
+    mean = np.empty(nruns, F32)
+    s2 = np.empty(nruns, F32)
+    for r in range(nruns):
+        run = a[r * dq_group:(r + 1) * dq_group]
+        total = 0.0                                   # Python float: fp64
+        for v in run:
+            total += float(v)
+        mu = F32(total / len(run))
+        d = (run - mu).astype(F32)
+        s = F32(np.abs(d).max() / F32(127.0))
+        if s == 0:
+            s = F32(1.0)
+        mean[r] = mu
+        s2[r] = s
+        c[r * dq_group:(r + 1) * dq_group] = np.clip(np.rint(d / s), -127, 127).astype(np.int8)
+    return c, mean, s2
+
+
+def nf4_absmax_mean_dequant(c: np.ndarray, mean: np.ndarray, s2: np.ndarray,
+                            dq_group: int = 256) -> np.ndarray:
+    """R20: absmax' = fp32(fp32(c * s2) + mean), per block (fp32 [nblocks])."""
+    cc = np.asarray(c, dtype=np.int8).astype(F32)
+    run = np.arange(cc.size) // dq_group
+    prod = (cc * np.asarray(s2, F32)[run]).astype(F32)          # fp32 product
+    return (prod + np.asarray(mean, F32)[run]).astype(F32)      # fp32 sum
+
+
+def nf4_quantize_meandq(W: np.ndarray, blocksize: int = 64, dq_group: int = 256):
+    """NF4 with R20 constants.  Returns (packed codes uint8 [N, K/2],
+    absmax codes int8 [N*K/blocksize], mean fp32 [runs], s2 fp32 [runs])."""
+    q = nf4_codes(W, blocksize)
+    c, mean, s2 = nf4_double_quant_mean(nf4_absmax(W, blocksize), dq_group)
+    return pack_nibbles(q), c, mean, s2
+
+
+def nf4_dequant_meandq(Wq: np.ndarray, absmax_q: np.ndarray, mean: np.ndarray,
+                       s2: np.ndarray, blocksize: int = 64, dq_group: int = 256) -> np.ndarray:
+    """R9 with R20 constants: bf16 bits [N, K] of fp32(T[q] * absmax')."""
+    q = unpack_nibbles(Wq)
+    shape = q.shape
+    qb = q.reshape(-1, blocksize)
+    nb = qb.shape[0]
+    a_dq = nf4_absmax_mean_dequant(np.asarray(absmax_q)[:nb], mean, s2, dq_group)
     vals = nf4_table()[qb] * a_dq[:, None]                    # fp32 product
     return bf16_round_bits(vals.reshape(shape))
 

@@ -564,6 +564,133 @@ def test_tolerance_ulp():
     assert ok and r <= 0.5
 
 
+# ------------------------------------------------- NF4 mean-offset double quant (R20)
+
+def test_meandq_worked_example():
+    # two runs of dq_group = 4 constants (the second one partial):
+    # run 0 = (1, 2, 3, 6): mean 12 / 4 = 3 exactly; residuals (-2, -1, 0, 3);
+    #   scale = 3 / 127; codes -2 / (3/127) = -84.67 -> -85, -1 -> -42.33 -> -42,
+    #   0 -> 0 and 3 -> 127; the residual 0 comes back as the mean itself
+    # run 1 = (10, 10, 10): equal constants, residuals 0, scale 1 (the zero
+    #   rule), codes 0, every constant back exactly
+    a = np.array([1, 2, 3, 6, 10, 10, 10], np.float32)
+    c, mean, s2 = O.nf4_double_quant_mean(a, 4)
+    assert c.dtype == np.int8 and c.tolist() == [-85, -42, 0, 127, 0, 0, 0]
+    assert mean.tolist() == [3.0, 10.0]
+    assert s2[0] == np.float32(3.0) / np.float32(127.0) and s2[1] == 1.0
+    back = O.nf4_absmax_mean_dequant(c, mean, s2, 4)
+    assert back[2] == 3.0 and back[4:].tolist() == [10.0, 10.0, 10.0]
+    assert np.all(np.abs(back[:4].astype(np.float64) - a[:4]) <= float(s2[0]) / 2)
+    # an all-zero run stays zero
+    c0, m0, s0 = O.nf4_double_quant_mean(np.zeros(5, np.float32), 256)
+    assert c0.tolist() == [0] * 5 and m0[0] == 0 and s0[0] == 1.0
+    assert np.all(O.nf4_absmax_mean_dequant(c0, m0, s0, 256) == 0)
+
+
+@pytest.mark.parametrize("dq_group", [256, 64])
+def test_meandq_bound_nearest_and_centring(dq_group):
+    W = _rand_w(40, 4096 + 64, 51)
+    W[3, :64] = 0.0                                   # one zero block
+    a = O.nf4_absmax(W)
+    c, mean, s2 = O.nf4_double_quant_mean(a, dq_group)
+    back = O.nf4_absmax_mean_dequant(c, mean, s2, dq_group).astype(np.float64)
+    run = np.arange(a.size) // dq_group
+    s = s2.astype(np.float64)[run]
+    # each code is the nearest of the 255 levels c * s2 to the residual
+    d = (a - mean[run]).astype(np.float32).astype(np.float64)
+    assert np.all(np.abs(c.astype(np.float64) - d / s) <= 0.5 + 1e-6)
+    # reconstruction within half a level plus fp32 rounding of the steps
+    amax = a.astype(np.float64).max()
+    assert np.all(np.abs(back - a) <= s / 2 + 4 * amax * 2.0 ** -24)
+    for r in range(mean.size):
+        blk = a[r * dq_group:(r + 1) * dq_group].astype(np.float64)
+        # the mean is the run's mean (against an exactly rounded sum)
+        exact = math.fsum(blk) / blk.size
+        assert abs(float(mean[r]) - exact) <= abs(exact) * 2.0 ** -23
+        # residuals centred: they sum to ~0, the largest maps to +-127
+        dr = d[r * dq_group:(r + 1) * dq_group]
+        assert abs(dr.sum()) <= blk.size * abs(exact) * 2.0 ** -22
+        assert np.abs(c[r * dq_group:(r + 1) * dq_group]).max() == 127
+
+
+def test_meandq_keeps_the_4bit_codes_and_bounds_w_hat():
+    # the second quantization touches only the constants: the 4-bit codes are
+    # those of the plain scheme; the dequantized weight stays within half a
+    # table gap of the block plus the constant's error and bf16 rounding
+    W = _rand_w(24, 1024, 52)
+    W[1, 64:128] = 0.0
+    Wq_plain, _, _ = O.nf4_quantize(W)
+    Wq, c, mean, s2 = O.nf4_quantize_meandq(W)
+    assert np.array_equal(Wq, Wq_plain)
+    what = O.bf16_bits_to_f32(O.nf4_dequant_meandq(Wq, c, mean, s2)).astype(np.float64)
+    B = W.reshape(-1, 64).astype(np.float64)
+    a = np.abs(B).max(axis=1, keepdims=True)
+    back = O.nf4_absmax_mean_dequant(c, mean, s2)[:, None].astype(np.float64)
+    half_gap = np.diff(O.nf4_table().astype(np.float64)).max() / 2
+    err = np.abs(what.reshape(B.shape) - B)
+    assert np.all(err <= a * half_gap + np.abs(back - a) + np.abs(B) * 2.0 ** -8 + 1e-12)
+    assert np.all(what.reshape(B.shape)[(1 * 1024 + 64) // 64] == 0)   # the zero block
+
+
+def test_planted_mistakes_meandq(monkeypatch):
+    import oracle.w4_oracle as M
+    checks = [test_meandq_worked_example,
+              lambda: test_meandq_bound_nearest_and_centring(256),
+              lambda: test_meandq_bound_nearest_and_centring(64)]
+
+    def caught(name, fn):
+        monkeypatch.setattr(M, name, fn)
+        monkeypatch.setattr(O, name, fn)
+        try:
+            for chk in checks:
+                try:
+                    chk()
+                except AssertionError:
+                    return True
+            return False
+        finally:
+            monkeypatch.undo()
+
+    orig_dq = M.nf4_double_quant_mean
+    orig_back = M.nf4_absmax_mean_dequant
+
+    def no_centring(absmax, dq_group=256):          # plain symmetric 8-bit, mean 0
+        a = np.asarray(absmax, np.float32)
+        c, mean, s2 = orig_dq(a, dq_group)
+        n = (a.size + dq_group - 1) // dq_group
+        s = np.array([max(a[r * dq_group:(r + 1) * dq_group].max() / np.float32(127), 1e-30)
+                      for r in range(n)], np.float32)
+        cc = np.clip(np.rint(a / s[np.arange(a.size) // dq_group]), -127, 127).astype(np.int8)
+        return cc, np.zeros(n, np.float32), s
+    assert caught("nf4_double_quant_mean", no_centring)
+
+    def global_mean(absmax, dq_group=256):          # one mean for every run
+        a = np.asarray(absmax, np.float32)
+        c, mean, s2 = orig_dq(a, dq_group)
+        mu = np.float32(a.astype(np.float64).mean())
+        d = (a - mu).astype(np.float32)
+        run = np.arange(a.size) // dq_group
+        s = np.array([np.abs(d[run == r]).max() / np.float32(127) for r in range(mean.size)],
+                     np.float32)
+        s[s == 0] = 1
+        cc = np.clip(np.rint(d / s[run]), -127, 127).astype(np.int8)
+        return cc, np.full(mean.size, mu, np.float32), s
+    assert caught("nf4_double_quant_mean", global_mean)
+
+    def over_255(absmax, dq_group=256):             # the unsigned 8-bit range
+        c, mean, s2 = orig_dq(absmax, dq_group)
+        s = (s2 * np.float32(127) / np.float32(255)).astype(np.float32)
+        a = np.asarray(absmax, np.float32)
+        run = np.arange(a.size) // dq_group
+        cc = np.clip(np.rint((a - mean[run]) / s[run]), -127, 127).astype(np.int8)
+        return cc, mean, s
+    assert caught("nf4_double_quant_mean", over_255)
+
+    def mean_dropped(c, mean, s2, dq_group=256):    # reconstruction without the mean
+        return orig_back(c, np.zeros_like(np.asarray(mean, np.float32)), s2, dq_group)
+    assert caught("nf4_absmax_mean_dequant", mean_dropped)
+
+
 # ---------------------------------------------------------------- planted mistakes
 
 # ---------------------------------------------------------------- FP4 (E2M1)
