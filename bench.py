@@ -482,6 +482,31 @@ def measure_rows(w4, peaks):
                                "frac_of_hbm": sum(nbytes) / tg / 1e6 / hbm,
                                "eager_TB/s": sum(nbytes) / sum(ts) / 1e9}
 
+    # NEXT row: NF4 with mean-offset double quantization of the constants,
+    # same shapes (8 bytes of constants per run instead of 4)
+    calls, nbytes = [], []
+    for (K, N) in nf["shapes"]:
+        W = torch.from_numpy(S.layer_w(nf, K, N)).cuda()
+        q4, c4, m4, s24 = w4.nf4_quantize_meandq(W)
+        if (K, N) == nf["shapes"][0]:
+            t = time_calls([lambda: w4.nf4_quantize_meandq(W)], reps=5)[0]
+            b = N * K * 4 + N * K / 2 + N * K / 64
+            rows["nf4_meandq_quantize"] = {"shape": [N, K], "ms": t, "GB/s": b / t / 1e6}
+        wp = w4.nf4_prepack(q4, c4.view(torch.uint8))
+        reps = [wp] + [wp.clone() for _ in range(_replicas_for(wp.numel(), l2) - 1)]
+        for M in nf["Ms"]:
+            X = bf16_dev(S.layer_x(nf, M, K, N))
+            for r in reps:
+                calls.append(lambda X=X, r=r, m=m4, s=s24, N=N, K=K:
+                             w4.nf4_gemm_meandq(X, r, m, s, N, K))
+                nbytes.append(nf4_bytes(M, N, K) + 4 * -(-(N * K // 64) // 256))
+        del W
+    tg = time_graph(calls)
+    rows["nf4_meandq_gemm_decode"] = {
+        "configs": "(K,N) in {(4096,14336),(14336,4096)} x M in {1,8,32}, mean-offset constants",
+        "timing": "CUDA graph of all calls",
+        "TB/s": sum(nbytes) / tg / 1e9, "frac_of_hbm": sum(nbytes) / tg / 1e6 / hbm}
+
     # NEXT row: FP4 (E2M1) table in the NF4 kernels, same shapes
     f4 = S.FP4_DECODE
     calls, nbytes = [], []

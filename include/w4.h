@@ -369,6 +369,35 @@ w4_status nf4_gemm(const uint16_t* X, const uint8_t* Wp, const float* s2, int M,
                    size_t workspace_bytes, w4_stream stream);
 
 /* ------------------------------------------------------------------------
+ * NF4 with mean-offset double quantization of the block constants.  The
+ * pages ask for the constants to be quantized a second time ([Survey] §6.2,
+ * the [Primer]'s §七, [Comparison] §6 bnb_4bit_use_double_quant) without
+ * saying how; this variant centres each run of dq_group constants on the
+ * run's mean and stores the residuals with the pages' symmetric 8-bit
+ * formula ([Comparison] §2.3: max|x| / 127, round):
+ *   mu = fp32(S / n), S the fp64 sum of the run's a in block order, n the
+ *        run's block count (the last run may be shorter);
+ *   d = fp32(a - mu); s2 = fp32(max|d| / 127) (1 if 0);
+ *   c = clamp(rint(d / s2), -127, 127) (int8); a' = fp32(fp32(c * s2) + mu)
+ *   w_hat = bf16_rne(fp32(T[q] * a')); codes q as for nf4_quantize.
+ *   absmax_q   out  int8 [N*K/64]
+ *   mean, s2   out  fp32 [ceil(N*K/64/dq_group)] each
+ *   all other arguments, layouts and errors as for nf4_quantize / nf4_dequant.
+ * Prepack the codes and the int8 constants with nf4_prepack (it moves the
+ * constant bytes unchanged; pass absmax_q as bytes) and multiply with
+ * nf4_gemm_meandq, which takes the run means beside s2 and otherwise the
+ * arguments, workspace and limits of nf4_gemm.                             */
+w4_status nf4_quantize_meandq(const float* W, int N, int K, int blocksize, int dq_group,
+                              uint8_t* Wq, int8_t* absmax_q, float* mean, float* s2,
+                              w4_stream stream);
+w4_status nf4_dequant_meandq(const uint8_t* Wq, const int8_t* absmax_q, const float* mean,
+                             const float* s2, int N, int K, int blocksize, int dq_group,
+                             uint16_t* W_out, w4_stream stream);
+w4_status nf4_gemm_meandq(const uint16_t* X, const uint8_t* Wp, const float* mean,
+                          const float* s2, int M, int N, int K, int dq_group, uint16_t* Y,
+                          void* workspace, size_t workspace_bytes, w4_stream stream);
+
+/* ------------------------------------------------------------------------
  * FP4: the second 4-bit type of the block-wise scheme ([Survey] §6.3: the
  * library offers NF4 and FP4; [Survey] §6.1: plain FP4 has three significant
  * bits and uneven spacing), with the 4-bit float layout [S:1][E:2][M:1]

@@ -173,3 +173,17 @@ def test_decode_row_limit_rejected_on_host():
     assert st == w4.W4_ERR_UNSUPPORTED
     st = w4.lib.w4a16_gemm_static_scratch(fake, fake, 1, limit + 32, 256, 128, 0, fake, None)
     assert st == w4.W4_ERR_UNSUPPORTED
+
+
+def test_meandq_entry_points_reject_missing_means():
+    fake = ctypes.c_void_p(1 << 20)
+    assert w4.lib.nf4_quantize_meandq(fake, 4, 128, 64, 256, fake, fake, None, fake,
+                                      None) == w4.W4_ERR_INVALID_ARG
+    assert w4.lib.nf4_dequant_meandq(fake, fake, None, fake, 4, 128, 64, 256, fake,
+                                     None) == w4.W4_ERR_INVALID_ARG
+    assert w4.lib.nf4_gemm_meandq(fake, fake, None, fake, 1, 4, 128, 256, fake, fake, 1 << 20,
+                                  None) == w4.W4_ERR_INVALID_ARG
+    # misaligned means
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    assert w4.lib.nf4_quantize_meandq(fake, 4, 128, 64, 256, fake, fake, odd, fake,
+                                      None) == w4.W4_ERR_INVALID_ARG

@@ -28,12 +28,13 @@ namespace w4 {
 
 enum WeightFormat : int { kFmtInt4 = 0, kFmtNf4 = 1 };
 
-template <int MT_, int STAGES_, int FMT_, int G_>
+template <int MT_, int STAGES_, int FMT_, int G_, bool MEAN_ = false>
 struct GemmCfg {
   static constexpr int MT = MT_;          // tokens per tile (MMA N)
   static constexpr int STAGES = STAGES_;  // shared-memory ring depth
   static constexpr int FMT = FMT_;
   static constexpr int G = G_;            // INT4 group size (ignored for NF4)
+  static constexpr bool MEAN = MEAN_;     // NF4 layout: mean-offset absmax constants
   static constexpr int kXBoxBytes = MT * 128;         // [MT][64] bf16, 128-byte rows
   static constexpr int kXStageBytes = 2 * kXBoxBytes;  // 128 channels
   static constexpr int kWStageBytes = FMT == kFmtInt4 ? int4_stage_bytes(G) : nf4_stage_bytes();
@@ -185,6 +186,7 @@ __device__ __forceinline__ void nf4_dq_word(uint32_t w, float a0, float a1, uint
 struct GemmArgs {
   const uint8_t* Wp;      // prepacked weights (tiles x stages blocks)
   const float* s2;        // NF4 second-level scales (NF4 only)
+  const float* mean;      // NF4 mean-offset double quantization: run means
   uint16_t* Y;            // bf16 [M, N]
   float* partial;         // split-K partials [tile][split][MT][128]
   unsigned int* counter;  // split-K arrival counters [tile]

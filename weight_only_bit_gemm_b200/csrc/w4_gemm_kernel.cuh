@@ -170,12 +170,18 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
           float a0 = 0.0f, a1 = 0.0f;
           if (blk_in_row * 64 < args.K) {
             const long long kb64 = args.K / 64;
-            if (r0 < args.N)
-              a0 = __fmul_rn(static_cast<float>(cp & 0xFFu),
-                             __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0) * kb64 + blk_in_row, args.by_dq)));
-            if (r0 + 8 < args.N)
-              a1 = __fmul_rn(static_cast<float>(cp >> 8),
-                             __ldg(args.s2 + fast_div(static_cast<unsigned long long>(r0 + 8) * kb64 + blk_in_row, args.by_dq)));
+            if (r0 < args.N) {
+              const unsigned long long i0 =
+                  fast_div(static_cast<unsigned long long>(r0) * kb64 + blk_in_row, args.by_dq);
+              a0 = absmax_from_code<C::MEAN>(cp, __ldg(args.s2 + i0),
+                                             C::MEAN ? __ldg(args.mean + i0) : 0.0f);
+            }
+            if (r0 + 8 < args.N) {
+              const unsigned long long i1 =
+                  fast_div(static_cast<unsigned long long>(r0 + 8) * kb64 + blk_in_row, args.by_dq);
+              a1 = absmax_from_code<C::MEAN>(cp >> 8, __ldg(args.s2 + i1),
+                                             C::MEAN ? __ldg(args.mean + i1) : 0.0f);
+            }
           }
 #pragma unroll
           for (int w = 0; w < 4; ++w) nf4_dq_word(words[w], a0, a1, smem_u32(Ts), &out[rgl][4 * w]);

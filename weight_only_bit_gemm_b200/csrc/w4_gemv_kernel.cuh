@@ -46,6 +46,7 @@ struct GemvArgs {
   const uint8_t* Wp;        // prepacked weights
   const uint16_t* X;        // bf16 [M, K] (act-order: already gathered)
   const float* s2;          // NF4 second-level scales
+  const float* mean;        // NF4 mean-offset double quantization: run means
   uint16_t* Y;              // bf16 [M, N]
   float* partial;           // [row group][slot][32 lanes][4 NB] fp32
   unsigned int* counter;    // [row group] arrivals
@@ -67,12 +68,13 @@ struct GemvArgs {
 __host__ __device__ constexpr int gemv_row_groups(int) { return 2; }
 __host__ __device__ constexpr int gemv_acc_split(int NB) { return NB >= 2 ? 1 : 2; }
 
-template <int NB_, int FMT_, int G_>
+template <int NB_, int FMT_, int G_, bool MEAN_ = false>
 struct GemvCfg {
   static constexpr int NB = NB_;   // token blocks of 8
   static constexpr int MT = 8 * NB;
   static constexpr int FMT = FMT_;
   static constexpr int G = G_;
+  static constexpr bool MEAN = MEAN_;  // NF4 layout: mean-offset absmax constants
   static constexpr int kStageBytes = FMT == kFmtInt4 ? int4_stage_bytes(G) : nf4_stage_bytes();
   static constexpr int kWarps = 8;
   static constexpr int kThreads = 32 * kWarps;
@@ -307,6 +309,7 @@ struct S2Cache {
   int rpg = -1;
   int lo[C::kRG][2], hi[C::kRG][2];
   float v[C::kRG][2];
+  float mu[C::kRG][2];  // the run's mean (mean-offset constants only)
 };
 
 // Registers of half h of stage st <- its activation fragments.
@@ -398,6 +401,7 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
           sc.lo[rr][hf] = 0;
           sc.hi[rr][hf] = 0;
           sc.v[rr][hf] = 0.0f;
+          sc.mu[rr][hf] = 0.0f;
         }
     }
     float a0[2][R], a1[2][R];
@@ -416,12 +420,14 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
               const unsigned long long rowb = static_cast<unsigned long long>(r) * kb64;
               const unsigned long long idx = fast_div(rowb + static_cast<unsigned long long>(blk), args.by_dq);
               sc.v[rr][hf] = __ldg(args.s2 + idx);
+              if constexpr (C::MEAN) sc.mu[rr][hf] = __ldg(args.mean + idx);
               const long long lo = static_cast<long long>(idx * static_cast<unsigned long long>(args.dq_group)) -
                                    static_cast<long long>(rowb);
               sc.lo[rr][hf] = static_cast<int>(lo);
               sc.hi[rr][hf] = static_cast<int>(lo + args.dq_group);
             }
-            a = __fmul_rn(static_cast<float>(hf == 0 ? (pair & 0xFFu) : (pair >> 8)), sc.v[rr][hf]);
+            a = absmax_from_code<C::MEAN>(hf == 0 ? pair : (pair >> 8), sc.v[rr][hf],
+                                          sc.mu[rr][hf]);
           }
           if (hf == 0) a0[h][rr] = a; else a1[h][rr] = a;
         }

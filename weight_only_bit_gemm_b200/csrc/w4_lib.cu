@@ -451,28 +451,43 @@ static bool nf4_shape_ok(int N, int K, int blocksize, int dq_group) {
 
 namespace {
 
+// mean == nullptr: the plain double quantization; otherwise the
+// mean-offset one, with the runs' means written to / read from `mean`.
 template <int TABLE>
 w4_status blockwise_quantize(const float* W, int N, int K, int blocksize, int dq_group,
-                             uint8_t* Wq, uint8_t* absmax_q, float* s2, w4_stream stream) {
+                             uint8_t* Wq, uint8_t* absmax_q, float* s2, float* mean,
+                             w4_stream stream) {
   if (!W || !Wq || !absmax_q || !s2) return W4_ERR_INVALID_ARG;
   if (!nf4_shape_ok(N, K, blocksize, dq_group)) return W4_ERR_INVALID_ARG;
-  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(s2, 4)) return W4_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(s2, 4) || !aligned(mean, 4))
+    return W4_ERR_INVALID_ARG;
   const long long nb = static_cast<long long>(N) * K / 64;
   const int runs = ceil_div(nb, dq_group);
-  nf4_quantize_kernel<TABLE><<<runs, dq_group, dq_group * sizeof(float), as_stream(stream)>>>(
-      W, nb, dq_group, Wq, absmax_q, s2);
+  if (mean)
+    nf4_quantize_kernel<TABLE, true>
+        <<<runs, dq_group, (2 * dq_group + 1) * sizeof(float), as_stream(stream)>>>(
+            W, nb, dq_group, Wq, absmax_q, s2, mean);
+  else
+    nf4_quantize_kernel<TABLE, false><<<runs, dq_group, dq_group * sizeof(float),
+                                        as_stream(stream)>>>(W, nb, dq_group, Wq, absmax_q, s2,
+                                                             nullptr);
   return launch_status(cudaGetLastError());
 }
 
-w4_status blockwise_dequant(const uint8_t* Wq, const uint8_t* absmax_q, const float* s2, int N,
-                            int K, int blocksize, int dq_group, int table, uint16_t* W_out,
-                            w4_stream stream) {
+w4_status blockwise_dequant(const uint8_t* Wq, const uint8_t* absmax_q, const float* s2,
+                            const float* mean, int N, int K, int blocksize, int dq_group,
+                            int table, uint16_t* W_out, w4_stream stream) {
   if (!Wq || !absmax_q || !s2 || !W_out) return W4_ERR_INVALID_ARG;
   if (!nf4_shape_ok(N, K, blocksize, dq_group)) return W4_ERR_INVALID_ARG;
-  if (!aligned(Wq, 4) || !aligned(W_out, 16) || !aligned(s2, 4)) return W4_ERR_INVALID_ARG;
+  if (!aligned(Wq, 4) || !aligned(W_out, 16) || !aligned(s2, 4) || !aligned(mean, 4))
+    return W4_ERR_INVALID_ARG;
   const long long total8 = static_cast<long long>(N) * K / 8;
-  nf4_dequant_kernel<<<ceil_div(total8, 256), 256, 0, as_stream(stream)>>>(
-      Wq, absmax_q, s2, total8, dq_group, table, W_out);
+  if (mean)
+    nf4_dequant_kernel<true><<<ceil_div(total8, 256), 256, 0, as_stream(stream)>>>(
+        Wq, absmax_q, s2, mean, total8, dq_group, table, W_out);
+  else
+    nf4_dequant_kernel<false><<<ceil_div(total8, 256), 256, 0, as_stream(stream)>>>(
+        Wq, absmax_q, s2, nullptr, total8, dq_group, table, W_out);
   return launch_status(cudaGetLastError());
 }
 
@@ -482,24 +497,42 @@ extern "C" {
 
 w4_status nf4_quantize(const float* W, int N, int K, int blocksize, int dq_group, uint8_t* Wq,
                        uint8_t* absmax_q, float* s2, w4_stream stream) {
-  return blockwise_quantize<kTableNf4>(W, N, K, blocksize, dq_group, Wq, absmax_q, s2, stream);
+  return blockwise_quantize<kTableNf4>(W, N, K, blocksize, dq_group, Wq, absmax_q, s2, nullptr,
+                                       stream);
 }
 
 w4_status nf4_dequant(const uint8_t* Wq, const uint8_t* absmax_q, const float* s2, int N, int K,
                       int blocksize, int dq_group, uint16_t* W_out, w4_stream stream) {
-  return blockwise_dequant(Wq, absmax_q, s2, N, K, blocksize, dq_group, kTableNf4, W_out,
-                           stream);
+  return blockwise_dequant(Wq, absmax_q, s2, nullptr, N, K, blocksize, dq_group, kTableNf4,
+                           W_out, stream);
 }
 
 w4_status fp4_quantize(const float* W, int N, int K, int blocksize, int dq_group, uint8_t* Wq,
                        uint8_t* absmax_q, float* s2, w4_stream stream) {
-  return blockwise_quantize<kTableFp4>(W, N, K, blocksize, dq_group, Wq, absmax_q, s2, stream);
+  return blockwise_quantize<kTableFp4>(W, N, K, blocksize, dq_group, Wq, absmax_q, s2, nullptr,
+                                       stream);
 }
 
 w4_status fp4_dequant(const uint8_t* Wq, const uint8_t* absmax_q, const float* s2, int N, int K,
                       int blocksize, int dq_group, uint16_t* W_out, w4_stream stream) {
-  return blockwise_dequant(Wq, absmax_q, s2, N, K, blocksize, dq_group, kTableFp4, W_out,
-                           stream);
+  return blockwise_dequant(Wq, absmax_q, s2, nullptr, N, K, blocksize, dq_group, kTableFp4,
+                           W_out, stream);
+}
+
+w4_status nf4_quantize_meandq(const float* W, int N, int K, int blocksize, int dq_group,
+                              uint8_t* Wq, int8_t* absmax_q, float* mean, float* s2,
+                              w4_stream stream) {
+  if (!mean) return W4_ERR_INVALID_ARG;
+  return blockwise_quantize<kTableNf4>(W, N, K, blocksize, dq_group, Wq,
+                                       reinterpret_cast<uint8_t*>(absmax_q), s2, mean, stream);
+}
+
+w4_status nf4_dequant_meandq(const uint8_t* Wq, const int8_t* absmax_q, const float* mean,
+                             const float* s2, int N, int K, int blocksize, int dq_group,
+                             uint16_t* W_out, w4_stream stream) {
+  if (!mean) return W4_ERR_INVALID_ARG;
+  return blockwise_dequant(Wq, reinterpret_cast<const uint8_t*>(absmax_q), s2, mean, N, K,
+                           blocksize, dq_group, kTableNf4, W_out, stream);
 }
 
 void fp4_levels(float out[16]) {

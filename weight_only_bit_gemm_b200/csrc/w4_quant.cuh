@@ -267,12 +267,19 @@ struct Fp4Mids {
 // One thread per 64-block, one CTA per run of dq_group blocks
 // (blockDim.x == dq_group).  Writes packed codes, absmax codes and s2.
 // TABLE selects the NF4 or the FP4 codes; everything else is shared.
-template <int TABLE>
+// MEAN selects the double quantization of the absmax constants:
+//   false  s2 = max(a) / 255 (1 if 0), c = clamp(rint(a / s2), 0, 255) (u8);
+//   true   mean-offset: mu = fp32(fp64 sum of the run's a in block order / n),
+//          d = a - mu, s2 = max|d| / 127 (1 if 0),
+//          c = clamp(rint(d / s2), -127, 127) (int8), mean[run] = mu.
+// Shared memory: dq_group floats (MEAN: 2 dq_group + 1).
+template <int TABLE, bool MEAN>
 __global__ void nf4_quantize_kernel(const float* __restrict__ W, long long nblocks, int dq_group,
                                     uint8_t* __restrict__ Wq, uint8_t* __restrict__ absmax_q,
-                                    float* __restrict__ s2) {
+                                    float* __restrict__ s2, float* __restrict__ mean) {
   extern __shared__ float sm_a[];
-  const long long b = static_cast<long long>(blockIdx.x) * dq_group + threadIdx.x;
+  const long long run0 = static_cast<long long>(blockIdx.x) * dq_group;
+  const long long b = run0 + threadIdx.x;
   const bool valid = b < nblocks;
   float w[64];
   float a = 0.0f;
@@ -289,7 +296,22 @@ __global__ void nf4_quantize_kernel(const float* __restrict__ W, long long nbloc
 #pragma unroll
     for (int i = 0; i < 64; ++i) a = fmaxf(a, fabsf(w[i]));
   }
-  sm_a[threadIdx.x] = a;
+  float key = a;  // what the run's scale is taken from: a, or |a - mu|
+  if constexpr (MEAN) {
+    float* sm_blk = sm_a + dq_group;  // the run's constants, in block order
+    sm_blk[threadIdx.x] = a;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const long long left = nblocks - run0;
+      const int n = left < dq_group ? static_cast<int>(left) : dq_group;
+      double sum = 0.0;
+      for (int i = 0; i < n; ++i) sum += static_cast<double>(sm_blk[i]);
+      sm_blk[dq_group] = static_cast<float>(sum / static_cast<double>(n));
+    }
+    __syncthreads();
+    key = valid ? fabsf(__fsub_rn(a, sm_blk[dq_group])) : 0.0f;
+  }
+  sm_a[threadIdx.x] = key;
   __syncthreads();
   for (int s = 1; s < blockDim.x; s <<= 1) {
     float other = 0.0f;
@@ -298,12 +320,21 @@ __global__ void nf4_quantize_kernel(const float* __restrict__ W, long long nbloc
     if ((threadIdx.x % (2 * s)) == 0) sm_a[threadIdx.x] = fmaxf(sm_a[threadIdx.x], other);
     __syncthreads();
   }
-  float sc = __fdiv_rn(sm_a[0], 255.0f);
+  float sc = __fdiv_rn(sm_a[0], MEAN ? 127.0f : 255.0f);
   if (sc == 0.0f) sc = 1.0f;
-  if (threadIdx.x == 0) s2[blockIdx.x] = sc;
+  if (threadIdx.x == 0) {
+    s2[blockIdx.x] = sc;
+    if constexpr (MEAN) mean[blockIdx.x] = sm_a[2 * dq_group];
+  }
   if (!valid) return;
-  const float c = fminf(fmaxf(rintf(__fdiv_rn(a, sc)), 0.0f), 255.0f);
-  absmax_q[b] = static_cast<uint8_t>(c);
+  if constexpr (MEAN) {
+    const float d = __fsub_rn(a, sm_a[2 * dq_group]);
+    const float c = fminf(fmaxf(rintf(__fdiv_rn(d, sc)), -127.0f), 127.0f);
+    absmax_q[b] = static_cast<uint8_t>(static_cast<int8_t>(c));
+  } else {
+    const float c = fminf(fmaxf(rintf(__fdiv_rn(a, sc)), 0.0f), 255.0f);
+    absmax_q[b] = static_cast<uint8_t>(c);
+  }
   uint32_t packed[8];
   const Fp4Mids fp4;
 #pragma unroll
@@ -321,11 +352,25 @@ __global__ void nf4_quantize_kernel(const float* __restrict__ W, long long nbloc
   dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
 }
 
-// w_hat = bf16_rne(fp32(T[q] * fp32(c * s2))): 8 weights per thread.
+// The reconstructed absmax of a block from its 8-bit code byte:
+//   plain      a' = fp32(c * s2), c unsigned;
+//   mean-offset a' = fp32(fp32(c * s2) + mu), c signed (int8).
+template <bool MEAN>
+__device__ __forceinline__ float absmax_from_code(uint32_t byte, float s2v, float mu) {
+  if constexpr (MEAN)
+    return __fadd_rn(__fmul_rn(static_cast<float>(static_cast<int8_t>(byte & 0xFFu)), s2v), mu);
+  else
+    return __fmul_rn(static_cast<float>(byte & 0xFFu), s2v);
+}
+
+// w_hat = bf16_rne(fp32(T[q] * a')), a' from the block's code byte (see
+// absmax_from_code): 8 weights per thread.
+template <bool MEAN>
 __global__ void nf4_dequant_kernel(const uint8_t* __restrict__ Wq,
                                    const uint8_t* __restrict__ absmax_q,
-                                   const float* __restrict__ s2, long long total8,
-                                   int dq_group, int table, uint16_t* __restrict__ out) {
+                                   const float* __restrict__ s2, const float* __restrict__ mean,
+                                   long long total8, int dq_group, int table,
+                                   uint16_t* __restrict__ out) {
   __shared__ float T[16];
   if (threadIdx.x < 16) T[threadIdx.x] = level_value(table, threadIdx.x);
   __syncthreads();
@@ -333,7 +378,8 @@ __global__ void nf4_dequant_kernel(const uint8_t* __restrict__ Wq,
   if (idx >= total8) return;
   const long long e0 = idx * 8;
   const long long b = e0 / 64;
-  const float a = __fmul_rn(static_cast<float>(absmax_q[b]), s2[b / dq_group]);
+  const long long run = b / dq_group;
+  const float a = absmax_from_code<MEAN>(absmax_q[b], s2[run], MEAN ? mean[run] : 0.0f);
   const uint32_t codes = *reinterpret_cast<const uint32_t*>(Wq + e0 / 2);
   uint32_t res[4];
 #pragma unroll

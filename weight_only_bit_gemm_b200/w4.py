@@ -60,6 +60,9 @@ _SIGS = {
     "nf4_prepack": (_i, [_p, _p, _i, _i, _p, _p]),
     "nf4_workspace_bytes": (_sz, [_i, _i, _i]),
     "nf4_gemm": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "nf4_quantize_meandq": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p, _p]),
+    "nf4_dequant_meandq": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p, _p]),
+    "nf4_gemm_meandq": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
     "fp4_quantize": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p]),
     "fp4_dequant": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p]),
     "fp4_levels": (None, [_p]),
@@ -380,6 +383,46 @@ def nf4_quantize(W, blocksize=64, dq_group=256):
 def nf4_dequant(Wq, absmax_q, s2, dq_group=256, blocksize=64):
     return _blockwise_dequant(lib.nf4_dequant, "nf4_dequant", Wq, absmax_q, s2, dq_group,
                               blocksize)
+
+
+def nf4_quantize_meandq(W, blocksize=64, dq_group=256):
+    """NF4 with mean-offset double quantization of the block constants:
+    (Wq, absmax codes int8, run means fp32, s2 fp32)."""
+    _cuda(W, torch.float32, "W")
+    N, K = W.shape
+    dev = W.device
+    nb = N * K // blocksize
+    runs = (nb + dq_group - 1) // dq_group
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    aq = torch.empty(nb, dtype=torch.int8, device=dev)
+    mean = torch.empty(runs, dtype=torch.float32, device=dev)
+    s2 = torch.empty(runs, dtype=torch.float32, device=dev)
+    _check(lib.nf4_quantize_meandq(_ptr(W), N, K, blocksize, dq_group, _ptr(Wq), _ptr(aq),
+                                   _ptr(mean), _ptr(s2), _stream()), "nf4_quantize_meandq")
+    return Wq, aq, mean, s2
+
+
+def nf4_dequant_meandq(Wq, absmax_q, mean, s2, dq_group=256, blocksize=64):
+    N, K = Wq.shape[0], Wq.shape[1] * 2
+    out = torch.empty((N, K), dtype=torch.bfloat16, device=Wq.device)
+    _check(lib.nf4_dequant_meandq(_ptr(Wq), _ptr(absmax_q), _ptr(mean), _ptr(s2), N, K,
+                                  blocksize, dq_group, _ptr(out), _stream()),
+           "nf4_dequant_meandq")
+    return out
+
+
+def nf4_gemm_meandq(X, Wp, mean, s2, N, K, dq_group=256, out=None, workspace=None):
+    """Y = X . w_hat^T for NF4 weights with mean-offset constants (Wp from
+    nf4_prepack of the codes and the int8 constants)."""
+    _cuda(X, torch.bfloat16, "X")
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    need = nf4_workspace_bytes(M, N, K)
+    ws = _ws_view(workspace if workspace is not None else _WS.get(need, X.device))
+    _check(lib.nf4_gemm_meandq(_ptr(X), _ptr(Wp), _ptr(mean), _ptr(s2), M, N, K, dq_group,
+                               _ptr(out), _ptr(ws), ws.numel(), _stream()), "nf4_gemm_meandq")
+    return out
 
 
 def fp4_quantize(W, blocksize=64, dq_group=256):
