@@ -55,8 +55,11 @@ enum {
   W4_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed            */
   W4_ERR_TIMEOUT = 4,     /* a device pipeline wait gave up (device status)  */
   W4_ERR_DEVICE_INPUT = 5, /* the device found bad input data (device status) */
-  W4_ERR_SCRATCH_LIMIT = 6 /* w4a16_gemm_static_scratch: the call needs more
-                              workspace than W4_STATIC_SCRATCH_BYTES           */
+  W4_ERR_SCRATCH_LIMIT = 6, /* w4a16_gemm_static_scratch: the call needs more
+                               workspace than W4_STATIC_SCRATCH_BYTES          */
+  W4_ERR_BOUNDS = 7        /* bounds-checked build only (device status): a
+                              kernel index fell outside its buffer; the access
+                              was skipped, so outputs are not to be trusted   */
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -66,9 +69,17 @@ const char* w4_status_string(w4_status s);
 int w4_version(void);
 
 /* Waits for `stream`, then returns and clears the error word that kernels of
- * this library set on the current device: W4_OK, W4_ERR_TIMEOUT or
- * W4_ERR_DEVICE_INPUT (or W4_ERR_CUDA if the synchronisation itself failed). */
+ * this library set on the current device: W4_OK, W4_ERR_BOUNDS (bounds-checked
+ * build only), W4_ERR_TIMEOUT or W4_ERR_DEVICE_INPUT, in that order of
+ * precedence (or W4_ERR_CUDA if the synchronisation itself failed). */
 w4_status w4_device_status(w4_stream stream);
+
+/* 1 for the bounds-checked build of this library (libw4b200_checked.so,
+ * compiled with W4_CHECKED: every global access of every kernel is checked
+ * against the extent of its buffer implied by the call's arguments; a
+ * violation is recorded as W4_ERR_BOUNDS and the access skipped), 0 for the
+ * normal build.  The two builds export the same functions. */
+int w4_checked_build(void);
 
 /* Failure-path check (no counterpart on the pages): launches one thread that
  * runs this library's bounded pipeline wait on a barrier nothing arrives on,

@@ -572,12 +572,22 @@ def gptq_eliminate(Hi: np.ndarray, j: int) -> np.ndarray:
 
 
 def gptq_quantize(W: np.ndarray, H: np.ndarray, G: int, act_order: bool = False,
-                  damp: float = 0.01):
+                  damp: float = 0.01, follow: np.ndarray | None = None,
+                  record: dict | None = None):
     """INT4 codes with GPTQ error compensation (R18).
 
     Returns (codes uint8 [N, K], scale fp16 [N, K/G], zero uint8 [N, K/G],
     g_idx int32 [K] or None): the canonical format of ``quantize_rtn``; with
-    act-order the channel processed j-th belongs to group j // G."""
+    act-order the channel processed j-th belongs to group j // G.
+
+    Observation hook for comparing another implementation step by step (the
+    arithmetic is unchanged): with ``follow`` (codes uint8 [N, K], canonical
+    channel order) the error of each column is computed from those codes
+    instead of this function's own, so that the compensated weights track the
+    other implementation's decisions; ``record`` (a dict) then receives
+    'own' (this function's own code decisions, canonical order) and 'tie'
+    (the distance of w / s to the nearest half-integer, in code units, for
+    each decision)."""
     W = np.array(W, dtype=np.float64, copy=True)
     N, K = W.shape
     if K % G:
@@ -596,8 +606,16 @@ def gptq_quantize(W: np.ndarray, H: np.ndarray, G: int, act_order: bool = False,
         sf = s16[:, g].astype(F32)
         zf = zp[:, g].astype(F32)
         w32 = Q[:, j].astype(F32)
-        q = np.clip(np.rint(w32 / sf) + zf, 0, 15)  # decided in fp32
+        ratio = w32 / sf
+        q = np.clip(np.rint(ratio) + zf, 0, 15)      # decided in fp32
         codes[:, j] = q.astype(np.uint8)
+        if record is not None:
+            record.setdefault("own", np.zeros((N, K), np.uint8))[:, perm[j]] = codes[:, j]
+            record.setdefault("tie", np.zeros((N, K)))[:, perm[j]] = np.abs(
+                np.abs(ratio.astype(np.float64) - np.rint(ratio)) - 0.5)
+        if follow is not None:
+            q = np.asarray(follow)[:, perm[j]].astype(F32)
+            codes[:, j] = q.astype(np.uint8)
         deq = ((q - zf) * sf).astype(F32).astype(np.float64)
         err = (Q[:, j] - deq) / Hi[0, 0]
         Q[:, j + 1:] -= np.outer(err, Hi[0, 1:])    # spread over the remaining columns

@@ -187,3 +187,14 @@ def test_meandq_entry_points_reject_missing_means():
     odd = ctypes.c_void_p((1 << 20) + 2)
     assert w4.lib.nf4_quantize_meandq(fake, 4, 128, 64, 256, fake, fake, odd, fake,
                                       None) == w4.W4_ERR_INVALID_ARG
+
+
+def test_checked_build_exports_the_same_functions():
+    # the bounds-checked twin of the library: same C ABI, reports itself
+    build.build(checked=True)
+    chk = w4.checked_library()
+    assert chk.w4_checked_build() == 1
+    assert w4.lib.w4_checked_build() == 0
+    missing = [n for n in w4.header_functions() if not hasattr(chk, n)]
+    assert missing == []
+    assert b"bounds" in w4.lib.w4_status_string(w4.W4_ERR_BOUNDS)

@@ -196,6 +196,8 @@ struct GemmArgs {
   int splits;
   FastDivIdx by_dq;        // NF4: 64-block index -> s2 index (double-quant run)
   int table;              // NF4 layout: level table (kTableNf4 / kTableFp4)
+  // buffer extents, read only by the bounds-checked build
+  unsigned long long wp_bytes, partial_floats, s2_count;
 };
 
 }  // namespace w4

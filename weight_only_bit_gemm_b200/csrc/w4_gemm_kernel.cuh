@@ -68,13 +68,21 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
       const uint64_t pol_x = policy_evict_last();   // X is shared by every CTA
       const uint8_t* wsrc =
           args.Wp + (static_cast<size_t>(nt) * args.KS + s0) * C::kWStageBytes;
+      // bounds-checked build: a stage outside Wp is flagged and replaced by the
+      // first stage (so that the barrier still completes)
+      auto stage_src = [&](int it) -> const uint8_t* {
+        const unsigned long long off = (static_cast<unsigned long long>(nt) * args.KS + s0 + it) *
+                                       C::kWStageBytes;
+        return in_bounds(off + C::kWStageBytes - 1, args.wp_bytes)
+                   ? wsrc + static_cast<size_t>(it) * C::kWStageBytes
+                   : args.Wp;
+      };
       // The weights do not depend on the previous kernel: start streaming the
       // first ring's worth before waiting for it, then add the X tiles.
       const int first = nst < C::STAGES ? nst : C::STAGES;
       for (int it = 0; it < first; ++it) {
         mbar_arrive_expect_tx(&full[it], C::kXStageBytes + C::kWStageBytes);
-        bulk_g2s(wsl + it * C::kWSlot, wsrc + static_cast<size_t>(it) * C::kWStageBytes,
-                 C::kWStageBytes, &full[it], pol_w);
+        bulk_g2s(wsl + it * C::kWSlot, stage_src(it), C::kWStageBytes, &full[it], pol_w);
       }
       grid_dep_wait();
       int issued = 0;
@@ -83,8 +91,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
         if (it >= C::STAGES) {
           if (!mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1)) break;
           mbar_arrive_expect_tx(&full[s], C::kXStageBytes + C::kWStageBytes);
-          bulk_g2s(wsl + s * C::kWSlot, wsrc + static_cast<size_t>(it) * C::kWStageBytes,
-                   C::kWStageBytes, &full[s], pol_w);
+          bulk_g2s(wsl + s * C::kWSlot, stage_src(it), C::kWStageBytes, &full[s], pol_w);
         }
         tma_load_3d(xs + s * C::kXStageBytes, &xmap, 0, mtile * C::MT, (s0 + it) * 2, &full[s],
                     pol_x);
@@ -171,14 +178,16 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
           if (blk_in_row * 64 < args.K) {
             const long long kb64 = args.K / 64;
             if (r0 < args.N) {
-              const unsigned long long i0 =
+              unsigned long long i0 =
                   fast_div(static_cast<unsigned long long>(r0) * kb64 + blk_in_row, args.by_dq);
+              if (!in_bounds(i0, args.s2_count)) i0 = 0;
               a0 = absmax_from_code<C::MEAN>(cp, __ldg(args.s2 + i0),
                                              C::MEAN ? __ldg(args.mean + i0) : 0.0f);
             }
             if (r0 + 8 < args.N) {
-              const unsigned long long i1 =
+              unsigned long long i1 =
                   fast_div(static_cast<unsigned long long>(r0 + 8) * kb64 + blk_in_row, args.by_dq);
+              if (!in_bounds(i1, args.s2_count)) i1 = 0;
               a1 = absmax_from_code<C::MEAN>(cp >> 8, __ldg(args.s2 + i1),
                                              C::MEAN ? __ldg(args.mean + i1) : 0.0f);
             }
@@ -233,7 +242,9 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
             if (m < args.M && n < args.N)
               args.Y[static_cast<size_t>(m) * args.N + n] =
                   __bfloat16_as_ushort(__float2bfloat16_rn(acc));
-          } else {
+          } else if (in_bounds(static_cast<unsigned long long>(part - args.partial) +
+                                   (cb + j) * kTileRows + row,
+                               args.partial_floats)) {
             part[(cb + j) * kTileRows + row] = acc;
           }
         }
@@ -248,7 +259,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
         if (lane == 0) mbar_arrive(epi1);
         bool have_flag = true;
         if (threadIdx.x == 64) {
-          if (mbar_wait(epi1, 0)) {
+          if (mbar_wait(epi1, 0) && in_bounds(tile_id, 65536)) {
             const unsigned prev = atomicAdd(args.counter + tile_id, 1u);
             *last_flag = (prev == static_cast<unsigned>(args.splits - 1)) ? 1 : 0;
           } else {
@@ -273,6 +284,10 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
             for (int sp = 0; sp < args.splits; ++sp) {
               const float* src = base + (static_cast<size_t>(sp) * C::MT + ml0) * kTileRows + row;
               float v[kCb];
+              if (!in_bounds(static_cast<unsigned long long>(src - args.partial) +
+                                 (kCb - 1) * kTileRows,
+                             args.partial_floats))
+                continue;
 #pragma unroll
               for (int j = 0; j < kCb; ++j) v[j] = __ldcg(src + j * kTileRows);
 #pragma unroll
@@ -328,6 +343,7 @@ __global__ void __launch_bounds__(256) x_prologue_kernel(const uint16_t* X,
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       c[e] = perm[j0 + e];
+      if (!in_bounds(static_cast<unsigned int>(c[e]), static_cast<unsigned int>(K))) c[e] = 0;
       v[e] = xr[c[e]];
     }
   } else {

@@ -11,8 +11,13 @@
 // m16n8k16 bf16 MMAs (one activation fragment serves both row groups) and
 // accumulates in fp32 registers.  No producer warp and no barriers between
 // warps: the only synchronisation is the deterministic reduction over the
-// warps that share a row pair (partials in a fixed slot per warp; the last
-// one to arrive sums them in slot order).
+// warps that share a row pair, in two levels.  Warps of one CTA combine in
+// shared memory (a CTA-scope arrival counter; the last local arrival sums
+// the warps' partials in warp order); a row pair that several CTAs share is
+// then combined once per CTA through global memory (a partial slot per CTA
+// and a device-scope arrival counter; the last CTA sums them in CTA order).
+// Measured on B200: the number of partials the last arrival reads from
+// global memory, not the arithmetic, sets the tail of each call.
 //
 // Why not tcgen05 here: a tcgen05.mma of kind::f16 occupies the SM's tensor
 // core for ~200 cycles whatever its N (measured on B200 for N = 16..256), so a
@@ -58,6 +63,8 @@ struct GemvArgs {
   FastDivIdx by_dq;          // NF4: 64-block index -> s2 index
   int dq_group;             // NF4: 64-blocks per second-level scale
   int table;                // NF4 layout: level table (kTableNf4 / kTableFp4)
+  // buffer extents, read only by the bounds-checked build
+  unsigned long long wp_bytes, partial_floats, s2_count;
 };
 
 // Row groups (16 rows each) per decode work unit: two share each activation
@@ -87,7 +94,15 @@ struct GemvCfg {
   static constexpr int kRG = gemv_row_groups(NB);  // row groups per work unit
   static constexpr int kAS = gemv_acc_split(NB);  // accumulators per (row group, token block)
   static constexpr int kSlot = kRG * 1024 + (kRG * (kScaleBytes + kZeroBytes) + 15) / 16 * 16;
-  static constexpr int kSmemBytes = kWarps * kDepth * kSlot;
+  static constexpr int kRingBytes = kWarps * kDepth * kSlot;
+  // CTA-level reduction (up to two token blocks; four would not leave room
+  // for two CTAs per SM): two partial slots per warp (the warp's first and
+  // last row-pair segments), [slot][V/4][32 lanes] float4, and one arrival
+  // counter per warp (the row pair that ends the warp's range).
+  static constexpr bool kCtaReduce = NB <= 2;
+  static constexpr int kV = kRG * NB * 4;  // partial floats per lane
+  static constexpr int kRedBytes = kCtaReduce ? kWarps * 2 * 32 * kV * 4 : 0;
+  static constexpr int kSmemBytes = kRingBytes + kRedBytes + kWarps * 4;
 };
 
 __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t (&a)[4],
@@ -121,9 +136,12 @@ struct StageRegs {
 
 template <class C>
 __device__ __forceinline__ void issue_stage(const uint8_t* __restrict__ blk, uint32_t slot, int rpl,
-                                            int lane) {
+                                            int lane, const GemvArgs& args) {
   constexpr int R = C::kRG;
   const int rgl0 = rpl * R;
+  if (kChecked && !in_bounds(static_cast<unsigned long long>(blk - args.Wp) + C::kStageBytes - 1,
+                             args.wp_bytes))
+    return;
   const uint8_t* cb = blk + rgl0 * 1024 + lane * 16;
 #pragma unroll
   for (int i = 0; i < 2 * R; ++i) cp_async16(slot + i * 512 + lane * 16, cb + i * 512);
@@ -218,12 +236,79 @@ __device__ __forceinline__ uint32_t owner_of(uint32_t u, const GemvArgs& a) {
   return u < big ? fast_div(u, a.by_q1) : a.r + fast_div(u - big, a.by_q);
 }
 
+// First unit after the range of warp w.
+__device__ __forceinline__ uint32_t range_end(uint32_t w, const GemvArgs& a) {
+  return w * a.q + (w < a.r ? w : a.r) + a.q + (w < a.r ? 1u : 0u);
+}
+
+// Shared-memory state of the CTA-level reduction.
+struct CtaRed {
+  float4* part;            // [warp][kind][V/4][32 lanes]
+  unsigned int* count;     // [warp]: arrivals for the row pair that ends its range
+};
+
+// Global level: this lane's partial `tot` in slot `slot` of row pair rpg,
+// `contrib` slots in all; returns true (with tot the full sum, added in slot
+// order) for the last of them to arrive, false for the others.
+template <class C>
+__device__ __forceinline__ bool global_combine(const GemvArgs& args,
+                                               float (&tot)[C::kRG][C::NB][4], int rpg,
+                                               uint32_t slot, uint32_t contrib, int lane) {
+  constexpr int R = C::kRG;
+  constexpr int V = C::kV;
+  float* dst = args.partial + ((static_cast<size_t>(rpg) * args.max_slots + slot) * 32 + lane) * V;
+  if (kChecked &&
+      !(in_bounds(((static_cast<unsigned long long>(rpg) * args.max_slots + contrib - 1) * 32 + lane) * V + V - 1,
+                  args.partial_floats) &&
+        in_bounds(slot, contrib) && in_bounds(static_cast<unsigned long long>(rpg) * 4 + 3, 65536ull * 4)))
+    return false;
+#pragma unroll
+  for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+    for (int nb = 0; nb < C::NB; ++nb)
+      *reinterpret_cast<float4*>(dst + (rr * C::NB + nb) * 4) =
+          make_float4(tot[rr][nb][0], tot[rr][nb][1], tot[rr][nb][2], tot[rr][nb][3]);
+  __syncwarp();
+  unsigned prev = 0;
+  if (lane == 0) prev = atom_add_acq_rel_gpu(args.counter + rpg, 1u);
+  prev = __shfl_sync(0xffffffffu, prev, 0);
+  // the shuffle carries lane 0's acquire to the other lanes as a value
+  // only; the warp barrier orders their partial loads after it
+  __syncwarp();
+  if (prev != contrib - 1) return false;
+#pragma unroll
+  for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+    for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tot[rr][nb][j] = 0.0f;
+  const float* base = args.partial + (static_cast<size_t>(rpg) * args.max_slots * 32 + lane) * V;
+  for (uint32_t sp = 0; sp < contrib; ++sp) {
+#pragma unroll
+    for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+      for (int nb = 0; nb < C::NB; ++nb) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(
+            base + static_cast<size_t>(sp) * 32 * V + (rr * C::NB + nb) * 4));
+        tot[rr][nb][0] += v.x;
+        tot[rr][nb][1] += v.y;
+        tot[rr][nb][2] += v.z;
+        tot[rr][nb][3] += v.w;
+      }
+  }
+  if (lane == 0) args.counter[rpg] = 0u;
+  return true;
+}
+
+// The warp's sums over units [seg0, seg1) of row pair rpg (its range ends at
+// unit wend) go to Y, directly when the warp covered the whole row pair,
+// otherwise through the two-level reduction.
 template <class C>
 __device__ __forceinline__ void flush_row_group(const GemvArgs& args,
                                                 float (&acc)[C::kRG][C::kAS][C::NB][4], int rpg,
-                                                uint32_t seg0, uint32_t seg1, uint32_t wid, int lane) {
+                                                uint32_t seg0, uint32_t seg1, uint32_t wid,
+                                                uint32_t wend, int lane, const CtaRed& cr) {
   constexpr int R = C::kRG;
-  constexpr int V = R * C::NB * 4;  // floats per lane
   const int g = lane >> 2, u = lane & 3;
   float tot[R][C::NB][4];
 #pragma unroll
@@ -240,45 +325,70 @@ __device__ __forceinline__ void flush_row_group(const GemvArgs& args,
   const uint32_t re = rs + static_cast<uint32_t>(args.KS);
   bool write_y = true;
   if (seg0 != rs || seg1 != re) {
-    const uint32_t first = owner_of(rs, args);
-    const uint32_t contributors = owner_of(re - 1, args) - first + 1;
-    float* slot = args.partial + ((static_cast<size_t>(rpg) * args.max_slots + (wid - first)) * 32 + lane) * V;
-#pragma unroll
-    for (int rr = 0; rr < R; ++rr)
-#pragma unroll
-      for (int nb = 0; nb < C::NB; ++nb)
-        *reinterpret_cast<float4*>(slot + (rr * C::NB + nb) * 4) =
-            make_float4(tot[rr][nb][0], tot[rr][nb][1], tot[rr][nb][2], tot[rr][nb][3]);
-    __syncwarp();
-    unsigned prev = 0;
-    if (lane == 0) prev = atom_add_acq_rel_gpu(args.counter + rpg, 1u);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    // the shuffle carries lane 0's acquire to the other lanes as a value
-    // only; the warp barrier orders their partial loads after it
-    __syncwarp();
-    write_y = prev == contributors - 1;
-    if (write_y) {
-#pragma unroll
-      for (int rr = 0; rr < R; ++rr)
-#pragma unroll
-        for (int nb = 0; nb < C::NB; ++nb)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) tot[rr][nb][j] = 0.0f;
-      const float* base = args.partial + (static_cast<size_t>(rpg) * args.max_slots * 32 + lane) * V;
-      for (uint32_t sp = 0; sp < contributors; ++sp) {
+    const uint32_t first = owner_of(rs, args);     // warps that touch the row pair
+    const uint32_t last = owner_of(re - 1, args);
+    const uint32_t cta_w0 = blockIdx.x * C::kWarps;
+    const uint32_t cta_w1 = cta_w0 + C::kWarps - 1;
+    bool done = false;  // the row pair lies within this CTA and has been summed here
+    if constexpr (C::kCtaReduce) {
+      const uint32_t lw0 = first > cta_w0 ? first : cta_w0;
+      const uint32_t lw1 = last < cta_w1 ? last : cta_w1;
+      if (lw1 > lw0) {
+        // level 1: deposit in this warp's slot; the last local arrival sums.
+        // Slot kind 1 holds a warp's last segment (the one ending its range),
+        // kind 0 its first segment when that ends earlier.
+        const uint32_t kind = seg1 == wend ? 1u : 0u;
+        float4* mine = cr.part + ((wid - cta_w0) * 2 + kind) * (C::kV / 4) * 32 + lane;
 #pragma unroll
         for (int rr = 0; rr < R; ++rr)
 #pragma unroll
-          for (int nb = 0; nb < C::NB; ++nb) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                base + static_cast<size_t>(sp) * 32 * V + (rr * C::NB + nb) * 4));
-            tot[rr][nb][0] += v.x;
-            tot[rr][nb][1] += v.y;
-            tot[rr][nb][2] += v.z;
-            tot[rr][nb][3] += v.w;
-          }
+          for (int nb = 0; nb < C::NB; ++nb)
+            mine[(rr * C::NB + nb) * 32] =
+                make_float4(tot[rr][nb][0], tot[rr][nb][1], tot[rr][nb][2], tot[rr][nb][3]);
+        __syncwarp();
+        unsigned prev = 0;
+        if (lane == 0) {
+          asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                       : "=r"(prev)
+                       : "r"(smem_u32(cr.count + (lw0 - cta_w0)))
+                       : "memory");
+        }
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        __syncwarp();
+        if (prev != lw1 - lw0) return;
+        // the first local contributor's range ends inside the row pair and so
+        // do the middle ones' (kind 1); the last one's segment is its last
+        // one only if its range ends inside the row pair too
+        const uint32_t kind_last = range_end(lw1, args) <= re ? 1u : 0u;
+#pragma unroll
+        for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+          for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tot[rr][nb][j] = 0.0f;
+        for (uint32_t w = lw0; w <= lw1; ++w) {
+          const uint32_t k = w < lw1 ? 1u : kind_last;
+          const float4* src = cr.part + ((w - cta_w0) * 2 + k) * (C::kV / 4) * 32 + lane;
+#pragma unroll
+          for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+            for (int nb = 0; nb < C::NB; ++nb) {
+              const float4 v = src[(rr * C::NB + nb) * 32];
+              tot[rr][nb][0] += v.x;
+              tot[rr][nb][1] += v.y;
+              tot[rr][nb][2] += v.z;
+              tot[rr][nb][3] += v.w;
+            }
+        }
+        done = first >= cta_w0 && last <= cta_w1;
       }
-      if (lane == 0) args.counter[rpg] = 0u;
+    }
+    if (!done) {
+      // level 2: one partial per CTA (per warp without the CTA level)
+      const uint32_t unit0 = C::kCtaReduce ? first / C::kWarps : first;
+      const uint32_t unit1 = C::kCtaReduce ? last / C::kWarps : last;
+      const uint32_t me = C::kCtaReduce ? blockIdx.x : wid;
+      write_y = global_combine<C>(args, tot, rpg, me - unit0, unit1 - unit0 + 1, lane);
     }
   }
   if (write_y) {
@@ -418,7 +528,8 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
           if (blk < kb64 && r < args.N) {
             if (blk < sc.lo[rr][hf] || blk >= sc.hi[rr][hf]) {
               const unsigned long long rowb = static_cast<unsigned long long>(r) * kb64;
-              const unsigned long long idx = fast_div(rowb + static_cast<unsigned long long>(blk), args.by_dq);
+              unsigned long long idx = fast_div(rowb + static_cast<unsigned long long>(blk), args.by_dq);
+              if (!in_bounds(idx, args.s2_count)) idx = 0;
               sc.v[rr][hf] = __ldg(args.s2 + idx);
               if constexpr (C::MEAN) sc.mu[rr][hf] = __ldg(args.mean + idx);
               const long long lo = static_cast<long long>(idx * static_cast<unsigned long long>(args.dq_group)) -
@@ -445,10 +556,13 @@ template <class C>
 __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(const GemvArgs args) {
   constexpr int R = C::kRG;
   __shared__ __align__(64) float Ts[16];  // NF4 / FP4 levels
-  if (C::FMT == kFmtNf4) {
-    if (threadIdx.x < 16) Ts[threadIdx.x] = level_value(args.table, threadIdx.x);
-    __syncthreads();
-  }
+  extern __shared__ __align__(16) uint8_t w4_gemv_smem[];
+  CtaRed cr;
+  cr.part = reinterpret_cast<float4*>(w4_gemv_smem + C::kRingBytes);
+  cr.count = reinterpret_cast<unsigned int*>(w4_gemv_smem + C::kRingBytes + C::kRedBytes);
+  if (C::FMT == kFmtNf4 && threadIdx.x < 16) Ts[threadIdx.x] = level_value(args.table, threadIdx.x);
+  if (threadIdx.x < C::kWarps) cr.count[threadIdx.x] = 0u;
+  __syncthreads();  // the only CTA-wide barrier: before any warp may leave
   grid_dep_launch();
 
   const int lane = threadIdx.x & 31;
@@ -465,6 +579,10 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
   for (int nb = 0; nb < C::NB; ++nb) {
     const int row = min(nb * 8 + g, args.M - 1);
     xrow[nb] = args.X + static_cast<size_t>(row) * args.K + 4 * u;
+    // the last fragment of the row: channels (K/16 - 1) * 16 + 4u .. + 3
+    if (kChecked && !in_bounds(static_cast<unsigned long long>(row) * args.K + (args.K - 16) + 4 * u + 3,
+                               static_cast<unsigned long long>(args.M) * args.K))
+      return;
   }
 
   const int rpg0 = static_cast<int>(fast_div(ua, args.by_ks));
@@ -482,13 +600,12 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
     }
   };
 
-  extern __shared__ __align__(16) uint8_t w4_gemv_smem[];
   uint8_t* ring = w4_gemv_smem + (threadIdx.x >> 5) * (C::kDepth * C::kSlot);
   const uint32_t ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
 #pragma unroll
   for (int i = 0; i < C::kDepth - 1; ++i) {
     if (i < left) {
-      issue_stage<C>(pf_ptr, ring_s + i * C::kSlot, pf_rpg % kPairsPerTile, lane);
+      issue_stage<C>(pf_ptr, ring_s + i * C::kSlot, pf_rpg % kPairsPerTile, lane, args);
       advance();
     }
     cp_async_commit();
@@ -523,7 +640,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
     read_stage<C>(ring + cs * C::kSlot, cur, lane);
     if (n + C::kDepth - 1 < left) {
       const int is = cs == 0 ? C::kDepth - 1 : cs - 1;
-      issue_stage<C>(pf_ptr, ring_s + is * C::kSlot, pf_rpg % kPairsPerTile, lane);
+      issue_stage<C>(pf_ptr, ring_s + is * C::kSlot, pf_rpg % kPairsPerTile, lane, args);
       advance();
     }
     cp_async_commit();
@@ -533,7 +650,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
                      acc);
     if (st == KS - 1 || n + 1 == left) {
       const uint32_t seg1 = ua + static_cast<uint32_t>(n) + 1;
-      flush_row_group<C>(args, acc, rpg, seg0, seg1, wid, lane);
+      flush_row_group<C>(args, acc, rpg, seg0, seg1, wid, ua + static_cast<uint32_t>(left), lane,
+                         cr);
       ++rpg;
       st = 0;
       seg0 = seg1;

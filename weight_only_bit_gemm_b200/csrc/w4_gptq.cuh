@@ -344,14 +344,18 @@ __global__ void __launch_bounds__(kGptqRows) gptq_block_kernel(
   float* Qb = sm_g + kGptqB * kGptqB;                 // [kGptqRows][kGptqB + 1]
   const int t = threadIdx.x;
   const int n0 = blockIdx.x * kGptqRows;
+  const unsigned long long kk = static_cast<unsigned long long>(K) * K;
   for (int e = t; e < bw * bw; e += kGptqRows) {
     const int a = e / bw, b = e - a * bw;
-    Ub[a * kGptqB + b] = b >= a ? U[static_cast<size_t>(j0 + a) * K + j0 + b] : 0.0f;
+    const unsigned long long ui = static_cast<unsigned long long>(j0 + a) * K + j0 + b;
+    Ub[a * kGptqB + b] = b >= a && in_bounds(ui, kk) ? U[ui] : 0.0f;
   }
   for (int e = t; e < kGptqRows * bw; e += kGptqRows) {
     const int r = e / bw, c = e - r * bw;
     const int n = n0 + r;
-    Qb[r * (kGptqB + 1) + c] = n < N ? Q[static_cast<size_t>(n) * K + j0 + c] : 0.0f;
+    const unsigned long long qi = static_cast<unsigned long long>(n) * K + j0 + c;
+    Qb[r * (kGptqB + 1) + c] =
+        n < N && in_bounds(qi, static_cast<unsigned long long>(N) * K) ? Q[qi] : 0.0f;
   }
   __syncthreads();
   const int n = n0 + t;
@@ -439,8 +443,12 @@ __global__ void gptq_pack_kernel(const uint8_t* __restrict__ codes_t,
   if (idx >= half * N) return;
   const size_t b = idx / N;
   const size_t n = idx - b * N;
-  const uint32_t lo = codes_t[static_cast<size_t>(pos[2 * b]) * N + n];
-  const uint32_t hi = codes_t[static_cast<size_t>(pos[2 * b + 1]) * N + n];
+  const int p0 = pos[2 * b], p1 = pos[2 * b + 1];
+  if (!in_bounds(static_cast<unsigned int>(p0), static_cast<unsigned int>(K)) ||
+      !in_bounds(static_cast<unsigned int>(p1), static_cast<unsigned int>(K)))
+    return;
+  const uint32_t lo = codes_t[static_cast<size_t>(p0) * N + n];
+  const uint32_t hi = codes_t[static_cast<size_t>(p1) * N + n];
   Wq[n * half + b] = static_cast<uint8_t>(lo | (hi << 4));
 }
 

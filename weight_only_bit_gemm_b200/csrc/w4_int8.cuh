@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(1024) int8_outliers_kernel(const uint16_t* __r
   __syncthreads();
   int base = incl - mine + (wid > 0 ? warp_sum[wid - 1] : 0);
   for (int k = k0; k < k1; ++k)
-    if (flag[k]) list[base++] = k;
+    if (flag[k] && in_bounds(static_cast<unsigned int>(base), static_cast<unsigned int>(K)))
+      list[base++] = k;
   if (t == 1023) *count = warp_sum[31];
 }
 
@@ -158,6 +159,7 @@ __global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(
     int d[kInt8MaxNB][4] = {};
     for (int k0 = kbeg; k0 < kend; k0 += 64) {
       const int kk = k0 + 16 * u;
+      if (!in_bounds(static_cast<unsigned int>(kk + 15), static_cast<unsigned int>(K))) continue;
       uint4 wa = make_uint4(0u, 0u, 0u, 0u), wb = make_uint4(0u, 0u, 0u, 0u);
       if (r0 < N) wa = *reinterpret_cast<const uint4*>(qw + static_cast<size_t>(r0) * K + kk);
       if (r1 < N) wb = *reinterpret_cast<const uint4*>(qw + static_cast<size_t>(r1) * K + kk);
@@ -199,7 +201,9 @@ __global__ void int8_epilogue_kernel(const int* __restrict__ acc, const float* _
   float y = __fmul_rn(__fmul_rn(static_cast<float>(acc[idx]), sx[m]), s);
   const int no = *count;
   for (int i = 0; i < no; ++i) {
+    if (!in_bounds(static_cast<unsigned int>(i), static_cast<unsigned int>(K))) break;
     const int k = list[i];
+    if (!in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(K))) continue;
     const float w16 = __bfloat162float(__float2bfloat16_rn(
         __fmul_rn(static_cast<float>(qw[static_cast<size_t>(n) * K + k]), s)));
     y = fmaf(bf16_bits_f32(X[static_cast<size_t>(m) * K + k]), w16, y);

@@ -80,6 +80,8 @@ const char* w4_status_string(w4_status s) {
     case W4_ERR_DEVICE_INPUT: return "device found invalid input data";
     case W4_ERR_SCRATCH_LIMIT:
       return "workspace needed exceeds the static scratch (W4_STATIC_SCRATCH_BYTES)";
+    case W4_ERR_BOUNDS:
+      return "bounds-checked build: a kernel index fell outside its buffer (access skipped)";
     default: return "unknown status";
   }
 }
@@ -94,10 +96,13 @@ w4_status w4_device_status(w4_stream stream) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return W4_ERR_CUDA;
   }
+  if (v & W4_DEV_ERR_BOUNDS) return W4_ERR_BOUNDS;
   if (v & W4_DEV_ERR_TIMEOUT) return W4_ERR_TIMEOUT;
   if (v & W4_DEV_ERR_INPUT) return W4_ERR_DEVICE_INPUT;
   return W4_OK;
 }
+
+int w4_checked_build(void) { return kChecked ? 1 : 0; }
 
 w4_status w4_selftest_wait_timeout(w4_stream stream) {
   wait_timeout_probe_kernel<<<1, 32, 0, as_stream(stream)>>>(kSelftestWaitCycles);
@@ -122,6 +127,27 @@ w4_status quantize_int4(const float* W, int N, int K, int G, const int32_t* g_id
   if (!int4_shape_ok(N, K, G)) return W4_ERR_INVALID_ARG;
   if (!aligned(W, 4) || !aligned(scales, 2) || (g_idx && !aligned(g_idx, 4)))
     return W4_ERR_INVALID_ARG;
+  const long long total = static_cast<long long>(N) * K;
+  if (!g_idx && total % 128 == 0 && aligned(W, 16) && aligned(Wq, 2)) {
+    // contiguous groups: the flat kernel, a persistent grid over 128-weight segments
+    const long long nseg = total / 128;
+    const long long warps = (nseg + 3) / 4;
+    const unsigned blocks = static_cast<unsigned>(
+        std::min<long long>((warps + 7) / 8, static_cast<long long>(sm_count()) * 8));
+    cudaStream_t st = as_stream(stream);
+    switch (G) {
+      case 32:
+        rtn_quantize_flat_kernel<SYM, 32><<<blocks, 256, 0, st>>>(W, nseg, Wq, scales, zeros);
+        break;
+      case 64:
+        rtn_quantize_flat_kernel<SYM, 64><<<blocks, 256, 0, st>>>(W, nseg, Wq, scales, zeros);
+        break;
+      default:
+        rtn_quantize_flat_kernel<SYM, 128><<<blocks, 256, 0, st>>>(W, nseg, Wq, scales, zeros);
+        break;
+    }
+    return launch_status(cudaGetLastError());
+  }
   const int ng = K / G;
   const size_t smem = static_cast<size_t>(ng) * 16;
   if (smem > 200 * 1024) return W4_ERR_UNSUPPORTED;
@@ -384,6 +410,24 @@ w4_status w4_dequant(const uint8_t* Wq, const uint16_t* scales, const uint8_t* z
   if (!aligned(Wq, 4) || !aligned(W_out, 16) || !aligned(scales, 2) ||
       (g_idx && !aligned(g_idx, 4)))
     return W4_ERR_INVALID_ARG;
+  if (!g_idx && aligned(Wq, 8)) {
+    // contiguous groups: 16 weights (one group) per thread over the flat array
+    const long long total16 = static_cast<long long>(N) * K / 16;
+    const unsigned blocks = static_cast<unsigned>(ceil_div(total16, 256));
+    cudaStream_t st = as_stream(stream);
+    switch (G) {
+      case 32:
+        rtn_dequant_flat_kernel<32><<<blocks, 256, 0, st>>>(Wq, scales, zeros, total16, W_out);
+        break;
+      case 64:
+        rtn_dequant_flat_kernel<64><<<blocks, 256, 0, st>>>(Wq, scales, zeros, total16, W_out);
+        break;
+      default:
+        rtn_dequant_flat_kernel<128><<<blocks, 256, 0, st>>>(Wq, scales, zeros, total16, W_out);
+        break;
+    }
+    return launch_status(cudaGetLastError());
+  }
   const long long total = static_cast<long long>(N) * (K / 8);
   rtn_dequant_kernel<<<ceil_div(total, 256), 256, 0, as_stream(stream)>>>(Wq, scales, zeros,
                                                                            g_idx, N, K, G, W_out);
@@ -463,14 +507,13 @@ w4_status blockwise_quantize(const float* W, int N, int K, int blocksize, int dq
     return W4_ERR_INVALID_ARG;
   const long long nb = static_cast<long long>(N) * K / 64;
   const int runs = ceil_div(nb, dq_group);
+  const size_t smem = (static_cast<size_t>(dq_group) + 288) * sizeof(float);
   if (mean)
     nf4_quantize_kernel<TABLE, true>
-        <<<runs, dq_group, (2 * dq_group + 1) * sizeof(float), as_stream(stream)>>>(
-            W, nb, dq_group, Wq, absmax_q, s2, mean);
+        <<<runs, 256, smem, as_stream(stream)>>>(W, nb, dq_group, Wq, absmax_q, s2, mean);
   else
-    nf4_quantize_kernel<TABLE, false><<<runs, dq_group, dq_group * sizeof(float),
-                                        as_stream(stream)>>>(W, nb, dq_group, Wq, absmax_q, s2,
-                                                             nullptr);
+    nf4_quantize_kernel<TABLE, false>
+        <<<runs, 256, smem, as_stream(stream)>>>(W, nb, dq_group, Wq, absmax_q, s2, nullptr);
   return launch_status(cudaGetLastError());
 }
 

@@ -76,7 +76,11 @@ __device__ __forceinline__ void pack_stage_words(const uint8_t* __restrict__ Wq,
       for (int e = 0; e < 2; ++e) {
         const int k = kbase + kb * 16 + 4 * u + 2 * (j & 1) + e;  // prepacked channel
         uint32_t code = 0;
-        if (r < N && k < K) code = nibble_at(row, perm ? perm[k] : k);
+        if (r < N && k < K) {
+          const int kk = perm ? perm[k] : k;
+          if (in_bounds(static_cast<unsigned int>(kk), static_cast<unsigned int>(K)))
+            code = nibble_at(row, kk);
+        }
         w |= code << (e ? 16 + 4 * j : 4 * j);
       }
     }

@@ -13,6 +13,7 @@ namespace w4 {
 enum : unsigned int {
   W4_DEV_ERR_TIMEOUT = 1u,
   W4_DEV_ERR_INPUT = 2u,
+  W4_DEV_ERR_BOUNDS = 4u,  // bounds-checked build: an access outside its buffer
 };
 
 // Per-device error word (one per loaded library image; read and cleared by
@@ -22,6 +23,26 @@ __device__ unsigned int g_dev_error;
 __device__ __forceinline__ void set_dev_error(unsigned int bits) {
   atomicOr(&g_dev_error, bits);
 }
+
+// Bounds-checked build (compiled with -DW4_CHECKED): every global access of
+// the kernels is preceded by in_bounds(index, extent), the extent being the
+// buffer's size implied by the call's arguments.  An index at or past the
+// extent records W4_DEV_ERR_BOUNDS in the error word and the access is
+// skipped (never a trap).  In the normal build the check is the constant
+// true and costs nothing.
+#ifdef W4_CHECKED
+constexpr bool kChecked = true;
+__device__ __forceinline__ bool in_bounds(unsigned long long i, unsigned long long n) {
+  if (i < n) return true;
+  set_dev_error(W4_DEV_ERR_BOUNDS);
+  return false;
+}
+#else
+constexpr bool kChecked = false;
+__device__ __forceinline__ constexpr bool in_bounds(unsigned long long, unsigned long long) {
+  return true;
+}
+#endif
 
 // ~2 s at 2 GHz: far above any legitimate wait inside one kernel.
 constexpr long long kWaitLimitCycles = 4000000000LL;

@@ -76,6 +76,8 @@ __global__ void __launch_bounds__(256) rtn_quantize_kernel(
   float* zp_s = sf_s + ng;
   const int n = blockIdx.x;
   const float* row = W + static_cast<size_t>(n) * K;
+  const unsigned long long nk = static_cast<unsigned long long>(N) * K;  // extents
+  const unsigned long long nrow0 = static_cast<unsigned long long>(n) * K;
 
   for (int g = threadIdx.x; g < ng; g += blockDim.x) {
     pos_bits[g] = 0u;
@@ -89,6 +91,7 @@ __global__ void __launch_bounds__(256) rtn_quantize_kernel(
     for (int g = warp; g < ng; g += blockDim.x >> 5) {
       float mx = 0.0f, nx = 0.0f;
       for (int k = lane; k < G; k += 32) {
+        if (!in_bounds(nrow0 + g * G + k, nk)) continue;
         const float w = row[g * G + k];
         if (w > mx) mx = w;
         if (-w > nx) nx = -w;
@@ -105,6 +108,7 @@ __global__ void __launch_bounds__(256) rtn_quantize_kernel(
     }
   } else {
     for (int k = threadIdx.x; k < K; k += blockDim.x) {
+      if (!in_bounds(nrow0 + k, nk)) continue;
       const int g = g_idx[k];
       if (g < 0 || g >= ng) {
         set_dev_error(W4_DEV_ERR_INPUT);
@@ -124,6 +128,9 @@ __global__ void __launch_bounds__(256) rtn_quantize_kernel(
     const RtnParam p = SYM ? sym_param(mx, nx) : rtn_param(mx, nx);
     sf_s[g] = p.sf;
     zp_s[g] = p.zp;
+    if (!in_bounds(static_cast<unsigned long long>(n) * ng + g,
+                   static_cast<unsigned long long>(N) * ng))
+      continue;
     scales[static_cast<size_t>(n) * ng + g] = p.s16;
     zeros[static_cast<size_t>(n) * ng + g] = static_cast<uint8_t>(p.zp);
   }
@@ -136,7 +143,7 @@ __global__ void __launch_bounds__(256) rtn_quantize_kernel(
     for (int e = 0; e < 2; ++e) {
       const int k = 2 * b + e;
       int g = g_idx ? g_idx[k] : k / G;
-      if (g < 0 || g >= ng) {
+      if (g < 0 || g >= ng || !in_bounds(nrow0 + k, nk)) {
         code[e] = 0;
         continue;
       }
@@ -146,8 +153,113 @@ __global__ void __launch_bounds__(256) rtn_quantize_kernel(
       p.lo = SYM ? 1.0f : 0.0f;
       code[e] = rtn_code(row[k], p);
     }
-    out[b] = static_cast<uint8_t>(code[0] | (code[1] << 4));
+    if (in_bounds(nrow0 / 2 + b, nk / 2)) out[b] = static_cast<uint8_t>(code[0] | (code[1] << 4));
   }
+}
+
+// rint(RN(w / s)) without a division in the common case.  With r = RN(1/s),
+// t = RN(w r) and the exact quotient Q = w / s differ by at most
+// |Q| (2^-23 + 2^-48), and so do RN(Q) and Q by |Q| 2^-24: when t lies
+// further than |t| 2^-19 from every half-integer, Q, RN(Q) and t all round to
+// the same integer (ties included, as RN(Q) cannot sit on a half-integer
+// either).  Otherwise the IEEE division decides.
+__device__ __forceinline__ float rint_quotient(float w, float s, float r) {
+  const float t = __fmul_rn(w, r);
+  const float c = rintf(t);
+  const float d = fabsf(__fsub_rn(t, c));  // exact: |t - c| <= 1/2
+  if (fabsf(__fsub_rn(d, 0.5f)) > __fmaf_rn(fabsf(t), 0x1p-19f, 0x1p-60f)) return c;
+  return rintf(__fdiv_rn(w, s));
+}
+
+// Contiguous groups (no g_idx): W is N*K/G consecutive groups of G weights in
+// row-major order (K % G == 0), so the kernel works on the flat array.  A lane
+// takes one float4 (4 consecutive weights of one group), a group spans G/4
+// lanes and a warp 128 weights (a segment); each warp loads kU segments at a
+// time so that enough loads are in flight, reduces each group's max(w, 0)
+// and max(-w, 0) with shuffles inside the group's lanes, and writes 2 bytes
+// of codes per lane plus the group's scale and zero point.
+template <bool SYM, int G>
+__global__ void __launch_bounds__(256) rtn_quantize_flat_kernel(
+    const float* __restrict__ W, long long nseg, uint8_t* __restrict__ Wq,
+    uint16_t* __restrict__ scales, uint8_t* __restrict__ zeros) {
+  constexpr int kLpg = G / 4;  // lanes per group
+  constexpr int kU = 4;
+  const int lane = threadIdx.x & 31;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const float4* src = reinterpret_cast<const float4*>(W);
+  for (long long s0 = warp * kU; s0 < nseg; s0 += nwarps * kU) {
+    float4 v[kU];
+    const unsigned long long n4 = static_cast<unsigned long long>(nseg) * 32;  // float4 extent
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      v[u] = s0 + u < nseg && in_bounds((s0 + u) * 32 + lane, n4)
+                 ? __ldcs(src + (s0 + u) * 32 + lane)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const long long seg = s0 + u;
+      if (seg >= nseg) break;  // the same for every lane of the warp
+      const float w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      // max(w, 0) and max(-w, 0) without ever producing -0
+      float mx = 0.0f, nx = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (w[e] > mx) mx = w[e];
+        if (-w[e] > nx) nx = -w[e];
+      }
+#pragma unroll
+      for (int o = 1; o < kLpg; o <<= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        nx = fmaxf(nx, __shfl_xor_sync(0xffffffffu, nx, o));
+      }
+      const RtnParam p = SYM ? sym_param(mx, nx) : rtn_param(mx, nx);
+      const float r = __frcp_rn(p.sf);
+      uint32_t codes = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float q = __fadd_rn(rint_quotient(w[e], p.sf, r), p.zp);
+        q = fminf(fmaxf(q, p.lo), 15.0f);
+        codes |= static_cast<uint32_t>(q) << (4 * e);
+      }
+      const long long flat = seg * 128 + lane * 4;
+      if (in_bounds(flat / 4, n4)) reinterpret_cast<uint16_t*>(Wq)[flat / 4] = static_cast<uint16_t>(codes);
+      if (lane % kLpg == 0 && in_bounds(flat / G, n4 * 4 / G)) {
+        scales[flat / G] = p.s16;
+        zeros[flat / G] = static_cast<uint8_t>(p.zp);
+      }
+    }
+  }
+}
+
+// Contiguous groups: 16 consecutive weights per thread (one group, as G is a
+// multiple of 16), flat over the row-major array.
+template <int G>
+__global__ void rtn_dequant_flat_kernel(const uint8_t* __restrict__ Wq,
+                                        const uint16_t* __restrict__ scales,
+                                        const uint8_t* __restrict__ zeros, long long total16,
+                                        uint16_t* __restrict__ out) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= total16) return;
+  const long long e0 = i * 16;
+  if (!in_bounds(e0 / G, static_cast<unsigned long long>(total16) * 16 / G)) return;
+  const uint2 codes = __ldcs(reinterpret_cast<const uint2*>(Wq) + i);
+  const float sf = __half2float(__ushort_as_half(scales[e0 / G]));
+  const float z = static_cast<float>(zeros[e0 / G]);
+  uint32_t res[8];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const uint32_t word = e < 8 ? codes.x : codes.y;
+    const float q = static_cast<float>((word >> (4 * (e & 7))) & 0xFu);
+    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__fsub_rn(q, z), sf)));
+    if (e & 1)
+      res[e >> 1] |= b << 16;
+    else
+      res[e >> 1] = b;
+  }
+  uint4* dst = reinterpret_cast<uint4*>(out + e0);
+  __stcs(dst, make_uint4(res[0], res[1], res[2], res[3]));
+  __stcs(dst + 1, make_uint4(res[4], res[5], res[6], res[7]));
 }
 
 // w_hat = bf16_rne(float(q - zp) * scale): 8 weights per thread.
@@ -162,6 +274,8 @@ __global__ void rtn_dequant_kernel(const uint8_t* __restrict__ Wq,
   if (idx >= per_row * N) return;
   const int n = static_cast<int>(idx / per_row);
   const int k0 = static_cast<int>(idx % per_row) * 8;
+  const unsigned long long nk = static_cast<unsigned long long>(N) * K;
+  if (!in_bounds(static_cast<unsigned long long>(n) * K + k0 + 7, nk)) return;
   const uint32_t codes = *reinterpret_cast<const uint32_t*>(Wq + static_cast<size_t>(n) * (K / 2) + k0 / 2);
   uint32_t res[4];
 #pragma unroll
@@ -169,7 +283,8 @@ __global__ void rtn_dequant_kernel(const uint8_t* __restrict__ Wq,
     const int k = k0 + e;
     const int g = g_idx ? g_idx[k] : k / G;
     float v = 0.0f;
-    if (g >= 0 && g < ng) {
+    if (g >= 0 && g < ng &&
+        in_bounds(static_cast<unsigned long long>(n) * ng + g, static_cast<unsigned long long>(N) * ng)) {
       const float sf = __half2float(__ushort_as_half(scales[static_cast<size_t>(n) * ng + g]));
       const float z = static_cast<float>(zeros[static_cast<size_t>(n) * ng + g]);
       const float q = static_cast<float>((codes >> (4 * e)) & 0xFu);
@@ -196,7 +311,8 @@ __global__ void awq_scale_weights_kernel(const float* W, const float* __restrict
   const size_t total = static_cast<size_t>(N) * K;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
-    W_out[i] = __fmul_rn(W[i], s[i % static_cast<size_t>(K)]);
+    if (in_bounds(i % static_cast<size_t>(K), static_cast<unsigned long long>(K)))
+      W_out[i] = __fmul_rn(W[i], s[i % static_cast<size_t>(K)]);
 }
 
 // ---------------------------------------------------------------- NF4
@@ -246,110 +362,156 @@ __device__ __forceinline__ float level_value(int table, int i) {
   return table == kTableFp4 ? kFp4Levels[i] : __uint_as_float(kNf4LevelBits[i]);
 }
 
-// Nearest magnitude among levels 0..7 (the lower one on a midpoint; the
-// midpoints are the fp32 averages of neighbours), sign bit only when the
-// magnitude is not zero.
-struct Fp4Mids {
-  float t[7];
-  __device__ __forceinline__ Fp4Mids() {
-#pragma unroll
-    for (int i = 0; i < 7; ++i) t[i] = __fmul_rn(__fadd_rn(kFp4Levels[i], kFp4Levels[i + 1]), 0.5f);
+// Decision thresholds of a block-wise table in shared memory, padded with
+// +inf to a power of two: NF4 the 15 midpoints t_i (code = #{i : v > t_i}),
+// FP4 the 7 magnitude midpoints (magnitude code = #{i : |v| > t_i}).
+template <int TABLE>
+struct LevelSearch {
+  static constexpr int kSteps = TABLE == kTableFp4 ? 3 : 4;  // 8 or 16 entries
+  static constexpr int kEntries = 1 << kSteps;
+  static __device__ __forceinline__ float threshold(int i) {
+    if (TABLE == kTableFp4)
+      return i < 7 ? __fmul_rn(__fadd_rn(kFp4Levels[i], kFp4Levels[i + 1]), 0.5f)
+                   : __int_as_float(0x7f800000);
+    return i < 15 ? __uint_as_float(kNf4MidBits[i]) : __int_as_float(0x7f800000);
   }
-  __device__ __forceinline__ uint32_t code(float v) const {
-    const float av = fabsf(v);
-    uint32_t mag = 0;
+  // #{i : x > t_i}, branch-free over the sorted thresholds
+  static __device__ __forceinline__ int count_below(const float* t, float x) {
+    int q = 0;
 #pragma unroll
-    for (int i = 0; i < 7; ++i) mag += (av > t[i]) ? 1u : 0u;
-    return (v < 0.0f && mag != 0u) ? (mag | 8u) : mag;
+    for (int step = kEntries / 2; step > 0; step >>= 1)
+      if (t[q + step - 1] < x) q += step;
+    return q;
+  }
+  // The code of v = w / a (a > 0, r = RN(1/a)): from t = RN(w r) when t is
+  // further than |t| 2^-20 from the thresholds around it (then t, the exact
+  // quotient and RN(w / a) lie on the same side of every threshold: they are
+  // within |w/a| 2^-23 of each other), else from the IEEE division.
+  static __device__ __forceinline__ uint32_t code(const float* t, float w, float a, float r) {
+    const float x = __fmul_rn(w, r);
+    const float ax = TABLE == kTableFp4 ? fabsf(x) : x;
+    int q = count_below(t, ax);
+    const float lo = q > 0 ? t[q - 1] : __int_as_float(0xff800000);
+    const float hi = t[q];
+    const float thr = __fmaf_rn(fabsf(x), 0x1p-20f, 0x1p-60f);
+    float v = x;
+    if (!(__fsub_rn(ax, lo) > thr && __fsub_rn(hi, ax) > thr)) {
+      v = __fdiv_rn(w, a);
+      q = count_below(t, TABLE == kTableFp4 ? fabsf(v) : v);
+    }
+    if (TABLE == kTableFp4) return (v < 0.0f && q != 0) ? (static_cast<uint32_t>(q) | 8u) : q;
+    return static_cast<uint32_t>(q);
   }
 };
 
-// One thread per 64-block, one CTA per run of dq_group blocks
-// (blockDim.x == dq_group).  Writes packed codes, absmax codes and s2.
-// TABLE selects the NF4 or the FP4 codes; everything else is shared.
-// MEAN selects the double quantization of the absmax constants:
-//   false  s2 = max(a) / 255 (1 if 0), c = clamp(rint(a / s2), 0, 255) (u8);
-//   true   mean-offset: mu = fp32(fp64 sum of the run's a in block order / n),
-//          d = a - mu, s2 = max|d| / 127 (1 if 0),
-//          c = clamp(rint(d / s2), -127, 127) (int8), mean[run] = mu.
-// Shared memory: dq_group floats (MEAN: 2 dq_group + 1).
+// One CTA (256 threads) per run of dq_group consecutive 64-weight blocks.
+// Codes: each warp takes pairs of blocks (half-warp per block, one float4 per
+// lane, kU pairs in flight); the block absmax is a 16-lane shuffle
+// reduction, the codes come from LevelSearch.  Then the run's constants:
+//   MEAN false  s2 = max(a) / 255 (1 if 0), c = clamp(rint(a / s2), 0, 255) (u8);
+//   MEAN true   mean-offset: mu = fp32(fp64 sum of the run's a in block order / n),
+//               d = a - mu, s2 = max|d| / 127 (1 if 0),
+//               c = clamp(rint(d / s2), -127, 127) (int8), mean[run] = mu.
+// TABLE selects the NF4 or the FP4 codes.  Shared memory: dq_group + 288
+// floats.
 template <int TABLE, bool MEAN>
-__global__ void nf4_quantize_kernel(const float* __restrict__ W, long long nblocks, int dq_group,
-                                    uint8_t* __restrict__ Wq, uint8_t* __restrict__ absmax_q,
-                                    float* __restrict__ s2, float* __restrict__ mean) {
-  extern __shared__ float sm_a[];
+__global__ void __launch_bounds__(256) nf4_quantize_kernel(const float* __restrict__ W,
+                                                           long long nblocks, int dq_group,
+                                                           uint8_t* __restrict__ Wq,
+                                                           uint8_t* __restrict__ absmax_q,
+                                                           float* __restrict__ s2,
+                                                           float* __restrict__ mean) {
+  using LS = LevelSearch<TABLE>;
+  constexpr int kU = 4;
+  extern __shared__ float sm_q4[];
+  float* a_s = sm_q4;                  // [dq_group] block absmax, block order
+  float* red = sm_q4 + dq_group;       // [256] reduction scratch, then [256] = mean
+  float* thr = red + 264;              // [16] decision thresholds
   const long long run0 = static_cast<long long>(blockIdx.x) * dq_group;
-  const long long b = run0 + threadIdx.x;
-  const bool valid = b < nblocks;
-  float w[64];
-  float a = 0.0f;
-  if (valid) {
-    const float4* src = reinterpret_cast<const float4*>(W + b * 64);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float4 v = src[i];
-      w[4 * i + 0] = v.x;
-      w[4 * i + 1] = v.y;
-      w[4 * i + 2] = v.z;
-      w[4 * i + 3] = v.w;
-    }
-#pragma unroll
-    for (int i = 0; i < 64; ++i) a = fmaxf(a, fabsf(w[i]));
-  }
-  float key = a;  // what the run's scale is taken from: a, or |a - mu|
-  if constexpr (MEAN) {
-    float* sm_blk = sm_a + dq_group;  // the run's constants, in block order
-    sm_blk[threadIdx.x] = a;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const long long left = nblocks - run0;
-      const int n = left < dq_group ? static_cast<int>(left) : dq_group;
-      double sum = 0.0;
-      for (int i = 0; i < n; ++i) sum += static_cast<double>(sm_blk[i]);
-      sm_blk[dq_group] = static_cast<float>(sum / static_cast<double>(n));
-    }
-    __syncthreads();
-    key = valid ? fabsf(__fsub_rn(a, sm_blk[dq_group])) : 0.0f;
-  }
-  sm_a[threadIdx.x] = key;
+  const long long left = nblocks - run0;
+  const int nrun = left < dq_group ? static_cast<int>(left) : dq_group;
+  if (threadIdx.x < LS::kEntries) thr[threadIdx.x] = LS::threshold(threadIdx.x);
   __syncthreads();
-  for (int s = 1; s < blockDim.x; s <<= 1) {
-    float other = 0.0f;
-    if ((threadIdx.x % (2 * s)) == 0 && threadIdx.x + s < blockDim.x) other = sm_a[threadIdx.x + s];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = lane >> 4, l16 = lane & 15;
+  const int npairs = (nrun + 1) / 2;
+  const float4* src = reinterpret_cast<const float4*>(W);
+  const unsigned long long n4 = static_cast<unsigned long long>(nblocks) * 16;
+  for (int p0 = warp; p0 < npairs; p0 += 8 * kU) {
+    float4 v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int b = 2 * (p0 + 8 * u) + half;
+      const unsigned long long i4 = static_cast<unsigned long long>(run0 + b) * 16 + l16;
+      v[u] = (p0 + 8 * u < npairs && b < nrun && in_bounds(i4, n4)) ? __ldcs(src + i4)
+                                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (p0 + 8 * u >= npairs) break;  // the same for the whole warp
+      const int b = 2 * (p0 + 8 * u) + half;
+      const float w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      float a = fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3])));
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      if (b >= nrun) continue;
+      if (l16 == 0) a_s[b] = a;
+      const float r = a > 0.0f ? __frcp_rn(a) : 0.0f;
+      uint32_t codes = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t c = a > 0.0f ? LS::code(thr, w[e], a, r)
+                                    : static_cast<uint32_t>(LS::count_below(thr, 0.0f));
+        codes |= c << (4 * e);
+      }
+      const unsigned long long byte = static_cast<unsigned long long>(run0 + b) * 32 + 2 * l16;
+      if (in_bounds(byte / 2, n4))
+        reinterpret_cast<uint16_t*>(Wq)[byte / 2] =
+            static_cast<uint16_t>((codes & 0xFu) | ((codes >> 4) & 0xFu) << 4 |
+                                  ((codes >> 8) & 0xFu) << 8 | ((codes >> 12) & 0xFu) << 12);
+    }
+  }
+  __syncthreads();
+
+  // the run's constants
+  float mu = 0.0f;
+  if constexpr (MEAN) {
+    if (threadIdx.x == 0) {
+      double sum = 0.0;
+      for (int i = 0; i < nrun; ++i) sum += static_cast<double>(a_s[i]);
+      red[256] = static_cast<float>(sum / static_cast<double>(nrun));
+    }
     __syncthreads();
-    if ((threadIdx.x % (2 * s)) == 0) sm_a[threadIdx.x] = fmaxf(sm_a[threadIdx.x], other);
+    mu = red[256];
+  }
+  float key = 0.0f;
+  for (int b = threadIdx.x; b < nrun; b += 256)
+    key = fmaxf(key, MEAN ? fabsf(__fsub_rn(a_s[b], mu)) : a_s[b]);
+  red[threadIdx.x] = key;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] = fmaxf(red[threadIdx.x], red[threadIdx.x + w]);
     __syncthreads();
   }
-  float sc = __fdiv_rn(sm_a[0], MEAN ? 127.0f : 255.0f);
+  float sc = __fdiv_rn(red[0], MEAN ? 127.0f : 255.0f);
   if (sc == 0.0f) sc = 1.0f;
   if (threadIdx.x == 0) {
     s2[blockIdx.x] = sc;
-    if constexpr (MEAN) mean[blockIdx.x] = sm_a[2 * dq_group];
+    if constexpr (MEAN) mean[blockIdx.x] = mu;
   }
-  if (!valid) return;
-  if constexpr (MEAN) {
-    const float d = __fsub_rn(a, sm_a[2 * dq_group]);
-    const float c = fminf(fmaxf(rintf(__fdiv_rn(d, sc)), -127.0f), 127.0f);
-    absmax_q[b] = static_cast<uint8_t>(static_cast<int8_t>(c));
-  } else {
-    const float c = fminf(fmaxf(rintf(__fdiv_rn(a, sc)), 0.0f), 255.0f);
-    absmax_q[b] = static_cast<uint8_t>(c);
-  }
-  uint32_t packed[8];
-  const Fp4Mids fp4;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float v = (a > 0.0f) ? __fdiv_rn(w[8 * i + e], a) : 0.0f;
-      word |= (TABLE == kTableFp4 ? fp4.code(v) : nf4_code(v)) << (4 * e);
+  for (int b = threadIdx.x; b < nrun; b += 256) {
+    const float a = a_s[b];
+    uint8_t byte;
+    if constexpr (MEAN) {
+      const float c = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(a, mu), sc)), -127.0f), 127.0f);
+      byte = static_cast<uint8_t>(static_cast<int8_t>(c));
+    } else {
+      byte = static_cast<uint8_t>(fminf(fmaxf(rintf(__fdiv_rn(a, sc)), 0.0f), 255.0f));
     }
-    packed[i] = word;
+    if (in_bounds(static_cast<unsigned long long>(run0 + b), static_cast<unsigned long long>(nblocks)))
+      absmax_q[run0 + b] = byte;
   }
-  uint4* dst = reinterpret_cast<uint4*>(Wq + b * 32);
-  dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-  dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
 }
 
 // The reconstructed absmax of a block from its 8-bit code byte:
@@ -379,6 +541,7 @@ __global__ void nf4_dequant_kernel(const uint8_t* __restrict__ Wq,
   const long long e0 = idx * 8;
   const long long b = e0 / 64;
   const long long run = b / dq_group;
+  if (!in_bounds(e0 + 7, static_cast<unsigned long long>(total8) * 8)) return;
   const float a = absmax_from_code<MEAN>(absmax_q[b], s2[run], MEAN ? mean[run] : 0.0f);
   const uint32_t codes = *reinterpret_cast<const uint32_t*>(Wq + e0 / 2);
   uint32_t res[4];

@@ -7,6 +7,7 @@ when the library has not been built.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import re
@@ -15,6 +16,7 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libw4b200.so")
+LIB_CHECKED_PATH = os.path.join(_PKG, "libw4b200_checked.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "w4.h")
 
 if not os.path.exists(LIB_PATH):
@@ -30,6 +32,7 @@ _sz = ctypes.c_size_t
 _SIGS = {
     "w4_status_string": (ctypes.c_char_p, [_i]),
     "w4_version": (_i, []),
+    "w4_checked_build": (_i, []),
     "w4_device_status": (_i, [_p]),
     "w4_selftest_wait_timeout": (_i, [_p]),
     "w4_weight_bytes": (ctypes.c_double, [_i, _i, _i]),
@@ -68,14 +71,47 @@ _SIGS = {
     "fp4_levels": (None, [_p]),
     "fp4_gemm": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
 }
-for _name, (_res, _args) in _SIGS.items():
-    _f = getattr(lib, _name)
-    _f.restype = _res
-    _f.argtypes = _args
+def _bind(handle):
+    for name, (res, args) in _SIGS.items():
+        f = getattr(handle, name)
+        f.restype = res
+        f.argtypes = args
+    return handle
+
+
+_bind(lib)
+_checked = None
+
+
+def checked_library():
+    """The bounds-checked build (libw4b200_checked.so), loaded on first use;
+    ImportError if it has not been built."""
+    global _checked
+    if _checked is None:
+        if not os.path.exists(LIB_CHECKED_PATH):
+            raise ImportError(f"{LIB_CHECKED_PATH} is missing: build it with "
+                              "`python -m weight_only_bit_gemm_b200.build --checked`")
+        _checked = _bind(ctypes.CDLL(LIB_CHECKED_PATH))
+    return _checked
+
+
+@contextlib.contextmanager
+def using(handle):
+    """Route every wrapper of this module through another build of the
+    library (e.g. checked_library()) inside the block."""
+    global lib
+    saved = lib
+    lib = handle
+    try:
+        yield handle
+    finally:
+        lib = saved
+
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA, W4_ERR_TIMEOUT, \
     W4_ERR_DEVICE_INPUT = range(6)
 W4_ERR_SCRATCH_LIMIT = 6
+W4_ERR_BOUNDS = 7
 W4_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
