@@ -832,6 +832,18 @@ def run_single(w4, args):
                       "TFLOP/s": flops / t / 1e9}), flush=True)
 
 
+def run_probe(name):
+    """Compile a microbenchmark for sm_100a into a temporary directory and run it."""
+    import subprocess
+    import tempfile
+    src = os.path.join(ROOT, "weight_only_bit_gemm_b200", "probes", name + ".cu")
+    with tempfile.TemporaryDirectory() as d:
+        exe = os.path.join(d, name)
+        subprocess.run([os.environ.get("NVCC", "nvcc"), "-gencode", "arch=compute_100a,code=sm_100a",
+                        "-O3", "-std=c++17", "-o", exe, src], check=True)
+        subprocess.run([exe], check=True)
+
+
 # --------------------------------------------------------------------- main
 
 def main():
@@ -842,12 +854,19 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-rows", action="store_true", help="skip the other-row measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--probe", choices=["pipes", "tcgen05_mma"],
+                    help="build and run one microbenchmark of weight_only_bit_gemm_b200/probes "
+                         "(the measurements the kernels' design rests on) and print its table")
     ap.add_argument("--single", nargs=4, metavar=("FMT", "K", "N", "M"),
                     help="profiling aid: run one layer call (FMT int4|nf4|fp4|awq|gptq|int8) warmup+steps times "
                          "eagerly and print its mean device time")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+
+    if args.probe:
+        run_probe(args.probe)
+        return
 
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -201,12 +201,17 @@ w4_status w4_gptq_hessian(const uint16_t* X, int n, int K, float* H, w4_stream s
  *     q_x = clamp(rint(x / s_x), -127, 127) outside O, 0 on O
  *     y[m,n] = (sum_k q_x q_w) s_x[m] s_w[n]             (exact int32 sum)
  *            + sum_{k in O} x[m,k] bf16(q_w[n,k] s_w[n])  (fp32)
- *     X bf16 [M, K]; qw 16-byte aligned; K % 64 == 0, K <= 65536;
- *     Y bf16 [M, N]; threshold >= 0 (the pages use 6.0);
+ *     X bf16 [M, K], 16-byte aligned; qw 16-byte aligned; K % 64 == 0,
+ *     K <= 65536; Y bf16 [M, N]; threshold >= 0 (the pages use 6.0);
  *     workspace of llm_int8_workspace_bytes(M, N, K) bytes, 256-byte aligned,
- *     contents irrelevant; the call leaves it dirty, so it must not be the
- *     workspace of w4a16_gemm / nf4_gemm (which must stay zeroed).  The INT8
- *     product uses warp-level s8 MMAs.                                      */
+ *     ZEROED ONCE before its first use: its accumulator and counters are
+ *     left zeroed by every call, the other regions are overwritten by every
+ *     call, so it must not double as the workspace of w4a16_gemm / nf4_gemm
+ *     (whose own regions must stay zeroed).  Calls that share a workspace
+ *     must be ordered on one stream.  Three launches (outlier scan, token
+ *     quantization, INT8 product with the 16-bit outlier part in its last
+ *     work item per row tile) chained by programmatic dependent launch; the
+ *     INT8 product uses warp-level s8 MMAs.                                 */
 w4_status llm_int8_quantize_weights(const float* W, int N, int K, int8_t* qw, float* sw,
                                     w4_stream stream);
 size_t llm_int8_workspace_bytes(int M, int N, int K);

@@ -8,7 +8,17 @@ propagates along its row.  Checked exactly: the Hessian's symmetry, the
 identity-Hessian case (equal to plain RTN), the first group's scales and
 zero points, the act-order map, dead channels.  Checked by property: code
 agreement with the oracle, the layer error tr((W - W_hat) H (W - W_hat)^T)
-against the oracle's and RTN's, and a GEMM on the result."""
+against the oracle's and RTN's, and a GEMM on the result.
+
+Step by step: the oracle is run again following the device's codes (its
+compensated weights then track the device's decisions), recording its own
+decision and the distance of w / s to the nearest half-integer at every
+step.  Every step where the two decide differently must be a rounding tie
+(within 1e-4 of a code unit: fp32 against fp64 arithmetic) or lie in a group
+whose fp16 scale came out one ulp apart (the scale itself at an fp16
+rounding tie); such scales must be rare and the zero points must agree
+wherever the scales do.  Measured on B200 over these cases: at most 2
+differing decisions per layer, all at ties below 2e-6 or in such groups."""
 import numpy as np
 import pytest
 import torch
@@ -76,6 +86,8 @@ GPTQ_CASES = [
     (300, 1024, 128, False, 512),
     (200, 768, 64, True, 384),
     (130, 1024, 32, True, 512),
+    (256, 2048, 32, True, 512),
+    (512, 1024, 64, False, 512),
 ]
 
 
@@ -101,14 +113,26 @@ def test_gptq_against_oracle(w4, N, K, G, act, n):
     gk = O.group_index(K, G, g)
     assert np.array_equal(q[:, 11], z[np.arange(N), gk[11]])
     agree = float(np.mean(q == qo))
-    assert agree >= 0.98, agree
+    assert agree >= 0.998, agree
+    # step by step, with the oracle following the device's decisions
+    rec = {}
+    _, sf, zf, _ = O.gptq_quantize(W, H.astype(np.float64), G, act, follow=q, record=rec)
+    scale_off = sf.view(np.uint16) != s.view(np.uint16)
+    assert np.all(np.abs(sf.view(np.uint16).astype(np.int32)[scale_off] -
+                         s.view(np.uint16).astype(np.int32)[scale_off]) == 1)
+    assert scale_off.mean() <= 2e-3, scale_off.mean()
+    assert np.array_equal(z[~scale_off], zf[~scale_off])
+    differ = rec["own"] != q
+    explained = (rec["tie"] < 1e-4) | scale_off[np.arange(N)[:, None], gk[None, :]]
+    assert not np.any(differ & ~explained), np.argwhere(differ & ~explained)[:5]
+    assert differ.sum() <= max(4, q.size // 50000), differ.sum()
     Wl = W.copy()
     Wl[:, 11] = 0.0
     l_dev = O.gptq_loss(Wl, O.dequant_rtn(O.pack_nibbles(q), s, z, G, g), H)
     l_ora = O.gptq_loss(Wl, O.dequant_rtn(O.pack_nibbles(qo), so, zo, G, go), H)
     qr, sr, zr_ = O.quantize_rtn(W, G)
     l_rtn = O.gptq_loss(Wl, O.dequant_rtn(O.pack_nibbles(qr), sr, zr_, G), H)
-    assert l_dev <= 1.02 * l_ora, (l_dev, l_ora)
+    assert l_dev <= 1.01 * l_ora, (l_dev, l_ora)
     assert l_dev < 0.5 * l_rtn, (l_dev, l_rtn)
 
 

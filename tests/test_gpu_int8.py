@@ -124,3 +124,24 @@ def test_int8_call_leaves_the_w4a16_workspace_clean(w4):
     y_ref, ab = O.matmul_ref(xb, O.dequant_rtn(Wq, s, z, G))
     ok, ratio = O.check_matmul(host_u16(y), y_ref, ab)
     assert ok, ratio
+
+
+def test_int8_calls_share_one_workspace(w4):
+    # the accumulator and row-tile counters are left zeroed by every call:
+    # calls of different shapes in turn on one workspace stay right, and the
+    # same call twice gives the same bits
+    ws = torch.zeros(w4.lib.llm_int8_workspace_bytes(16, 1000, 11008) + 256, dtype=torch.uint8,
+                     device="cuda")
+    shapes = [(16, 1000, 11008), (1, 4096, 4096), (3, 77, 320), (16, 1000, 11008)]
+    for i, (M, N, K) in enumerate(shapes * 2):
+        W = S.draw_w(N, K, 0.02, seed=i % 4, tag=64)
+        xb = S.draw_x(M, K, seed=i % 4, tag=64, N=N, outlier_frac=0.003, outlier_scale=50.0)
+        qw, sw = w4.llm_int8_quantize_weights(dev(W))
+        y1 = w4.llm_int8_gemm(x_dev(xb), qw, sw, workspace=ws)
+        y2 = w4.llm_int8_gemm(x_dev(xb), qw, sw, workspace=ws)
+        status_ok(w4)
+        assert torch.equal(y1, y2)
+        q_r, s_r = O.int8_quantize_weights(W)
+        y_ref, ab = O.int8_mixed_ref(xb, q_r, s_r)
+        ok, ratio = O.check_matmul(host_u16(y1), y_ref, ab)
+        assert ok, f"call {i}: worst error / tolerance = {ratio}"

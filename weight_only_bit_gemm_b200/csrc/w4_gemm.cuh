@@ -194,6 +194,8 @@ struct GemmArgs {
   int KS;                 // stages per tile row = ceil(K / 128)
   int tiles_n;
   int splits;
+  int tiles_m;            // token tiles
+  int group_m;            // token tiles per group of the CTA order (see the kernel)
   FastDivIdx by_dq;        // NF4: 64-block index -> s2 index (double-quant run)
   int table;              // NF4 layout: level table (kTableNf4 / kTableFp4)
   // buffer extents, read only by the bounds-checked build

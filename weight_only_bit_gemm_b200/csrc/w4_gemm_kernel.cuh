@@ -28,9 +28,19 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nt = blockIdx.x / args.splits;
-  const int split = blockIdx.x % args.splits;
-  const int mtile = blockIdx.y;
+  // CTA order: groups of group_m token tiles; inside a group the token tile
+  // runs fastest, so the CTAs that read one weight tile (and split range)
+  // run together and share it through L2, as do the weight tiles of a wave
+  // for the group's activation tiles.
+  const int ns = args.tiles_n * args.splits;
+  const int gsize = args.group_m * ns;
+  const int grp = static_cast<int>(blockIdx.x) / gsize;
+  const int gm = min(args.group_m, args.tiles_m - grp * args.group_m);
+  const int lin = static_cast<int>(blockIdx.x) - grp * gsize;
+  const int mtile = grp * args.group_m + lin % gm;
+  const int nts = lin / gm;
+  const int nt = nts / args.splits;
+  const int split = nts % args.splits;
   const int s0 = static_cast<int>(static_cast<long long>(split) * args.KS / args.splits);
   const int s1 = static_cast<int>(static_cast<long long>(split + 1) * args.KS / args.splits);
   const int nst = s1 - s0;

@@ -63,6 +63,7 @@ struct GemvArgs {
   FastDivIdx by_dq;          // NF4: 64-block index -> s2 index
   int dq_group;             // NF4: 64-blocks per second-level scale
   int table;                // NF4 layout: level table (kTableNf4 / kTableFp4)
+  int cluster;              // CTAs per thread-block cluster (1: no cluster level)
   // buffer extents, read only by the bounds-checked build
   unsigned long long wp_bytes, partial_floats, s2_count;
 };
@@ -102,7 +103,12 @@ struct GemvCfg {
   static constexpr bool kCtaReduce = NB <= 2;
   static constexpr int kV = kRG * NB * 4;  // partial floats per lane
   static constexpr int kRedBytes = kCtaReduce ? kWarps * 2 * 32 * kV * 4 : 0;
-  static constexpr int kSmemBytes = kRingBytes + kRedBytes + kWarps * 4;
+  // cluster level (with the CTA level): the row pair that ends this CTA's
+  // range, if it continues in the next CTAs of the cluster, is combined here:
+  // one partial slot per CTA of the cluster and one arrival counter
+  static constexpr int kMaxCluster = 4;
+  static constexpr int kClusterBytes = kCtaReduce ? kMaxCluster * 32 * kV * 4 : 0;
+  static constexpr int kSmemBytes = kRingBytes + kRedBytes + kClusterBytes + kWarps * 4 + 16;
 };
 
 __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t (&a)[4],
@@ -245,7 +251,41 @@ __device__ __forceinline__ uint32_t range_end(uint32_t w, const GemvArgs& a) {
 struct CtaRed {
   float4* part;            // [warp][kind][V/4][32 lanes]
   unsigned int* count;     // [warp]: arrivals for the row pair that ends its range
+  float4* cpart;           // [CTA of the cluster][V/4][32 lanes]
+  unsigned int* ccount;    // arrivals of the cluster's CTAs
 };
+
+// Distributed shared memory of the CTAs of a cluster.
+__device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_peer(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ float4 ld_peer(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned atom_add_peer(uint32_t addr) {
+  unsigned old;
+  asm volatile("atom.acq_rel.cluster.shared::cluster.add.u32 %0, [%1], 1;"
+               : "=r"(old)
+               : "r"(addr)
+               : "memory");
+  return old;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
 
 // Global level: this lane's partial `tot` in slot `slot` of row pair rpg,
 // `contrib` slots in all; returns true (with tot the full sum, added in slot
@@ -383,11 +423,59 @@ __device__ __forceinline__ void flush_row_group(const GemvArgs& args,
         done = first >= cta_w0 && last <= cta_w1;
       }
     }
+    uint32_t cs = 1;  // CTAs per global contributor
+    if constexpr (C::kCtaReduce) {
+      if (!done && args.cluster > 1) {
+        // level 2: the CTAs of one cluster that share the row pair combine in
+        // the shared memory of the first of them (the row pair ends its range)
+        cs = static_cast<uint32_t>(args.cluster);
+        const uint32_t cta = blockIdx.x;
+        const uint32_t cl0 = cta / cs * cs, cl1 = cl0 + cs - 1;
+        const uint32_t fc = first / C::kWarps, lc = last / C::kWarps;
+        const uint32_t k0 = fc > cl0 ? fc : cl0, k1 = lc < cl1 ? lc : cl1;
+        if (k1 > k0) {
+          const uint32_t owner = k0 - cl0;
+#pragma unroll
+          for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+            for (int nb = 0; nb < C::NB; ++nb)
+              st_peer(peer_addr(cr.cpart + ((cta - k0) * (C::kV / 4) + rr * C::NB + nb) * 32 + lane, owner),
+                      make_float4(tot[rr][nb][0], tot[rr][nb][1], tot[rr][nb][2], tot[rr][nb][3]));
+          __syncwarp();
+          unsigned prev = 0;
+          if (lane == 0) prev = atom_add_peer(peer_addr(cr.ccount, owner));
+          prev = __shfl_sync(0xffffffffu, prev, 0);
+          __syncwarp();
+          if (prev != k1 - k0) return;
+#pragma unroll
+          for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+            for (int nb = 0; nb < C::NB; ++nb)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) tot[rr][nb][j] = 0.0f;
+          for (uint32_t c = k0; c <= k1; ++c) {
+#pragma unroll
+            for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+              for (int nb = 0; nb < C::NB; ++nb) {
+                const float4 v = ld_peer(
+                    peer_addr(cr.cpart + ((c - k0) * (C::kV / 4) + rr * C::NB + nb) * 32 + lane, owner));
+                tot[rr][nb][0] += v.x;
+                tot[rr][nb][1] += v.y;
+                tot[rr][nb][2] += v.z;
+                tot[rr][nb][3] += v.w;
+              }
+          }
+          done = fc >= cl0 && lc <= cl1;
+        }
+      }
+    }
     if (!done) {
-      // level 2: one partial per CTA (per warp without the CTA level)
-      const uint32_t unit0 = C::kCtaReduce ? first / C::kWarps : first;
-      const uint32_t unit1 = C::kCtaReduce ? last / C::kWarps : last;
-      const uint32_t me = C::kCtaReduce ? blockIdx.x : wid;
+      // last level, through global memory: one partial per cluster (per CTA
+      // without clusters, per warp without the CTA level)
+      const uint32_t per = C::kCtaReduce ? C::kWarps * cs : 1u;
+      const uint32_t unit0 = first / per, unit1 = last / per;
+      const uint32_t me = C::kCtaReduce ? blockIdx.x / cs : wid;
       write_y = global_combine<C>(args, tot, rpg, me - unit0, unit1 - unit0 + 1, lane);
     }
   }
@@ -552,19 +640,11 @@ __device__ __forceinline__ void stage_compute(const GemvArgs& args, const StageR
   }
 }
 
+// One warp's whole share of the launch (returns when the warp is done).
 template <class C>
-__global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(const GemvArgs args) {
+__device__ __forceinline__ void decode_warp(const GemvArgs& args, const CtaRed& cr,
+                                            uint8_t* w4_gemv_smem, const float* Ts) {
   constexpr int R = C::kRG;
-  __shared__ __align__(64) float Ts[16];  // NF4 / FP4 levels
-  extern __shared__ __align__(16) uint8_t w4_gemv_smem[];
-  CtaRed cr;
-  cr.part = reinterpret_cast<float4*>(w4_gemv_smem + C::kRingBytes);
-  cr.count = reinterpret_cast<unsigned int*>(w4_gemv_smem + C::kRingBytes + C::kRedBytes);
-  if (C::FMT == kFmtNf4 && threadIdx.x < 16) Ts[threadIdx.x] = level_value(args.table, threadIdx.x);
-  if (threadIdx.x < C::kWarps) cr.count[threadIdx.x] = 0u;
-  __syncthreads();  // the only CTA-wide barrier: before any warp may leave
-  grid_dep_launch();
-
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, u = lane & 3;
   const uint32_t wid = blockIdx.x * C::kWarps + (threadIdx.x >> 5);
@@ -659,6 +739,32 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(con
       ++st;
     }
   }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(const GemvArgs args) {
+  __shared__ __align__(64) float Ts[16];  // NF4 / FP4 levels
+  extern __shared__ __align__(16) uint8_t w4_gemv_smem[];
+  CtaRed cr;
+  cr.part = reinterpret_cast<float4*>(w4_gemv_smem + C::kRingBytes);
+  cr.cpart = reinterpret_cast<float4*>(w4_gemv_smem + C::kRingBytes + C::kRedBytes);
+  cr.count = reinterpret_cast<unsigned int*>(w4_gemv_smem + C::kRingBytes + C::kRedBytes +
+                                             C::kClusterBytes);
+  cr.ccount = cr.count + C::kWarps;
+  if (C::FMT == kFmtNf4 && threadIdx.x < 16) Ts[threadIdx.x] = level_value(args.table, threadIdx.x);
+  if (threadIdx.x <= C::kWarps) cr.count[threadIdx.x] = 0u;  // and the cluster counter
+  // Every thread of every CTA meets here (counters initialised before any
+  // peer may count on them) and again at the end (no CTA leaves while its
+  // shared memory may still be read or written by the cluster's others).
+  const bool clustered = C::kCtaReduce && args.cluster > 1;
+  if (clustered)
+    cluster_sync_all();
+  else
+    __syncthreads();
+  grid_dep_launch();
+  decode_warp<C>(args, cr, w4_gemv_smem, Ts);
+  __syncwarp();
+  if (clustered) cluster_sync_all();
 }
 
 }  // namespace w4

@@ -5,15 +5,22 @@
 // (input channels whose activation exceeds the threshold, 6.0, in magnitude
 // go through a 16-bit product, the others through INT8, and the two results
 // are added); "【推理与部署篇05】模型量化部署深度对比" §6.1: llm_int8_threshold 6.0,
-// no 16-bit copy of the weights.  Per call:
-//   outliers  one CTA: flag[k] = |x[m,k]| > threshold for some token m, and
-//             the ascending list of flagged channels (block prefix sum);
-//   quantize  one CTA per token: s_x = max over unflagged |x| / 127,
-//             q_x = clamp(rint(x / s_x), +-127), 0 on flagged channels;
+// no 16-bit copy of the weights.  Per call, three launches:
+//   scan      one CTA per 256 input channels: flag[k] = |x[m,k]| > threshold
+//             for some token m; the CTA's flagged channels in ascending
+//             order in its own list region; per token the largest unflagged
+//             |x| of the CTA's channels (a partial maximum);
+//   quantize  s_x = max of the partial maxima / 127 per token, q_x =
+//             clamp(rint(x / s_x), +-127), 0 on flagged channels; the first
+//             CTA also concatenates the scan CTAs' lists into one ascending
+//             list of outlier channels;
 //   product   warp-level INT8 MMAs (m16n8k32, s32 accumulate) over
 //             (16-row tile, K slice) work items, exact int32 partial sums
-//             added atomically (exact, so the order does not matter);
-//   epilogue  y = acc s_x s_w + sum over flagged k of x * bf16(q_w s_w).
+//             added atomically (exact, so the order does not matter); the
+//             last work item of a row tile to finish (an arrival counter)
+//             runs the epilogue y = acc s_x s_w + sum over flagged k of
+//             x * bf16(q_w s_w) for the tile and zeroes its accumulators and
+//             counter again, so the workspace is left as it was found.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -54,76 +61,121 @@ __global__ void __launch_bounds__(256) int8_quantize_weights_kernel(const float*
   }
 }
 
-// Outlier channels of the call (one CTA of 1024 threads; thread t owns the
-// contiguous channel range [t c, (t + 1) c)), listed in ascending order.
-__global__ void __launch_bounds__(1024) int8_outliers_kernel(const uint16_t* __restrict__ X, int M,
-                                                             int K, float threshold,
-                                                             uint8_t* __restrict__ flag,
-                                                             int32_t* __restrict__ list,
-                                                             int32_t* __restrict__ count) {
-  __shared__ int warp_sum[32];
-  const int t = threadIdx.x;
-  const int c = (K + 1023) / 1024;
-  const int k0 = min(K, t * c), k1 = min(K, k0 + c);
-  int mine = 0;
-  for (int k = k0; k < k1; ++k) {
-    bool o = false;
+// One CTA per 256 input channels (thread = channel).
+__global__ void __launch_bounds__(256) int8_scan_kernel(const uint16_t* __restrict__ X, int M,
+                                                        int K, float threshold,
+                                                        uint8_t* __restrict__ flag,
+                                                        int32_t* __restrict__ list,
+                                                        int32_t* __restrict__ cnt,
+                                                        float* __restrict__ part) {
+  __shared__ int warp_cnt[8];
+  __shared__ float red[8][8];
+  grid_dep_launch();
+  grid_dep_wait();  // X may come from the previous kernel
+  const int c = blockIdx.x, t = threadIdx.x, lane = t & 31, wid = t >> 5;
+  const int k = c * 256 + t;
+  const bool in = k < K;
+  bool o = false;
+  if (in)
     for (int m = 0; m < M && !o; ++m)
       o = fabsf(bf16_bits_f32(X[static_cast<size_t>(m) * K + k])) > threshold;
-    flag[k] = o ? 1 : 0;
-    mine += o ? 1 : 0;
-  }
-  // exclusive prefix sum of `mine` over the block
-  const int lane = t & 31, wid = t >> 5;
-  int incl = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) warp_sum[wid] = incl;
+  if (in) flag[k] = o ? 1 : 0;
+  // the CTA's flagged channels, ascending, in its list region
+  const unsigned bal = __ballot_sync(0xffffffffu, o);
+  if (lane == 0) warp_cnt[wid] = __popc(bal);
   __syncthreads();
-  if (wid == 0) {
-    int v = warp_sum[lane];
+  int before = 0, total = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += u;
+  for (int w = 0; w < 8; ++w) {
+    before += w < wid ? warp_cnt[w] : 0;
+    total += warp_cnt[w];
+  }
+  if (o) {
+    const int pos = before + __popc(bal & ((1u << lane) - 1u));
+    if (in_bounds(static_cast<unsigned>(c * 256 + pos), static_cast<unsigned>(gridDim.x * 256)))
+      list[c * 256 + pos] = k;
+  }
+  if (t == 0) cnt[c] = total;
+  // per token, the largest unflagged |x| among the CTA's channels
+  for (int m0 = 0; m0 < M; m0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      v[j] = (in && !o && m0 + j < M) ? fabsf(bf16_bits_f32(X[static_cast<size_t>(m0 + j) * K + k]))
+                                      : 0.0f;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v[j] = fmaxf(v[j], __shfl_xor_sync(0xffffffffu, v[j], off));
     }
-    warp_sum[lane] = v;  // inclusive over warps
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) red[j][wid] = v[j];
+    }
+    __syncthreads();
+    if (t < 8 && m0 + t < M) {
+      float a = red[t][0];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) a = fmaxf(a, red[t][w]);
+      part[static_cast<size_t>(c) * M + m0 + t] = a;
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  int base = incl - mine + (wid > 0 ? warp_sum[wid - 1] : 0);
-  for (int k = k0; k < k1; ++k)
-    if (flag[k] && in_bounds(static_cast<unsigned int>(base), static_cast<unsigned int>(K)))
-      list[base++] = k;
-  if (t == 1023) *count = warp_sum[31];
 }
 
-// Per token: s_x = max over unflagged channels |x| / 127 (1 if 0); q_x.
-__global__ void __launch_bounds__(256) int8_quantize_x_kernel(const uint16_t* __restrict__ X,
-                                                              const uint8_t* __restrict__ flag,
-                                                              int K, int8_t* __restrict__ qx,
-                                                              float* __restrict__ sx) {
+// grid (M, ceil(K / 2048)), 256 threads x 8 channels: q_x of one token.
+// s_x = max over the scan CTAs' partial maxima / 127 (1 if 0).  CTA (0, 0)
+// also writes the ascending list of all outlier channels and its length.
+__global__ void __launch_bounds__(256) int8_quantize_x_kernel(
+    const uint16_t* __restrict__ X, const uint8_t* __restrict__ flag,
+    const float* __restrict__ part, const int32_t* __restrict__ list,
+    const int32_t* __restrict__ cnt, int nscan, int M, int K, int8_t* __restrict__ qx,
+    float* __restrict__ sx, int32_t* __restrict__ olist, int32_t* __restrict__ ocount) {
   __shared__ float red[256];
-  const int m = blockIdx.x;
-  const uint16_t* row = X + static_cast<size_t>(m) * K;
+  __shared__ int pre[257];
+  grid_dep_launch();
+  grid_dep_wait();
+  const int m = blockIdx.x, t = threadIdx.x;
   float a = 0.0f;
-  for (int k = threadIdx.x; k < K; k += 256)
-    if (!flag[k]) a = fmaxf(a, fabsf(bf16_bits_f32(row[k])));
-  red[threadIdx.x] = a;
+  for (int c = t; c < nscan; c += 256) a = fmaxf(a, part[static_cast<size_t>(c) * M + m]);
+  red[t] = a;
   __syncthreads();
   for (int w = 128; w > 0; w >>= 1) {
-    if (threadIdx.x < w) red[threadIdx.x] = fmaxf(red[threadIdx.x], red[threadIdx.x + w]);
+    if (t < w) red[t] = fmaxf(red[t], red[t + w]);
     __syncthreads();
   }
   float s = __fdiv_rn(red[0], 127.0f);
   if (s == 0.0f) s = 1.0f;
-  if (threadIdx.x == 0) sx[m] = s;
-  for (int k = threadIdx.x; k < K; k += 256) {
-    float q = 0.0f;
-    if (!flag[k]) q = fminf(fmaxf(rintf(__fdiv_rn(bf16_bits_f32(row[k]), s)), -127.0f), 127.0f);
-    qx[static_cast<size_t>(m) * K + k] = static_cast<int8_t>(q);
+  if (blockIdx.y == 0 && t == 0) sx[m] = s;
+  const int k0 = blockIdx.y * 2048 + t * 8;
+  if (k0 < K) {
+    const uint4 xv = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K + k0);
+    const uint2 fv = *reinterpret_cast<const uint2*>(flag + k0);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    uint32_t q[2] = {0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x = bf16_bits_f32(static_cast<uint16_t>(xw[e >> 1] >> (16 * (e & 1))));
+      const uint32_t fl = ((e < 4 ? fv.x : fv.y) >> (8 * (e & 3))) & 0xFFu;
+      const float qq = fl ? 0.0f : fminf(fmaxf(rintf(__fdiv_rn(x, s)), -127.0f), 127.0f);
+      q[e >> 2] |= (static_cast<uint32_t>(static_cast<int32_t>(qq)) & 0xFFu) << (8 * (e & 3));
+    }
+    *reinterpret_cast<uint2*>(qx + static_cast<size_t>(m) * K + k0) = make_uint2(q[0], q[1]);
+  }
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    // concatenate the scan CTAs' ascending lists (nscan <= 256)
+    const int n = t < nscan ? cnt[t] : 0;
+    pre[t + 1] = n;
+    if (t == 0) pre[0] = 0;
+    __syncthreads();
+    for (int off = 1; off < 256; off <<= 1) {
+      const int v = t + 1 - off >= 1 ? pre[t + 1 - off] : 0;
+      __syncthreads();
+      pre[t + 1] += v;
+      __syncthreads();
+    }
+    for (int i = 0; i < n; ++i)
+      if (in_bounds(static_cast<unsigned>(pre[t] + i), static_cast<unsigned>(K)))
+        olist[pre[t] + i] = list[t * 256 + i];
+    if (t == 0) *ocount = pre[256];
   }
 }
 
@@ -136,39 +188,69 @@ __device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+struct Int8Args {
+  const int8_t* qw;        // [N, K]
+  const int8_t* qx;        // [M, K]
+  const float* sx;         // [M]
+  const float* sw;         // [N]
+  const uint16_t* X;       // bf16 [M, K] (outlier channels)
+  const int32_t* olist;    // ascending outlier channels
+  const int32_t* ocount;
+  int* acc;                // [M, N] int32, zero at rest
+  unsigned int* counter;   // [row tiles], zero at rest
+  uint16_t* Y;             // bf16 [M, N]
+  int M, N, K, row_tiles, slices, steps;
+};
+
 // acc[m][n] += sum over the warp's K slice of q_x[m][k] q_w[n][k].
 // Work item = (16-row tile, slice of `steps` 64-channel steps); lane (g, u)
 // = (lane / 4, lane % 4) loads 16 consecutive bytes of weight rows g and
 // g + 8 and of token row g at channel k0 + 16u: bytes 0-3 / 4-7 feed the
 // first MMA's k-slots 4u.. / 16 + 4u.., bytes 8-15 the second MMA's.  A and
 // B use the same channel-to-slot map, so the exact sum is the plain dot
-// product.  Tokens in passes of up to kInt8MaxNB blocks of 8.
-__global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(
-    const int8_t* __restrict__ qw, const int8_t* __restrict__ qx, int M, int N, int K,
-    int row_tiles, int slices, int steps, int* __restrict__ acc) {
+// product.  Tokens in passes of up to kInt8MaxNB blocks of 8.  The last of a
+// row tile's work items to finish (counted after a release fence on the
+// tile's counter) applies the epilogue to the tile's outputs.
+__global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(const Int8Args a) {
+  grid_dep_launch();
   const int lane = threadIdx.x & 31, g = lane >> 2, u = lane & 3;
   const long long item = static_cast<long long>(blockIdx.x) * kInt8Warps + (threadIdx.x >> 5);
-  if (item >= static_cast<long long>(row_tiles) * slices) return;
-  const int rt = static_cast<int>(item % row_tiles);
-  const int sl = static_cast<int>(item / row_tiles);
+  if (item >= static_cast<long long>(a.row_tiles) * a.slices) {
+    grid_dep_wait();
+    return;
+  }
+  const int rt = static_cast<int>(item % a.row_tiles);
+  const int sl = static_cast<int>(item / a.row_tiles);
   const int r0 = rt * 16 + g, r1 = r0 + 8;
-  const int kbeg = sl * steps * 64;
-  const int kend = min(K, kbeg + steps * 64);
-  const int NB = (M + 7) / 8;
+  const int kbeg = sl * a.steps * 64;
+  const int kend = min(a.K, kbeg + a.steps * 64);
+  const int NB = (a.M + 7) / 8;
+  // the first step's weights do not depend on the previous kernels
+  uint4 wa0 = make_uint4(0u, 0u, 0u, 0u), wb0 = make_uint4(0u, 0u, 0u, 0u);
+  if (kbeg < kend && in_bounds(static_cast<unsigned int>(kbeg + 16 * u + 15),
+                               static_cast<unsigned int>(a.K))) {
+    if (r0 < a.N) wa0 = *reinterpret_cast<const uint4*>(a.qw + static_cast<size_t>(r0) * a.K + kbeg + 16 * u);
+    if (r1 < a.N) wb0 = *reinterpret_cast<const uint4*>(a.qw + static_cast<size_t>(r1) * a.K + kbeg + 16 * u);
+  }
+  grid_dep_wait();  // q_x, s_x and the outlier list come from the previous kernels
   for (int tb0 = 0; tb0 < NB; tb0 += kInt8MaxNB) {
     int d[kInt8MaxNB][4] = {};
     for (int k0 = kbeg; k0 < kend; k0 += 64) {
       const int kk = k0 + 16 * u;
-      if (!in_bounds(static_cast<unsigned int>(kk + 15), static_cast<unsigned int>(K))) continue;
-      uint4 wa = make_uint4(0u, 0u, 0u, 0u), wb = make_uint4(0u, 0u, 0u, 0u);
-      if (r0 < N) wa = *reinterpret_cast<const uint4*>(qw + static_cast<size_t>(r0) * K + kk);
-      if (r1 < N) wb = *reinterpret_cast<const uint4*>(qw + static_cast<size_t>(r1) * K + kk);
+      if (!in_bounds(static_cast<unsigned int>(kk + 15), static_cast<unsigned int>(a.K))) continue;
+      uint4 wa = wa0, wb = wb0;
+      if (k0 != kbeg || tb0 != 0) {
+        wa = make_uint4(0u, 0u, 0u, 0u);
+        wb = make_uint4(0u, 0u, 0u, 0u);
+        if (r0 < a.N) wa = *reinterpret_cast<const uint4*>(a.qw + static_cast<size_t>(r0) * a.K + kk);
+        if (r1 < a.N) wb = *reinterpret_cast<const uint4*>(a.qw + static_cast<size_t>(r1) * a.K + kk);
+      }
 #pragma unroll
       for (int j = 0; j < kInt8MaxNB; ++j) {
         const int tok = (tb0 + j) * 8 + g;
         if (tb0 + j >= NB) break;
         uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-        if (tok < M) xv = *reinterpret_cast<const uint4*>(qx + static_cast<size_t>(tok) * K + kk);
+        if (tok < a.M) xv = *reinterpret_cast<const uint4*>(a.qx + static_cast<size_t>(tok) * a.K + kk);
         mma_s8_16832(d[j], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
         mma_s8_16832(d[j], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
       }
@@ -178,37 +260,39 @@ __global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(
       if (tb0 + j >= NB) break;
       const int t0 = (tb0 + j) * 8 + 2 * u;
       // d0, d1: row r0, tokens t0, t0 + 1; d2, d3: row r1
-      if (r0 < N && t0 < M) atomicAdd(&acc[static_cast<size_t>(t0) * N + r0], d[j][0]);
-      if (r0 < N && t0 + 1 < M) atomicAdd(&acc[static_cast<size_t>(t0 + 1) * N + r0], d[j][1]);
-      if (r1 < N && t0 < M) atomicAdd(&acc[static_cast<size_t>(t0) * N + r1], d[j][2]);
-      if (r1 < N && t0 + 1 < M) atomicAdd(&acc[static_cast<size_t>(t0 + 1) * N + r1], d[j][3]);
+      if (r0 < a.N && t0 < a.M) atomicAdd(&a.acc[static_cast<size_t>(t0) * a.N + r0], d[j][0]);
+      if (r0 < a.N && t0 + 1 < a.M) atomicAdd(&a.acc[static_cast<size_t>(t0 + 1) * a.N + r0], d[j][1]);
+      if (r1 < a.N && t0 < a.M) atomicAdd(&a.acc[static_cast<size_t>(t0) * a.N + r1], d[j][2]);
+      if (r1 < a.N && t0 + 1 < a.M) atomicAdd(&a.acc[static_cast<size_t>(t0 + 1) * a.N + r1], d[j][3]);
     }
   }
-}
-
-// y[m][n] = acc s_x s_w + sum over listed outlier channels x * bf16(q_w s_w).
-__global__ void int8_epilogue_kernel(const int* __restrict__ acc, const float* __restrict__ sx,
-                                     const float* __restrict__ sw, const uint16_t* __restrict__ X,
-                                     const int8_t* __restrict__ qw,
-                                     const int32_t* __restrict__ list,
-                                     const int32_t* __restrict__ count, int M, int N, int K,
-                                     uint16_t* __restrict__ Y) {
-  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<size_t>(M) * N) return;
-  const int m = static_cast<int>(idx / N);
-  const int n = static_cast<int>(idx - static_cast<size_t>(m) * N);
-  const float s = sw[n];
-  float y = __fmul_rn(__fmul_rn(static_cast<float>(acc[idx]), sx[m]), s);
-  const int no = *count;
-  for (int i = 0; i < no; ++i) {
-    if (!in_bounds(static_cast<unsigned int>(i), static_cast<unsigned int>(K))) break;
-    const int k = list[i];
-    if (!in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(K))) continue;
-    const float w16 = __bfloat162float(__float2bfloat16_rn(
-        __fmul_rn(static_cast<float>(qw[static_cast<size_t>(n) * K + k]), s)));
-    y = fmaf(bf16_bits_f32(X[static_cast<size_t>(m) * K + k]), w16, y);
+  // arrival on the row tile's counter; the last item runs the epilogue
+  __syncwarp();
+  unsigned prev = 0;
+  if (lane == 0 && in_bounds(static_cast<unsigned int>(rt), static_cast<unsigned int>(a.row_tiles)))
+    prev = atom_add_acq_rel_gpu(a.counter + rt, 1u);
+  prev = __shfl_sync(0xffffffffu, prev, 0);
+  __syncwarp();
+  if (prev != static_cast<unsigned>(a.slices - 1)) return;
+  // y[m][n] = acc s_x s_w + sum over outlier channels (ascending) of x * bf16(q_w s_w)
+  const int no = min(*a.ocount, a.K);
+  for (int idx = lane; idx < 16 * a.M; idx += 32) {
+    const int m = idx >> 4, n = rt * 16 + (idx & 15);
+    if (n >= a.N) continue;
+    const size_t o = static_cast<size_t>(m) * a.N + n;
+    const float s = a.sw[n];
+    float y = __fmul_rn(__fmul_rn(static_cast<float>(__ldcg(a.acc + o)), a.sx[m]), s);
+    for (int i = 0; i < no; ++i) {
+      const int k = a.olist[i];
+      if (!in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K))) continue;
+      const float w16 = __bfloat162float(__float2bfloat16_rn(
+          __fmul_rn(static_cast<float>(a.qw[static_cast<size_t>(n) * a.K + k]), s)));
+      y = fmaf(bf16_bits_f32(a.X[static_cast<size_t>(m) * a.K + k]), w16, y);
+    }
+    a.Y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+    a.acc[o] = 0;  // leave the accumulator zeroed for the next call
   }
-  Y[idx] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+  if (lane == 0) a.counter[rt] = 0u;
 }
 
 }  // namespace w4

@@ -322,20 +322,29 @@ w4_status w4_gptq_quantize(const float* W, const float* H, int N, int K, int G, 
 // LLM.int8: workspace regions (each 256-byte aligned).
 namespace {
 
+// Regions of the LLM.int8 workspace (each 256-byte aligned).  The
+// accumulator and the row-tile counters are zero at rest (every call leaves
+// them zeroed); the rest is rewritten by every call.
 struct Int8Layout {
-  size_t flag, list, count, qx, sx, acc, total;
+  size_t counter, acc, flag, list, cnt, part, olist, ocount, qx, sx, total;
+  int nscan;  // scan CTAs (256 channels each)
 };
 
 Int8Layout int8_layout(int M, int N, int K) {
   auto r = [](size_t v) { return (v + 255) / 256 * 256; };
   Int8Layout l{};
+  l.nscan = (K + 255) / 256;
   size_t o = 0;
-  l.flag = o;  o += r(static_cast<size_t>(K));
-  l.list = o;  o += r(static_cast<size_t>(K) * 4);
-  l.count = o; o += 256;
-  l.qx = o;    o += r(static_cast<size_t>(M) * K);
-  l.sx = o;    o += r(static_cast<size_t>(M) * 4);
-  l.acc = o;   o += r(static_cast<size_t>(M) * N * 4);
+  l.counter = o; o += r(static_cast<size_t>((N + 15) / 16) * 4);
+  l.acc = o;     o += r(static_cast<size_t>(M) * N * 4);
+  l.flag = o;    o += r(static_cast<size_t>(K));
+  l.list = o;    o += r(static_cast<size_t>(l.nscan) * 256 * 4);
+  l.cnt = o;     o += r(static_cast<size_t>(l.nscan) * 4);
+  l.part = o;    o += r(static_cast<size_t>(l.nscan) * M * 4);
+  l.olist = o;   o += r(static_cast<size_t>(K) * 4);
+  l.ocount = o;  o += 256;
+  l.qx = o;      o += r(static_cast<size_t>(M) * K);
+  l.sx = o;      o += r(static_cast<size_t>(M) * 4);
   l.total = o;
   return l;
 }
@@ -367,7 +376,7 @@ w4_status llm_int8_gemm(const uint16_t* X, const int8_t* qw, const float* sw, in
                         w4_stream stream) {
   if (!X || !qw || !sw || !Y || !workspace) return W4_ERR_INVALID_ARG;
   if (!int8_shape_ok(M, N, K) || !(threshold >= 0.0f)) return W4_ERR_INVALID_ARG;
-  if (!aligned(X, 2) || !aligned(qw, 16) || !aligned(sw, 4) || !aligned(Y, 2) ||
+  if (!aligned(X, 16) || !aligned(qw, 16) || !aligned(sw, 4) || !aligned(Y, 2) ||
       !aligned(workspace, 256))
     return W4_ERR_INVALID_ARG;
   const Int8Layout l = int8_layout(M, N, K);
@@ -376,30 +385,56 @@ w4_status llm_int8_gemm(const uint16_t* X, const int8_t* qw, const float* sw, in
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* flag = ws + l.flag;
   int32_t* list = reinterpret_cast<int32_t*>(ws + l.list);
-  int32_t* count = reinterpret_cast<int32_t*>(ws + l.count);
-  int8_t* qx = reinterpret_cast<int8_t*>(ws + l.qx);
-  float* sx = reinterpret_cast<float*>(ws + l.sx);
-  int* acc = reinterpret_cast<int*>(ws + l.acc);
-  int8_outliers_kernel<<<1, 1024, 0, st>>>(X, M, K, threshold, flag, list, count);
-  int8_quantize_x_kernel<<<M, 256, 0, st>>>(X, flag, K, qx, sx);
-  if (cudaMemsetAsync(acc, 0, static_cast<size_t>(M) * N * 4, st) != cudaSuccess) {
-    cudaGetLastError();
-    return W4_ERR_CUDA;
-  }
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + l.cnt);
+  float* part = reinterpret_cast<float*>(ws + l.part);
+  Int8Args a{};
+  a.qw = qw;
+  a.qx = reinterpret_cast<int8_t*>(ws + l.qx);
+  a.sx = reinterpret_cast<float*>(ws + l.sx);
+  a.sw = sw;
+  a.X = X;
+  a.olist = reinterpret_cast<int32_t*>(ws + l.olist);
+  a.ocount = reinterpret_cast<int32_t*>(ws + l.ocount);
+  a.acc = reinterpret_cast<int*>(ws + l.acc);
+  a.counter = reinterpret_cast<unsigned int*>(ws + l.counter);
+  a.Y = Y;
+  a.M = M;
+  a.N = N;
+  a.K = K;
   // work items: (16-row tile, K slice), about 24 warps per SM
-  const int row_tiles = ceil_div(N, 16);
+  a.row_tiles = ceil_div(N, 16);
   const int steps_total = K / 64;
   const int target = sm_count() * 24;
-  int slices = std::min(steps_total, std::max(1, ceil_div(target, row_tiles)));
-  const int steps = ceil_div(steps_total, slices);
-  slices = ceil_div(steps_total, steps);
-  const long long items = static_cast<long long>(row_tiles) * slices;
-  int8_product_kernel<<<static_cast<unsigned>((items + kInt8Warps - 1) / kInt8Warps),
-                        kInt8Warps * 32, 0, st>>>(qw, qx, M, N, K, row_tiles, slices, steps, acc);
-  const size_t outs = static_cast<size_t>(M) * N;
-  int8_epilogue_kernel<<<static_cast<unsigned>((outs + 255) / 256), 256, 0, st>>>(
-      acc, sx, sw, X, qw, list, count, M, N, K, Y);
-  return launch_status(cudaGetLastError());
+  a.slices = std::min(steps_total, std::max(1, ceil_div(target, a.row_tiles)));
+  a.steps = ceil_div(steps_total, a.slices);
+  a.slices = ceil_div(steps_total, a.steps);
+  const long long items = static_cast<long long>(a.row_tiles) * a.slices;
+  // three launches chained by programmatic dependent launch
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(l.nscan);
+  cfg.blockDim = dim3(256);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, int8_scan_kernel, X, M, K, threshold, flag, list, cnt,
+                                     part);
+  if (e == cudaSuccess) {
+    cfg.gridDim = dim3(M, ceil_div(K, 2048));
+    e = cudaLaunchKernelEx(&cfg, int8_quantize_x_kernel, X, static_cast<const uint8_t*>(flag),
+                           static_cast<const float*>(part), static_cast<const int32_t*>(list),
+                           static_cast<const int32_t*>(cnt), l.nscan, M, K,
+                           const_cast<int8_t*>(a.qx), const_cast<float*>(a.sx),
+                           const_cast<int32_t*>(a.olist), const_cast<int32_t*>(a.ocount));
+  }
+  if (e == cudaSuccess) {
+    cfg.gridDim = dim3(static_cast<unsigned>((items + kInt8Warps - 1) / kInt8Warps));
+    cfg.blockDim = dim3(kInt8Warps * 32);
+    e = cudaLaunchKernelEx(&cfg, int8_product_kernel, a);
+  }
+  return launch_status(e);
 }
 
 w4_status w4_dequant(const uint8_t* Wq, const uint16_t* scales, const uint8_t* zeros,

@@ -317,8 +317,8 @@ class Workspace:
 
 
 _WS = Workspace()
-# scratch whose contents the library does not keep zeroed (LLM.int8): never
-# the zero-kept workspace of the W4A16 / NF4 GEMMs
+# LLM.int8's workspace: its own layout (zero-kept accumulator and counters,
+# regions that every call overwrites), so never the W4A16 / NF4 workspace
 _WS_SCRATCH = Workspace()
 
 
