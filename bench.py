@@ -638,6 +638,20 @@ def measure_rows(w4, peaks):
         "frac_of_hbm": sum(i8_bytes) / tg / 1e6 / hbm,
         "eager_TB/s": sum(i8_bytes) / sum(ts) / 1e9}
 
+    # NEXT row: LLM.int8 at prefill sizes (the tensor-core kind::i8 product)
+    pre = {}
+    for (K, N) in [(4096, 12288), (11008, 4096)]:
+        W = torch.from_numpy(S.layer_w(WL, K, N)).cuda()
+        qw, sw = w4.llm_int8_quantize_weights(W)
+        del W
+        for M in (256, 2048):
+            X = bf16_dev(S.layer_x(WL, M, K, N))
+            t = time_graph([lambda X=X, qw=qw, sw=sw: w4.llm_int8_gemm(X, qw, sw)])
+            pre[f"K{K}_N{N}_M{M}"] = {"us": t * 1e3, "TOPS": 2.0 * M * N * K / t / 1e9}
+            del X
+        del qw, sw
+    rows["llm_int8_prefill"] = {"timing": "CUDA graph of one call (3 launches)", "per_shape": pre}
+
     # NEXT row: GPTQ at quantization time (13B MLP up-projection, act-order, G = 32,
     # 512 calibration tokens): Hessian, then the compensated quantization
     K, N, G, ncal = 5120, 13824, ao["G"], 512

@@ -204,11 +204,10 @@ w4_status w4_gptq_hessian(const uint16_t* X, int n, int K, float* H, w4_stream s
  *     X bf16 [M, K], 16-byte aligned; qw 16-byte aligned; K % 64 == 0,
  *     K <= 65536; Y bf16 [M, N]; threshold >= 0 (the pages use 6.0);
  *     workspace of llm_int8_workspace_bytes(M, N, K) bytes, 256-byte aligned,
- *     ZEROED ONCE before its first use: its accumulator and counters are
- *     left zeroed by every call, the other regions are overwritten by every
- *     call, so it must not double as the workspace of w4a16_gemm / nf4_gemm
- *     (whose own regions must stay zeroed).  Calls that share a workspace
- *     must be ordered on one stream.  Three launches (outlier scan, token
+ *     contents irrelevant (the call clears what it needs cleared); the call
+ *     leaves it dirty, so it must not be the workspace of w4a16_gemm /
+ *     nf4_gemm (which must stay zeroed).  Calls that share a workspace must
+ *     be ordered on one stream.  Three launches (outlier scan, token
  *     quantization, INT8 product with the 16-bit outlier part in its last
  *     work item per row tile) chained by programmatic dependent launch; the
  *     INT8 product uses warp-level s8 MMAs.                                 */

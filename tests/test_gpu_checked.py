@@ -106,7 +106,8 @@ def test_checked_blockwise_path(libs, M, N, K):
     _same(*_both(w4, chk, lambda: w4.nf4_gemm_meandq(X, wp, m, s2, N, K)))
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 100, 256), (16, 300, 1024), (40, 64, 512)])
+@pytest.mark.parametrize("M,N,K", [(1, 100, 256), (16, 300, 1024), (40, 64, 512),
+                                   (130, 300, 1088)])
 def test_checked_llm_int8(libs, M, N, K):
     w4, chk = libs
     W = torch.from_numpy(S.draw_w(N, K, 0.02, seed=M, tag=63)).cuda()

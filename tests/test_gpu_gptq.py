@@ -13,12 +13,17 @@ against the oracle's and RTN's, and a GEMM on the result.
 Step by step: the oracle is run again following the device's codes (its
 compensated weights then track the device's decisions), recording its own
 decision and the distance of w / s to the nearest half-integer at every
-step.  Every step where the two decide differently must be a rounding tie
-(within 1e-4 of a code unit: fp32 against fp64 arithmetic) or lie in a group
-whose fp16 scale came out one ulp apart (the scale itself at an fp16
-rounding tie); such scales must be rare and the zero points must agree
-wherever the scales do.  Measured on B200 over these cases: at most 2
-differing decisions per layer, all at ties below 2e-6 or in such groups."""
+step.  Every step where the two decide differently must be near a rounding
+tie (within 1e-2 of a code unit: the device compensates in fp32, the oracle
+in fp64, and with fewer calibration tokens than channels the damped Hessian
+is ill-conditioned enough for the fp32 weights to drift by a few 1e-3 of a
+step) or lie in a group whose fp16 scale came out one ulp apart (the scale
+itself at an fp16 rounding tie); such events must be rare, and the zero
+points must agree wherever the scales do.  A wrong group or column would
+instead give many differences at distances spread over the whole [0, 1/2].
+Measured on B200 over these cases: at most 2 differing decisions per layer,
+at tie distances up to 5.6e-3 (act-order, 512 tokens for 2048 channels) and
+below 2e-6 elsewhere."""
 import numpy as np
 import pytest
 import torch
@@ -123,7 +128,7 @@ def test_gptq_against_oracle(w4, N, K, G, act, n):
     assert scale_off.mean() <= 2e-3, scale_off.mean()
     assert np.array_equal(z[~scale_off], zf[~scale_off])
     differ = rec["own"] != q
-    explained = (rec["tie"] < 1e-4) | scale_off[np.arange(N)[:, None], gk[None, :]]
+    explained = (rec["tie"] < 1e-2) | scale_off[np.arange(N)[:, None], gk[None, :]]
     assert not np.any(differ & ~explained), np.argwhere(differ & ~explained)[:5]
     assert differ.sum() <= max(4, q.size // 50000), differ.sum()
     Wl = W.copy()

@@ -59,7 +59,10 @@ INT8_CASES = [
     (1, 4096, 4096, 6.0, 0.001),       # Llama-7B decode inputs: 0.1% of channels x50
     (4, 1000, 2048, 6.0, 0.001),       # ragged N
     (16, 512, 11008, 6.0, 0.001),
-    (40, 256, 1024, 6.0, 0.01),        # more than 32 tokens: two passes over the weights
+    (40, 256, 1024, 6.0, 0.01),        # more than 32 tokens: the tensor-core (kind::i8) product
+    (64, 4096, 4096, 6.0, 0.001),      # prefill-sized LLM.int8, split K
+    (256, 512, 2048, 6.0, 0.001),
+    (300, 200, 1088, 6.0, 0.002),      # ragged token tile and rows, K = 8.5 stages
     (7, 33, 64, 6.0, 0.05),            # tiny, ragged
     (5, 300, 512, 1e30, 0.0),          # no outliers
     (3, 128, 256, 0.0, 0.0),           # every nonzero channel an outlier
@@ -79,12 +82,13 @@ def test_int8_gemm_tolerance(w4, M, N, K, thr, frac):
     assert ok, f"worst error / tolerance = {ratio}"
 
 
-def test_int8_gemm_exact_on_exact_inputs(w4):
+@pytest.mark.parametrize("M,N,K", [(3, 48, 128), (64, 256, 1024), (256, 130, 512)])
+def test_int8_gemm_exact_on_exact_inputs(w4, M, N, K):
     # weights k/32 with a row maximum of 127/32 and activations k/64 with a
     # token maximum of 127/64 (plus one outlier channel of 8): every scale is
-    # a power of two, every code exact, every sum exact in fp32
+    # a power of two, every code exact, every sum exact in fp32 (warp-level
+    # and, above 32 tokens, tensor-core INT8 products)
     rng = np.random.default_rng(7)
-    M, N, K = 3, 48, 128
     W = rng.integers(-127, 128, (N, K)).astype(np.float32) / 32
     W[:, 0] = 127.0 / 32
     x = rng.integers(-127, 128, (M, K)).astype(np.float32) / 64
@@ -127,11 +131,12 @@ def test_int8_call_leaves_the_w4a16_workspace_clean(w4):
 
 
 def test_int8_calls_share_one_workspace(w4):
-    # the accumulator and row-tile counters are left zeroed by every call:
-    # calls of different shapes in turn on one workspace stay right, and the
-    # same call twice gives the same bits
-    ws = torch.zeros(w4.lib.llm_int8_workspace_bytes(16, 1000, 11008) + 256, dtype=torch.uint8,
-                     device="cuda")
+    # the workspace's regions move with the shape, so each call clears the
+    # counters and the accumulator it uses: calls of different shapes in turn
+    # on one (initially garbage) workspace stay right, and the same call
+    # twice gives the same bits
+    ws = torch.randint(0, 255, (w4.lib.llm_int8_workspace_bytes(16, 1000, 11008) + 256,),
+                       dtype=torch.uint8, device="cuda")
     shapes = [(16, 1000, 11008), (1, 4096, 4096), (3, 77, 320), (16, 1000, 11008)]
     for i, (M, N, K) in enumerate(shapes * 2):
         W = S.draw_w(N, K, 0.02, seed=i % 4, tag=64)

@@ -308,14 +308,17 @@ __device__ __forceinline__ bool global_combine(const GemvArgs& args,
     for (int nb = 0; nb < C::NB; ++nb)
       *reinterpret_cast<float4*>(dst + (rr * C::NB + nb) * 4) =
           make_float4(tot[rr][nb][0], tot[rr][nb][1], tot[rr][nb][2], tot[rr][nb][3]);
+  // every lane's partial visible device-wide before the arrival; the last
+  // arrival's lanes fence again before reading the others' partials (the
+  // shuffle carries lane 0's acquire to them only as a value)
+  __threadfence();
   __syncwarp();
   unsigned prev = 0;
   if (lane == 0) prev = atom_add_acq_rel_gpu(args.counter + rpg, 1u);
   prev = __shfl_sync(0xffffffffu, prev, 0);
-  // the shuffle carries lane 0's acquire to the other lanes as a value
-  // only; the warp barrier orders their partial loads after it
   __syncwarp();
   if (prev != contrib - 1) return false;
+  __threadfence();
 #pragma unroll
   for (int rr = 0; rr < R; ++rr)
 #pragma unroll
@@ -441,12 +444,14 @@ __device__ __forceinline__ void flush_row_group(const GemvArgs& args,
             for (int nb = 0; nb < C::NB; ++nb)
               st_peer(peer_addr(cr.cpart + ((cta - k0) * (C::kV / 4) + rr * C::NB + nb) * 32 + lane, owner),
                       make_float4(tot[rr][nb][0], tot[rr][nb][1], tot[rr][nb][2], tot[rr][nb][3]));
+          asm volatile("fence.acq_rel.cluster;" ::: "memory");  // every lane's slot
           __syncwarp();
           unsigned prev = 0;
           if (lane == 0) prev = atom_add_peer(peer_addr(cr.ccount, owner));
           prev = __shfl_sync(0xffffffffu, prev, 0);
           __syncwarp();
           if (prev != k1 - k0) return;
+          asm volatile("fence.acq_rel.cluster;" ::: "memory");
 #pragma unroll
           for (int rr = 0; rr < R; ++rr)
 #pragma unroll

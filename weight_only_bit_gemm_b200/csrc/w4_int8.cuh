@@ -19,8 +19,9 @@
 //             added atomically (exact, so the order does not matter); the
 //             last work item of a row tile to finish (an arrival counter)
 //             runs the epilogue y = acc s_x s_w + sum over flagged k of
-//             x * bf16(q_w s_w) for the tile and zeroes its accumulators and
-//             counter again, so the workspace is left as it was found.
+//             x * bf16(q_w s_w) for the tile.
+// The scan clears the row-tile counters and the quantization clears the
+// accumulator, so the workspace's contents before the call do not matter.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -67,12 +68,15 @@ __global__ void __launch_bounds__(256) int8_scan_kernel(const uint16_t* __restri
                                                         uint8_t* __restrict__ flag,
                                                         int32_t* __restrict__ list,
                                                         int32_t* __restrict__ cnt,
-                                                        float* __restrict__ part) {
+                                                        float* __restrict__ part,
+                                                        unsigned int* __restrict__ counter,
+                                                        int row_tiles) {
   __shared__ int warp_cnt[8];
   __shared__ float red[8][8];
   grid_dep_launch();
   grid_dep_wait();  // X may come from the previous kernel
   const int c = blockIdx.x, t = threadIdx.x, lane = t & 31, wid = t >> 5;
+  for (int i = c * 256 + t; i < row_tiles; i += gridDim.x * 256) counter[i] = 0u;
   const int k = c * 256 + t;
   const bool in = k < K;
   bool o = false;
@@ -128,12 +132,15 @@ __global__ void __launch_bounds__(256) int8_quantize_x_kernel(
     const uint16_t* __restrict__ X, const uint8_t* __restrict__ flag,
     const float* __restrict__ part, const int32_t* __restrict__ list,
     const int32_t* __restrict__ cnt, int nscan, int M, int K, int8_t* __restrict__ qx,
-    float* __restrict__ sx, int32_t* __restrict__ olist, int32_t* __restrict__ ocount) {
+    float* __restrict__ sx, int32_t* __restrict__ olist, int32_t* __restrict__ ocount,
+    int* __restrict__ acc, int N) {
   __shared__ float red[256];
   __shared__ int pre[257];
   grid_dep_launch();
   grid_dep_wait();
   const int m = blockIdx.x, t = threadIdx.x;
+  // this token's row of the INT8 accumulator starts at zero
+  for (int n = blockIdx.y * 256 + t; n < N; n += gridDim.y * 256) acc[static_cast<size_t>(m) * N + n] = 0;
   float a = 0.0f;
   for (int c = t; c < nscan; c += 256) a = fmaxf(a, part[static_cast<size_t>(c) * M + m]);
   red[t] = a;
@@ -188,7 +195,7 @@ __device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-struct Int8Args {
+struct Int8Args {  // (acc and counter are cleared by the call's first two kernels)
   const int8_t* qw;        // [N, K]
   const int8_t* qx;        // [M, K]
   const float* sx;         // [M]
@@ -196,8 +203,8 @@ struct Int8Args {
   const uint16_t* X;       // bf16 [M, K] (outlier channels)
   const int32_t* olist;    // ascending outlier channels
   const int32_t* ocount;
-  int* acc;                // [M, N] int32, zero at rest
-  unsigned int* counter;   // [row tiles], zero at rest
+  int* acc;                // [M, N] int32
+  unsigned int* counter;   // [row tiles]
   uint16_t* Y;             // bf16 [M, N]
   int M, N, K, row_tiles, slices, steps;
 };
@@ -266,7 +273,11 @@ __global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(const Int
       if (r1 < a.N && t0 + 1 < a.M) atomicAdd(&a.acc[static_cast<size_t>(t0 + 1) * a.N + r1], d[j][3]);
     }
   }
-  // arrival on the row tile's counter; the last item runs the epilogue
+  // arrival on the row tile's counter; the last item runs the epilogue.
+  // Every lane's atomics are made visible device-wide before the arrival
+  // (a fence by each lane, not only by the lane that counts), and every lane
+  // of the last item fences again before it reads the sums.
+  __threadfence();
   __syncwarp();
   unsigned prev = 0;
   if (lane == 0 && in_bounds(static_cast<unsigned int>(rt), static_cast<unsigned int>(a.row_tiles)))
@@ -274,6 +285,7 @@ __global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(const Int
   prev = __shfl_sync(0xffffffffu, prev, 0);
   __syncwarp();
   if (prev != static_cast<unsigned>(a.slices - 1)) return;
+  __threadfence();
   // y[m][n] = acc s_x s_w + sum over outlier channels (ascending) of x * bf16(q_w s_w)
   const int no = min(*a.ocount, a.K);
   for (int idx = lane; idx < 16 * a.M; idx += 32) {
@@ -290,9 +302,7 @@ __global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(const Int
       y = fmaf(bf16_bits_f32(a.X[static_cast<size_t>(m) * a.K + k]), w16, y);
     }
     a.Y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-    a.acc[o] = 0;  // leave the accumulator zeroed for the next call
   }
-  if (lane == 0) a.counter[rt] = 0u;
 }
 
 }  // namespace w4

@@ -15,6 +15,7 @@
 #include "w4_gemv_kernel.cuh"
 #include "w4_gptq.cuh"
 #include "w4_int8.cuh"
+#include "w4_int8_tc.cuh"
 #include "w4_prepack.cuh"
 #include "w4_quant.cuh"
 #include "w4_ptx.cuh"
@@ -322,21 +323,50 @@ w4_status w4_gptq_quantize(const float* W, const float* H, int N, int K, int G, 
 // LLM.int8: workspace regions (each 256-byte aligned).
 namespace {
 
-// Regions of the LLM.int8 workspace (each 256-byte aligned).  The
-// accumulator and the row-tile counters are zero at rest (every call leaves
-// them zeroed); the rest is rewritten by every call.
+// Regions of the LLM.int8 workspace (each 256-byte aligned), all written by
+// the call before they are read (the counters and the accumulator cleared by
+// its first two kernels).
+// More than this many tokens: the tensor-core (kind::i8) product.
+constexpr int kInt8TcMinM = 33;
+
+// The tensor-core product's tiling and split-K plan.
+struct I8Plan {
+  int MT, tiles_n, tiles_m, KS, splits;
+};
+
+I8Plan int8_tc_plan(int M, int N, int K) {
+  I8Plan p{};
+  p.MT = M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  p.tiles_n = (N + 127) / 128;
+  p.tiles_m = (M + p.MT - 1) / p.MT;
+  p.KS = (K + 127) / 128;
+  const long long tiles = static_cast<long long>(p.tiles_n) * p.tiles_m;
+  // split K until the tiles fill the SMs (at most 16 ways, 4 stages each)
+  long long s = (148 + tiles - 1) / tiles;
+  s = std::min<long long>(s, std::max(1, p.KS / 4));
+  s = std::min<long long>(s, 16);
+  if (tiles > 65536) s = 1;
+  p.splits = static_cast<int>(std::max<long long>(1, s));
+  return p;
+}
+
 struct Int8Layout {
-  size_t counter, acc, flag, list, cnt, part, olist, ocount, qx, sx, total;
-  int nscan;  // scan CTAs (256 channels each)
+  size_t counter, acc, flag, list, cnt, part, olist, ocount, qx, sx, tcpart, total;
+  int nscan;         // scan CTAs (256 channels each)
+  int counters;      // counters the scan clears
 };
 
 Int8Layout int8_layout(int M, int N, int K) {
   auto r = [](size_t v) { return (v + 255) / 256 * 256; };
   Int8Layout l{};
   l.nscan = (K + 255) / 256;
+  const bool tc = M >= kInt8TcMinM;
+  const I8Plan tp = int8_tc_plan(M, N, K);
+  const long long tiles = static_cast<long long>(tp.tiles_n) * tp.tiles_m;
+  l.counters = std::max((N + 15) / 16, tc ? static_cast<int>(std::min<long long>(tiles, 65536)) : 0);
   size_t o = 0;
-  l.counter = o; o += r(static_cast<size_t>((N + 15) / 16) * 4);
-  l.acc = o;     o += r(static_cast<size_t>(M) * N * 4);
+  l.counter = o; o += r(static_cast<size_t>(l.counters) * 4);
+  l.acc = o;     o += tc ? 0 : r(static_cast<size_t>(M) * N * 4);
   l.flag = o;    o += r(static_cast<size_t>(K));
   l.list = o;    o += r(static_cast<size_t>(l.nscan) * 256 * 4);
   l.cnt = o;     o += r(static_cast<size_t>(l.nscan) * 4);
@@ -345,8 +375,35 @@ Int8Layout int8_layout(int M, int N, int K) {
   l.ocount = o;  o += 256;
   l.qx = o;      o += r(static_cast<size_t>(M) * K);
   l.sx = o;      o += r(static_cast<size_t>(M) * 4);
+  l.tcpart = o;
+  if (tc && tp.splits > 1)
+    o += r(static_cast<size_t>(tiles) * tp.splits * tp.MT * kI8Rows * 4);
   l.total = o;
   return l;
+}
+
+// 3-D tensor map over an int8 [rows, K] matrix: {K, rows, 1}, box {128,
+// box_rows, 1}, 128-byte swizzle (one 128-channel stage = one 128-byte row),
+// rows past the end read as zero.
+bool encode_i8_map(CUtensorMap* map, const int8_t* base, int rows, int K, int box_rows);
+
+template <class C>
+cudaError_t launch_i8_tc(const CUtensorMap& wmap, const CUtensorMap& xmap, const I8TcArgs& a,
+                         int ctas, cudaStream_t st) {
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t attr_err = ensure_smem_limit(int8_tc_kernel<C>, C::kSmemBytes, smem_set);
+  if (attr_err != cudaSuccess) return attr_err;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, int8_tc_kernel<C>, wmap, xmap, a);
 }
 
 bool int8_shape_ok(int M, int N, int K) {
@@ -420,14 +477,47 @@ w4_status llm_int8_gemm(const uint16_t* X, const int8_t* qw, const float* sw, in
   cfg.gridDim = dim3(l.nscan);
   cfg.blockDim = dim3(256);
   cudaError_t e = cudaLaunchKernelEx(&cfg, int8_scan_kernel, X, M, K, threshold, flag, list, cnt,
-                                     part);
+                                     part, a.counter, l.counters);
   if (e == cudaSuccess) {
     cfg.gridDim = dim3(M, ceil_div(K, 2048));
     e = cudaLaunchKernelEx(&cfg, int8_quantize_x_kernel, X, static_cast<const uint8_t*>(flag),
                            static_cast<const float*>(part), static_cast<const int32_t*>(list),
                            static_cast<const int32_t*>(cnt), l.nscan, M, K,
                            const_cast<int8_t*>(a.qx), const_cast<float*>(a.sx),
-                           const_cast<int32_t*>(a.olist), const_cast<int32_t*>(a.ocount));
+                           const_cast<int32_t*>(a.olist), const_cast<int32_t*>(a.ocount), a.acc,
+                           M >= kInt8TcMinM ? 0 : N);
+  }
+  if (e == cudaSuccess && M >= kInt8TcMinM) {
+    // tensor-core product with the epilogue fused
+    const I8Plan tp = int8_tc_plan(M, N, K);
+    CUtensorMap wmap, xmap;
+    if (!encode_i8_map(&wmap, qw, N, K, kI8Rows) || !encode_i8_map(&xmap, a.qx, M, K, tp.MT))
+      return W4_ERR_CUDA;
+    I8TcArgs t{};
+    t.sx = a.sx;
+    t.sw = sw;
+    t.X = X;
+    t.qw = qw;
+    t.olist = a.olist;
+    t.ocount = a.ocount;
+    t.Y = Y;
+    t.partial = reinterpret_cast<int*>(ws + l.tcpart);
+    t.counter = a.counter;
+    t.M = M;
+    t.N = N;
+    t.K = K;
+    t.KS = tp.KS;
+    t.tiles_n = tp.tiles_n;
+    t.tiles_m = tp.tiles_m;
+    t.splits = tp.splits;
+    t.partial_count = (l.total - l.tcpart) / 4;
+    const int ctas = tp.tiles_n * tp.tiles_m * tp.splits;
+    switch (tp.MT) {
+      case 64: e = launch_i8_tc<I8Cfg<64, 6>>(wmap, xmap, t, ctas, st); break;
+      case 128: e = launch_i8_tc<I8Cfg<128, 5>>(wmap, xmap, t, ctas, st); break;
+      default: e = launch_i8_tc<I8Cfg<256, 4>>(wmap, xmap, t, ctas, st); break;
+    }
+    return launch_status(e);
   }
   if (e == cudaSuccess) {
     cfg.gridDim = dim3(static_cast<unsigned>((items + kInt8Warps - 1) / kInt8Warps));

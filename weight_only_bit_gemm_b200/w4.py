@@ -317,8 +317,8 @@ class Workspace:
 
 
 _WS = Workspace()
-# LLM.int8's workspace: its own layout (zero-kept accumulator and counters,
-# regions that every call overwrites), so never the W4A16 / NF4 workspace
+# scratch whose contents the library does not keep zeroed (LLM.int8): never
+# the zero-kept workspace of the W4A16 / NF4 GEMMs
 _WS_SCRATCH = Workspace()
 
 
