@@ -314,6 +314,12 @@ def time_graph(calls, reps: int = 5, warm: int = 2):
     return a.elapsed_time(b) / reps
 
 
+def time_per_call(f, n: int = 5):
+    """Device time (ms) of one call of f, from a CUDA graph of n back-to-back
+    calls (launch latency hidden, as in the decode step's timing)."""
+    return time_graph([f] * n) / n
+
+
 def measure_decode(step, args, pg, local):
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
@@ -434,7 +440,8 @@ def _replicas_for(nbytes_each: int, l2: int) -> int:
 
 
 def measure_rows(w4, peaks):
-    """The other steps of the path, each timed alone (device time, CUDA events)."""
+    """The other steps of the path, each timed alone (device time, CUDA events;
+    the standalone kernels as CUDA graphs of 5 back-to-back calls)."""
     rows = {}
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
     hbm = peaks["hbm_gbs"]
@@ -443,15 +450,15 @@ def measure_rows(w4, peaks):
     K, N, G = 4096, 22016, 128
     W = torch.from_numpy(S.layer_w(WL, K, N)).cuda()
     Wq, sc, zr = w4.quantize_rtn(W, G)
-    t = time_calls([lambda: w4.quantize_rtn(W, G)], reps=5)[0]
+    t = time_per_call(lambda: w4.quantize_rtn(W, G))
     qb = N * K * 4 + N * K / 2 + N * (K // G) * 3
     rows["quantize_rtn"] = {"shape": [N, K], "G": G, "ms": t, "GB/s": qb / t / 1e6,
                             "frac_of_hbm": qb / t / 1e6 / hbm}
-    t = time_calls([lambda: w4.dequant(Wq, sc, zr, G)], reps=5)[0]
+    t = time_per_call(lambda: w4.dequant(Wq, sc, zr, G))
     db = N * K / 2 + N * (K // G) * 3 + N * K * 2
     rows["dequant"] = {"shape": [N, K], "G": G, "ms": t, "GB/s": db / t / 1e6,
                        "frac_of_hbm": db / t / 1e6 / hbm}
-    t = time_calls([lambda: w4.prepack(Wq, sc, zr, G)], reps=5)[0]
+    t = time_per_call(lambda: w4.prepack(Wq, sc, zr, G))
     pb = 2 * (N * K / 2 + N * (K // G) * 2.5)
     rows["prepack"] = {"shape": [N, K], "G": G, "ms": t, "GB/s": pb / t / 1e6}
     del W, Wq, sc, zr
@@ -463,7 +470,7 @@ def measure_rows(w4, peaks):
         W = torch.from_numpy(S.layer_w(nf, K, N)).cuda()
         q4, c4, s24 = w4.nf4_quantize(W)
         if (K, N) == nf["shapes"][0]:
-            t = time_calls([lambda: w4.nf4_quantize(W)], reps=5)[0]
+            t = time_per_call(lambda: w4.nf4_quantize(W))
             b = N * K * 4 + N * K / 2 + N * K / 64
             rows["nf4_quantize"] = {"shape": [N, K], "ms": t, "GB/s": b / t / 1e6}
         wp = w4.nf4_prepack(q4, c4)
@@ -489,7 +496,7 @@ def measure_rows(w4, peaks):
         W = torch.from_numpy(S.layer_w(nf, K, N)).cuda()
         q4, c4, m4, s24 = w4.nf4_quantize_meandq(W)
         if (K, N) == nf["shapes"][0]:
-            t = time_calls([lambda: w4.nf4_quantize_meandq(W)], reps=5)[0]
+            t = time_per_call(lambda: w4.nf4_quantize_meandq(W))
             b = N * K * 4 + N * K / 2 + N * K / 64
             rows["nf4_meandq_quantize"] = {"shape": [N, K], "ms": t, "GB/s": b / t / 1e6}
         wp = w4.nf4_prepack(q4, c4.view(torch.uint8))
@@ -514,7 +521,7 @@ def measure_rows(w4, peaks):
         W = torch.from_numpy(S.layer_w(f4, K, N)).cuda()
         q4, c4, s24 = w4.fp4_quantize(W)
         if (K, N) == f4["shapes"][0]:
-            t = time_calls([lambda: w4.fp4_quantize(W)], reps=5)[0]
+            t = time_per_call(lambda: w4.fp4_quantize(W))
             b = N * K * 4 + N * K / 2 + N * K / 64
             rows["fp4_quantize"] = {"shape": [N, K], "ms": t, "GB/s": b / t / 1e6}
         wp = w4.nf4_prepack(q4, c4)
@@ -581,11 +588,11 @@ def measure_rows(w4, peaks):
         Ws = w4.awq_scale_weights(W, sd)
         Wq, sc, zr = w4.quantize_sym(Ws, G)
         if (K, N) == (4096, 22016):
-            t = time_calls([lambda: w4.awq_scale_weights(W, sd, out=Ws)], reps=5)[0]
+            t = time_per_call(lambda: w4.awq_scale_weights(W, sd, out=Ws))
             b = 2 * N * K * 4 + K * 4
             rows["awq_scale_weights"] = {"shape": [N, K], "ms": t, "GB/s": b / t / 1e6,
                                          "frac_of_hbm": b / t / 1e6 / hbm}
-            t = time_calls([lambda: w4.quantize_sym(Ws, G)], reps=5)[0]
+            t = time_per_call(lambda: w4.quantize_sym(Ws, G))
             qb = N * K * 4 + N * K / 2 + N * (K // G) * 3
             rows["quantize_sym"] = {"shape": [N, K], "G": G, "ms": t, "GB/s": qb / t / 1e6,
                                     "frac_of_hbm": qb / t / 1e6 / hbm}
@@ -618,7 +625,7 @@ def measure_rows(w4, peaks):
         W = torch.from_numpy(S.layer_w(WL, K, N)).cuda()
         qw, sw = w4.llm_int8_quantize_weights(W)
         if (K, N) == (4096, 22016):
-            t = time_calls([lambda: w4.llm_int8_quantize_weights(W)], reps=5)[0]
+            t = time_per_call(lambda: w4.llm_int8_quantize_weights(W))
             b = N * K * 4 + N * K + 4 * N
             rows["llm_int8_quantize"] = {"shape": [N, K], "ms": t, "GB/s": b / t / 1e6}
         reps = [qw] + [qw.clone() for _ in range(_replicas_for(qw.numel(), l2) - 1)]

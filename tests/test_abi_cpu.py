@@ -87,6 +87,25 @@ def test_fp4_levels_equal_oracle_table():
     assert np.array_equal(np.array(got, np.float32).view(np.uint32), want.view(np.uint32))
 
 
+def test_prefill_tail_split_workspace():
+    # 148 SMs (the planner's count without a device).  (40, 19000, 2560):
+    # 149 tiles of 64 tokens x 128 rows, 20 stages; one full wave of whole
+    # tiles (cost 21.5) and the remaining tile in 5 K ranges (4 + 13.5) beats
+    # two waves of whole tiles (43): partials for 5 ranges of one 64 x 128
+    # tile after the 65536 arrival counters.
+    assert w4.workspace_bytes(40, 19000, 2560, 128) == 65536 * 4 + 5 * 64 * 128 * 4
+    # (512, 28672, 8192): 448 tiles of 256 tokens, 64 stages; three full
+    # waves (196.5) and 4 tail tiles in 4 K ranges each (16 + 1.5 + 12; more
+    # ranges cost more reduction round trips than they save) against 262 for
+    # four waves of whole tiles
+    assert w4.workspace_bytes(512, 28672, 8192, 128) == 65536 * 4 + 4 * 4 * 256 * 128 * 4
+    # (2048, 8192, 28672): 512 tiles, 224 stages; 3 waves whole and 68 tiles in
+    # 2 ranges (802) against every tile in 2 ranges (878)
+    assert w4.workspace_bytes(2048, 8192, 28672, 128) == 65536 * 4 + 68 * 2 * 256 * 128 * 4
+    # one partial wave (128 tiles): whole tiles, no partials
+    assert w4.workspace_bytes(512, 8192, 28672, 128) == 65536 * 4
+
+
 def test_workspace_sizes_of_the_variants():
     r256 = lambda v: (v + 255) // 256 * 256
     # the AWQ call adds the rewritten activations, M x K bf16, to the plain plan

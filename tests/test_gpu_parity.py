@@ -101,6 +101,25 @@ def test_nf4_quantize_dequant_bit_exact(w4, N, K):
     assert np.array_equal(host_u16(what), O.nf4_dequant(Wq_r, c_r, s2_r))
 
 
+@pytest.mark.parametrize("table", ["nf4", "fp4"])
+@pytest.mark.parametrize("N,K,dq", [(37, 1024, 300), (64, 4096, 1024), (20, 640, 3)])
+def test_blockwise_quantize_dq_group_bit_exact(w4, table, N, K, dq):
+    # runs longer than one pass of the kernel (256 blocks), a last run
+    # shorter than the others, and very short runs
+    W = S.draw_w(N, K, 0.02, seed=N, tag=3)
+    W[1, 64:128] = 0.0
+    oq, odq = (O.nf4_quantize, O.nf4_dequant) if table == "nf4" else (O.fp4_quantize,
+                                                                      O.fp4_dequant)
+    dq_dev = w4.nf4_dequant if table == "nf4" else w4.fp4_dequant
+    Wq_r, c_r, s2_r = oq(W, 64, dq)
+    Wq, c, s2 = (w4.nf4_quantize if table == "nf4" else w4.fp4_quantize)(dev(W), 64, dq)
+    status_ok(w4)
+    assert np.array_equal(Wq.cpu().numpy(), Wq_r)
+    assert np.array_equal(c.cpu().numpy(), c_r)
+    assert np.array_equal(s2.cpu().numpy().view(np.uint32), s2_r.view(np.uint32))
+    assert np.array_equal(host_u16(dq_dev(Wq, c, s2, dq)), odq(Wq_r, c_r, s2_r, 64, dq))
+
+
 # ----------------------------------------------------------------- prepack
 
 @pytest.mark.parametrize("N,K,G,act", [(300, 320, 64, False), (256, 1024, 32, True),
@@ -201,6 +220,10 @@ GEMM_CASES = [
     (2, 1, 128, 128, False),         # one output row
     (8, 77, 320, 32, False),         # last stage has no second half, ragged N
     (32, 1000, 4096, 128, False),    # four token blocks, ragged N
+    # prefill work split: one full wave of whole tiles, then the last partial
+    # wave's tiles split in K (149 and 150 tiles on 148 SMs)
+    (40, 19000, 2560, 128, False),   # ragged N, one tail tile in 5 K ranges
+    (300, 9550, 2560, 64, True),     # two token tiles, act-order, two tail tiles
     (5, 4096, 4160, 64, False),      # K = 32.5 stages: last stage half, G = 64
 ]
 

@@ -56,7 +56,7 @@ struct GemmCfg {
   static constexpr int kNumBars = 2 * STAGES + 2 * kASlots + 3;
   static constexpr int kSmemBytes =
       1024 /* alignment slack */ + STAGES * (kXStageBytes + kWSlot) + kNumBars * 8 + 16 + 64 +
-      64 /* NF4 level table alignment */;
+      256 /* NF4 level table alignment */;
   static constexpr int kMinBlocks = kTmemCols <= 256 && kSmemBytes <= 113 * 1024 ? 2 : 1;
   static_assert(MT % 16 == 0 && MT >= 16 && MT <= 256, "MMA N for M=128 is 16..256 step 16");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -149,23 +149,24 @@ __device__ __forceinline__ void int4_dq_word(uint32_t w, const Int4Dq& p0, const
 }
 
 // NF4 dequant of one word: w_hat = bf16_rne(fp32(T[q] * a')), with the 16
-// levels T in shared memory at the 64-byte-aligned shared address tb (so that
-// a level's address is tb | 4q), a0 / a1 the reconstructed absmax of rows
-// r0 / r1.  One asm block: per code one shift and one LOP3 for the address,
-// one shared load, one fp32 multiply; one conversion per pair.
+// levels T in shared memory at the 256-byte-aligned shared address tb (so
+// that a level's address is tb with its low byte replaced by 4q), a0 / a1 the
+// reconstructed absmax of rows r0 / r1.  One asm block: two shift + mask
+// pairs put 4q of all eight codes into the bytes of two registers (t0: codes
+// 0, 2, 4, 6; t1: codes 1, 3, 5, 7), one byte permute per code makes its
+// address; then one shared load and one fp32 multiply per code and one
+// conversion per pair.  The pairs are (code i, code i + 4), i = 0..3, as the
+// prepacked layout orders them for the MMA fragment.
 __device__ __forceinline__ void nf4_dq_word(uint32_t w, float a0, float a1, uint32_t tb,
                                             uint32_t* out) {
-  const uint32_t m = 0x3Cu;
-  asm("{\n\t.reg .b32 o0, o1, o2, o3, o4, o5, o6, o7;\n\t"
+  asm("{\n\t.reg .b32 t0, t1, o0, o1, o2, o3, o4, o5, o6, o7;\n\t"
       ".reg .f32 v0, v1, v2, v3, v4, v5, v6, v7;\n\t"
-      "shl.b32 o0, %4, 2;\n\t  lop3.b32 o0, o0, %7, %8, 0xEA;\n\t"
-      "shr.b32 o1, %4, 14;\n\t lop3.b32 o1, o1, %7, %8, 0xEA;\n\t"
-      "shr.b32 o2, %4, 2;\n\t  lop3.b32 o2, o2, %7, %8, 0xEA;\n\t"
-      "shr.b32 o3, %4, 18;\n\t lop3.b32 o3, o3, %7, %8, 0xEA;\n\t"
-      "shr.b32 o4, %4, 6;\n\t  lop3.b32 o4, o4, %7, %8, 0xEA;\n\t"
-      "shr.b32 o5, %4, 22;\n\t lop3.b32 o5, o5, %7, %8, 0xEA;\n\t"
-      "shr.b32 o6, %4, 10;\n\t lop3.b32 o6, o6, %7, %8, 0xEA;\n\t"
-      "shr.b32 o7, %4, 26;\n\t lop3.b32 o7, o7, %7, %8, 0xEA;\n\t"
+      "shl.b32 t0, %4, 2;\n\t  and.b32 t0, t0, 0x3C3C3C3C;\n\t"
+      "shr.b32 t1, %4, 2;\n\t  and.b32 t1, t1, 0x3C3C3C3C;\n\t"
+      "prmt.b32 o0, t0, %7, 0x7650;\n\t prmt.b32 o1, t0, %7, 0x7652;\n\t"
+      "prmt.b32 o2, t1, %7, 0x7650;\n\t prmt.b32 o3, t1, %7, 0x7652;\n\t"
+      "prmt.b32 o4, t0, %7, 0x7651;\n\t prmt.b32 o5, t0, %7, 0x7653;\n\t"
+      "prmt.b32 o6, t1, %7, 0x7651;\n\t prmt.b32 o7, t1, %7, 0x7653;\n\t"
       "ld.shared.f32 v0, [o0];\n\t ld.shared.f32 v1, [o1];\n\t"
       "ld.shared.f32 v2, [o2];\n\t ld.shared.f32 v3, [o3];\n\t"
       "ld.shared.f32 v4, [o4];\n\t ld.shared.f32 v5, [o5];\n\t"
@@ -179,7 +180,7 @@ __device__ __forceinline__ void nf4_dq_word(uint32_t w, float a0, float a1, uint
       "cvt.rn.bf16x2.f32 %2, v5, v4;\n\t"
       "cvt.rn.bf16x2.f32 %3, v7, v6;\n\t}"
       : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
-      : "r"(w), "f"(a0), "f"(a1), "r"(m), "r"(tb)
+      : "r"(w), "f"(a0), "f"(a1), "r"(tb)
       : "memory");
 }
 
@@ -193,7 +194,9 @@ struct GemmArgs {
   int M, N, K;
   int KS;                 // stages per tile row = ceil(K / 128)
   int tiles_n;
-  int splits;
+  int splits;             // K ranges of every tile (tail_splits == 0)
+  int head_tiles;         // tail_splits > 0: tiles (in CTA order) computed whole,
+  int tail_splits;        //   then each remaining tile in tail_splits K ranges
   int tiles_m;            // token tiles
   int group_m;            // token tiles per group of the CTA order (see the kernel)
   FastDivIdx by_dq;        // NF4: 64-block index -> s2 index (double-quant run)

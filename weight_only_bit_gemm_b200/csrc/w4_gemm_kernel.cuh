@@ -23,8 +23,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
   uint64_t* epi2 = epi1 + 1;                            // last-arrival known (1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi2 + 1);
   int* last_flag = reinterpret_cast<int*>(tmem_holder + 1);
-  float* Ts = reinterpret_cast<float*>(                   // NF4 levels [16], 64-byte aligned
-      (reinterpret_cast<uintptr_t>(tmem_holder + 4) + 63) & ~static_cast<uintptr_t>(63));
+  float* Ts = reinterpret_cast<float*>(                   // NF4 levels [16], 256-byte aligned
+      (reinterpret_cast<uintptr_t>(tmem_holder + 4) + 255) & ~static_cast<uintptr_t>(255));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -32,17 +32,46 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
   // runs fastest, so the CTAs that read one weight tile (and split range)
   // run together and share it through L2, as do the weight tiles of a wave
   // for the group's activation tiles.
-  const int ns = args.tiles_n * args.splits;
-  const int gsize = args.group_m * ns;
-  const int grp = static_cast<int>(blockIdx.x) / gsize;
-  const int gm = min(args.group_m, args.tiles_m - grp * args.group_m);
-  const int lin = static_cast<int>(blockIdx.x) - grp * gsize;
-  const int mtile = grp * args.group_m + lin % gm;
-  const int nts = lin / gm;
-  const int nt = nts / args.splits;
-  const int split = nts % args.splits;
-  const int s0 = static_cast<int>(static_cast<long long>(split) * args.KS / args.splits);
-  const int s1 = static_cast<int>(static_cast<long long>(split + 1) * args.KS / args.splits);
+  // Two work splits: every tile in `splits` K ranges (tail_splits == 0), or
+  // the first head_tiles tiles whole and the remaining (tail) tiles in
+  // tail_splits K ranges each, so that the last partial wave of CTAs still
+  // spreads over the SMs.  pbase: the partial slot of K range 0 of this
+  // tile; cidx: its arrival counter.
+  int mtile, nt, split, nsplit, cidx;
+  size_t pbase;
+  {
+    const int b = static_cast<int>(blockIdx.x);
+    const int ns = args.tail_splits == 0 ? args.tiles_n * args.splits : args.tiles_n;
+    int lt = b;  // CTA position in the group order (tail: the tile's)
+    if (args.tail_splits == 0) {
+      nsplit = args.splits;
+    } else if (b < args.head_tiles) {
+      nsplit = 1;
+    } else {
+      const int t = b - args.head_tiles;
+      nsplit = args.tail_splits;
+      lt = args.head_tiles + t / nsplit;
+    }
+    const int gsize = args.group_m * ns;
+    const int grp = lt / gsize;
+    const int gm = min(args.group_m, args.tiles_m - grp * args.group_m);
+    const int lin = lt - grp * gsize;
+    mtile = grp * args.group_m + lin % gm;
+    const int nts = lin / gm;
+    if (args.tail_splits == 0) {
+      nt = nts / nsplit;
+      split = nts % nsplit;
+      cidx = mtile * args.tiles_n + nt;
+      pbase = static_cast<size_t>(cidx) * nsplit;
+    } else {
+      nt = nts;
+      split = b < args.head_tiles ? 0 : (b - args.head_tiles) % nsplit;
+      cidx = lt - args.head_tiles;
+      pbase = static_cast<size_t>(cidx) * nsplit;
+    }
+  }
+  const int s0 = static_cast<int>(static_cast<long long>(split) * args.KS / nsplit);
+  const int s1 = static_cast<int>(static_cast<long long>(split + 1) * args.KS / nsplit);
   const int nst = s1 - s0;
 
   if (threadIdx.x == 0) {
@@ -61,6 +90,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     grid_dep_launch();  // the next kernel on the stream may start its prologue
   }
   if (C::FMT == kFmtNf4 && threadIdx.x < 16) Ts[threadIdx.x] = level_value(args.table, threadIdx.x);
+  // the level addresses need a 256-byte-aligned table (bounds-checked build: verified)
+  if (C::FMT == kFmtNf4 && kChecked && threadIdx.x == 0) in_bounds(smem_u32(Ts) & 0xFFu, 1u);
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::kTmemCols);
     tmem_relinquish();
@@ -228,10 +259,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
       grid_dep_wait();  // Y and the workspace may still be in use by the previous kernel
       constexpr int kHalfCols = C::MT / 2;
       const int m_base = mtile * C::MT + h * kHalfCols;
-      const int tile_id = mtile * args.tiles_n + nt;
-      float* part = args.partial +
-                    ((static_cast<size_t>(tile_id) * args.splits + split) * C::MT + h * kHalfCols) *
-                        kTileRows;
+      float* part = args.partial + ((pbase + split) * C::MT + h * kHalfCols) * kTileRows;
 #pragma unroll 1
       for (int cb = 0; cb < kHalfCols; cb += 8) {
         float sum[8];
@@ -248,7 +276,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
         for (int j = 0; j < 8; ++j) {
           const int m = m_base + cb + j;
           const float acc = sum[j];
-          if (args.splits == 1) {
+          if (nsplit == 1) {
             if (m < args.M && n < args.N)
               args.Y[static_cast<size_t>(m) * args.N + n] =
                   __bfloat16_as_ushort(__float2bfloat16_rn(acc));
@@ -260,7 +288,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
         }
       }
       tc_fence_before();
-      if (args.splits > 1) {
+      if (nsplit > 1) {
         // the last CTA of this tile to arrive sums the partials in split order
         // (mbarriers with bounded waits, not bar.sync, so that a warp that gave
         // up earlier cannot leave the others blocked)
@@ -269,9 +297,9 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
         if (lane == 0) mbar_arrive(epi1);
         bool have_flag = true;
         if (threadIdx.x == 64) {
-          if (mbar_wait(epi1, 0) && in_bounds(tile_id, 65536)) {
-            const unsigned prev = atomicAdd(args.counter + tile_id, 1u);
-            *last_flag = (prev == static_cast<unsigned>(args.splits - 1)) ? 1 : 0;
+          if (mbar_wait(epi1, 0) && in_bounds(cidx, 65536)) {
+            const unsigned prev = atomicAdd(args.counter + cidx, 1u);
+            *last_flag = (prev == static_cast<unsigned>(nsplit - 1)) ? 1 : 0;
           } else {
             *last_flag = 0;
           }
@@ -280,28 +308,38 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
         have_flag = __all_sync(0xffffffffu, mbar_wait(epi2, 0));
         if (have_flag && *last_flag) {
           __threadfence();
-          const float* base =
-              args.partial + static_cast<size_t>(tile_id) * args.splits * C::MT * kTileRows;
-          // kCb columns at a time, so that kCb loads per split are in flight
-          // (one column at a time leaves the reduction L2-latency bound)
-          constexpr int kCb = kHalfCols < 16 ? kHalfCols : 16;
+          const float* base = args.partial + pbase * C::MT * kTileRows;
+          // kCb columns of kSu K ranges at a time: kCb * kSu loads in flight per
+          // L2 round trip (one range at a time, a 16-range tile took 128 round
+          // trips); the sums are still taken in range order
+          constexpr int kCb = kHalfCols < 8 ? kHalfCols : 8;
+          constexpr int kSu = 4;
 #pragma unroll 1
           for (int c0 = 0; c0 < kHalfCols; c0 += kCb) {
             const int ml0 = h * kHalfCols + c0;
             float acc[kCb];
 #pragma unroll
             for (int j = 0; j < kCb; ++j) acc[j] = 0.0f;
-            for (int sp = 0; sp < args.splits; ++sp) {
-              const float* src = base + (static_cast<size_t>(sp) * C::MT + ml0) * kTileRows + row;
-              float v[kCb];
-              if (!in_bounds(static_cast<unsigned long long>(src - args.partial) +
-                                 (kCb - 1) * kTileRows,
-                             args.partial_floats))
-                continue;
+#pragma unroll 1
+            for (int sp0 = 0; sp0 < nsplit; sp0 += kSu) {
+              float v[kSu][kCb];
+              bool ok[kSu];
 #pragma unroll
-              for (int j = 0; j < kCb; ++j) v[j] = __ldcg(src + j * kTileRows);
+              for (int u = 0; u < kSu; ++u) {
+                const float* src =
+                    base + (static_cast<size_t>(sp0 + u) * C::MT + ml0) * kTileRows + row;
+                ok[u] = sp0 + u < nsplit &&
+                        in_bounds(static_cast<unsigned long long>(src - args.partial) +
+                                      (kCb - 1) * kTileRows,
+                                  args.partial_floats);
 #pragma unroll
-              for (int j = 0; j < kCb; ++j) acc[j] += v[j];
+                for (int j = 0; j < kCb; ++j) v[u][j] = ok[u] ? __ldcg(src + j * kTileRows) : 0.0f;
+              }
+#pragma unroll
+              for (int u = 0; u < kSu; ++u)
+#pragma unroll
+                for (int j = 0; j < kCb; ++j)
+                  if (ok[u]) acc[j] += v[u][j];
             }
 #pragma unroll
             for (int j = 0; j < kCb; ++j) {
@@ -311,7 +349,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
                     __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
             }
           }
-          if (threadIdx.x == 64) args.counter[tile_id] = 0u;  // leave the workspace zeroed
+          if (threadIdx.x == 64) args.counter[cidx] = 0u;  // leave the workspace zeroed
         }
       }
     }

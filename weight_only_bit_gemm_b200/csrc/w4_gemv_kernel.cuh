@@ -63,7 +63,6 @@ struct GemvArgs {
   FastDivIdx by_dq;          // NF4: 64-block index -> s2 index
   int dq_group;             // NF4: 64-blocks per second-level scale
   int table;                // NF4 layout: level table (kTableNf4 / kTableFp4)
-  int cluster;              // CTAs per thread-block cluster (1: no cluster level)
   // buffer extents, read only by the bounds-checked build
   unsigned long long wp_bytes, partial_floats, s2_count;
 };
@@ -74,6 +73,14 @@ struct GemvArgs {
 // each other; with two or four token blocks the blocks themselves give that
 // independence, and one set keeps the registers within budget.
 __host__ __device__ constexpr int gemv_row_groups(int) { return 2; }
+
+// CTA shape of the decode kernel: warps per CTA and resident CTAs per SM (one
+// wave of CTAs covers the GPU; the planner sizes the grid from these).  One
+// CTA of 16 warps per SM (128 registers a thread): measured on B200, the
+// same warps as two CTAs of 8 per SM but half as many CTA partials per row
+// pair in the global level of the reduction, 0.6 us less per call.
+constexpr int kGemvWarps = 16;
+constexpr int kGemvCtasPerSm = 1;
 __host__ __device__ constexpr int gemv_acc_split(int NB) { return NB >= 2 ? 1 : 2; }
 
 template <int NB_, int FMT_, int G_, bool MEAN_ = false>
@@ -84,9 +91,9 @@ struct GemvCfg {
   static constexpr int G = G_;
   static constexpr bool MEAN = MEAN_;  // NF4 layout: mean-offset absmax constants
   static constexpr int kStageBytes = FMT == kFmtInt4 ? int4_stage_bytes(G) : nf4_stage_bytes();
-  static constexpr int kWarps = 8;
+  static constexpr int kWarps = kGemvWarps;
   static constexpr int kThreads = 32 * kWarps;
-  static constexpr int kMinBlocks = 2;  // resident CTAs per SM (128 registers a thread)
+  static constexpr int kMinBlocks = kGemvCtasPerSm;
   // groups per 128-channel stage (INT4); NF4 keeps its absmax pairs in sp[0] / zp[0]
   static constexpr int kNq = FMT == kFmtInt4 ? 128 / G : 1;
   static constexpr int kDepth = 4;  // per-warp ring slots (3 units in flight)
@@ -103,12 +110,8 @@ struct GemvCfg {
   static constexpr bool kCtaReduce = NB <= 2;
   static constexpr int kV = kRG * NB * 4;  // partial floats per lane
   static constexpr int kRedBytes = kCtaReduce ? kWarps * 2 * 32 * kV * 4 : 0;
-  // cluster level (with the CTA level): the row pair that ends this CTA's
-  // range, if it continues in the next CTAs of the cluster, is combined here:
-  // one partial slot per CTA of the cluster and one arrival counter
-  static constexpr int kMaxCluster = 4;
-  static constexpr int kClusterBytes = kCtaReduce ? kMaxCluster * 32 * kV * 4 : 0;
-  static constexpr int kSmemBytes = kRingBytes + kRedBytes + kClusterBytes + kWarps * 4 + 16;
+  static constexpr int kSmemBytes = kRingBytes + kRedBytes + kWarps * 4;
+  static_assert(kSmemBytes + 64 <= 227 * 1024, "shared memory of one CTA");
 };
 
 __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t (&a)[4],
@@ -251,41 +254,7 @@ __device__ __forceinline__ uint32_t range_end(uint32_t w, const GemvArgs& a) {
 struct CtaRed {
   float4* part;            // [warp][kind][V/4][32 lanes]
   unsigned int* count;     // [warp]: arrivals for the row pair that ends its range
-  float4* cpart;           // [CTA of the cluster][V/4][32 lanes]
-  unsigned int* ccount;    // arrivals of the cluster's CTAs
 };
-
-// Distributed shared memory of the CTAs of a cluster.
-__device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void st_peer(uint32_t addr, float4 v) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y),
-               "f"(v.z), "f"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ float4 ld_peer(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ unsigned atom_add_peer(uint32_t addr) {
-  unsigned old;
-  asm volatile("atom.acq_rel.cluster.shared::cluster.add.u32 %0, [%1], 1;"
-               : "=r"(old)
-               : "r"(addr)
-               : "memory");
-  return old;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
-                   "memory");
-}
 
 // Global level: this lane's partial `tot` in slot `slot` of row pair rpg,
 // `contrib` slots in all; returns true (with tot the full sum, added in slot
@@ -308,17 +277,16 @@ __device__ __forceinline__ bool global_combine(const GemvArgs& args,
     for (int nb = 0; nb < C::NB; ++nb)
       *reinterpret_cast<float4*>(dst + (rr * C::NB + nb) * 4) =
           make_float4(tot[rr][nb][0], tot[rr][nb][1], tot[rr][nb][2], tot[rr][nb][3]);
-  // every lane's partial visible device-wide before the arrival; the last
-  // arrival's lanes fence again before reading the others' partials (the
-  // shuffle carries lane 0's acquire to them only as a value)
-  __threadfence();
+  // The warp barrier orders every lane's partial before lane 0's release
+  // (the arrival) and, on the last arrival, lane 0's acquire before every
+  // lane's reads of the other partials (the shuffle carries the count only
+  // as a value).
   __syncwarp();
   unsigned prev = 0;
   if (lane == 0) prev = atom_add_acq_rel_gpu(args.counter + rpg, 1u);
   prev = __shfl_sync(0xffffffffu, prev, 0);
   __syncwarp();
   if (prev != contrib - 1) return false;
-  __threadfence();
 #pragma unroll
   for (int rr = 0; rr < R; ++rr)
 #pragma unroll
@@ -426,61 +394,12 @@ __device__ __forceinline__ void flush_row_group(const GemvArgs& args,
         done = first >= cta_w0 && last <= cta_w1;
       }
     }
-    uint32_t cs = 1;  // CTAs per global contributor
-    if constexpr (C::kCtaReduce) {
-      if (!done && args.cluster > 1) {
-        // level 2: the CTAs of one cluster that share the row pair combine in
-        // the shared memory of the first of them (the row pair ends its range)
-        cs = static_cast<uint32_t>(args.cluster);
-        const uint32_t cta = blockIdx.x;
-        const uint32_t cl0 = cta / cs * cs, cl1 = cl0 + cs - 1;
-        const uint32_t fc = first / C::kWarps, lc = last / C::kWarps;
-        const uint32_t k0 = fc > cl0 ? fc : cl0, k1 = lc < cl1 ? lc : cl1;
-        if (k1 > k0) {
-          const uint32_t owner = k0 - cl0;
-#pragma unroll
-          for (int rr = 0; rr < R; ++rr)
-#pragma unroll
-            for (int nb = 0; nb < C::NB; ++nb)
-              st_peer(peer_addr(cr.cpart + ((cta - k0) * (C::kV / 4) + rr * C::NB + nb) * 32 + lane, owner),
-                      make_float4(tot[rr][nb][0], tot[rr][nb][1], tot[rr][nb][2], tot[rr][nb][3]));
-          asm volatile("fence.acq_rel.cluster;" ::: "memory");  // every lane's slot
-          __syncwarp();
-          unsigned prev = 0;
-          if (lane == 0) prev = atom_add_peer(peer_addr(cr.ccount, owner));
-          prev = __shfl_sync(0xffffffffu, prev, 0);
-          __syncwarp();
-          if (prev != k1 - k0) return;
-          asm volatile("fence.acq_rel.cluster;" ::: "memory");
-#pragma unroll
-          for (int rr = 0; rr < R; ++rr)
-#pragma unroll
-            for (int nb = 0; nb < C::NB; ++nb)
-#pragma unroll
-              for (int j = 0; j < 4; ++j) tot[rr][nb][j] = 0.0f;
-          for (uint32_t c = k0; c <= k1; ++c) {
-#pragma unroll
-            for (int rr = 0; rr < R; ++rr)
-#pragma unroll
-              for (int nb = 0; nb < C::NB; ++nb) {
-                const float4 v = ld_peer(
-                    peer_addr(cr.cpart + ((c - k0) * (C::kV / 4) + rr * C::NB + nb) * 32 + lane, owner));
-                tot[rr][nb][0] += v.x;
-                tot[rr][nb][1] += v.y;
-                tot[rr][nb][2] += v.z;
-                tot[rr][nb][3] += v.w;
-              }
-          }
-          done = fc >= cl0 && lc <= cl1;
-        }
-      }
-    }
     if (!done) {
-      // last level, through global memory: one partial per cluster (per CTA
-      // without clusters, per warp without the CTA level)
-      const uint32_t per = C::kCtaReduce ? C::kWarps * cs : 1u;
+      // level 2, through global memory: one partial per CTA (per warp
+      // without the CTA level)
+      const uint32_t per = C::kCtaReduce ? C::kWarps : 1u;
       const uint32_t unit0 = first / per, unit1 = last / per;
-      const uint32_t me = C::kCtaReduce ? blockIdx.x / cs : wid;
+      const uint32_t me = C::kCtaReduce ? blockIdx.x : wid;
       write_y = global_combine<C>(args, tot, rpg, me - unit0, unit1 - unit0 + 1, lane);
     }
   }
@@ -748,28 +667,18 @@ __device__ __forceinline__ void decode_warp(const GemvArgs& args, const CtaRed& 
 
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4_gemv_kernel(const GemvArgs args) {
-  __shared__ __align__(64) float Ts[16];  // NF4 / FP4 levels
+  __shared__ __align__(256) float Ts[16];  // NF4 / FP4 levels (see nf4_dq_word)
   extern __shared__ __align__(16) uint8_t w4_gemv_smem[];
   CtaRed cr;
   cr.part = reinterpret_cast<float4*>(w4_gemv_smem + C::kRingBytes);
-  cr.cpart = reinterpret_cast<float4*>(w4_gemv_smem + C::kRingBytes + C::kRedBytes);
-  cr.count = reinterpret_cast<unsigned int*>(w4_gemv_smem + C::kRingBytes + C::kRedBytes +
-                                             C::kClusterBytes);
-  cr.ccount = cr.count + C::kWarps;
+  cr.count = reinterpret_cast<unsigned int*>(w4_gemv_smem + C::kRingBytes + C::kRedBytes);
   if (C::FMT == kFmtNf4 && threadIdx.x < 16) Ts[threadIdx.x] = level_value(args.table, threadIdx.x);
-  if (threadIdx.x <= C::kWarps) cr.count[threadIdx.x] = 0u;  // and the cluster counter
-  // Every thread of every CTA meets here (counters initialised before any
-  // peer may count on them) and again at the end (no CTA leaves while its
-  // shared memory may still be read or written by the cluster's others).
-  const bool clustered = C::kCtaReduce && args.cluster > 1;
-  if (clustered)
-    cluster_sync_all();
-  else
-    __syncthreads();
+  // the level addresses need a 256-byte-aligned table (bounds-checked build: verified)
+  if (C::FMT == kFmtNf4 && kChecked && threadIdx.x == 0) in_bounds(smem_u32(Ts) & 0xFFu, 1u);
+  if (threadIdx.x < C::kWarps) cr.count[threadIdx.x] = 0u;
+  __syncthreads();
   grid_dep_launch();
   decode_warp<C>(args, cr, w4_gemv_smem, Ts);
-  __syncwarp();
-  if (clustered) cluster_sync_all();
 }
 
 }  // namespace w4

@@ -273,11 +273,10 @@ __global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(const Int
       if (r1 < a.N && t0 + 1 < a.M) atomicAdd(&a.acc[static_cast<size_t>(t0 + 1) * a.N + r1], d[j][3]);
     }
   }
-  // arrival on the row tile's counter; the last item runs the epilogue.
-  // Every lane's atomics are made visible device-wide before the arrival
-  // (a fence by each lane, not only by the lane that counts), and every lane
-  // of the last item fences again before it reads the sums.
-  __threadfence();
+  // arrival on the row tile's counter; the last item runs the epilogue.  The
+  // warp barrier orders every lane's atomics before lane 0's release (the
+  // arrival) and, on the last item, lane 0's acquire before every lane's
+  // reads of the sums.
   __syncwarp();
   unsigned prev = 0;
   if (lane == 0 && in_bounds(static_cast<unsigned int>(rt), static_cast<unsigned int>(a.row_tiles)))
@@ -285,7 +284,6 @@ __global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(const Int
   prev = __shfl_sync(0xffffffffu, prev, 0);
   __syncwarp();
   if (prev != static_cast<unsigned>(a.slices - 1)) return;
-  __threadfence();
   // y[m][n] = acc s_x s_w + sum over outlier channels (ascending) of x * bf16(q_w s_w)
   const int no = min(*a.ocount, a.K);
   for (int idx = lane; idx < 16 * a.M; idx += 32) {

@@ -130,21 +130,21 @@ w4_status quantize_int4(const float* W, int N, int K, int G, const int32_t* g_id
     return W4_ERR_INVALID_ARG;
   const long long total = static_cast<long long>(N) * K;
   if (!g_idx && total % 128 == 0 && aligned(W, 16) && aligned(Wq, 2)) {
-    // contiguous groups: the flat kernel, a persistent grid over 128-weight segments
-    const long long nseg = total / 128;
-    const long long warps = (nseg + 3) / 4;
+    // contiguous groups: the flat kernel, a persistent grid over 512-weight chunks
+    const long long ngroups = total / G;
+    const long long warps = (total + 511) / 512;
     const unsigned blocks = static_cast<unsigned>(
         std::min<long long>((warps + 7) / 8, static_cast<long long>(sm_count()) * 8));
     cudaStream_t st = as_stream(stream);
     switch (G) {
       case 32:
-        rtn_quantize_flat_kernel<SYM, 32><<<blocks, 256, 0, st>>>(W, nseg, Wq, scales, zeros);
+        rtn_quantize_flat_kernel<SYM, 32><<<blocks, 256, 0, st>>>(W, ngroups, Wq, scales, zeros);
         break;
       case 64:
-        rtn_quantize_flat_kernel<SYM, 64><<<blocks, 256, 0, st>>>(W, nseg, Wq, scales, zeros);
+        rtn_quantize_flat_kernel<SYM, 64><<<blocks, 256, 0, st>>>(W, ngroups, Wq, scales, zeros);
         break;
       default:
-        rtn_quantize_flat_kernel<SYM, 128><<<blocks, 256, 0, st>>>(W, nseg, Wq, scales, zeros);
+        rtn_quantize_flat_kernel<SYM, 128><<<blocks, 256, 0, st>>>(W, ngroups, Wq, scales, zeros);
         break;
     }
     return launch_status(cudaGetLastError());
@@ -632,13 +632,13 @@ w4_status blockwise_quantize(const float* W, int N, int K, int blocksize, int dq
     return W4_ERR_INVALID_ARG;
   const long long nb = static_cast<long long>(N) * K / 64;
   const int runs = ceil_div(nb, dq_group);
-  const size_t smem = (static_cast<size_t>(dq_group) + 288) * sizeof(float);
+  const size_t smem = (static_cast<size_t>(dq_group) + 64) * sizeof(float);
   if (mean)
     nf4_quantize_kernel<TABLE, true>
-        <<<runs, 256, smem, as_stream(stream)>>>(W, nb, dq_group, Wq, absmax_q, s2, mean);
+        <<<runs, kNf4QThreads, smem, as_stream(stream)>>>(W, nb, dq_group, Wq, absmax_q, s2, mean);
   else
     nf4_quantize_kernel<TABLE, false>
-        <<<runs, 256, smem, as_stream(stream)>>>(W, nb, dq_group, Wq, absmax_q, s2, nullptr);
+        <<<runs, kNf4QThreads, smem, as_stream(stream)>>>(W, nb, dq_group, Wq, absmax_q, s2, nullptr);
   return launch_status(cudaGetLastError());
 }
 

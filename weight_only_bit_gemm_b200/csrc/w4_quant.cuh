@@ -172,49 +172,58 @@ __device__ __forceinline__ float rint_quotient(float w, float s, float r) {
 }
 
 // Contiguous groups (no g_idx): W is N*K/G consecutive groups of G weights in
-// row-major order (K % G == 0), so the kernel works on the flat array.  A lane
-// takes one float4 (4 consecutive weights of one group), a group spans G/4
-// lanes and a warp 128 weights (a segment); each warp loads kU segments at a
-// time so that enough loads are in flight, reduces each group's max(w, 0)
-// and max(-w, 0) with shuffles inside the group's lanes, and writes 2 bytes
-// of codes per lane plus the group's scale and zero point.
+// row-major order (K % G == 0), so the kernel works on the flat array.  A warp
+// takes a chunk of 512 weights (512 / G whole groups); a group belongs to G/16
+// lanes, each holding 16 of its weights as four float4 loads (load u of lane j
+// of the group is float4 u * G/16 + j, so that every load instruction reads
+// whole 32..128-byte runs).  Each lane reduces max(w, 0) and max(-w, 0) over
+// its 16 weights, the group's lanes combine them with shuffles, and every lane
+// derives the group's scale and zero point itself and writes 2 bytes of codes
+// per float4; the group's first lane writes the scale and zero point.
 template <bool SYM, int G>
 __global__ void __launch_bounds__(256) rtn_quantize_flat_kernel(
-    const float* __restrict__ W, long long nseg, uint8_t* __restrict__ Wq,
+    const float* __restrict__ W, long long ngroups, uint8_t* __restrict__ Wq,
     uint16_t* __restrict__ scales, uint8_t* __restrict__ zeros) {
-  constexpr int kLpg = G / 4;  // lanes per group
-  constexpr int kU = 4;
+  constexpr int kLpg = G / 16;     // lanes per group
+  constexpr int kGpc = 32 / kLpg;  // groups per 512-weight chunk
   const int lane = threadIdx.x & 31;
+  const int gi = lane / kLpg, j = lane % kLpg;
   const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const long long nchunks = (ngroups + kGpc - 1) / kGpc;
+  const unsigned long long n4 = static_cast<unsigned long long>(ngroups) * (G / 4);  // float4s
   const float4* src = reinterpret_cast<const float4*>(W);
-  for (long long s0 = warp * kU; s0 < nseg; s0 += nwarps * kU) {
-    float4 v[kU];
-    const unsigned long long n4 = static_cast<unsigned long long>(nseg) * 32;  // float4 extent
+  for (long long c = warp; c < nchunks; c += nwarps) {
+    const long long grp = c * kGpc + gi;
+    const bool valid = grp < ngroups;  // whole groups only: the same for a group's lanes
+    const long long f0 = grp * (G / 4) + j;  // this lane's first float4
+    float4 v[4];
 #pragma unroll
-    for (int u = 0; u < kU; ++u)
-      v[u] = s0 + u < nseg && in_bounds((s0 + u) * 32 + lane, n4)
-                 ? __ldcs(src + (s0 + u) * 32 + lane)
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < 4; ++u)
+      v[u] = valid && in_bounds(f0 + u * kLpg, n4) ? __ldcs(src + f0 + u * kLpg)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    // max(w, 0) and max(-w, 0) without ever producing -0
+    float mx = 0.0f, nx = 0.0f;
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const long long seg = s0 + u;
-      if (seg >= nseg) break;  // the same for every lane of the warp
+    for (int u = 0; u < 4; ++u) {
       const float w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      // max(w, 0) and max(-w, 0) without ever producing -0
-      float mx = 0.0f, nx = 0.0f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         if (w[e] > mx) mx = w[e];
         if (-w[e] > nx) nx = -w[e];
       }
+    }
 #pragma unroll
-      for (int o = 1; o < kLpg; o <<= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        nx = fmaxf(nx, __shfl_xor_sync(0xffffffffu, nx, o));
-      }
-      const RtnParam p = SYM ? sym_param(mx, nx) : rtn_param(mx, nx);
-      const float r = __frcp_rn(p.sf);
+    for (int o = 1; o < kLpg; o <<= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      nx = fmaxf(nx, __shfl_xor_sync(0xffffffffu, nx, o));
+    }
+    if (!valid) continue;
+    const RtnParam p = SYM ? sym_param(mx, nx) : rtn_param(mx, nx);
+    const float r = __frcp_rn(p.sf);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
       uint32_t codes = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -222,12 +231,13 @@ __global__ void __launch_bounds__(256) rtn_quantize_flat_kernel(
         q = fminf(fmaxf(q, p.lo), 15.0f);
         codes |= static_cast<uint32_t>(q) << (4 * e);
       }
-      const long long flat = seg * 128 + lane * 4;
-      if (in_bounds(flat / 4, n4)) reinterpret_cast<uint16_t*>(Wq)[flat / 4] = static_cast<uint16_t>(codes);
-      if (lane % kLpg == 0 && in_bounds(flat / G, n4 * 4 / G)) {
-        scales[flat / G] = p.s16;
-        zeros[flat / G] = static_cast<uint8_t>(p.zp);
-      }
+      // float4 f0 + u * kLpg holds weights 4 (f0 + u * kLpg) .. + 3: code bytes 2 (f0 + ...)
+      const unsigned long long h = static_cast<unsigned long long>(f0 + u * kLpg);
+      if (in_bounds(h, n4)) reinterpret_cast<uint16_t*>(Wq)[h] = static_cast<uint16_t>(codes);
+    }
+    if (j == 0 && in_bounds(static_cast<unsigned long long>(grp), static_cast<unsigned long long>(ngroups))) {
+      scales[grp] = p.s16;
+      zeros[grp] = static_cast<uint8_t>(p.zp);
     }
   }
 }
@@ -404,29 +414,33 @@ struct LevelSearch {
   }
 };
 
-// One CTA (256 threads) per run of dq_group consecutive 64-weight blocks.
-// Codes: each warp takes pairs of blocks (half-warp per block, one float4 per
-// lane, kU pairs in flight); the block absmax is a 16-lane shuffle
-// reduction, the codes come from LevelSearch.  Then the run's constants:
+// One CTA (kNf4QThreads threads) per run of dq_group consecutive 64-weight blocks.
+// Codes: kNf4QLanes lanes per block, 64 / kNf4QLanes weights each (load u of
+// lane j is float4 u kNf4QLanes + j of the block, so that every load
+// instruction reads whole runs of 16 kNf4QLanes bytes), all of a lane's loads
+// issued at once; the block absmax is a shuffle reduction over the block's
+// lanes and the codes come from LevelSearch.  Then
+// the run's constants:
 //   MEAN false  s2 = max(a) / 255 (1 if 0), c = clamp(rint(a / s2), 0, 255) (u8);
 //   MEAN true   mean-offset: mu = fp32(fp64 sum of the run's a in block order / n),
 //               d = a - mu, s2 = max|d| / 127 (1 if 0),
 //               c = clamp(rint(d / s2), -127, 127) (int8), mean[run] = mu.
-// TABLE selects the NF4 or the FP4 codes.  Shared memory: dq_group + 288
-// floats.
+// TABLE selects the NF4 or the FP4 codes.  Shared memory: dq_group + 64 floats.
+constexpr int kNf4QThreads = 512;  // threads per CTA (a multiple of 128)
+constexpr int kNf4QCtasPerSm = 4;  // resident CTAs per SM (caps the registers)
+constexpr int kNf4QLanes = 8;       // lanes per 64-weight block (4 or 8)
 template <int TABLE, bool MEAN>
-__global__ void __launch_bounds__(256) nf4_quantize_kernel(const float* __restrict__ W,
-                                                           long long nblocks, int dq_group,
-                                                           uint8_t* __restrict__ Wq,
-                                                           uint8_t* __restrict__ absmax_q,
-                                                           float* __restrict__ s2,
-                                                           float* __restrict__ mean) {
+__global__ void __launch_bounds__(kNf4QThreads, kNf4QCtasPerSm) nf4_quantize_kernel(const float* __restrict__ W,
+                                                            long long nblocks, int dq_group,
+                                                            uint8_t* __restrict__ Wq,
+                                                            uint8_t* __restrict__ absmax_q,
+                                                            float* __restrict__ s2,
+                                                            float* __restrict__ mean) {
   using LS = LevelSearch<TABLE>;
-  constexpr int kU = 4;
   extern __shared__ float sm_q4[];
-  float* a_s = sm_q4;                  // [dq_group] block absmax, block order
-  float* red = sm_q4 + dq_group;       // [256] reduction scratch, then [256] = mean
-  float* thr = red + 264;              // [16] decision thresholds
+  float* a_s = sm_q4;             // [dq_group] block absmax, block order
+  float* red = sm_q4 + dq_group;  // [32] warp maxima, [32] the run's max, [33] its mean
+  float* thr = red + 48;          // [16] decision thresholds
   const long long run0 = static_cast<long long>(blockIdx.x) * dq_group;
   const long long left = nblocks - run0;
   const int nrun = left < dq_group ? static_cast<int>(left) : dq_group;
@@ -434,42 +448,40 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float* __restri
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = lane >> 4, l16 = lane & 15;
-  const int npairs = (nrun + 1) / 2;
+  constexpr int kL = kNf4QLanes;  // lanes per block
+  constexpr int kF = 16 / kL;     // float4 loads per lane
+  const int j = threadIdx.x % kL;
   const float4* src = reinterpret_cast<const float4*>(W);
   const unsigned long long n4 = static_cast<unsigned long long>(nblocks) * 16;
-  for (int p0 = warp; p0 < npairs; p0 += 8 * kU) {
-    float4 v[kU];
+  for (int b0 = 0; b0 < nrun; b0 += kNf4QThreads / kL) {
+    const int b = b0 + static_cast<int>(threadIdx.x) / kL;
+    const bool valid = b < nrun;  // the same for a block's lanes
+    const unsigned long long f0 = static_cast<unsigned long long>(run0 + b) * 16 + j;
+    float4 v[kF];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int b = 2 * (p0 + 8 * u) + half;
-      const unsigned long long i4 = static_cast<unsigned long long>(run0 + b) * 16 + l16;
-      v[u] = (p0 + 8 * u < npairs && b < nrun && in_bounds(i4, n4)) ? __ldcs(src + i4)
-                                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    for (int u = 0; u < kF; ++u)
+      v[u] = valid && in_bounds(f0 + kL * u, n4) ? __ldcs(src + f0 + kL * u)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    float a = 0.0f;
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      if (p0 + 8 * u >= npairs) break;  // the same for the whole warp
-      const int b = 2 * (p0 + 8 * u) + half;
+    for (int u = 0; u < kF; ++u)
+      a = fmaxf(a, fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w))));
+#pragma unroll
+    for (int o = 1; o < kL; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (!valid) continue;
+    if (j == 0) a_s[b] = a;
+    const float r = a > 0.0f ? __frcp_rn(a) : 0.0f;
+    const uint32_t zc = static_cast<uint32_t>(LS::count_below(thr, 0.0f));
+#pragma unroll
+    for (int u = 0; u < kF; ++u) {
       const float w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      float a = fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3])));
-#pragma unroll
-      for (int o = 1; o < 16; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-      if (b >= nrun) continue;
-      if (l16 == 0) a_s[b] = a;
-      const float r = a > 0.0f ? __frcp_rn(a) : 0.0f;
       uint32_t codes = 0;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t c = a > 0.0f ? LS::code(thr, w[e], a, r)
-                                    : static_cast<uint32_t>(LS::count_below(thr, 0.0f));
-        codes |= c << (4 * e);
-      }
-      const unsigned long long byte = static_cast<unsigned long long>(run0 + b) * 32 + 2 * l16;
-      if (in_bounds(byte / 2, n4))
-        reinterpret_cast<uint16_t*>(Wq)[byte / 2] =
-            static_cast<uint16_t>((codes & 0xFu) | ((codes >> 4) & 0xFu) << 4 |
-                                  ((codes >> 8) & 0xFu) << 8 | ((codes >> 12) & 0xFu) << 12);
+      for (int e = 0; e < 4; ++e)
+        codes |= (a > 0.0f ? LS::code(thr, w[e], a, r) : zc) << (4 * e);
+      // float4 f0 + kL u holds weights 4 (f0 + kL u) .. + 3: code bytes 2 (f0 + kL u) ..
+      if (in_bounds(f0 + kL * u, n4))
+        reinterpret_cast<uint16_t*>(Wq)[f0 + kL * u] = static_cast<uint16_t>(codes);
     }
   }
   __syncthreads();
@@ -480,27 +492,32 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float* __restri
     if (threadIdx.x == 0) {
       double sum = 0.0;
       for (int i = 0; i < nrun; ++i) sum += static_cast<double>(a_s[i]);
-      red[256] = static_cast<float>(sum / static_cast<double>(nrun));
+      red[33] = static_cast<float>(sum / static_cast<double>(nrun));
     }
     __syncthreads();
-    mu = red[256];
+    mu = red[33];
   }
   float key = 0.0f;
-  for (int b = threadIdx.x; b < nrun; b += 256)
+  for (int b = threadIdx.x; b < nrun; b += kNf4QThreads)
     key = fmaxf(key, MEAN ? fabsf(__fsub_rn(a_s[b], mu)) : a_s[b]);
-  red[threadIdx.x] = key;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) key = fmaxf(key, __shfl_xor_sync(0xffffffffu, key, o));
+  if (lane == 0) red[warp] = key;
   __syncthreads();
-  for (int w = 128; w > 0; w >>= 1) {
-    if (threadIdx.x < w) red[threadIdx.x] = fmaxf(red[threadIdx.x], red[threadIdx.x + w]);
-    __syncthreads();
+  if (warp == 0) {
+    key = lane < kNf4QThreads / 32 ? red[lane] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) key = fmaxf(key, __shfl_xor_sync(0xffffffffu, key, o));
+    if (lane == 0) red[32] = key;
   }
-  float sc = __fdiv_rn(red[0], MEAN ? 127.0f : 255.0f);
+  __syncthreads();
+  float sc = __fdiv_rn(red[32], MEAN ? 127.0f : 255.0f);
   if (sc == 0.0f) sc = 1.0f;
   if (threadIdx.x == 0) {
     s2[blockIdx.x] = sc;
     if constexpr (MEAN) mean[blockIdx.x] = mu;
   }
-  for (int b = threadIdx.x; b < nrun; b += 256) {
+  for (int b = threadIdx.x; b < nrun; b += kNf4QThreads) {
     const float a = a_s[b];
     uint8_t byte;
     if constexpr (MEAN) {
