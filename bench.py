@@ -53,9 +53,9 @@ def nf4_bytes(M, N, K):
 # DRAM bytes of one decode-kernel launch from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of w4_gemv_kernel.cuh).
 TRAFFIC_CAPTURE = {
-    "kernel_sha256": "4218176cac61511b085dca981eb0bef8f64c9445de3552d5b0ceea6ab48dec90",
+    "kernel_sha256": "ed31b8887930dec824e91550d9b6cf38f2bbc38667bf05f64b636fcc584136da",
     "shape": {"M": 1, "N": 12288, "K": 4096, "G": 128},
-    "dram_bytes": 26178304,
+    "dram_bytes": 26182400,
 }
 
 
@@ -815,6 +815,15 @@ def run_single(w4, args):
         gemm = w4.nf4_gemm if fmt == "nf4" else w4.fp4_gemm
         f = (lambda: gemm(X, wp, s2, N, K))
         nbytes, flops = nf4_bytes(M, N, K), 2.0 * M * N * K
+    elif fmt in ("quant", "nf4q"):
+        # the quantize kernels alone (M unused): INT4 RTN g128, or NF4 with
+        # double-quantized constants
+        wl = WL if fmt == "quant" else S.NF4_DECODE
+        W = torch.from_numpy(S.layer_w(wl, K, N)).cuda()
+        f = ((lambda W=W: w4.quantize_rtn(W, WL["G"])) if fmt == "quant"
+             else (lambda W=W: w4.nf4_quantize(W)))
+        nbytes = N * K * 4 + N * K / 2 + (N * (K // WL["G"]) * 3 if fmt == "quant" else N * K // 64)
+        flops = 0.0
     elif fmt == "gptq":
         # M = calibration tokens; act-order, G = 32 (the 13B act-order family)
         G = S.ACT_ORDER_13B["G"]
@@ -879,7 +888,8 @@ def main():
                     help="build and run one microbenchmark of weight_only_bit_gemm_b200/probes "
                          "(the measurements the kernels' design rests on) and print its table")
     ap.add_argument("--single", nargs=4, metavar=("FMT", "K", "N", "M"),
-                    help="profiling aid: run one layer call (FMT int4|nf4|fp4|awq|gptq|int8) warmup+steps times "
+                    help="profiling aid: run one layer call (FMT int4|nf4|fp4|awq|gptq|int8, or the "
+                         "quantize kernels quant|nf4q) warmup+steps times "
                          "eagerly and print its mean device time")
     args = ap.parse_args()
     if args.warmup < 3:

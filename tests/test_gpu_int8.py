@@ -66,6 +66,10 @@ INT8_CASES = [
     (7, 33, 64, 6.0, 0.05),            # tiny, ragged
     (5, 300, 512, 1e30, 0.0),          # no outliers
     (3, 128, 256, 0.0, 0.0),           # every nonzero channel an outlier
+    # tensor-core product: ~120 outlier channels gathered into shared memory
+    # for the epilogue, and 2048 (more than fit) read from global memory
+    (100, 300, 4096, 6.0, 0.03),
+    (48, 256, 2048, 0.0, 0.0),
 ]
 
 

@@ -32,6 +32,8 @@ namespace w4 {
 
 constexpr int kInt8Warps = 8;      // warps per product CTA
 constexpr int kInt8MaxNB = 4;      // token blocks of 8 per pass over the weights
+constexpr int kInt8EpiChunk = 8;   // outlier channels per step of the epilogue
+constexpr int kInt8EpiDirectM = 4; // up to this many tokens the epilogue reads global memory
 
 __device__ __forceinline__ float bf16_bits_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
@@ -62,65 +64,96 @@ __global__ void __launch_bounds__(256) int8_quantize_weights_kernel(const float*
   }
 }
 
-// One CTA per 256 input channels (thread = channel).
-__global__ void __launch_bounds__(256) int8_scan_kernel(const uint16_t* __restrict__ X, int M,
-                                                        int K, float threshold,
-                                                        uint8_t* __restrict__ flag,
-                                                        int32_t* __restrict__ list,
-                                                        int32_t* __restrict__ cnt,
-                                                        float* __restrict__ part,
-                                                        unsigned int* __restrict__ counter,
-                                                        int row_tiles) {
+// One CTA per 256 input channels, 1024 threads: warp w takes channels
+// 32 (w % 8) .. + 31 of the CTA's and the tokens m = w / 8 (mod 4), eight
+// tokens' loads at a time (independent), so a long prefill batch is read in
+// M / 32 round trips per thread.  Flags: OR over the four token groups in
+// shared memory.  The per-token maximum of the unflagged |x| over the CTA's
+// channels: a warp maximum (shuffles), then an atomic maximum of the
+// non-negative float's bits in shared memory, 256 tokens at a time.
+__global__ void __launch_bounds__(1024) int8_scan_kernel(const uint16_t* __restrict__ X, int M,
+                                                         int K, float threshold,
+                                                         uint8_t* __restrict__ flag,
+                                                         int32_t* __restrict__ list,
+                                                         int32_t* __restrict__ cnt,
+                                                         float* __restrict__ part,
+                                                         unsigned int* __restrict__ counter,
+                                                         int row_tiles) {
+  __shared__ uint8_t grp_flag[4][256];
   __shared__ int warp_cnt[8];
-  __shared__ float red[8][8];
+  __shared__ unsigned int tok_max[256];
   grid_dep_launch();
   grid_dep_wait();  // X may come from the previous kernel
   const int c = blockIdx.x, t = threadIdx.x, lane = t & 31, wid = t >> 5;
-  for (int i = c * 256 + t; i < row_tiles; i += gridDim.x * 256) counter[i] = 0u;
-  const int k = c * 256 + t;
+  const int kl = (wid & 7) * 32 + lane;  // channel within the CTA
+  const int tg = wid >> 3;               // token group
+  for (int i = c * 1024 + t; i < row_tiles; i += gridDim.x * 1024) counter[i] = 0u;
+  const int k = c * 256 + kl;
   const bool in = k < K;
-  bool o = false;
-  if (in)
-    for (int m = 0; m < M && !o; ++m)
-      o = fabsf(bf16_bits_f32(X[static_cast<size_t>(m) * K + k])) > threshold;
-  if (in) flag[k] = o ? 1 : 0;
-  // the CTA's flagged channels, ascending, in its list region
-  const unsigned bal = __ballot_sync(0xffffffffu, o);
-  if (lane == 0) warp_cnt[wid] = __popc(bal);
-  __syncthreads();
-  int before = 0, total = 0;
-#pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    before += w < wid ? warp_cnt[w] : 0;
-    total += warp_cnt[w];
-  }
-  if (o) {
-    const int pos = before + __popc(bal & ((1u << lane) - 1u));
-    if (in_bounds(static_cast<unsigned>(c * 256 + pos), static_cast<unsigned>(gridDim.x * 256)))
-      list[c * 256 + pos] = k;
-  }
-  if (t == 0) cnt[c] = total;
-  // per token, the largest unflagged |x| among the CTA's channels
-  for (int m0 = 0; m0 < M; m0 += 8) {
+  bool og = false;
+  for (int m0 = tg; m0 < M; m0 += 32) {
     float v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      v[j] = (in && !o && m0 + j < M) ? fabsf(bf16_bits_f32(X[static_cast<size_t>(m0 + j) * K + k]))
-                                      : 0.0f;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) v[j] = fmaxf(v[j], __shfl_xor_sync(0xffffffffu, v[j], off));
+      const int m = m0 + 4 * j;
+      v[j] = in && m < M ? fabsf(bf16_bits_f32(X[static_cast<size_t>(m) * K + k])) : 0.0f;
     }
-    if (lane == 0) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) red[j][wid] = v[j];
+    for (int j = 0; j < 8; ++j) og = og || v[j] > threshold;
+  }
+  grp_flag[tg][kl] = og ? 1 : 0;
+  __syncthreads();
+  const bool o = grp_flag[0][kl] | grp_flag[1][kl] | grp_flag[2][kl] | grp_flag[3][kl];
+  // the CTA's flagged channels, ascending, in its list region (token group 0)
+  unsigned bal = 0;
+  if (tg == 0) {
+    if (in) flag[k] = o ? 1 : 0;
+    bal = __ballot_sync(0xffffffffu, o);
+    if (lane == 0) warp_cnt[wid] = __popc(bal);
+  }
+  __syncthreads();
+  if (tg == 0) {
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      before += w < wid ? warp_cnt[w] : 0;
+      total += warp_cnt[w];
+    }
+    if (o) {
+      const int pos = before + __popc(bal & ((1u << lane) - 1u));
+      if (in_bounds(static_cast<unsigned>(c * 256 + pos), static_cast<unsigned>(gridDim.x * 256)))
+        list[c * 256 + pos] = k;
+    }
+    if (t == 0) cnt[c] = total;
+  }
+  // per token, the largest unflagged |x| among the CTA's channels
+  for (int mc = 0; mc < M; mc += 256) {
+    const int me = min(M, mc + 256);
+    if (t < 256) tok_max[t] = 0u;
+    __syncthreads();
+    for (int m0 = mc + tg; m0 < me; m0 += 32) {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int m = m0 + 4 * j;
+        v[j] = in && !o && m < me ? fabsf(bf16_bits_f32(X[static_cast<size_t>(m) * K + k])) : 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v[j] = fmaxf(v[j], __shfl_xor_sync(0xffffffffu, v[j], off));
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int m = m0 + 4 * j;
+          // non-negative floats order as their bits; a NaN counts as 0
+          if (m < me) atomicMax(&tok_max[m - mc], __float_as_uint(fmaxf(v[j], 0.0f)));
+        }
+      }
     }
     __syncthreads();
-    if (t < 8 && m0 + t < M) {
-      float a = red[t][0];
-#pragma unroll
-      for (int w = 1; w < 8; ++w) a = fmaxf(a, red[t][w]);
-      part[static_cast<size_t>(c) * M + m0 + t] = a;
-    }
+    if (t < me - mc) part[static_cast<size_t>(c) * M + mc + t] = __uint_as_float(tok_max[t]);
     __syncthreads();
   }
 }
@@ -209,6 +242,117 @@ struct Int8Args {  // (acc and counter are cleared by the call's first two kerne
   int M, N, K, row_tiles, slices, steps;
 };
 
+// The epilogue of row tile rt, run by the last of its work items' warps.
+__device__ __forceinline__ void int8_epilogue(const Int8Args& a, int rt, int lane) {
+  // y[m][n] = acc s_x s_w + sum over outlier channels (ascending) of
+  // x * bf16(q_w s_w), one fp32 fma per channel in ascending order.  Up to
+  // kInt8EpiDirectM tokens (at most two outputs per lane) each output's chain
+  // reads its operands from global memory (measured faster there).  Above,
+  // lane l owns outputs l + 32 j (token idx / 16, row idx % 16 of the tile);
+  // the outlier channels go kInt8EpiChunk at a time: the warp gathers their 16
+  // rows' weights bf16(q_w s_w) and the M tokens' activations into its slice
+  // of shared memory (independent loads spread over the lanes), then every
+  // lane advances its outputs' fma chains over the chunk.  The slice is kept
+  // small so that the L1 left beside it still holds the activation codes
+  // every warp streams.
+  if (a.M <= kInt8EpiDirectM) {
+    // a few outputs per lane: each lane's output straight from global memory
+    const int no = min(*a.ocount, a.K);
+    for (int idx = lane; idx < 16 * a.M; idx += 32) {
+      const int m = idx >> 4, n = rt * 16 + (idx & 15);
+      if (n >= a.N) continue;
+      const size_t o = static_cast<size_t>(m) * a.N + n;
+      const float s = a.sw[n];
+      float y = __fmul_rn(__fmul_rn(static_cast<float>(__ldcg(a.acc + o)), a.sx[m]), s);
+      for (int i = 0; i < no; ++i) {
+        const int k = a.olist[i];
+        if (!in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K))) continue;
+        const float w16 = __bfloat162float(__float2bfloat16_rn(
+            __fmul_rn(static_cast<float>(a.qw[static_cast<size_t>(n) * a.K + k]), s)));
+        y = fmaf(bf16_bits_f32(a.X[static_cast<size_t>(m) * a.K + k]), w16, y);
+      }
+      a.Y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+    }
+    return;
+  }
+  extern __shared__ float i8_epi[];
+  const int per = 16 + a.M;  // rows, then tokens
+  float* wsm = i8_epi + (threadIdx.x >> 5) * (per * kInt8EpiChunk + kInt8EpiChunk);
+  float* xsm = wsm + 16 * kInt8EpiChunk;
+  float* okm = wsm + per * kInt8EpiChunk;  // 1: the channel is inside K
+  const int no = min(*a.ocount, a.K);
+  const int nout = 16 * a.M;  // at most 512: 16 outputs per lane
+  float y[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int idx = lane + 32 * j;
+    y[j] = 0.0f;
+    if (idx < nout) {
+      const int m = idx >> 4, n = rt * 16 + (idx & 15);
+      if (n < a.N)
+        y[j] = __fmul_rn(__fmul_rn(static_cast<float>(__ldcg(a.acc + static_cast<size_t>(m) * a.N + n)),
+                                   a.sx[m]),
+                         a.sw[n]);
+    }
+  }
+  static_assert(32 % kInt8EpiChunk == 0, "a lane keeps one channel of the chunk");
+  constexpr int kMaxV = (16 + 32) * kInt8EpiChunk / 32;  // values a lane gathers at most
+  for (int c0 = 0; c0 < no; c0 += kInt8EpiChunk) {
+    // lane l gathers channel l % chunk of the chunk for rows / tokens
+    // l / chunk + (32 / chunk) t: the channel index once, then all its loads
+    // at once
+    const int ch = lane % kInt8EpiChunk;
+    int k = 0;
+    bool ok = false;
+    if (c0 + ch < no) {
+      k = a.olist[c0 + ch];
+      ok = in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K));
+    }
+    if (lane < kInt8EpiChunk) okm[lane] = ok ? 1.0f : 0.0f;
+    float vals[kMaxV];
+#pragma unroll
+    for (int t = 0; t < kMaxV; ++t) {
+      const int v = lane + 32 * t, rr = v / kInt8EpiChunk;
+      vals[t] = 0.0f;
+      if (ok && rr < per) {
+        if (rr < 16) {
+          const int n = rt * 16 + rr;
+          if (n < a.N)
+            vals[t] = __bfloat162float(__float2bfloat16_rn(
+                __fmul_rn(static_cast<float>(a.qw[static_cast<size_t>(n) * a.K + k]), a.sw[n])));
+        } else {
+          vals[t] = bf16_bits_f32(a.X[static_cast<size_t>(rr - 16) * a.K + k]);
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kMaxV; ++t) {
+      const int v = lane + 32 * t;
+      if (v < per * kInt8EpiChunk) wsm[v] = vals[t];  // rows, then tokens (xsm)
+    }
+    __syncwarp();
+    const int cn = min(kInt8EpiChunk, no - c0);
+    for (int ii = 0; ii < cn; ++ii) {
+      if (okm[ii] == 0.0f) continue;  // a channel outside K (bounds-checked build)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int idx = lane + 32 * j;
+        if (idx < nout)
+          y[j] = fmaf(xsm[(idx >> 4) * kInt8EpiChunk + ii], wsm[(idx & 15) * kInt8EpiChunk + ii], y[j]);
+      }
+    }
+    __syncwarp();
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int idx = lane + 32 * j;
+    if (idx < nout) {
+      const int m = idx >> 4, n = rt * 16 + (idx & 15);
+      if (n < a.N) a.Y[static_cast<size_t>(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y[j]));
+    }
+  }
+}
+
 // acc[m][n] += sum over the warp's K slice of q_x[m][k] q_w[n][k].
 // Work item = (16-row tile, slice of `steps` 64-channel steps); lane (g, u)
 // = (lane / 4, lane % 4) loads 16 consecutive bytes of weight rows g and
@@ -218,7 +362,7 @@ struct Int8Args {  // (acc and counter are cleared by the call's first two kerne
 // product.  Tokens in passes of up to kInt8MaxNB blocks of 8.  The last of a
 // row tile's work items to finish (counted after a release fence on the
 // tile's counter) applies the epilogue to the tile's outputs.
-__global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(const Int8Args a) {
+__global__ void __launch_bounds__(kInt8Warps * 32, 3) int8_product_kernel(const Int8Args a) {
   grid_dep_launch();
   const int lane = threadIdx.x & 31, g = lane >> 2, u = lane & 3;
   const long long item = static_cast<long long>(blockIdx.x) * kInt8Warps + (threadIdx.x >> 5);
@@ -284,23 +428,7 @@ __global__ void __launch_bounds__(kInt8Warps * 32) int8_product_kernel(const Int
   prev = __shfl_sync(0xffffffffu, prev, 0);
   __syncwarp();
   if (prev != static_cast<unsigned>(a.slices - 1)) return;
-  // y[m][n] = acc s_x s_w + sum over outlier channels (ascending) of x * bf16(q_w s_w)
-  const int no = min(*a.ocount, a.K);
-  for (int idx = lane; idx < 16 * a.M; idx += 32) {
-    const int m = idx >> 4, n = rt * 16 + (idx & 15);
-    if (n >= a.N) continue;
-    const size_t o = static_cast<size_t>(m) * a.N + n;
-    const float s = a.sw[n];
-    float y = __fmul_rn(__fmul_rn(static_cast<float>(__ldcg(a.acc + o)), a.sx[m]), s);
-    for (int i = 0; i < no; ++i) {
-      const int k = a.olist[i];
-      if (!in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K))) continue;
-      const float w16 = __bfloat162float(__float2bfloat16_rn(
-          __fmul_rn(static_cast<float>(a.qw[static_cast<size_t>(n) * a.K + k]), s)));
-      y = fmaf(bf16_bits_f32(a.X[static_cast<size_t>(m) * a.K + k]), w16, y);
-    }
-    a.Y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-  }
+  int8_epilogue(a, rt, lane);
 }
 
 }  // namespace w4

@@ -33,7 +33,8 @@ struct I8Cfg {
   static constexpr int kXStage = MT * 128;   // activation tile bytes per stage
   static constexpr int kThreads = 64 + 4 * 32;
   static constexpr int kTmemCols = MT <= 32 ? 32 : MT <= 64 ? 64 : MT <= 128 ? 128 : 256;
-  static constexpr int kSmemBytes = 1024 + STAGES * (kWStage + kXStage) + (2 * STAGES + 4) * 8 + 16;
+  static constexpr int kRingBytes = STAGES * (kWStage + kXStage);
+  static constexpr int kSmemBytes = 1024 + kRingBytes + (2 * STAGES + 5) * 8 + 16;
   static_assert(MT % 16 == 0 && MT >= 16 && MT <= 256, "MMA N for M = 128");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -85,7 +86,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   uint64_t* accf = empty + C::STAGES;              // accumulator ready (commit)
   uint64_t* epi1 = accf + 1;                       // partials stored (4 warps)
   uint64_t* epi2 = epi1 + 1;                       // last-arrival known (1)
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi2 + 1);
+  uint64_t* epi3 = epi2 + 1;                       // outlier operands gathered (4 warps)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi3 + 1);
   int* last_flag = reinterpret_cast<int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -107,6 +109,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     mbar_init(accf, 1);
     mbar_init(epi1, 4);
     mbar_init(epi2, 1);
+    mbar_init(epi3, 4);
     fence_barrier_init();
     grid_dep_launch();
   }
@@ -177,19 +180,61 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       grid_dep_wait();  // s_x, the outlier list, Y and the workspace
       const float swn = n < a.N ? a.sw[n] : 0.0f;
       const int no = min(*a.ocount, a.K);
+      // The outlier operands, gathered once into the (now idle) operand ring
+      // when they fit: the tile's tokens' activations xo[token][i] and this
+      // thread's row's 16-bit weights wo[row][i] = bf16(q_w s_w) (row stride
+      // odd, so that the lanes' rows fall in different banks); otherwise each
+      // output reads them from global memory.  Either way one fp32 fma per
+      // outlier channel in ascending order.  (An outlier channel outside K,
+      // bounds-checked build only, contributes nothing.)
+      const int wstr = no | 1;
+      const bool gathered =
+          no > 0 && (static_cast<long long>(C::MT) * no + 128ll * wstr) * 4 <= C::kRingBytes;
+      float* xo = reinterpret_cast<float*>(ws);
+      float* wo = xo + C::MT * no;
+      bool ready = false;
+      auto gather = [&]() {
+        const int e = threadIdx.x - 64;  // epilogue thread 0..127
+        for (int i = 0; i < no; ++i) {
+          const int k = a.olist[i];
+          const bool ok = in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K));
+          for (int ml = e; ml < C::MT; ml += 128) {
+            const int m = mtile * C::MT + ml;
+            xo[ml * no + i] = ok && m < a.M ? bf16_bits_f32(a.X[static_cast<size_t>(m) * a.K + k]) : 0.0f;
+          }
+          wo[row * wstr + i] =
+              ok && n < a.N ? __bfloat162float(__float2bfloat16_rn(
+                                  __fmul_rn(static_cast<float>(a.qw[static_cast<size_t>(n) * a.K + k]), swn)))
+                            : 0.0f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi3);
+        ready = __all_sync(0xffffffffu, mbar_wait(epi3, 0));
+      };
       auto finish = [&](int m, int v) {
         if (m >= a.M || n >= a.N) return;
         float y = __fmul_rn(__fmul_rn(static_cast<float>(v), a.sx[m]), swn);
-        for (int i = 0; i < no; ++i) {
-          const int k = a.olist[i];
-          if (!in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K))) continue;
-          const float w16 = __bfloat162float(__float2bfloat16_rn(
-              __fmul_rn(static_cast<float>(a.qw[static_cast<size_t>(n) * a.K + k]), swn)));
-          y = fmaf(bf16_bits_f32(a.X[static_cast<size_t>(m) * a.K + k]), w16, y);
+        if (ready) {
+          const float* xr = xo + (m - mtile * C::MT) * no;
+          const float* wr = wo + row * wstr;
+          for (int i = 0; i < no; ++i) {
+            if (kChecked && !(static_cast<unsigned int>(a.olist[i]) < static_cast<unsigned int>(a.K)))
+              continue;
+            y = fmaf(xr[i], wr[i], y);
+          }
+        } else {
+          for (int i = 0; i < no; ++i) {
+            const int k = a.olist[i];
+            if (!in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K))) continue;
+            const float w16 = __bfloat162float(__float2bfloat16_rn(
+                __fmul_rn(static_cast<float>(a.qw[static_cast<size_t>(n) * a.K + k]), swn)));
+            y = fmaf(bf16_bits_f32(a.X[static_cast<size_t>(m) * a.K + k]), w16, y);
+          }
         }
         a.Y[static_cast<size_t>(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
       };
       int* part = a.partial + (static_cast<size_t>(tile_id) * a.splits + split) * C::MT * kI8Rows;
+      if (a.splits == 1 && gathered) gather();
 #pragma unroll 1
       for (int cb = 0; cb < C::MT; cb += 8) {
         uint32_t v[8];
@@ -223,17 +268,30 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         }
         if (__all_sync(0xffffffffu, mbar_wait(epi2, 0)) && *last_flag) {
           __threadfence();
+          if (gathered) gather();
           const int* base = a.partial + static_cast<size_t>(tile_id) * a.splits * C::MT * kI8Rows;
+          // 8 columns of 4 K ranges at a time: 32 loads in flight per L2 round
+          // trip (exact integer sums, so the order is free)
+          constexpr int kSu = 4;
 #pragma unroll 1
           for (int c0 = 0; c0 < C::MT; c0 += 8) {
             int acc[8] = {};
-            for (int sp = 0; sp < a.splits; ++sp) {
-              const int* src = base + (static_cast<size_t>(sp) * C::MT + c0) * kI8Rows + row;
-              if (!in_bounds(static_cast<unsigned long long>(src - a.partial) + 7 * kI8Rows,
-                             a.partial_count))
-                continue;
+#pragma unroll 1
+            for (int sp0 = 0; sp0 < a.splits; sp0 += kSu) {
+              int v[kSu][8];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) acc[j] += __ldcg(src + j * kI8Rows);
+              for (int u = 0; u < kSu; ++u) {
+                const int* src = base + (static_cast<size_t>(sp0 + u) * C::MT + c0) * kI8Rows + row;
+                const bool ok = sp0 + u < a.splits &&
+                                in_bounds(static_cast<unsigned long long>(src - a.partial) + 7 * kI8Rows,
+                                          a.partial_count);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[u][j] = ok ? __ldcg(src + j * kI8Rows) : 0;
+              }
+#pragma unroll
+              for (int u = 0; u < kSu; ++u)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] += v[u][j];
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j) finish(mtile * C::MT + c0 + j, acc[j]);

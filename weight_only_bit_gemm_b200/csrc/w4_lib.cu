@@ -341,12 +341,26 @@ I8Plan int8_tc_plan(int M, int N, int K) {
   p.tiles_m = (M + p.MT - 1) / p.MT;
   p.KS = (K + 127) / 128;
   const long long tiles = static_cast<long long>(p.tiles_n) * p.tiles_m;
-  // split K until the tiles fill the SMs (at most 16 ways, 4 stages each)
-  long long s = (148 + tiles - 1) / tiles;
-  s = std::min<long long>(s, std::max(1, p.KS / 4));
-  s = std::min<long long>(s, 16);
-  if (tiles > 65536) s = 1;
-  p.splits = static_cast<int>(std::max<long long>(1, s));
+  // K split by a cost model over the SMs, in stages of 4 MMAs: per CTA the
+  // prologue and epilogue count 1.5 stages, a split tile's round trip at
+  // least 12 more, and more when the last CTA's reduction needs more than
+  // 8 L2 round trips (MT / 8 column chunks times one per 4 K ranges, about
+  // 1.2 stages each); at most 16 ranges of at least 4 stages
+  const long long sms = sm_count();
+  const long long smax =
+      tiles > 65536 ? 1 : std::min<long long>(16, std::max<long long>(1, p.KS / 4));
+  double best = 1e30;
+  p.splits = 1;
+  for (long long s = 1; s <= smax; ++s) {
+    const double rounds = static_cast<double>(p.MT / 8) * static_cast<double>((s + 3) / 4);
+    const double rt = s > 1 ? std::max(12.0, 4.0 + 1.2 * rounds) : 0.0;
+    const double cost = static_cast<double>((tiles * s + sms - 1) / sms) *
+                        (static_cast<double>((p.KS + s - 1) / s) + 1.5 + rt);
+    if (cost < best - 1e-9) {
+      best = cost;
+      p.splits = static_cast<int>(s);
+    }
+  }
   return p;
 }
 
@@ -475,11 +489,12 @@ w4_status llm_int8_gemm(const uint16_t* X, const int8_t* qw, const float* sw, in
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cfg.gridDim = dim3(l.nscan);
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(1024);
   cudaError_t e = cudaLaunchKernelEx(&cfg, int8_scan_kernel, X, M, K, threshold, flag, list, cnt,
                                      part, a.counter, l.counters);
   if (e == cudaSuccess) {
     cfg.gridDim = dim3(M, ceil_div(K, 2048));
+    cfg.blockDim = dim3(256);
     e = cudaLaunchKernelEx(&cfg, int8_quantize_x_kernel, X, static_cast<const uint8_t*>(flag),
                            static_cast<const float*>(part), static_cast<const int32_t*>(list),
                            static_cast<const int32_t*>(cnt), l.nscan, M, K,
@@ -522,6 +537,12 @@ w4_status llm_int8_gemm(const uint16_t* X, const int8_t* qw, const float* sw, in
   if (e == cudaSuccess) {
     cfg.gridDim = dim3(static_cast<unsigned>((items + kInt8Warps - 1) / kInt8Warps));
     cfg.blockDim = dim3(kInt8Warps * 32);
+    // the epilogue's per-warp slice: one chunk of outlier channels for 16
+    // rows and M tokens, and the chunk's in-bounds flags
+    cfg.dynamicSmemBytes =
+        M <= kInt8EpiDirectM
+            ? 0
+            : static_cast<size_t>(kInt8Warps) * ((16 + M) * kInt8EpiChunk + kInt8EpiChunk) * sizeof(float);
     e = cudaLaunchKernelEx(&cfg, int8_product_kernel, a);
   }
   return launch_status(e);
