@@ -120,6 +120,40 @@ def test_blockwise_quantize_dq_group_bit_exact(w4, table, N, K, dq):
     assert np.array_equal(host_u16(dq_dev(Wq, c, s2, dq)), odq(Wq_r, c_r, s2_r, 64, dq))
 
 
+@pytest.mark.parametrize("table", ["nf4", "fp4"])
+def test_blockwise_codes_at_decision_thresholds(w4, table):
+    # weights whose quotient w / absmax falls on a decision threshold or a few
+    # ulps to either side (the codes' exact-division path), for several block
+    # scales, both signs
+    mids = O.nf4_midpoints() if table == "nf4" else O.fp4_midpoints()
+    vals = []
+    for t in mids.astype(np.float32):
+        for sgn in ((1.0, -1.0) if table == "fp4" else (1.0,)):
+            v = t
+            for _ in range(2):
+                v = np.nextafter(v, np.float32(-np.inf))
+            for _ in range(5):                            # t - 2 ulps .. t + 2 ulps
+                vals.append(np.float32(sgn) * v)
+                v = np.nextafter(v, np.float32(np.inf))
+    vals = np.array(vals, np.float32)
+    rows = []
+    for a in (1.0, 0.7, 0.013, 3.1e-5, 1234.5):
+        a = np.float32(a)
+        body = (vals * a).astype(np.float32)              # w / a rounds to within ulps of vals
+        body = body[np.abs(body) <= a]
+        blk = np.concatenate([[a], body])                 # a: the absmax of every block
+        blk = np.resize(blk, ((blk.size + 127) // 128) * 128).astype(np.float32)
+        rows.append(blk)
+    W = np.ascontiguousarray(np.concatenate(rows).reshape(-1, 128).astype(np.float32))
+    oq = O.nf4_quantize if table == "nf4" else O.fp4_quantize
+    Wq_r, c_r, s2_r = oq(W)
+    Wq, c, s2 = (w4.nf4_quantize if table == "nf4" else w4.fp4_quantize)(dev(W))
+    status_ok(w4)
+    assert np.array_equal(Wq.cpu().numpy(), Wq_r)
+    assert np.array_equal(c.cpu().numpy(), c_r)
+    assert np.array_equal(s2.cpu().numpy().view(np.uint32), s2_r.view(np.uint32))
+
+
 # ----------------------------------------------------------------- prepack
 
 @pytest.mark.parametrize("N,K,G,act", [(300, 320, 64, False), (256, 1024, 32, True),

@@ -653,7 +653,7 @@ w4_status blockwise_quantize(const float* W, int N, int K, int blocksize, int dq
     return W4_ERR_INVALID_ARG;
   const long long nb = static_cast<long long>(N) * K / 64;
   const int runs = ceil_div(nb, dq_group);
-  const size_t smem = (static_cast<size_t>(dq_group) + 64) * sizeof(float);
+  const size_t smem = (512 + static_cast<size_t>(dq_group) + 64) * sizeof(float);
   if (mean)
     nf4_quantize_kernel<TABLE, true>
         <<<runs, kNf4QThreads, smem, as_stream(stream)>>>(W, nb, dq_group, Wq, absmax_q, s2, mean);

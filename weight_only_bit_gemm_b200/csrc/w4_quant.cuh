@@ -374,7 +374,8 @@ __device__ __forceinline__ float level_value(int table, int i) {
 
 // Decision thresholds of a block-wise table in shared memory, padded with
 // +inf to a power of two: NF4 the 15 midpoints t_i (code = #{i : v > t_i}),
-// FP4 the 7 magnitude midpoints (magnitude code = #{i : |v| > t_i}).
+// FP4 the 7 magnitude midpoints (magnitude code = #{i : |v| > t_i}); the
+// count by binary search (the exact-division path of LevelBuckets::code).
 template <int TABLE>
 struct LevelSearch {
   static constexpr int kSteps = TABLE == kTableFp4 ? 3 : 4;  // 8 or 16 entries
@@ -393,21 +394,61 @@ struct LevelSearch {
       if (t[q + step - 1] < x) q += step;
     return q;
   }
-  // The code of v = w / a (a > 0, r = RN(1/a)): from t = RN(w r) when t is
-  // further than |t| 2^-20 from the thresholds around it (then t, the exact
-  // quotient and RN(w / a) lie on the same side of every threshold: they are
-  // within |w/a| 2^-23 of each other), else from the IEEE division.
-  static __device__ __forceinline__ uint32_t code(const float* t, float w, float a, float r) {
+};
+
+// The code of v = w / a (a > 0, r = RN(1/a)): from t = RN(w r) when t is
+// further than |t| 2^-20 from the thresholds around it (then t, the exact
+// quotient and RN(w / a) lie on the same side of every threshold: they are
+// within |w/a| 2^-23 of each other), else from the IEEE division.  The
+// decision uses a bucket table rather than a search over the thresholds: the
+// range of x (NF4: [-1, 1], FP4: |x| in [0, 1]) cut into buckets 1/64 (NF4)
+// or 1/128 (FP4) wide, bucket b = round(x S + O) taken from the low mantissa
+// bits of one fused multiply-add with a 1.5 * 2^23 offset.  No bucket holds
+// more than one threshold, and every threshold lies at least 7e-4 from a
+// bucket edge (checked for both tables, far above the 2^-20 |x| margin), so
+// #{i : x > t_i} = (thresholds below the bucket) + (x > the bucket's
+// threshold), and the margin test needs only the bucket's threshold: the
+// others are further from x than its bucket edges.  Entry b = {the bucket's
+// threshold (+inf if none), the count below the bucket}; 256 entries so that
+// any mantissa bits index inside.  An infinite or NaN t (a subnormal absmax
+// overflows 1/a) fails the margin test and takes the IEEE division.
+template <int TABLE>
+struct LevelBuckets {
+  static constexpr float kScale = TABLE == kTableFp4 ? 128.0f : 64.0f;
+  static constexpr float kOffset = TABLE == kTableFp4 ? 0.0f : 64.0f;
+  static constexpr int kUsed = 129;  // buckets 0..128 cover the range
+  // thr: LevelSearch<TABLE>'s thresholds in shared memory (built first)
+  static __device__ void build(float2* bk, const float* thr) {
+    using LS = LevelSearch<TABLE>;
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+      float tau = __int_as_float(0x7f800000);
+      int below = LS::kEntries - 1;  // unused entries: +inf (no decision made here)
+      if (b < kUsed) {
+        const float lo = (static_cast<float>(b) - 0.5f - kOffset) / kScale;
+        const float hi = (static_cast<float>(b) + 0.5f - kOffset) / kScale;
+        below = 0;
+        for (int i = 0; i < LS::kEntries; ++i) {
+          const float t = thr[i];
+          if (t < lo) ++below;
+          else if (t < hi) tau = t;
+        }
+      }
+      bk[b] = make_float2(tau, __int_as_float(below));
+    }
+  }
+  static __device__ __forceinline__ uint32_t code(const float2* bk, const float* thr, float w,
+                                                  float a, float r) {
+    using LS = LevelSearch<TABLE>;
     const float x = __fmul_rn(w, r);
     const float ax = TABLE == kTableFp4 ? fabsf(x) : x;
-    int q = count_below(t, ax);
-    const float lo = q > 0 ? t[q - 1] : __int_as_float(0xff800000);
-    const float hi = t[q];
-    const float thr = __fmaf_rn(fabsf(x), 0x1p-20f, 0x1p-60f);
+    const float y = __fmaf_rn(ax, kScale, 12582912.0f + kOffset);
+    const float2 e = bk[__float_as_uint(y) & 0xFFu];
+    int q = __float_as_int(e.y) + (ax > e.x ? 1 : 0);
+    const float m = __fmaf_rn(fabsf(x), 0x1p-20f, 0x1p-60f);
     float v = x;
-    if (!(__fsub_rn(ax, lo) > thr && __fsub_rn(hi, ax) > thr)) {
+    if (!(fabsf(__fsub_rn(ax, e.x)) > m)) {
       v = __fdiv_rn(w, a);
-      q = count_below(t, TABLE == kTableFp4 ? fabsf(v) : v);
+      q = LS::count_below(thr, TABLE == kTableFp4 ? fabsf(v) : v);
     }
     if (TABLE == kTableFp4) return (v < 0.0f && q != 0) ? (static_cast<uint32_t>(q) | 8u) : q;
     return static_cast<uint32_t>(q);
@@ -419,13 +460,14 @@ struct LevelSearch {
 // lane j is float4 u kNf4QLanes + j of the block, so that every load
 // instruction reads whole runs of 16 kNf4QLanes bytes), all of a lane's loads
 // issued at once; the block absmax is a shuffle reduction over the block's
-// lanes and the codes come from LevelSearch.  Then
+// lanes and the codes come from LevelBuckets.  Then
 // the run's constants:
 //   MEAN false  s2 = max(a) / 255 (1 if 0), c = clamp(rint(a / s2), 0, 255) (u8);
 //   MEAN true   mean-offset: mu = fp32(fp64 sum of the run's a in block order / n),
 //               d = a - mu, s2 = max|d| / 127 (1 if 0),
 //               c = clamp(rint(d / s2), -127, 127) (int8), mean[run] = mu.
-// TABLE selects the NF4 or the FP4 codes.  Shared memory: dq_group + 64 floats.
+// TABLE selects the NF4 or the FP4 codes.  Shared memory: 2 KB of level
+// buckets, then dq_group + 64 floats.
 constexpr int kNf4QThreads = 512;  // threads per CTA (a multiple of 128)
 constexpr int kNf4QCtasPerSm = 4;  // resident CTAs per SM (caps the registers)
 constexpr int kNf4QLanes = 8;       // lanes per 64-weight block (4 or 8)
@@ -437,14 +479,18 @@ __global__ void __launch_bounds__(kNf4QThreads, kNf4QCtasPerSm) nf4_quantize_ker
                                                             float* __restrict__ s2,
                                                             float* __restrict__ mean) {
   using LS = LevelSearch<TABLE>;
+  using LB = LevelBuckets<TABLE>;
   extern __shared__ float sm_q4[];
-  float* a_s = sm_q4;             // [dq_group] block absmax, block order
-  float* red = sm_q4 + dq_group;  // [32] warp maxima, [32] the run's max, [33] its mean
+  float2* bk = reinterpret_cast<float2*>(sm_q4);  // [256] level buckets
+  float* a_s = sm_q4 + 512;       // [dq_group] block absmax, block order
+  float* red = a_s + dq_group;    // [32] warp maxima, [32] the run's max, [33] its mean
   float* thr = red + 48;          // [16] decision thresholds
   const long long run0 = static_cast<long long>(blockIdx.x) * dq_group;
   const long long left = nblocks - run0;
   const int nrun = left < dq_group ? static_cast<int>(left) : dq_group;
   if (threadIdx.x < LS::kEntries) thr[threadIdx.x] = LS::threshold(threadIdx.x);
+  __syncthreads();
+  LB::build(bk, thr);
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -478,7 +524,7 @@ __global__ void __launch_bounds__(kNf4QThreads, kNf4QCtasPerSm) nf4_quantize_ker
       uint32_t codes = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        codes |= (a > 0.0f ? LS::code(thr, w[e], a, r) : zc) << (4 * e);
+        codes |= (a > 0.0f ? LB::code(bk, thr, w[e], a, r) : zc) << (4 * e);
       // float4 f0 + kL u holds weights 4 (f0 + kL u) .. + 3: code bytes 2 (f0 + kL u) ..
       if (in_bounds(f0 + kL * u, n4))
         reinterpret_cast<uint16_t*>(Wq)[f0 + kL * u] = static_cast<uint16_t>(codes);
