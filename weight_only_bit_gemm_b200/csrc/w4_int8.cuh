@@ -34,6 +34,8 @@ constexpr int kInt8Warps = 8;      // warps per product CTA
 constexpr int kInt8MaxNB = 4;      // token blocks of 8 per pass over the weights
 constexpr int kInt8EpiChunk = 8;   // outlier channels per step of the epilogue
 constexpr int kInt8EpiDirectM = 4; // up to this many tokens the epilogue reads global memory
+constexpr int kInt8StepsAhead = 2; // 64-channel weight steps loaded together per warp
+constexpr int kInt8CtasPerSm = 3;  // resident product CTAs per SM (caps the registers)
 
 __device__ __forceinline__ float bf16_bits_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
@@ -362,7 +364,7 @@ __device__ __forceinline__ void int8_epilogue(const Int8Args& a, int rt, int lan
 // product.  Tokens in passes of up to kInt8MaxNB blocks of 8.  The last of a
 // row tile's work items to finish (counted after a release fence on the
 // tile's counter) applies the epilogue to the tile's outputs.
-__global__ void __launch_bounds__(kInt8Warps * 32, 3) int8_product_kernel(const Int8Args a) {
+__global__ void __launch_bounds__(kInt8Warps * 32, kInt8CtasPerSm) int8_product_kernel(const Int8Args a) {
   grid_dep_launch();
   const int lane = threadIdx.x & 31, g = lane >> 2, u = lane & 3;
   const long long item = static_cast<long long>(blockIdx.x) * kInt8Warps + (threadIdx.x >> 5);
@@ -376,34 +378,45 @@ __global__ void __launch_bounds__(kInt8Warps * 32, 3) int8_product_kernel(const 
   const int kbeg = sl * a.steps * 64;
   const int kend = min(a.K, kbeg + a.steps * 64);
   const int NB = (a.M + 7) / 8;
-  // the first step's weights do not depend on the previous kernels
-  uint4 wa0 = make_uint4(0u, 0u, 0u, 0u), wb0 = make_uint4(0u, 0u, 0u, 0u);
-  if (kbeg < kend && in_bounds(static_cast<unsigned int>(kbeg + 16 * u + 15),
-                               static_cast<unsigned int>(a.K))) {
-    if (r0 < a.N) wa0 = *reinterpret_cast<const uint4*>(a.qw + static_cast<size_t>(r0) * a.K + kbeg + 16 * u);
-    if (r1 < a.N) wb0 = *reinterpret_cast<const uint4*>(a.qw + static_cast<size_t>(r1) * a.K + kbeg + 16 * u);
-  }
+  // weights of kInt8StepsAhead 64-channel steps requested together (the
+  // first batch before the launch dependency: weights do not depend on the
+  // previous kernels), so that enough bytes are in flight to cover the HBM
+  // latency with one wave of warps
+  constexpr int kU = kInt8StepsAhead;
+  uint4 wa[kU], wb[kU];
+  auto load_batch = [&](int k0) {
+#pragma unroll
+    for (int st = 0; st < kU; ++st) {
+      const int kk = k0 + 64 * st + 16 * u;
+      wa[st] = make_uint4(0u, 0u, 0u, 0u);
+      wb[st] = make_uint4(0u, 0u, 0u, 0u);
+      if (k0 + 64 * st < kend &&
+          in_bounds(static_cast<unsigned int>(kk + 15), static_cast<unsigned int>(a.K))) {
+        if (r0 < a.N) wa[st] = *reinterpret_cast<const uint4*>(a.qw + static_cast<size_t>(r0) * a.K + kk);
+        if (r1 < a.N) wb[st] = *reinterpret_cast<const uint4*>(a.qw + static_cast<size_t>(r1) * a.K + kk);
+      }
+    }
+  };
+  load_batch(kbeg);
   grid_dep_wait();  // q_x, s_x and the outlier list come from the previous kernels
   for (int tb0 = 0; tb0 < NB; tb0 += kInt8MaxNB) {
     int d[kInt8MaxNB][4] = {};
-    for (int k0 = kbeg; k0 < kend; k0 += 64) {
-      const int kk = k0 + 16 * u;
-      if (!in_bounds(static_cast<unsigned int>(kk + 15), static_cast<unsigned int>(a.K))) continue;
-      uint4 wa = wa0, wb = wb0;
-      if (k0 != kbeg || tb0 != 0) {
-        wa = make_uint4(0u, 0u, 0u, 0u);
-        wb = make_uint4(0u, 0u, 0u, 0u);
-        if (r0 < a.N) wa = *reinterpret_cast<const uint4*>(a.qw + static_cast<size_t>(r0) * a.K + kk);
-        if (r1 < a.N) wb = *reinterpret_cast<const uint4*>(a.qw + static_cast<size_t>(r1) * a.K + kk);
-      }
+    for (int k0 = kbeg; k0 < kend; k0 += 64 * kU) {
+      if (k0 != kbeg || tb0 != 0) load_batch(k0);
 #pragma unroll
-      for (int j = 0; j < kInt8MaxNB; ++j) {
-        const int tok = (tb0 + j) * 8 + g;
-        if (tb0 + j >= NB) break;
-        uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-        if (tok < a.M) xv = *reinterpret_cast<const uint4*>(a.qx + static_cast<size_t>(tok) * a.K + kk);
-        mma_s8_16832(d[j], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
-        mma_s8_16832(d[j], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
+      for (int st = 0; st < kU; ++st) {
+        if (k0 + 64 * st >= kend) break;  // the same for the whole warp
+        const int kk = k0 + 64 * st + 16 * u;
+#pragma unroll
+        for (int j = 0; j < kInt8MaxNB; ++j) {
+          const int tok = (tb0 + j) * 8 + g;
+          if (tb0 + j >= NB) break;
+          uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+          if (tok < a.M && in_bounds(static_cast<unsigned int>(kk + 15), static_cast<unsigned int>(a.K)))
+            xv = *reinterpret_cast<const uint4*>(a.qx + static_cast<size_t>(tok) * a.K + kk);
+          mma_s8_16832(d[j], wa[st].x, wb[st].x, wa[st].y, wb[st].y, xv.x, xv.y);
+          mma_s8_16832(d[j], wa[st].z, wb[st].z, wa[st].w, wb[st].w, xv.z, xv.w);
+        }
       }
     }
 #pragma unroll

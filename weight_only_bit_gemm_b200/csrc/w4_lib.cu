@@ -472,11 +472,12 @@ w4_status llm_int8_gemm(const uint16_t* X, const int8_t* qw, const float* sw, in
   a.M = M;
   a.N = N;
   a.K = K;
-  // work items: (16-row tile, K slice), about 24 warps per SM
+  // work items: (16-row tile, K slice), one wave of warps (kInt8CtasPerSm
+  // CTAs of kInt8Warps per SM)
   a.row_tiles = ceil_div(N, 16);
   const int steps_total = K / 64;
-  const int target = sm_count() * 24;
-  a.slices = std::min(steps_total, std::max(1, ceil_div(target, a.row_tiles)));
+  const int target = sm_count() * kInt8Warps * kInt8CtasPerSm;
+  a.slices = std::min(steps_total, std::max(1, target / a.row_tiles));
   a.steps = ceil_div(steps_total, a.slices);
   a.slices = ceil_div(steps_total, a.steps);
   const long long items = static_cast<long long>(a.row_tiles) * a.slices;
