@@ -6,7 +6,7 @@
 // go through a 16-bit product, the others through INT8, and the two results
 // are added); "【推理与部署篇05】模型量化部署深度对比" §6.1: llm_int8_threshold 6.0,
 // no 16-bit copy of the weights.  Per call, three launches:
-//   scan      one CTA per 256 input channels: flag[k] = |x[m,k]| > threshold
+//   scan      one CTA per 32 input channels: flag[k] = |x[m,k]| > threshold
 //             for some token m; the CTA's flagged channels in ascending
 //             order in its own list region; per token the largest unflagged
 //             |x| of the CTA's channels (a partial maximum);
@@ -32,6 +32,7 @@ namespace w4 {
 
 constexpr int kInt8Warps = 8;      // warps per product CTA
 constexpr int kInt8MaxNB = 4;      // token blocks of 8 per pass over the weights
+constexpr int kInt8ScanCh = 32;    // input channels per outlier-scan CTA
 constexpr int kInt8EpiChunk = 8;   // outlier channels per step of the epilogue
 constexpr int kInt8EpiDirectM = 4; // up to this many tokens the epilogue reads global memory
 constexpr int kInt8StepsAhead = 2; // 64-channel weight steps loaded together per warp
@@ -66,13 +67,14 @@ __global__ void __launch_bounds__(256) int8_quantize_weights_kernel(const float*
   }
 }
 
-// One CTA per 256 input channels, 1024 threads: warp w takes channels
-// 32 (w % 8) .. + 31 of the CTA's and the tokens m = w / 8 (mod 4), eight
-// tokens' loads at a time (independent), so a long prefill batch is read in
-// M / 32 round trips per thread.  Flags: OR over the four token groups in
-// shared memory.  The per-token maximum of the unflagged |x| over the CTA's
-// channels: a warp maximum (shuffles), then an atomic maximum of the
-// non-negative float's bits in shared memory, 256 tokens at a time.
+// One CTA of min(M, 32) warps per kInt8ScanCh = 32 input channels: lane =
+// channel, warp w of nw = the tokens m = w (mod nw), eight of them loaded at
+// once (independent loads), so a long prefill batch is read in M / 256 round
+// trips per thread, short K still gives many CTAs, and a short batch does
+// not launch idle warps.  Flags: a ballot per warp,
+// OR-ed over the warps in shared memory.  The per-token maximum of the
+// unflagged |x| over the CTA's channels is one warp's maximum (shuffles), so
+// each partial is written by exactly one lane.
 __global__ void __launch_bounds__(1024) int8_scan_kernel(const uint16_t* __restrict__ X, int M,
                                                          int K, float threshold,
                                                          uint8_t* __restrict__ flag,
@@ -81,82 +83,60 @@ __global__ void __launch_bounds__(1024) int8_scan_kernel(const uint16_t* __restr
                                                          float* __restrict__ part,
                                                          unsigned int* __restrict__ counter,
                                                          int row_tiles) {
-  __shared__ uint8_t grp_flag[4][256];
-  __shared__ int warp_cnt[8];
-  __shared__ unsigned int tok_max[256];
+  __shared__ unsigned int warp_bits[32];
   grid_dep_launch();
   grid_dep_wait();  // X may come from the previous kernel
-  const int c = blockIdx.x, t = threadIdx.x, lane = t & 31, wid = t >> 5;
-  const int kl = (wid & 7) * 32 + lane;  // channel within the CTA
-  const int tg = wid >> 3;               // token group
-  for (int i = c * 1024 + t; i < row_tiles; i += gridDim.x * 1024) counter[i] = 0u;
-  const int k = c * 256 + kl;
+  const int c = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const int nw = static_cast<int>(blockDim.x) >> 5;
+  for (int i = c * blockDim.x + t; i < row_tiles; i += gridDim.x * blockDim.x) counter[i] = 0u;
+  const int k = c * kInt8ScanCh + lane;
   const bool in = k < K;
   bool og = false;
-  for (int m0 = tg; m0 < M; m0 += 32) {
+  for (int m0 = w; m0 < M; m0 += nw * 8) {
     float v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int m = m0 + 4 * j;
+      const int m = m0 + nw * j;
       v[j] = in && m < M ? fabsf(bf16_bits_f32(X[static_cast<size_t>(m) * K + k])) : 0.0f;
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) og = og || v[j] > threshold;
   }
-  grp_flag[tg][kl] = og ? 1 : 0;
+  const unsigned bits = __ballot_sync(0xffffffffu, og);
+  if (lane == 0) warp_bits[w] = bits;
   __syncthreads();
-  const bool o = grp_flag[0][kl] | grp_flag[1][kl] | grp_flag[2][kl] | grp_flag[3][kl];
-  // the CTA's flagged channels, ascending, in its list region (token group 0)
-  unsigned bal = 0;
-  if (tg == 0) {
+  unsigned flagged = 0u;
+  for (int i = 0; i < nw; ++i) flagged |= warp_bits[i];
+  const bool o = (flagged >> lane) & 1u;
+  // the CTA's flagged channels, ascending, in its list region
+  if (w == 0) {
     if (in) flag[k] = o ? 1 : 0;
-    bal = __ballot_sync(0xffffffffu, o);
-    if (lane == 0) warp_cnt[wid] = __popc(bal);
-  }
-  __syncthreads();
-  if (tg == 0) {
-    int before = 0, total = 0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      before += w < wid ? warp_cnt[w] : 0;
-      total += warp_cnt[w];
-    }
     if (o) {
-      const int pos = before + __popc(bal & ((1u << lane) - 1u));
-      if (in_bounds(static_cast<unsigned>(c * 256 + pos), static_cast<unsigned>(gridDim.x * 256)))
-        list[c * 256 + pos] = k;
+      const int pos = __popc(flagged & ((1u << lane) - 1u));
+      if (in_bounds(static_cast<unsigned>(c * kInt8ScanCh + pos),
+                    static_cast<unsigned>(gridDim.x * kInt8ScanCh)))
+        list[c * kInt8ScanCh + pos] = k;
     }
-    if (t == 0) cnt[c] = total;
+    if (lane == 0) cnt[c] = __popc(flagged);
   }
   // per token, the largest unflagged |x| among the CTA's channels
-  for (int mc = 0; mc < M; mc += 256) {
-    const int me = min(M, mc + 256);
-    if (t < 256) tok_max[t] = 0u;
-    __syncthreads();
-    for (int m0 = mc + tg; m0 < me; m0 += 32) {
-      float v[8];
+  for (int m0 = w; m0 < M; m0 += nw * 8) {
+    float v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int m = m0 + 4 * j;
-        v[j] = in && !o && m < me ? fabsf(bf16_bits_f32(X[static_cast<size_t>(m) * K + k])) : 0.0f;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v[j] = fmaxf(v[j], __shfl_xor_sync(0xffffffffu, v[j], off));
-      }
-      if (lane == 0) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int m = m0 + 4 * j;
-          // non-negative floats order as their bits; a NaN counts as 0
-          if (m < me) atomicMax(&tok_max[m - mc], __float_as_uint(fmaxf(v[j], 0.0f)));
-        }
-      }
+    for (int j = 0; j < 8; ++j) {
+      const int m = m0 + nw * j;
+      v[j] = in && !o && m < M ? fabsf(bf16_bits_f32(X[static_cast<size_t>(m) * K + k])) : 0.0f;
     }
-    __syncthreads();
-    if (t < me - mc) part[static_cast<size_t>(c) * M + mc + t] = __uint_as_float(tok_max[t]);
-    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v[j] = fmaxf(v[j], __shfl_xor_sync(0xffffffffu, v[j], off));
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (m0 + nw * j < M) part[static_cast<size_t>(c) * M + m0 + nw * j] = v[j];
+    }
   }
 }
 
@@ -203,8 +183,14 @@ __global__ void __launch_bounds__(256) int8_quantize_x_kernel(
     *reinterpret_cast<uint2*>(qx + static_cast<size_t>(m) * K + k0) = make_uint2(q[0], q[1]);
   }
   if (blockIdx.x == 0 && blockIdx.y == 0) {
-    // concatenate the scan CTAs' ascending lists (nscan <= 256)
-    const int n = t < nscan ? cnt[t] : 0;
+    // concatenate the scan CTAs' ascending lists: thread t takes scan CTAs
+    // t per .. t per + per - 1, in order
+    const int per = (nscan + 255) / 256;
+    int n = 0;
+    for (int i = 0; i < per; ++i) {
+      const int cc = t * per + i;
+      if (cc < nscan) n += cnt[cc];
+    }
     pre[t + 1] = n;
     if (t == 0) pre[0] = 0;
     __syncthreads();
@@ -214,9 +200,16 @@ __global__ void __launch_bounds__(256) int8_quantize_x_kernel(
       pre[t + 1] += v;
       __syncthreads();
     }
-    for (int i = 0; i < n; ++i)
-      if (in_bounds(static_cast<unsigned>(pre[t] + i), static_cast<unsigned>(K)))
-        olist[pre[t] + i] = list[t * 256 + i];
+    int pos = pre[t];
+    for (int i = 0; i < per; ++i) {
+      const int cc = t * per + i;
+      if (cc >= nscan) break;
+      const int nc = cnt[cc];
+      for (int j = 0; j < nc; ++j, ++pos)
+        if (in_bounds(static_cast<unsigned>(pos), static_cast<unsigned>(K)) &&
+            in_bounds(static_cast<unsigned>(j), static_cast<unsigned>(kInt8ScanCh)))
+          olist[pos] = list[cc * kInt8ScanCh + j];
+    }
     if (t == 0) *ocount = pre[256];
   }
 }

@@ -181,20 +181,25 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       const float swn = n < a.N ? a.sw[n] : 0.0f;
       const int no = min(*a.ocount, a.K);
       // The outlier operands, gathered once into the (now idle) operand ring
-      // when they fit: the tile's tokens' activations xo[token][i] and this
-      // thread's row's 16-bit weights wo[row][i] = bf16(q_w s_w) (row stride
-      // odd, so that the lanes' rows fall in different banks); otherwise each
-      // output reads them from global memory.  Either way one fp32 fma per
+      // when they fit: the tile's tokens' scales so[token] and activations
+      // xo[token][i] and this thread's row's 16-bit weights wo[row][i] =
+      // bf16(q_w s_w) (row stride odd, so that the lanes' rows fall in
+      // different banks); otherwise each output reads them from global memory.  Either way one fp32 fma per
       // outlier channel in ascending order.  (An outlier channel outside K,
       // bounds-checked build only, contributes nothing.)
       const int wstr = no | 1;
       const bool gathered =
-          no > 0 && (static_cast<long long>(C::MT) * no + 128ll * wstr) * 4 <= C::kRingBytes;
-      float* xo = reinterpret_cast<float*>(ws);
+          (static_cast<long long>(C::MT) * (no + 1) + 128ll * wstr) * 4 <= C::kRingBytes;
+      float* so = reinterpret_cast<float*>(ws);  // the tile's tokens' s_x
+      float* xo = so + C::MT;
       float* wo = xo + C::MT * no;
       bool ready = false;
       auto gather = [&]() {
         const int e = threadIdx.x - 64;  // epilogue thread 0..127
+        for (int ml = e; ml < C::MT; ml += 128) {
+          const int m = mtile * C::MT + ml;
+          so[ml] = m < a.M ? a.sx[m] : 0.0f;
+        }
         for (int i = 0; i < no; ++i) {
           const int k = a.olist[i];
           const bool ok = in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K));
@@ -213,7 +218,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       };
       auto finish = [&](int m, int v) {
         if (m >= a.M || n >= a.N) return;
-        float y = __fmul_rn(__fmul_rn(static_cast<float>(v), a.sx[m]), swn);
+        float y = __fmul_rn(__fmul_rn(static_cast<float>(v), ready ? so[m - mtile * C::MT] : a.sx[m]), swn);
         if (ready) {
           const float* xr = xo + (m - mtile * C::MT) * no;
           const float* wr = wo + row * wstr;

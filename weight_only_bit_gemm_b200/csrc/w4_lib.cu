@@ -366,14 +366,14 @@ I8Plan int8_tc_plan(int M, int N, int K) {
 
 struct Int8Layout {
   size_t counter, acc, flag, list, cnt, part, olist, ocount, qx, sx, tcpart, total;
-  int nscan;         // scan CTAs (256 channels each)
+  int nscan;         // scan CTAs (kInt8ScanCh channels each)
   int counters;      // counters the scan clears
 };
 
 Int8Layout int8_layout(int M, int N, int K) {
   auto r = [](size_t v) { return (v + 255) / 256 * 256; };
   Int8Layout l{};
-  l.nscan = (K + 255) / 256;
+  l.nscan = (K + kInt8ScanCh - 1) / kInt8ScanCh;
   const bool tc = M >= kInt8TcMinM;
   const I8Plan tp = int8_tc_plan(M, N, K);
   const long long tiles = static_cast<long long>(tp.tiles_n) * tp.tiles_m;
@@ -382,7 +382,7 @@ Int8Layout int8_layout(int M, int N, int K) {
   l.counter = o; o += r(static_cast<size_t>(l.counters) * 4);
   l.acc = o;     o += tc ? 0 : r(static_cast<size_t>(M) * N * 4);
   l.flag = o;    o += r(static_cast<size_t>(K));
-  l.list = o;    o += r(static_cast<size_t>(l.nscan) * 256 * 4);
+  l.list = o;    o += r(static_cast<size_t>(l.nscan) * kInt8ScanCh * 4);
   l.cnt = o;     o += r(static_cast<size_t>(l.nscan) * 4);
   l.part = o;    o += r(static_cast<size_t>(l.nscan) * M * 4);
   l.olist = o;   o += r(static_cast<size_t>(K) * 4);
@@ -490,7 +490,7 @@ w4_status llm_int8_gemm(const uint16_t* X, const int8_t* qw, const float* sw, in
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cfg.gridDim = dim3(l.nscan);
-  cfg.blockDim = dim3(1024);
+  cfg.blockDim = dim3(32 * std::min(M, 32));
   cudaError_t e = cudaLaunchKernelEx(&cfg, int8_scan_kernel, X, M, K, threshold, flag, list, cnt,
                                      part, a.counter, l.counters);
   if (e == cudaSuccess) {
