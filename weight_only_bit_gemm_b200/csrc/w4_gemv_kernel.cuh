@@ -103,8 +103,8 @@ struct GemvCfg {
   static constexpr int kAS = gemv_acc_split(NB);  // accumulators per (row group, token block)
   static constexpr int kSlot = kRG * 1024 + (kRG * (kScaleBytes + kZeroBytes) + 15) / 16 * 16;
   static constexpr int kRingBytes = kWarps * kDepth * kSlot;
-  // CTA-level reduction (up to two token blocks; four would not leave room
-  // for two CTAs per SM): two partial slots per warp (the warp's first and
+  // CTA-level reduction (up to two token blocks; the slots of four would not
+  // fit beside the ring): two partial slots per warp (the warp's first and
   // last row-pair segments), [slot][V/4][32 lanes] float4, and one arrival
   // counter per warp (the row pair that ends the warp's range).
   static constexpr bool kCtaReduce = NB <= 2;
