@@ -28,18 +28,25 @@ namespace w4 {
 
 enum WeightFormat : int { kFmtInt4 = 0, kFmtNf4 = 1 };
 
-template <int MT_, int STAGES_, int FMT_, int G_, bool MEAN_ = false>
+template <int MT_, int STAGES_, int FMT_, int G_, bool MEAN_ = false, bool PAIR_ = false>
 struct GemmCfg {
   static constexpr int MT = MT_;          // tokens per tile (MMA N)
   static constexpr int STAGES = STAGES_;  // shared-memory ring depth
   static constexpr int FMT = FMT_;
   static constexpr int G = G_;            // INT4 group size (ignored for NF4)
   static constexpr bool MEAN = MEAN_;     // NF4 layout: mean-offset absmax constants
-  static constexpr int kXBoxBytes = MT * 128;         // [MT][64] bf16, 128-byte rows
+  // CTA pair (cluster of 2, cta_group::2): the pair computes 256 weight rows
+  // x MT tokens with one MMA stream issued by the even CTA; each CTA holds its
+  // 128 weight rows (dequantized into its own tensor memory) and half of the
+  // tile's tokens (MT / 2 rows of the activation boxes), so each CTA streams
+  // half the activation bytes per MMA of a single-CTA tile.
+  static constexpr bool PAIR = PAIR_;
+  static constexpr int kXTok = PAIR ? MT / 2 : MT;    // token rows of this CTA's boxes
+  static constexpr int kXBoxBytes = kXTok * 128;      // [kXTok][64] bf16, 128-byte rows
   static constexpr int kXStageBytes = 2 * kXBoxBytes;  // 128 channels
   static constexpr int kWStageBytes = FMT == kFmtInt4 ? int4_stage_bytes(G) : nf4_stage_bytes();
   static constexpr int kWSlot = (kWStageBytes + 127) / 128 * 128;
-  static constexpr int kASlots = 3;                   // TMEM A ring (64 columns each)
+  static constexpr int kASlots = PAIR ? 4 : 3;        // TMEM A ring (64 columns each)
   // Independent accumulators: consecutive MMAs of a stage write different
   // ones, so that narrow (decode) tiles are not serialised on the
   // accumulator dependency; the epilogue sums them in a fixed order.
@@ -53,11 +60,15 @@ struct GemmCfg {
                                    : kColsNeeded <= 256 ? 256 : 512;
   static constexpr int kDqWarps = 8;
   static constexpr int kThreads = 64 + kDqWarps * 32;
-  static constexpr int kNumBars = 2 * STAGES + 2 * kASlots + 3;
+  // full, empty (STAGES each), afull, aempty (kASlots each), accf, epi1,
+  // epi2, and for a pair xfull (STAGES: the activation halves of both CTAs)
+  static constexpr int kNumBars = (PAIR ? 3 : 2) * STAGES + 2 * kASlots + 3;
   static constexpr int kSmemBytes =
       1024 /* alignment slack */ + STAGES * (kXStageBytes + kWSlot) + kNumBars * 8 + 16 + 64 +
       256 /* NF4 level table alignment */;
-  static constexpr int kMinBlocks = kTmemCols <= 256 && kSmemBytes <= 113 * 1024 ? 2 : 1;
+  static constexpr int kMinBlocks =
+      !PAIR && kTmemCols <= 256 && kSmemBytes <= 113 * 1024 ? 2 : 1;
+  static_assert(!PAIR || (MT == 256 && kAcc == 1), "CTA pairs: 256-token tiles");
   static_assert(MT % 16 == 0 && MT >= 16 && MT <= 256, "MMA N for M=128 is 16..256 step 16");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   static_assert(kColsNeeded <= 512, "tensor memory");

@@ -21,13 +21,17 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
   uint64_t* accf = aempty + C::kASlots;                 // accumulator ready  (commit)
   uint64_t* epi1 = accf + 1;                            // partials stored    (8 warps)
   uint64_t* epi2 = epi1 + 1;                            // last-arrival known (1)
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi2 + 1);
+  uint64_t* xfull = epi2 + 1;                           // pair: both X halves landed (tx)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xfull + (C::PAIR ? C::STAGES : 0));
   int* last_flag = reinterpret_cast<int*>(tmem_holder + 1);
   float* Ts = reinterpret_cast<float*>(                   // NF4 levels [16], 256-byte aligned
       (reinterpret_cast<uintptr_t>(tmem_holder + 4) + 255) & ~static_cast<uintptr_t>(255));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA pair: rank 0 (the leader) issues the MMAs; the barriers of the
+  // shared MMA stream (xfull, afull) live in the leader's shared memory.
+  const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
   // CTA order: groups of group_m token tiles; inside a group the token tile
   // runs fastest, so the CTAs that read one weight tile (and split range)
   // run together and share it through L2, as do the weight tiles of a wave
@@ -39,9 +43,12 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
   // tile; cidx: its arrival counter.
   int mtile, nt, split, nsplit, cidx;
   size_t pbase;
+  // For a CTA pair every count below is in pair tiles of 256 weight rows
+  // (tiles_n / 2 of them); the CTA then takes 128-row tile 2 nt + rank.
   {
-    const int b = static_cast<int>(blockIdx.x);
-    const int ns = args.tail_splits == 0 ? args.tiles_n * args.splits : args.tiles_n;
+    const int b = static_cast<int>(C::PAIR ? blockIdx.x >> 1 : blockIdx.x);
+    const int tn = C::PAIR ? args.tiles_n >> 1 : args.tiles_n;
+    const int ns = args.tail_splits == 0 ? tn * args.splits : tn;
     int lt = b;  // CTA position in the group order (tail: the tile's)
     if (args.tail_splits == 0) {
       nsplit = args.splits;
@@ -61,12 +68,13 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     if (args.tail_splits == 0) {
       nt = nts / nsplit;
       split = nts % nsplit;
+      if (C::PAIR) nt = 2 * nt + static_cast<int>(rank);
       cidx = mtile * args.tiles_n + nt;
       pbase = static_cast<size_t>(cidx) * nsplit;
     } else {
-      nt = nts;
+      nt = C::PAIR ? 2 * nts + static_cast<int>(rank) : nts;
       split = b < args.head_tiles ? 0 : (b - args.head_tiles) % nsplit;
-      cidx = lt - args.head_tiles;
+      cidx = C::PAIR ? 2 * (lt - args.head_tiles) + static_cast<int>(rank) : lt - args.head_tiles;
       pbase = static_cast<size_t>(cidx) * nsplit;
     }
   }
@@ -80,12 +88,14 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < C::kASlots; ++i) {
-      mbar_init(&afull[i], C::kDqWarps);
+      mbar_init(&afull[i], C::PAIR ? 2 * C::kDqWarps : C::kDqWarps);
       mbar_init(&aempty[i], 1);
     }
     mbar_init(accf, 1);
     mbar_init(epi1, C::kDqWarps);
     mbar_init(epi2, 1);
+    if (C::PAIR)
+      for (int i = 0; i < C::STAGES; ++i) mbar_init(&xfull[i], 1);
     fence_barrier_init();
     grid_dep_launch();  // the next kernel on the stream may start its prologue
   }
@@ -93,11 +103,21 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
   // the level addresses need a 256-byte-aligned table (bounds-checked build: verified)
   if (C::FMT == kFmtNf4 && kChecked && threadIdx.x == 0) in_bounds(smem_u32(Ts) & 0xFFu, 1u);
   if (warp == 1) {
-    tmem_alloc(tmem_holder, C::kTmemCols);
-    tmem_relinquish();
+    if constexpr (C::PAIR) {
+      tmem_alloc_pair(tmem_holder, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  // a pair: the peer's copies and arrivals may target this CTA's barriers
+  // as soon as it passes here, so both CTAs' initialisations come first
+  if constexpr (C::PAIR)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
@@ -120,9 +140,13 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
       };
       // The weights do not depend on the previous kernel: start streaming the
       // first ring's worth before waiting for it, then add the X tiles.
+      // full[s] counts this CTA's weight bytes (and for a single CTA its X
+      // bytes); a pair's X halves are counted on the leader's xfull[s], which
+      // the leader alone arms, with both halves' bytes.
+      constexpr uint32_t kFullBytes = C::PAIR ? C::kWStageBytes : C::kXStageBytes + C::kWStageBytes;
       const int first = nst < C::STAGES ? nst : C::STAGES;
       for (int it = 0; it < first; ++it) {
-        mbar_arrive_expect_tx(&full[it], C::kXStageBytes + C::kWStageBytes);
+        mbar_arrive_expect_tx(&full[it], kFullBytes);
         bulk_g2s(wsl + it * C::kWSlot, stage_src(it), C::kWStageBytes, &full[it], pol_w);
       }
       grid_dep_wait();
@@ -131,11 +155,18 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
         const int s = it % C::STAGES;
         if (it >= C::STAGES) {
           if (!mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1)) break;
-          mbar_arrive_expect_tx(&full[s], C::kXStageBytes + C::kWStageBytes);
+          mbar_arrive_expect_tx(&full[s], kFullBytes);
           bulk_g2s(wsl + s * C::kWSlot, stage_src(it), C::kWStageBytes, &full[s], pol_w);
         }
-        tma_load_3d(xs + s * C::kXStageBytes, &xmap, 0, mtile * C::MT, (s0 + it) * 2, &full[s],
-                    pol_x);
+        if constexpr (C::PAIR) {
+          if (rank == 0) mbar_arrive_expect_tx(&xfull[s], 2 * C::kXStageBytes);
+          tma_load_3d_pair(xs + s * C::kXStageBytes, &xmap, 0,
+                           mtile * C::MT + static_cast<int>(rank) * C::kXTok, (s0 + it) * 2,
+                           mapa_shared(smem_u32(&xfull[s]), 0), pol_x);
+        } else {
+          tma_load_3d(xs + s * C::kXStageBytes, &xmap, 0, mtile * C::MT, (s0 + it) * 2,
+                      &full[s], pol_x);
+        }
         ++issued;
       }
       if (issued < first) {
@@ -143,18 +174,28 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
         for (int it = issued; it < first; ++it) mbar_wait(&full[it], 0);
       }
       // never leave with copies in flight: wait for the last issued stages
-      for (int it = issued - 1; it >= 0 && it >= issued - C::STAGES; --it)
+      // (the leader's xfull also covers the peer's halves)
+      for (int it = issued - 1; it >= 0 && it >= issued - C::STAGES; --it) {
         mbar_wait(&full[it % C::STAGES], (it / C::STAGES) & 1);
+        if (C::PAIR && rank == 0) mbar_wait(&xfull[it % C::STAGES], (it / C::STAGES) & 1);
+      }
+      // a pair: the leader's MMA completions arrive on this CTA's empty
+      // barriers from the other SM; wait for the last ones before leaving
+      if (C::PAIR && issued == nst)
+        for (int it = nst - 1; it >= 0 && it >= nst - C::STAGES; --it)
+          mbar_wait(&empty[it % C::STAGES], (it / C::STAGES) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, C::MT);
+    // (a pair: the leader's thread alone; its MMAs span both CTAs, and each
+    // commit arrives on the barrier at the same offset in both)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(C::PAIR ? 256 : 128, C::MT);
       const uint32_t d_tmem = tmem + C::kDCol;
       for (int it = 0; it < nst; ++it) {
         const int s = it % C::STAGES;
         const int a = it % C::kASlots;
-        if (!mbar_wait(&full[s], (it / C::STAGES) & 1)) break;
+        if (!mbar_wait(C::PAIR ? &xfull[s] : &full[s], (it / C::STAGES) & 1)) break;
         if (!mbar_wait(&afull[a], (it / C::kASlots) & 1)) break;
         tc_fence_after();
         const uint32_t xaddr = smem_u32(xs + s * C::kXStageBytes);
@@ -164,13 +205,25 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
               smem_desc_sw128(xaddr + (kk >> 2) * C::kXBoxBytes + (kk & 3) * 32);
           const uint32_t a_tmem = tmem + C::kACol + a * 64 + kk * 8;
           const int acc = kk % C::kAcc;
-          mma_bf16_ts(d_tmem + acc * C::MT, a_tmem, bdesc, idesc,
-                      (it > 0 || kk >= C::kAcc) ? 1u : 0u);
+          if constexpr (C::PAIR)
+            mma_bf16_ts_pair(d_tmem, a_tmem, bdesc, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+          else
+            mma_bf16_ts(d_tmem + acc * C::MT, a_tmem, bdesc, idesc,
+                        (it > 0 || kk >= C::kAcc) ? 1u : 0u);
         }
-        mma_commit(&empty[s]);
-        mma_commit(&aempty[a]);
+        if constexpr (C::PAIR) {
+          mma_commit_pair(&empty[s], 3);
+          mma_commit_pair(&aempty[a], 3);
+        } else {
+          mma_commit(&empty[s]);
+          mma_commit(&aempty[a]);
+        }
       }
-      mma_commit(accf);  // also on an early exit, so that TMEM is quiet before dealloc
+      // also on an early exit, so that TMEM is quiet before dealloc
+      if constexpr (C::PAIR)
+        mma_commit_pair(accf, 3);
+      else
+        mma_commit(accf);
     }
   } else {
     // ------------------------------------------------------------ dequant
@@ -237,10 +290,12 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
           for (int w = 0; w < 4; ++w) nf4_dq_word(words[w], a0, a1, smem_u32(Ts), &out[rgl][4 * w]);
         }
       }
-      if (it >= C::kASlots &&
-          !__all_sync(0xffffffffu, mbar_wait(&aempty[a], ((it / C::kASlots) - 1) & 1))) {
-        ok = false;
-        break;
+      if (it >= C::kASlots) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&aempty[a], ((it / C::kASlots) - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();  // the MMAs that read this slot are complete
       }
 #pragma unroll
       for (int rgl = 0; rgl < 2; ++rgl)
@@ -250,8 +305,18 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[a]);
+      if (lane == 0) {
+        if constexpr (C::PAIR)
+          mbar_arrive_cluster(mapa_shared(smem_u32(&afull[a]), 0));  // the leader's
+        else
+          mbar_arrive(&afull[a]);
+      }
     }
+    // a pair: the last slot releases arrive from the other SM; wait for them
+    // before the CTA can leave
+    if (C::PAIR && ok)
+      for (int it = nst - 1; it >= 0 && it >= nst - C::kASlots; --it)
+        mbar_wait(&aempty[it % C::kASlots], (it / C::kASlots) & 1);
 
     // ------------------------------------------------------------ epilogue
     if (ok && __all_sync(0xffffffffu, mbar_wait(accf, 0))) {
@@ -355,11 +420,23 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     }
   }
 
-  __syncthreads();
-  if (warp == 1) {
-    mbar_wait(accf, 0);  // every issued MMA has completed
-    tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+  if constexpr (C::PAIR) {
+    // neither CTA of a pair leaves (or frees its tensor memory) while the
+    // other may still reach its shared or tensor memory
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 1) {
+      mbar_wait(accf, 0);  // every issued MMA has completed
+      tc_fence_after();
+      tmem_dealloc_pair(tmem, C::kTmemCols);
+    }
+  } else {
+    __syncthreads();
+    if (warp == 1) {
+      mbar_wait(accf, 0);  // every issued MMA has completed
+      tc_fence_after();
+      tmem_dealloc(tmem, C::kTmemCols);
+    }
   }
 }
 
