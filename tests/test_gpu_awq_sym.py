@@ -78,7 +78,10 @@ def test_quantize_sym_bit_exact(w4, N, K, G, act):
 
 # ----------------------------------------------------------------- AWQ factor
 
-@pytest.mark.parametrize("N,K", [(64, 4096), (3, 10), (1000, 777)])
+# (64, 4096), (300, 1028), (5, 8): the float4 row kernel (K % 4 == 0; 257
+# float4 per row leave a ragged last trip, 2 per row fewer than one trip);
+# (3, 10), (1000, 777): the element kernel
+@pytest.mark.parametrize("N,K", [(64, 4096), (300, 1028), (5, 8), (3, 10), (1000, 777)])
 def test_awq_scale_weights_bit_exact(w4, N, K):
     W = S.draw_w(N, K, 0.02, seed=2, tag=21)
     s = S.draw_awq_s(K, seed=2, tag=21, lo=0.25, hi=4.0)

@@ -60,6 +60,10 @@ INT4_CASES = [
     (100, 640, 2048, 128, False),
     (300, 384, 1024, 128, False),
     (256, 256, 2048, 32, True),
+    # CTA pairs: ragged token halves, K-split partials, head and tail tiles
+    (129, 512, 2048, 128, False),
+    (520, 2304, 4096, 64, False),
+    (300, 9728, 4096, 128, False),
 ]
 
 
@@ -84,7 +88,7 @@ def test_checked_int4_path(libs, M, N, K, G, act):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 40, 64), (8, 300, 1024), (32, 200, 1536), (48, 256, 512),
-                                   (300, 256, 512)])
+                                   (300, 256, 512), (260, 1024, 4096)])
 def test_checked_blockwise_path(libs, M, N, K):
     w4, chk = libs
     W = torch.from_numpy(S.draw_w(N, K, 0.02, seed=M, tag=62)).cuda()

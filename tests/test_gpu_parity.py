@@ -259,6 +259,13 @@ GEMM_CASES = [
     (40, 19000, 2560, 128, False),   # ragged N, one tail tile in 5 K ranges
     (300, 9550, 2560, 64, True),     # two token tiles, act-order, two tail tiles
     (5, 4096, 4160, 64, False),      # K = 32.5 stages: last stage half, G = 64
+    # CTA pairs (256-token tiles over an even number of 128-row tiles): the
+    # odd CTA holds tokens 128..255 of a tile, its 128 rows the pair's second
+    (129, 512, 2048, 128, False),    # the odd CTA's token half holds one token
+    (520, 2304, 4096, 64, False),    # every tile in 2 K ranges, third token tile 8 tokens
+    (700, 1536, 8192, 128, False),   # 4 K ranges, ragged third token tile
+    (260, 1024, 4096, 32, True),     # act-order, 4 K ranges
+    (300, 9728, 4096, 128, False),   # one wave of 74 pairs whole, 2 tail pairs in 4 K ranges
 ]
 
 
@@ -299,7 +306,8 @@ def test_nf4_gemm_unit_vectors_exact(w4):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 512, 4096), (8, 384, 1024), (32, 200, 1536),
-                                   (300, 256, 512), (1, 40, 64), (3, 4096, 14336)])
+                                   (300, 256, 512), (1, 40, 64), (3, 4096, 14336),
+                                   (260, 1024, 4096)])   # CTA pairs, 4 K ranges
 def test_nf4_gemm_tolerance(w4, M, N, K):
     W = S.draw_w(N, K, 0.02, seed=M, tag=3)
     Wq_r, c_r, s2_r = O.nf4_quantize(W)

@@ -181,6 +181,15 @@ w4_status w4_awq_scale_weights(const float* W, const float* s, int N, int K, flo
   if (!W || !s || !W_out) return W4_ERR_INVALID_ARG;
   if (N < 1 || K < 1) return W4_ERR_INVALID_ARG;
   if (!aligned(W, 4) || !aligned(s, 4) || !aligned(W_out, 4)) return W4_ERR_INVALID_ARG;
+  if (K % 4 == 0 && aligned(W, 16) && aligned(s, 16) && aligned(W_out, 16)) {
+    // one CTA per row at a time, 8 resident per SM
+    const int blocks = std::min(N, sm_count() * 8);
+    awq_scale_weights_vec_kernel<<<static_cast<unsigned>(blocks), kAwqThreads, 0,
+                                   as_stream(stream)>>>(
+        reinterpret_cast<const float4*>(W), reinterpret_cast<const float4*>(s), N, K / 4,
+        reinterpret_cast<float4*>(W_out));
+    return launch_status(cudaGetLastError());
+  }
   const size_t total = static_cast<size_t>(N) * K;
   const size_t blocks =
       std::min<size_t>((total + 255) / 256, static_cast<size_t>(sm_count()) * 16);

@@ -325,6 +325,38 @@ __global__ void awq_scale_weights_kernel(const float* W, const float* __restrict
       W_out[i] = __fmul_rn(W[i], s[i % static_cast<size_t>(K)]);
 }
 
+// The same product for K % 4 == 0 and 16-byte aligned W, s, W_out: CTAs walk
+// whole rows (no index division), each thread 4 float4 of a row per trip,
+// all 4 loads issued before the stores.  W_out may be W (each element is
+// read and written by the same thread).
+constexpr int kAwqThreads = 256;
+__global__ void __launch_bounds__(kAwqThreads) awq_scale_weights_vec_kernel(
+    const float4* W, const float4* __restrict__ s, int N, int K4, float4* W_out) {
+  const unsigned long long total = static_cast<unsigned long long>(N) * K4;
+  for (int n = blockIdx.x; n < N; n += gridDim.x) {
+    const size_t row = static_cast<size_t>(n) * K4;
+    for (int k0 = threadIdx.x; k0 < K4; k0 += 4 * kAwqThreads) {
+      float4 v[4], f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int k = k0 + u * kAwqThreads;
+        if (k < K4 && in_bounds(row + k, total)) {
+          v[u] = __ldcs(W + row + k);
+          f[u] = __ldg(s + k);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int k = k0 + u * kAwqThreads;
+        if (k < K4 && in_bounds(row + k, total))
+          __stcs(W_out + row + k,
+                 make_float4(__fmul_rn(v[u].x, f[u].x), __fmul_rn(v[u].y, f[u].y),
+                             __fmul_rn(v[u].z, f[u].z), __fmul_rn(v[u].w, f[u].w)));
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- NF4
 // "大模型量化选型" §6.1 (normal quantiles), §6.3 (blocks of 64),
 // §6.2 (double quantization).  Levels: normal quantiles at equally spaced
