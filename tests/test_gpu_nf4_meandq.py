@@ -53,10 +53,11 @@ def test_meandq_quantize_dequant_bit_exact(w4, N, K, dq):
     assert np.array_equal(_u16(got), what)
 
 
-@pytest.mark.parametrize("M", [32, 48])
+@pytest.mark.parametrize("M", [32, 48, 300])
 def test_meandq_gemm_unit_vectors_exact(w4, M):
-    # decode kernel (M = 32) and tensor-core kernel (M = 48): each output is
-    # one w_hat, so the in-kernel reconstruction of the constants is exact
+    # decode kernel (M = 32), tensor-core kernel (M = 48) and its CTA pairs
+    # (M = 300: two 256-token tiles over the two 128-row tiles): each output
+    # is one w_hat, so the in-kernel reconstruction of the constants is exact
     N, K = 256, 1024
     what, (Wq, c, m, s2) = _layer(w4, N, K, 256, seed=5)
     Wp = w4.nf4_prepack(Wq, c.view(torch.uint8))

@@ -11,9 +11,17 @@
 // bytes per instruction.  Warp roles: warp 0 the producer (the weight tiles
 // of the first ring are requested before the launch dependency resolves),
 // warp 1 tensor-memory allocation and the single MMA thread, warps 2..5 the
-// epilogue (one weight row per thread: y = acc s_x s_w plus the 16-bit
-// product of the outlier channels, bf16 out; with split K the fp32-free int32
-// partials go to the workspace and the last CTA of the tile sums them).
+// epilogue (one weight row per thread: y = acc s_x s_w + d, bf16 out; with
+// split K the int32 partials go to the workspace and the last CTA of the
+// tile sums them).  d, the 16-bit product of the outlier channels
+// (§2.2's second matrix multiplication), is itself a small GEMM,
+// D2 = W_o X_o^T over the outlier channels: once the INT8 accumulator is
+// complete the operand ring is idle, the epilogue warps write
+// W_o[row][i] = bf16(q_w s_w) and X_o[token][i] = x into it (128-byte swizzled,
+// K-major, 64 channels per chunk, zero beyond the last outlier) and one of
+// them issues kind::f16 MMAs into a second accumulator in tensor memory.
+// Operands that do not fit the ring (more than about 256 outlier channels)
+// are read from global memory by each output instead, one fma per channel.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -32,9 +40,13 @@ struct I8Cfg {
   static constexpr int kWStage = 128 * 128;  // weight tile bytes per stage
   static constexpr int kXStage = MT * 128;   // activation tile bytes per stage
   static constexpr int kThreads = 64 + 4 * 32;
-  static constexpr int kTmemCols = MT <= 32 ? 32 : MT <= 64 ? 64 : MT <= 128 ? 128 : 256;
+  // the s32 accumulator in columns [0, MT), the outlier product's fp32 one in [MT, 2 MT)
+  static constexpr int kTmemCols = MT <= 16 ? 32 : MT <= 32 ? 64 : MT <= 64 ? 128 : MT <= 128 ? 256 : 512;
   static constexpr int kRingBytes = STAGES * (kWStage + kXStage);
-  static constexpr int kSmemBytes = 1024 + kRingBytes + (2 * STAGES + 5) * 8 + 16;
+  // one 64-channel chunk of the outlier operands: 128 weight rows and MT
+  // token rows of 128 bytes (a multiple of 1024: swizzle atoms stay aligned)
+  static constexpr int kOChunkBytes = (128 + MT) * 128;
+  static constexpr int kSmemBytes = 1024 + kRingBytes + (2 * STAGES + 6) * 8 + 16;
   static_assert(MT % 16 == 0 && MT >= 16 && MT <= 256, "MMA N for M = 128");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -56,6 +68,12 @@ __device__ __forceinline__ void mma_s8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// bf16_rne of two floats, packed with the first in the low half.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
+         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
 }
 
 struct I8TcArgs {
@@ -87,7 +105,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   uint64_t* epi1 = accf + 1;                       // partials stored (4 warps)
   uint64_t* epi2 = epi1 + 1;                       // last-arrival known (1)
   uint64_t* epi3 = epi2 + 1;                       // outlier operands gathered (4 warps)
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi3 + 1);
+  uint64_t* ofull = epi3 + 1;                      // outlier product ready (commit)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ofull + 1);
   int* last_flag = reinterpret_cast<int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -110,6 +129,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     mbar_init(epi1, 4);
     mbar_init(epi2, 1);
     mbar_init(epi3, 4);
+    mbar_init(ofull, 1);
     fence_barrier_init();
     grid_dep_launch();
   }
@@ -180,53 +200,89 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       grid_dep_wait();  // s_x, the outlier list, Y and the workspace
       const float swn = n < a.N ? a.sw[n] : 0.0f;
       const int no = min(*a.ocount, a.K);
-      // The outlier operands, gathered once into the (now idle) operand ring
-      // when they fit: the tile's tokens' scales so[token] and activations
-      // xo[token][i] and this thread's row's 16-bit weights wo[row][i] =
-      // bf16(q_w s_w) (row stride odd, so that the lanes' rows fall in
-      // different banks); otherwise each output reads them from global memory.  Either way one fp32 fma per
-      // outlier channel in ascending order.  (An outlier channel outside K,
-      // bounds-checked build only, contributes nothing.)
-      const int wstr = no | 1;
-      const bool gathered =
-          (static_cast<long long>(C::MT) * (no + 1) + 128ll * wstr) * 4 <= C::kRingBytes;
-      float* so = reinterpret_cast<float*>(ws);  // the tile's tokens' s_x
-      float* xo = so + C::MT;
-      float* wo = xo + C::MT * no;
-      bool ready = false;
-      auto gather = [&]() {
+      const int nch = (no + 63) >> 6;  // 64-channel chunks of the outlier operands
+      const bool tc_out =
+          no > 0 && static_cast<long long>(nch) * C::kOChunkBytes <= C::kRingBytes;
+      // byte offset of 16-byte unit u (channels 8u..8u+7) of row r in a
+      // 128-byte swizzled K-major operand (8-row atoms of 1024 bytes)
+      auto sw_off = [](int r, int u) { return (r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4); };
+      // the outlier product D2 into tensor-memory columns [MT, 2 MT)
+      bool have_d2 = false;
+      auto outlier_mma = [&]() {
         const int e = threadIdx.x - 64;  // epilogue thread 0..127
-        for (int ml = e; ml < C::MT; ml += 128) {
-          const int m = mtile * C::MT + ml;
-          so[ml] = m < a.M ? a.sx[m] : 0.0f;
-        }
-        for (int i = 0; i < no; ++i) {
-          const int k = a.olist[i];
-          const bool ok = in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K));
-          for (int ml = e; ml < C::MT; ml += 128) {
-            const int m = mtile * C::MT + ml;
-            xo[ml * no + i] = ok && m < a.M ? bf16_bits_f32(a.X[static_cast<size_t>(m) * a.K + k]) : 0.0f;
+        for (int c = 0; c < nch; ++c) {
+          uint8_t* A = ws + c * C::kOChunkBytes;
+          uint8_t* B = A + 128 * 128;
+          for (int u = 0; u < 8; ++u) {  // this thread's weight row
+            uint32_t pk[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              float v[2];
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                const int i = c * 64 + u * 8 + 2 * h + t;
+                v[t] = 0.0f;
+                if (i < no && n < a.N) {
+                  const int k = a.olist[i];
+                  if (in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K)))
+                    v[t] = __fmul_rn(static_cast<float>(a.qw[static_cast<size_t>(n) * a.K + k]), swn);
+                }
+              }
+              pk[h] = bf16x2_rn(v[0], v[1]);
+            }
+            *reinterpret_cast<uint4*>(A + sw_off(row, u)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
-          wo[row * wstr + i] =
-              ok && n < a.N ? __bfloat162float(__float2bfloat16_rn(
-                                  __fmul_rn(static_cast<float>(a.qw[static_cast<size_t>(n) * a.K + k]), swn)))
-                            : 0.0f;
+          for (int idx = e; idx < C::MT * 8; idx += 128) {  // token rows
+            const int r = idx >> 3, u = idx & 7;
+            const int m = mtile * C::MT + r;
+            uint32_t pk[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              uint32_t b2[2];
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                const int i = c * 64 + u * 8 + 2 * h + t;
+                b2[t] = 0u;
+                if (i < no && m < a.M) {
+                  const int k = a.olist[i];
+                  if (in_bounds(static_cast<unsigned int>(k), static_cast<unsigned int>(a.K)))
+                    b2[t] = a.X[static_cast<size_t>(m) * a.K + k];
+                }
+              }
+              pk[h] = b2[0] | (b2[1] << 16);
+            }
+            *reinterpret_cast<uint4*>(B + sw_off(r, u)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
         }
+        fence_proxy_async_smem();  // the stores above are read by the tensor core
         __syncwarp();
         if (lane == 0) mbar_arrive(epi3);
-        ready = __all_sync(0xffffffffu, mbar_wait(epi3, 0));
-      };
-      auto finish = [&](int m, int v) {
-        if (m >= a.M || n >= a.N) return;
-        float y = __fmul_rn(__fmul_rn(static_cast<float>(v), ready ? so[m - mtile * C::MT] : a.sx[m]), swn);
-        if (ready) {
-          const float* xr = xo + (m - mtile * C::MT) * no;
-          const float* wr = wo + row * wstr;
-          for (int i = 0; i < no; ++i) {
-            if (kChecked && !(static_cast<unsigned int>(a.olist[i]) < static_cast<unsigned int>(a.K)))
-              continue;
-            y = fmaf(xr[i], wr[i], y);
+        if (threadIdx.x == 64) {
+          if (mbar_wait(epi3, 0)) {
+            tc_fence_after();
+            constexpr uint32_t idesc = idesc_bf16_f32(128, C::MT);
+            int step = 0;
+            for (int c = 0; c < nch; ++c) {
+              const uint32_t Aa = smem_u32(ws + c * C::kOChunkBytes);
+              const uint32_t Ba = Aa + 128 * 128;
+              const int ksteps = min(4, (no - 64 * c + 15) >> 4);  // K = 16 each
+              for (int kk = 0; kk < ksteps; ++kk, ++step)
+                mma_bf16_ss(tmem + C::MT, smem_desc_sw128(Aa + kk * 32), smem_desc_sw128(Ba + kk * 32),
+                            idesc, step > 0 ? 1u : 0u);
+            }
           }
+          mma_commit(ofull);  // (with no MMA issued it arrives at once)
+        }
+        have_d2 = __all_sync(0xffffffffu, mbar_wait(ofull, 0));
+        tc_fence_after();
+      };
+      // y = acc s_x s_w + d; d from D2, or (operands beyond the ring) one fma
+      // per outlier channel in ascending order from global memory
+      auto finish = [&](int m, int v, float d2) {
+        if (m >= a.M || n >= a.N) return;
+        float y = __fmul_rn(__fmul_rn(static_cast<float>(v), a.sx[m]), swn);
+        if (have_d2) {
+          y = __fadd_rn(y, d2);
         } else {
           for (int i = 0; i < no; ++i) {
             const int k = a.olist[i];
@@ -239,17 +295,18 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         a.Y[static_cast<size_t>(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
       };
       int* part = a.partial + (static_cast<size_t>(tile_id) * a.splits + split) * C::MT * kI8Rows;
-      if (a.splits == 1 && gathered) gather();
+      if (a.splits == 1 && tc_out) outlier_mma();
 #pragma unroll 1
       for (int cb = 0; cb < C::MT; cb += 8) {
-        uint32_t v[8];
+        uint32_t v[8], d[8];
         tmem_ld8(tmem + lane_base + cb, v);
+        if (a.splits == 1 && have_d2) tmem_ld8(tmem + lane_base + C::MT + cb, d);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int m = mtile * C::MT + cb + j;
           if (a.splits == 1) {
-            finish(m, static_cast<int>(v[j]));
+            finish(m, static_cast<int>(v[j]), have_d2 ? __uint_as_float(d[j]) : 0.0f);
           } else if (in_bounds(static_cast<unsigned long long>(part - a.partial) + (cb + j) * kI8Rows + row,
                                a.partial_count)) {
             part[(cb + j) * kI8Rows + row] = static_cast<int>(v[j]);
@@ -273,7 +330,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         }
         if (__all_sync(0xffffffffu, mbar_wait(epi2, 0)) && *last_flag) {
           __threadfence();
-          if (gathered) gather();
+          if (tc_out) outlier_mma();
           const int* base = a.partial + static_cast<size_t>(tile_id) * a.splits * C::MT * kI8Rows;
           // 8 columns of 4 K ranges at a time: 32 loads in flight per L2 round
           // trip (exact integer sums, so the order is free)
@@ -298,8 +355,16 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[j] += v[u][j];
             }
+            float d2[8] = {};
+            if (have_d2) {
+              uint32_t d[8];
+              tmem_ld8(tmem + lane_base + C::MT + c0, d);
+              tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 8; ++j) finish(mtile * C::MT + c0 + j, acc[j]);
+              for (int j = 0; j < 8; ++j) d2[j] = __uint_as_float(d[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) finish(mtile * C::MT + c0 + j, acc[j], d2[j]);
           }
         }
       }
