@@ -46,7 +46,8 @@ struct I8Cfg {
   // one 64-channel chunk of the outlier operands: 128 weight rows and MT
   // token rows of 128 bytes (a multiple of 1024: swizzle atoms stay aligned)
   static constexpr int kOChunkBytes = (128 + MT) * 128;
-  static constexpr int kSmemBytes = 1024 + kRingBytes + (2 * STAGES + 6) * 8 + 16;
+  // + per epilogue warp, its copy of the tile's token scales s_x
+  static constexpr int kSmemBytes = 1024 + kRingBytes + (2 * STAGES + 6) * 8 + 16 + 4 * MT * 4;
   static_assert(MT % 16 == 0 && MT >= 16 && MT <= 256, "MMA N for M = 128");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   uint64_t* ofull = epi3 + 1;                      // outlier product ready (commit)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ofull + 1);
   int* last_flag = reinterpret_cast<int*>(tmem_holder + 1);
+  float* sxs = reinterpret_cast<float*>(tmem_holder + 4);  // [4 warps][MT]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // tile order: token tile fastest, so the CTAs that share a weight tile run together
@@ -200,6 +202,15 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       grid_dep_wait();  // s_x, the outlier list, Y and the workspace
       const float swn = n < a.N ? a.sw[n] : 0.0f;
       const int no = min(*a.ocount, a.K);
+      // the tile's token scales, one copy per warp (all loads in flight at
+      // once; the outputs then read them without a global round trip each)
+      float* so = sxs + (warp - 2) * C::MT;
+#pragma unroll
+      for (int j = lane; j < C::MT; j += 32) {
+        const int m = mtile * C::MT + j;
+        so[j] = m < a.M ? a.sx[m] : 0.0f;
+      }
+      __syncwarp();
       const int nch = (no + 63) >> 6;  // 64-channel chunks of the outlier operands
       const bool tc_out =
           no > 0 && static_cast<long long>(nch) * C::kOChunkBytes <= C::kRingBytes;
@@ -280,7 +291,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       // per outlier channel in ascending order from global memory
       auto finish = [&](int m, int v, float d2) {
         if (m >= a.M || n >= a.N) return;
-        float y = __fmul_rn(__fmul_rn(static_cast<float>(v), a.sx[m]), swn);
+        float y = __fmul_rn(__fmul_rn(static_cast<float>(v), so[m - mtile * C::MT]), swn);
         if (have_d2) {
           y = __fadd_rn(y, d2);
         } else {
