@@ -325,20 +325,31 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
       constexpr int kHalfCols = C::MT / 2;
       const int m_base = mtile * C::MT + h * kHalfCols;
       float* part = args.partial + ((pbase + split) * C::MT + h * kHalfCols) * kTileRows;
+      // columns per tensor-memory wait: 32 with one accumulator (every
+      // tile of 64 tokens or more), else 8 per accumulator, summed in order
+      constexpr int kCw = C::kAcc == 1 && kHalfCols % 32 == 0 ? 32 : 8;
 #pragma unroll 1
-      for (int cb = 0; cb < kHalfCols; cb += 8) {
-        float sum[8];
-#pragma unroll
-        for (int ai = 0; ai < C::kAcc; ++ai) {
-          uint32_t v[8];
-          tmem_ld8(tmem + lane_base + C::kDCol + ai * C::MT + h * kHalfCols + cb, v);
+      for (int cb = 0; cb < kHalfCols; cb += kCw) {
+        float sum[kCw];
+        if constexpr (kCw == 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + C::kDCol + h * kHalfCols + cb, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            sum[j] = ai == 0 ? __uint_as_float(v[j]) : sum[j] + __uint_as_float(v[j]);
+          for (int j = 0; j < 32; ++j) sum[j] = __uint_as_float(v[j]);
+        } else {
+#pragma unroll
+          for (int ai = 0; ai < C::kAcc; ++ai) {
+            uint32_t v[8];
+            tmem_ld8(tmem + lane_base + C::kDCol + ai * C::MT + h * kHalfCols + cb, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              sum[j] = ai == 0 ? __uint_as_float(v[j]) : sum[j] + __uint_as_float(v[j]);
+          }
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < kCw; ++j) {
           const int m = m_base + cb + j;
           const float acc = sum[j];
           if (nsplit == 1) {
