@@ -5,6 +5,9 @@
 
 namespace w4 {
 
+// CTA mask of a pair's multicast commits: ranks 0 and 1 of the cluster
+constexpr uint16_t kPairCtas = 0x3;
+
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     w4_tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs args) {
@@ -212,8 +215,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
                         (it > 0 || kk >= C::kAcc) ? 1u : 0u);
         }
         if constexpr (C::PAIR) {
-          mma_commit_pair(&empty[s], 3);
-          mma_commit_pair(&aempty[a], 3);
+          mma_commit_pair(&empty[s], kPairCtas);
+          mma_commit_pair(&aempty[a], kPairCtas);
         } else {
           mma_commit(&empty[s]);
           mma_commit(&aempty[a]);
@@ -221,7 +224,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
       }
       // also on an early exit, so that TMEM is quiet before dealloc
       if constexpr (C::PAIR)
-        mma_commit_pair(accf, 3);
+        mma_commit_pair(accf, kPairCtas);
       else
         mma_commit(accf);
     }
